@@ -1,0 +1,181 @@
+"""NVFP4 quantisation and the NVFP4 layer forward, in the oracle.
+
+TEST INFRASTRUCTURE ONLY (see lmoe_oracle.py).  Shares no code with the CUDA library.
+
+Format.  NVFP4 stores each value as an E2M1 code (1 sign, 2 exponent, 1 mantissa bit: magnitudes
+0, 0.5, 1, 1.5, 2, 3, 4, 6) with two scale levels: a fine scale per 16-element block stored as
+E4M3, and one fp32 scale per tensor ("Nemotron 3 Super" notes, section 3.6: a per-tensor global
+scale plus per-block fine scales; "Nemotron 3 Ultra" summary, method steps: E2M1 data and the
+remark that E2M1 weights carry E4M3 block scales).  The pages fix neither the block size nor the
+rounding rule; this library reads them as: 16 consecutive elements along the reduction dimension
+per block, round-to-nearest-even everywhere, saturating to the largest finite value.
+
+Scale rules (all decisions in float32, the precision the kernels use):
+  per-tensor     g   = amax(|W|) / 2688            (2688 = 6 * 448: E2M1 max times E4M3 max;
+                                                    an all-zero tensor gets g = 1)
+  per-block      s   = E4M3_rne_sat( amax_blk / (6 * g) )
+  element        q   = E2M1_rne_sat( v / (s * g) )  (s decoded back to float32 first; s == 0
+                                                    gives q = 0)
+  dequantised    v'  = q * s * g                     (exact)
+Weights (W1_e, W2_e, W_s1, W_s2) get one g per matrix per expert.  Activations: x and h get a
+dynamic g from the amax of the whole call's tensor; u and u_s (produced inside a GEMM epilogue,
+before any tensor-wide amax exists) use the static g = 1.
+"""
+from __future__ import annotations
+
+from typing import Optional, Sequence
+
+import numpy as np
+
+from . import lmoe_oracle as lo
+
+__all__ = [
+    "E2M1_VALUES", "e2m1_encode", "e2m1_decode", "e4m3_encode", "e4m3_decode", "tensor_scale",
+    "quantize", "dequantize", "qdq", "forward_nvfp4",
+]
+
+E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
+BLOCK = 16
+F32 = np.float32
+
+
+def e2m1_encode(r: np.ndarray) -> np.ndarray:
+    """float32 -> 4-bit code (bit 3 = sign of r, bits 0-2 = magnitude index), nearest-even, saturating."""
+    r = np.asarray(r, dtype=np.float32)
+    a = np.abs(r).astype(np.float64)
+    a = np.minimum(a, 6.0)                               # saturate to the largest finite magnitude
+    hi = np.searchsorted(E2M1_VALUES, a, side="left")    # first grid point >= a
+    hi = np.minimum(hi, 7)
+    lo = np.where(E2M1_VALUES[hi] == a, hi, hi - 1)
+    lo = np.maximum(lo, 0)
+    dlo = a - E2M1_VALUES[lo]
+    dhi = E2M1_VALUES[hi] - a
+    pick = np.where(dlo < dhi, lo, np.where(dhi < dlo, hi, np.where(lo % 2 == 0, lo, hi)))
+    sign = np.signbit(r).astype(np.uint8)
+    return (sign << 3 | pick.astype(np.uint8)).astype(np.uint8)
+
+
+def e2m1_decode(code: np.ndarray) -> np.ndarray:
+    code = np.asarray(code, dtype=np.uint8)
+    mag = E2M1_VALUES[code & 7]
+    return np.where(code & 8, -mag, mag)
+
+
+def e4m3_encode(s: np.ndarray) -> np.ndarray:
+    """Non-negative float32 -> E4M3 byte (bias 7, no infinities, max 448), nearest-even, saturating."""
+    s = np.asarray(s, dtype=np.float32).astype(np.float64)
+    if np.any(s < 0) or np.any(~np.isfinite(s)):
+        raise ValueError("block scales are non-negative and finite")
+    s = np.minimum(s, 448.0)
+    out = np.zeros(s.shape, dtype=np.uint8)
+    sub = s < 2.0 ** -6
+    # subnormals: m * 2^-9, m in 0..8 (m == 8 is the smallest normal 2^-6)
+    m = np.rint(s[sub] / 2.0 ** -9)                     # np.rint rounds half to even
+    out[sub] = np.where(m >= 8, (1 << 3), m).astype(np.uint8)
+    nrm = ~sub
+    if np.any(nrm):
+        v = s[nrm]
+        e = np.floor(np.log2(v))
+        # guard log2 rounding at exact powers of two
+        e = np.where(2.0 ** e > v, e - 1, e)
+        e = np.where(2.0 ** (e + 1) <= v, e + 1, e)
+        q = np.rint(v / 2.0 ** (e - 3))                 # 8..16 (16 = carry into next binade)
+        carry = q >= 16
+        e = np.where(carry, e + 1, e)
+        q = np.where(carry, 8, q)
+        byte = ((e + 7).astype(np.int64) << 3) | (q.astype(np.int64) - 8)
+        byte = np.minimum(byte, 0x7E)                   # 0x7E = 448 (0x7F would be NaN)
+        out[nrm] = byte.astype(np.uint8)
+    return out
+
+
+def e4m3_decode(b: np.ndarray) -> np.ndarray:
+    b = np.asarray(b, dtype=np.uint8).astype(np.int64)
+    e = (b >> 3) & 0xF
+    m = b & 7
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    return np.where(b & 0x80, -val, val)
+
+
+def tensor_scale(a: np.ndarray) -> np.float32:
+    """Per-tensor scale g = amax / 2688 in float32 (1 for an all-zero tensor)."""
+    amax = F32(np.max(np.abs(np.asarray(a, dtype=np.float32)))) if np.size(a) else F32(0)
+    if amax == 0:
+        return F32(1.0)
+    return F32(amax / F32(2688.0))
+
+
+def quantize(a: np.ndarray, g: Optional[np.float32] = None):
+    """Quantise a [rows, cols] matrix along cols in 16-element blocks.
+
+    Returns (codes uint8 [rows, cols] one code per element, scales uint8 [rows, cols/16] E4M3
+    bytes, g float32).  Values are taken as float32 (exact for bf16 inputs)."""
+    a = np.asarray(a, dtype=np.float32)
+    rows, cols = a.shape
+    if cols % BLOCK:
+        raise ValueError("reduction dimension must be a multiple of 16")
+    g = tensor_scale(a) if g is None else F32(g)
+    blk = a.reshape(rows, cols // BLOCK, BLOCK)
+    amax_blk = np.max(np.abs(blk), axis=2)                      # float32, exact
+    den6 = F32(F32(6.0) * g)
+    s_f = (amax_blk / den6).astype(np.float32)                  # float32 division, RNE
+    s_b = e4m3_encode(s_f)
+    s_dec = e4m3_decode(s_b).astype(np.float32)                 # exact
+    den = (s_dec * g).astype(np.float32)                        # float32 product, RNE
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = np.where(den[..., None] > 0, blk / den[..., None], F32(0)).astype(np.float32)
+    # keep the sign of v for exact zeros produced by an all-zero block (s == 0)
+    r = np.where(den[..., None] > 0, r, np.copysign(F32(0), blk)).astype(np.float32)
+    codes = e2m1_encode(r).reshape(rows, cols)
+    return codes, s_b, g
+
+
+def dequantize(codes: np.ndarray, scales: np.ndarray, g) -> np.ndarray:
+    rows, cols = codes.shape
+    v = e2m1_decode(codes).reshape(rows, cols // BLOCK, BLOCK)
+    s = e4m3_decode(scales)[..., None]
+    return (v * s * float(g)).reshape(rows, cols)
+
+
+def qdq(a: np.ndarray, g: Optional[np.float32] = None) -> np.ndarray:
+    """Quantise then dequantise (float64 result)."""
+    c, s, gg = quantize(a, g)
+    return dequantize(c, s, gg)
+
+
+def forward_nvfp4(w: "lo.OracleWeights", x: np.ndarray, k: int, idx: Optional[np.ndarray] = None,
+                  g_x: Optional[np.float32] = None, g_h: Optional[np.float32] = None):
+    """Layer forward with NVFP4 routed and shared experts (weights and activations); router,
+    W_down and W_up stay at the device's bf16 values.
+
+    g_x / g_h: per-call activation scales.  They depend on the whole call's x / h, so a caller that
+    evaluates a sample of tokens passes the full batch's values."""
+    logits = lo.router_logits(x, w.w_router, w.b_router)
+    if idx is None:
+        idx = lo.topk(logits, k)
+    gate = lo.softmax_gates(logits, idx)
+    h = x @ w.w_down.T
+    if g_x is None:
+        g_x = tensor_scale(x.astype(np.float32))
+    if g_h is None:
+        g_h = tensor_scale(h.astype(np.float32))
+    hq = qdq(h.astype(np.float32), g_h)
+    xq = qdq(x.astype(np.float32), g_x)
+    one = F32(1.0)
+    z = np.zeros_like(h)
+    for e in range(w.n_experts):
+        tt, kk = np.nonzero(idx == e)
+        if tt.size == 0:
+            continue
+        w1 = qdq(w.w1(e).astype(np.float32))
+        w2 = qdq(w.w2(e).astype(np.float32))
+        u = lo.sqrelu(hq[tt] @ w1.T)
+        o = qdq(u.astype(np.float32), one) @ w2.T
+        z[tt] += gate[tt, kk][:, None] * o
+    ws1 = qdq(w.ws1.astype(np.float32))
+    ws2 = qdq(w.ws2.astype(np.float32))
+    us = lo.sqrelu(xq @ ws1.T)
+    s = qdq(us.astype(np.float32), one) @ ws2.T
+    y = z @ w.w_up.T + s
+    return {"y": y, "idx": idx, "gate": gate, "logits": logits, "h": h, "z": z,
+            "g_x": g_x, "g_h": g_h}
