@@ -1,0 +1,364 @@
+"""Throughput of the B200 LatentMoE layer (Super shape) on seeded synthetic inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|skewed|tiny]
+                    [--impl ours|reference]
+
+One step = one full forward of the layer (router, top-K, dispatch, W_down, routed experts, combine,
+W_up, shared expert) over one batch.  The default workload is the Super-shaped decode/verify batch
+(T = 256).  With N > 1 (torchrun, one process per GPU) every rank runs an independent replica:
+the layer has no cross-GPU step, so nothing is exchanged and scaling is weak.
+
+Prints ONE JSON line on rank 0.  `value` is whole-job tokens/s with inputs resident in HBM; `e2e`
+is the same through lmoe_forward_host (pinned host x in, y/idx/gate out, copies inside the timed
+region); `roofline` reports the dominant kernel's algorithmic bytes (or FLOPs) per launch over its
+CUDA-event duration against the measured peak; `cpu_baseline` times the fp64 oracle on a bounded
+sample on the host cores.  `--impl reference` times that oracle alone as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import lmoe_inputs as inp  # noqa: E402
+
+METRIC = "LatentMoE layer tokens/s (Super shape, T=256 & 16K); % of HBM / TC roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DEFAULT_STEPS = {"tiny": 200, "decode": 400, "skewed": 40, "prefill": 20}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------ helpers
+def algorithmic_work(wl, counts: np.ndarray):
+    """Bytes and FLOPs one forward must move / compute, from the actual routing (counts per expert)."""
+    s = wl.shape
+    d, l, n, k, m, ms = s.d, s.latent, s.n_experts, s.top_k, s.expert_ffn, s.shared_ffn
+    t = wl.tokens
+    tk = t * k
+    touched = int((counts > 0).sum())
+    w_exp = touched * m * l * 2                                  # bf16 bytes of one expert matrix set (W1 or W2)
+    up = {"bytes": w_exp + tk * l * 2 + tk * m * 2, "flops": 2 * tk * m * l}
+    down = {"bytes": w_exp + tk * m * 2 + tk * l * 2 + tk * 4, "flops": 2 * tk * m * l}
+    layer_bytes = (2 * w_exp + (n + l) * d * 2 + ms * d * 2 + d * (l + ms) * 2 + 2 * t * d * 2 + tk * 8)
+    layer_flops = 2 * t * ((n + l) * d + ms * d + d * (l + ms)) + 4 * tk * m * l
+    return {"expert_up": up, "expert_down": down, "layer": {"bytes": layer_bytes, "flops": layer_flops},
+            "touched_experts": touched}
+
+
+def make_device_layer(wl, device):
+    import torch
+
+    import latentmoe_expert_layer_b200 as lm
+    w = inp.make_weights(wl)
+    to = lambda a: (torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+                    if w.dtype == "bf16" else torch.from_numpy(np.ascontiguousarray(a))).to(device)
+    dev = {k: to(getattr(w, k)) for k in ("w_router", "w_down", "w_up", "w1", "w2", "ws1", "ws2")}
+    b = torch.from_numpy(w.b_router).to(device) if w.b_router is not None else None
+    layer = lm.LatentMoE(wl.shape, wl.tokens, precision=wl.precision, router_bias=wl.router_bias,
+                         device=device.index)
+    layer.load_weights(b_router=b, **dev)
+    torch.cuda.synchronize(device)
+    del dev
+    torch.cuda.empty_cache()
+    return layer, w
+
+
+def cpu_baseline(wl, w, budget_s: float = 20.0):
+    """The fp64 oracle, as it stands, on a bounded token sample of the same workload."""
+    from oracle import lmoe_oracle as lo
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    ow = lo.OracleWeights(w)
+    x = lo.lift(inp.make_x(wl), "bf16")
+    done, t0, sample = 0, time.perf_counter(), 0
+    while time.perf_counter() - t0 < budget_s and done < wl.tokens:
+        n = min(4, wl.tokens - done)
+        lo.forward(ow, x[done:done + n], wl.shape.top_k)
+        done += n
+    el = time.perf_counter() - t0
+    return {"value": done / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {done} of the {wl.tokens} tokens, fp64 numpy oracle, {el:.1f} s"}
+
+
+# ------------------------------------------------------------------------------------------ arms
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return
+    from oracle import lmoe_oracle as lo
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    w = inp.make_weights(wl)
+    ow = lo.OracleWeights(w)
+    x = lo.lift(inp.make_x(wl), "bf16")
+    per_step = 1 if wl.shape.n_experts > 64 else wl.tokens   # bounded sample per step
+    pos = 0
+
+    def step():
+        nonlocal pos
+        lo.forward(ow, x[pos:pos + per_step], wl.shape.top_k)
+        pos = (pos + per_step) % max(1, wl.tokens - per_step + 1)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    val = per_step * args.steps / el
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "tokens": wl.tokens, "sample_tokens_per_step": per_step},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{per_step} token(s) of the {wl.tokens}-token batch per step"},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, wl, rank, world):
+    import torch
+    import torch.distributed as dist
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    layer, w = make_device_layer(wl, device)
+    x_bits = inp.make_x(wl)
+    x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).to(device)
+    t = wl.tokens
+    y = torch.empty((t, wl.shape.d), dtype=torch.bfloat16, device=device)
+    idx = torch.empty((t, wl.shape.top_k), dtype=torch.int32, device=device)
+    gate = torch.empty((t, wl.shape.top_k), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        layer.forward(x, y, idx, gate)
+    torch.cuda.synchronize(device)
+    st = layer.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    counts = layer.inspect("counts").cpu().numpy()
+
+    # ---- device-timed region (inputs resident in HBM) ----
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    layer.profile(True)
+    barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            layer.forward(x, y, idx, gate)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+    barrier()
+    layer.profile(False)
+    ms = e0.elapsed_time(e1)
+    stage_ms, recorded, launches = layer.profile_read()
+    if layer.device_status() != 0:
+        raise RuntimeError("device status not clean after the timed region")
+    ms_max = ms
+    if world > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_max = float(tt.item())
+
+    # ---- end to end through the host-buffer entry point ----
+    xh = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty((t, wl.shape.d), dtype=torch.bfloat16).pin_memory()
+    ih = torch.empty((t, wl.shape.top_k), dtype=torch.int32).pin_memory()
+    gh = torch.empty((t, wl.shape.top_k), dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 200))
+    for _ in range(2):
+        layer.forward_host(xh, yh, ih, gh)
+    torch.cuda.synchronize(device)
+    barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        layer.forward_host(xh, yh, ih, gh)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+
+    if rank != 0:
+        layer.close()
+        return
+    work = algorithmic_work(wl, counts)
+    pk, pk_kind = peaks()
+    # dominant kernel: the stage with the largest device time
+    dom = max(stage_ms, key=stage_ms.get)
+    per_launch_ms = stage_ms[dom] / max(1, recorded)
+    decode_like = wl.tokens * wl.shape.top_k <= 48 * wl.shape.n_experts
+    if dom in ("expert_up", "expert_down"):
+        unit_work = work[dom]
+    else:
+        unit_work = None
+    roof = None
+    if unit_work is not None:
+        if decode_like:
+            ach = unit_work["bytes"] / (per_launch_ms * 1e-3) / 1e9
+            roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": ach / pk["hbm_gbs"], "traffic": None, "algorithmic_bytes": unit_work["bytes"],
+                    "launch_ms": per_launch_ms, "peak_source": pk_kind}
+        else:
+            ach = unit_work["flops"] / (per_launch_ms * 1e-3) / 1e12
+            p = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+            roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": p, "unit": "TFLOP/s",
+                    "frac": ach / p, "traffic": None, "algorithmic_flops": unit_work["flops"],
+                    "launch_ms": per_launch_ms, "peak_source": pk_kind + " (sustained)"}
+    step_ms = ms_max / args.steps
+    lay = work["layer"]
+    layer_roof = {"bytes_per_step": lay["bytes"], "flops_per_step": lay["flops"],
+                  "hbm_frac": lay["bytes"] / (step_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                  "tc_frac": lay["flops"] / (step_ms * 1e-3) / 1e12 / pk.get("bf16_tflops_sustained",
+                                                                               pk["bf16_tflops"])}
+    line = {
+        "metric": METRIC,
+        "value": world * t * args.steps / (ms_max * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1/fan_in) weights, N(0,1) x, bf16",
+        "config": {"workload": wl.name, "tokens": t, "d": wl.shape.d, "latent": wl.shape.latent,
+                   "experts": wl.shape.n_experts, "top_k": wl.shape.top_k, "expert_ffn": wl.shape.expert_ffn,
+                   "shared_ffn": wl.shape.shared_ffn, "precision": wl.precision,
+                   "parallelism": f"{world} independent replica(s)",
+                   "l2": "inputs larger than L2: every step streams all touched expert weights "
+                         f"({work['touched_experts']} experts, {2 * work['touched_experts'] * wl.shape.expert_ffn * wl.shape.latent * 2 / 1e9:.2f} GB)"},
+        "roofline": roof,
+        "layer_roofline": layer_roof,
+        "stages_ms_per_step": {k: v / max(1, recorded) for k, v in stage_ms.items()},
+        "e2e": {"value": world * t * e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": t * wl.shape.d * 2,
+                "d2h_bytes_per_step": t * wl.shape.d * 2 + t * wl.shape.top_k * 8, "steps": e2e_steps},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, w)
+    layer.close()
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode", choices=sorted(inp.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = inp.workload(args.workload)
+    if args.steps is None:
+        args.steps = DEFAULT_STEPS.get(args.workload.split("_")[0], 20)
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, wl, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

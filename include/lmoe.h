@@ -1,0 +1,155 @@
+/*
+ * lmoe.h - C ABI of a B200 (sm_100a) LatentMoE expert layer, forward pass.
+ *
+ * The layer (LatentMoE, "Nemotron 3 Super" notes on guokunwang.com, section 3.2; shapes from the
+ * section 3.1 architecture table), per token x in R^d:
+ *   logits = W_r x (+ b)                       gating network, full dimension d
+ *   S, g   = top-K of the logits (value desc, lower expert index first on ties);
+ *            g = softmax over the K selected logits
+ *   h      = W_down x                          W_down in R^{l x d}
+ *   z      = sum_k g_k * W2_{S_k} sqrelu(W1_{S_k} h)   routed experts in the latent space l -> m -> l
+ *   y      = W_up z + W_s2 sqrelu(W_s1 x)      W_up in R^{d x l}; shared expert d -> m_s -> d
+ * where sqrelu(v) = max(v, 0)^2 elementwise.  The pages leave the expert nonlinearity, the router
+ * normalisation and the NVFP4 block size open; this library fixes them to squared ReLU (non-gated,
+ * no biases), softmax over the selected K, and 16-element E2M1 blocks with E4M3 block scales and an
+ * fp32 per-tensor scale.
+ *
+ * Conventions
+ *   - Every call returns lmoe_status; nothing throws across the ABI.
+ *   - Matrices are row-major [out, in] (the pages' W_down in R^{l x d}, W_up in R^{d x l}).
+ *   - bf16 means IEEE bfloat16 bit patterns (uint16).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Device calls are asynchronous on
+ *     it; no call below synchronises the host unless it says so.
+ *   - Device pointers must be 16-byte aligned; a misaligned pointer returns LMOE_ERR_INVALID_ARG.
+ *   - Thread safety: one handle must not be used by two host threads at once; forward calls on one
+ *     handle share its workspace, so two forward calls on different streams must not overlap.
+ */
+#ifndef LMOE_H
+#define LMOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct lmoe_ctx* lmoe_handle;
+
+typedef enum {
+  LMOE_OK = 0,
+  LMOE_ERR_INVALID_ARG = 1,    /* null/misaligned pointer, bad enum value */
+  LMOE_ERR_SHAPE = 2,          /* T > max_tokens, T < 0 */
+  LMOE_ERR_UNSUPPORTED = 3,    /* a config this build does not implement (see lmoe_create) */
+  LMOE_ERR_OOM = 4,            /* device allocation failed */
+  LMOE_ERR_CUDA = 5,           /* a CUDA runtime/driver call failed */
+  LMOE_ERR_NOT_LOADED = 6,     /* forward before lmoe_load_weights */
+  LMOE_ERR_DEVICE_TIMEOUT = 7, /* a kernel's bounded wait gave up (see lmoe_get_device_status) */
+  LMOE_ERR_DEVICE_INDEX = 8,   /* a kernel found an out-of-range index and skipped the access */
+  LMOE_ERR_NO_DEVICE = 9       /* no sm_100 device, or the device index is invalid */
+} lmoe_status;
+
+typedef enum { LMOE_PREC_BF16 = 0, LMOE_PREC_NVFP4 = 1 } lmoe_precision;
+typedef enum { LMOE_DTYPE_BF16 = 0, LMOE_DTYPE_F32 = 1 } lmoe_dtype;
+
+typedef struct {
+  int32_t d;           /* model dimension (multiple of 64) */
+  int32_t latent;      /* latent dimension l (multiple of 64) */
+  int32_t n_experts;   /* N, 1..1024 */
+  int32_t top_k;       /* K, 1..min(32, N) */
+  int32_t expert_ffn;  /* m, routed expert hidden (multiple of 64) */
+  int32_t shared_ffn;  /* m_s, shared expert hidden (multiple of 64) */
+  int32_t max_tokens;  /* largest T a forward call may pass; sizes the workspace */
+  int32_t precision;   /* lmoe_precision: NVFP4 quantises routed+shared experts (weights and inputs) */
+  int32_t has_router_bias; /* 1: a per-expert fp32 bias is added to the router logits */
+} lmoe_config;
+
+/* Device pointers to the caller's weights, all of element type `dtype`, row-major [out, in].
+ * With LMOE_DTYPE_F32 the router stays fp32 (scored with fp32 FMAs) and every other matrix is
+ * converted to bf16 (round to nearest even) at load.  The library copies everything into its own
+ * memory; the caller may free these buffers once `stream` has passed the load. */
+typedef struct {
+  const void* w_router;  /* [N, d] */
+  const float* b_router; /* [N] fp32, or NULL (required iff has_router_bias) */
+  const void* w_down;    /* [l, d]   (W_down) */
+  const void* w_up;      /* [d, l]   (W_up) */
+  const void* w1;        /* [N, m, l] expert up matrices */
+  const void* w2;        /* [N, l, m] expert down matrices */
+  const void* ws1;       /* [m_s, d] shared expert */
+  const void* ws2;       /* [d, m_s] shared expert */
+  int32_t dtype;         /* lmoe_dtype */
+} lmoe_weights;
+
+/* Create a layer on CUDA device `device` and allocate its workspace for cfg->max_tokens tokens.
+ * Errors: INVALID_ARG (null), UNSUPPORTED (a dimension not a multiple of 64, N > 1024, K > 32,
+ * K > N), NO_DEVICE (device missing or not compute capability 10.0), OOM. */
+lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out);
+
+/* Copy (and, for NVFP4, quantise) the weights into library-owned device memory, enqueued on
+ * `stream`.  May be called again to replace the weights. */
+lmoe_status lmoe_load_weights(lmoe_handle h, const lmoe_weights* w, void* stream);
+
+/* y = LatentMoE(x) for T tokens, all pointers on the device:
+ *   x         [T, d]  bf16, read only
+ *   y         [T, d]  bf16, written
+ *   topk_idx  [T, K]  int32 expert ids per token in slot order, written; may be NULL
+ *   topk_gate [T, K]  fp32 softmax gates, written; may be NULL
+ * T = 0 returns LMOE_OK and enqueues nothing.  T > max_tokens: LMOE_ERR_SHAPE.
+ * Enqueued on `stream`; device-side faults are reported by lmoe_get_device_status. */
+lmoe_status lmoe_forward(lmoe_handle h, const void* x, int32_t T, void* y, int32_t* topk_idx, float* topk_gate,
+                         void* stream);
+
+/* Same as lmoe_forward, with x/y/topk_idx/topk_gate in HOST memory (pinned memory gives
+ * asynchronous copies).  The host-to-device copy of x, the layer and the device-to-host copies of
+ * the outputs are all enqueued on `stream`; the caller synchronises before reading the outputs. */
+lmoe_status lmoe_forward_host(lmoe_handle h, const void* x_host, int32_t T, void* y_host, int32_t* topk_idx_host,
+                              float* topk_gate_host, void* stream);
+
+/* Synchronise the handle's device and return the sticky device status raised by any kernel since
+ * the last call (DEVICE_TIMEOUT or DEVICE_INDEX), then clear it.  LMOE_OK if none. */
+lmoe_status lmoe_get_device_status(lmoe_handle h);
+
+/* Intermediate buffers of the last forward call, for inspection and tests (device pointers owned by
+ * the handle, valid until the next forward / destroy).  `count` receives the element count. */
+typedef enum {
+  LMOE_BUF_LOGITS = 0,     /* fp32 [T, N]   router logits (bias not included) */
+  LMOE_BUF_COUNTS = 1,     /* int32 [N]     assignments per expert */
+  LMOE_BUF_OFFSETS = 2,    /* int32 [N+1]   exclusive prefix sum of counts */
+  LMOE_BUF_ROW_OF = 3,     /* int32 [T*K]   grouped row of assignment (t, k) */
+  LMOE_BUF_TOK_OF_ROW = 4, /* int32 [T*K]   token of grouped row r */
+  LMOE_BUF_H = 5,          /* bf16 [T, l]   latent h = W_down x */
+  LMOE_BUF_Z = 6,          /* bf16 [T, l + m_s] columns 0..l-1: latent sum z; the rest: sqrelu(W_s1 x) */
+  LMOE_BUF_U = 7           /* bf16 [T*K, m] expert hidden activations, grouped rows */
+} lmoe_buffer;
+lmoe_status lmoe_inspect(lmoe_handle h, int32_t which, void** dev_ptr, int64_t* count);
+
+/* Per-stage device timing of forward calls (CUDA events recorded on the forward's own stream
+ * between consecutive kernels).  lmoe_profile(h, 1) clears the record and starts recording the next
+ * forward calls (at most 1024); lmoe_profile(h, 0) stops.  lmoe_profile_read synchronises on the
+ * recorded events and returns, per stage, the summed milliseconds over the recorded calls, the
+ * number of recorded calls, and the number of kernel launches one forward call makes. */
+typedef enum {
+  LMOE_STAGE_ROUTER = 0,      /* router logits + W_down (one fused GEMM when the router is bf16) */
+  LMOE_STAGE_SHARED_UP = 1,   /* sqrelu(W_s1 x) */
+  LMOE_STAGE_TOPK = 2,        /* top-K, softmax gates, per-chunk expert histogram */
+  LMOE_STAGE_GROUPING = 3,    /* expert offsets and grouped-GEMM work lists */
+  LMOE_STAGE_SCATTER = 4,     /* stable row assignment + gather of latent rows */
+  LMOE_STAGE_EXPERT_UP = 5,   /* u = sqrelu(W1_e h), grouped */
+  LMOE_STAGE_EXPERT_DOWN = 6, /* o = g * W2_e u, grouped */
+  LMOE_STAGE_COMBINE = 7,     /* z = sum_k o */
+  LMOE_STAGE_OUTPUT = 8,      /* y = W_up z + W_s2 u_s */
+  LMOE_NUM_STAGES = 9
+} lmoe_stage;
+lmoe_status lmoe_profile(lmoe_handle h, int32_t enable);
+lmoe_status lmoe_profile_read(lmoe_handle h, double* stage_ms /* [LMOE_NUM_STAGES] */, int32_t* forwards,
+                              int32_t* launches_per_forward);
+
+/* Human-readable name of a status code (static string). */
+const char* lmoe_status_string(lmoe_status s);
+
+/* Free everything the handle owns (synchronises its device first).  NULL is ignored. */
+void lmoe_destroy(lmoe_handle h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LMOE_H */

@@ -1,0 +1,180 @@
+"""Python binding of the sm_100a LatentMoE layer library (liblmoe.so).
+
+Argument marshalling only: tensors are passed to the C ABI as raw device pointers plus the current
+CUDA stream.  Every step of the layer runs in the library's CUDA kernels; there is no Python or CPU
+fallback, and importing this package raises if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = ["LatentMoE", "LmoeError", "lib", "STATUS", "BUF", "SYMBOLS", "STAGES", "library_path"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "liblmoe.so")
+
+if not os.path.exists(library_path):
+    raise ImportError(f"{library_path} is missing: build it with `python latentmoe_expert_layer_b200/build.py`"
+                      " or __graft_entry__.build()")
+
+lib = ctypes.CDLL(library_path)
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "shape out of range", 3: "unsupported configuration",
+          4: "device out of memory", 5: "CUDA error", 6: "weights not loaded",
+          7: "device-side wait timed out", 8: "device-side index out of range", 9: "no suitable CUDA device"}
+BUF = {"logits": 0, "counts": 1, "offsets": 2, "row_of": 3, "tok_of_row": 4, "h": 5, "z": 6, "u": 7}
+PREC = {"bf16": 0, "nvfp4": 1}
+DTYPE = {torch.bfloat16: 0, torch.float32: 1}
+
+# every extern "C" symbol declared in include/lmoe.h
+SYMBOLS = ("lmoe_create", "lmoe_load_weights", "lmoe_forward", "lmoe_forward_host", "lmoe_get_device_status",
+           "lmoe_inspect", "lmoe_profile", "lmoe_profile_read", "lmoe_status_string", "lmoe_destroy")
+STAGES = ("router", "shared_up", "topk", "grouping", "scatter", "expert_up", "expert_down", "combine", "output")
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("d", "latent", "n_experts", "top_k", "expert_ffn", "shared_ffn",
+                                             "max_tokens", "precision", "has_router_bias")]
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [("w_router", ctypes.c_void_p), ("b_router", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
+                ("w_up", ctypes.c_void_p), ("w1", ctypes.c_void_p), ("w2", ctypes.c_void_p),
+                ("ws1", ctypes.c_void_p), ("ws2", ctypes.c_void_p), ("dtype", ctypes.c_int32)]
+
+
+_vp, _i32, _i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+lib.lmoe_create.argtypes = [ctypes.POINTER(_Config), ctypes.c_int, ctypes.POINTER(_vp)]
+lib.lmoe_load_weights.argtypes = [_vp, ctypes.POINTER(_Weights), _vp]
+lib.lmoe_forward.argtypes = [_vp, _vp, _i32, _vp, _vp, _vp, _vp]
+lib.lmoe_forward_host.argtypes = [_vp, _vp, _i32, _vp, _vp, _vp, _vp]
+lib.lmoe_get_device_status.argtypes = [_vp]
+lib.lmoe_inspect.argtypes = [_vp, _i32, ctypes.POINTER(_vp), ctypes.POINTER(_i64)]
+lib.lmoe_profile.argtypes = [_vp, _i32]
+lib.lmoe_profile_read.argtypes = [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i32), ctypes.POINTER(_i32)]
+lib.lmoe_status_string.argtypes = [ctypes.c_int]
+lib.lmoe_status_string.restype = ctypes.c_char_p
+lib.lmoe_destroy.argtypes = [_vp]
+lib.lmoe_destroy.restype = None
+for _f in ("lmoe_create", "lmoe_load_weights", "lmoe_forward", "lmoe_forward_host", "lmoe_get_device_status",
+           "lmoe_inspect", "lmoe_profile", "lmoe_profile_read"):
+    getattr(lib, _f).restype = ctypes.c_int
+
+
+class LmoeError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({code})")
+        self.code = code
+
+
+def _check(code: int, what: str) -> None:
+    if code != 0:
+        raise LmoeError(code, what)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return t.data_ptr()
+
+
+class _DevArray:
+    """__cuda_array_interface__ view of a library-owned device buffer (for lmoe_inspect)."""
+
+    def __init__(self, ptr: int, count: int, typestr: str):
+        self.__cuda_array_interface__ = {"shape": (count,), "typestr": typestr, "data": (ptr, True),
+                                         "version": 3, "strides": None}
+
+
+_BUF_TYPES = {"logits": "<f4", "counts": "<i4", "offsets": "<i4", "row_of": "<i4", "tok_of_row": "<i4",
+              "h": "<u2", "z": "<u2", "u": "<u2"}
+
+
+class LatentMoE:
+    """One LatentMoE layer on one GPU.
+
+    shape: object with d, latent, n_experts, top_k, expert_ffn, shared_ffn attributes.
+    """
+
+    def __init__(self, shape, max_tokens: int, precision: str = "bf16", router_bias: bool = False,
+                 device: int = 0):
+        cfg = _Config(shape.d, shape.latent, shape.n_experts, shape.top_k, shape.expert_ffn, shape.shared_ffn,
+                      max_tokens, PREC[precision], int(router_bias))
+        h = _vp()
+        _check(lib.lmoe_create(ctypes.byref(cfg), device, ctypes.byref(h)), "lmoe_create")
+        self._h = h
+        self.shape = shape
+        self.max_tokens = max_tokens
+        self.device = torch.device("cuda", device)
+
+    def load_weights(self, w_router, w_down, w_up, w1, w2, ws1, ws2, b_router=None, stream=None) -> None:
+        ts = (w_router, w_down, w_up, w1, w2, ws1, ws2)
+        dt = {t.dtype for t in ts}
+        if len(dt) != 1 or next(iter(dt)) not in DTYPE:
+            raise ValueError("all weight matrices must share one dtype, bf16 or fp32")
+        w = _Weights(_ptr(w_router), _ptr(b_router), _ptr(w_down), _ptr(w_up), _ptr(w1), _ptr(w2), _ptr(ws1),
+                     _ptr(ws2), DTYPE[next(iter(dt))])
+        _check(lib.lmoe_load_weights(self._h, ctypes.byref(w), self._stream(stream)), "lmoe_load_weights")
+
+    def _stream(self, stream) -> int:
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        return s.cuda_stream
+
+    def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                gate: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+        t = x.shape[0]
+        k = self.shape.top_k
+        if y is None:
+            y = torch.empty((t, self.shape.d), dtype=torch.bfloat16, device=self.device)
+        if idx is None:
+            idx = torch.empty((t, k), dtype=torch.int32, device=self.device)
+        if gate is None:
+            gate = torch.empty((t, k), dtype=torch.float32, device=self.device)
+        _check(lib.lmoe_forward(self._h, _ptr(x), t, _ptr(y), _ptr(idx), _ptr(gate), self._stream(stream)),
+               "lmoe_forward")
+        return y, idx, gate
+
+    def forward_host(self, x: torch.Tensor, y: torch.Tensor, idx: Optional[torch.Tensor] = None,
+                     gate: Optional[torch.Tensor] = None, stream=None) -> None:
+        """x, y, idx, gate are CPU tensors (pinned for asynchronous copies)."""
+        _check(lib.lmoe_forward_host(self._h, _ptr(x), x.shape[0], _ptr(y), _ptr(idx), _ptr(gate),
+                                     self._stream(stream)), "lmoe_forward_host")
+
+    def device_status(self) -> int:
+        return lib.lmoe_get_device_status(self._h)
+
+    def inspect(self, name: str) -> torch.Tensor:
+        p, n = _vp(), _i64()
+        _check(lib.lmoe_inspect(self._h, BUF[name], ctypes.byref(p), ctypes.byref(n)), "lmoe_inspect")
+        if n.value == 0:
+            return torch.empty(0)
+        t = torch.as_tensor(_DevArray(p.value, n.value, _BUF_TYPES[name]), device=self.device)
+        return t.clone()
+
+    def profile(self, enable: bool) -> None:
+        """Start (clearing the record) or stop per-stage CUDA-event timing of forward calls."""
+        _check(lib.lmoe_profile(self._h, int(enable)), "lmoe_profile")
+
+    def profile_read(self):
+        """(dict stage -> summed ms over the recorded calls, recorded calls, kernel launches per call)."""
+        ms = (ctypes.c_double * len(STAGES))()
+        n, launches = _i32(), _i32()
+        _check(lib.lmoe_profile_read(self._h, ms, ctypes.byref(n), ctypes.byref(launches)), "lmoe_profile_read")
+        return dict(zip(STAGES, list(ms))), n.value, launches.value
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            lib.lmoe_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

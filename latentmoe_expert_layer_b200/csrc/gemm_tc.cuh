@@ -1,0 +1,341 @@
+// Persistent, warp-specialised tcgen05 GEMM used for every contraction of the LatentMoE layer.
+//
+//   out[tok, f] = epi( sum_k W[f, k] * act[tok, k] )
+//
+// W (weights, K-major, bf16) is the MMA's A operand: 128 output features per tile fill the
+// M = 128 rows of the tensor core.  The activations (K-major, bf16) are the B operand: up to BN_MAX
+// tokens per tile form N, rounded up to a multiple of 16.  With tokens on N, an expert that holds
+// only ~11 tokens (the T = 256 decode batch spread over 512 experts) costs an N = 16 MMA instead of a
+// 128-row tile that is 90 % padding, and every expert weight byte is streamed exactly once per token
+// tile.
+//
+// Roles (192 threads):
+//   warp 0      TMA producer: one lane streams W and activation tiles into a STAGES-deep ring
+//   warp 1      MMA issuer: allocates TMEM, one lane issues tcgen05.mma into one of two TMEM
+//               accumulators (double buffered, so the epilogue of tile i overlaps the MMAs of i+1)
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes 32*(w%4)..),
+//               elementwise op, transpose through shared memory, coalesced 16-byte stores
+//
+// Work units are (weight row block, token block) pairs.  Dense GEMMs enumerate them from the
+// launch arguments; the grouped expert GEMMs read a unit list that the routing kernels built on the
+// device, so no host round trip sits between routing and the experts.
+#pragma once
+#include "ptx.cuh"
+
+namespace lmoe {
+
+enum EpiKind : int {
+  EPI_BF16 = 0,           // out = bf16(acc)
+  EPI_F32 = 1,            // out = acc (fp32)
+  EPI_SQRELU_BF16 = 2,    // out = bf16(max(acc, 0)^2)
+  EPI_ROWSCALE_BF16 = 3,  // out = bf16(acc * row_scale[token row])
+  EPI_ROUTER = 4,         // features < split_feat: fp32 to out2; others: bf16 to out (column f - split)
+};
+
+// One unit of GEMM work.  a_row: first W row of the tile; b_row: first activation row (also the
+// output row); f0: first output feature (column) of the tile; nm = n_valid | (m_valid << 16) with
+// n_valid tokens (1..BN_MAX) and m_valid features (1..128, a multiple of 32).
+struct GemmUnit {
+  int a_row, b_row, f0, nm;
+};
+
+struct GemmArgs {
+  int num_k_blocks;           // K / 64
+  // dense schedule (units == nullptr)
+  int dense_units;            // number of units
+  int dense_ftiles;           // feature tiles
+  int dense_feat;             // output features (rows of W)
+  int dense_tokens;           // tokens (rows of act)
+  // grouped schedule
+  const GemmUnit* units;      // device list
+  const int* num_units;       // device count
+  // epilogue
+  int epi;
+  void* out;
+  long long ldo;              // output row pitch (elements)
+  int out_col0;               // output column offset
+  float* out2;                // EPI_ROUTER fp32 destination
+  long long ld2;
+  int split_feat;
+  const float* row_scale;     // EPI_ROWSCALE_BF16
+  unsigned* status;           // device status word
+  unsigned long long timeout_ns;
+};
+
+constexpr int GEMM_THREADS = 192;
+constexpr int BLOCK_M = 128;
+constexpr int BLOCK_K = 64;                 // 64 bf16 = one 128-byte swizzle row
+constexpr int A_STAGE_BYTES = BLOCK_M * BLOCK_K * 2;
+constexpr int EPI_STAGE_BYTES = 32 * 32 * 4;  // per epilogue warp: 32 tokens x 32 features fp32
+
+template <int BN_MAX, int STAGES>
+struct GemmSmem {
+  static constexpr int B_STAGE_BYTES = BN_MAX * BLOCK_K * 2;
+  static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+  static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
+  static constexpr int BAR_OFF = EPI_OFF + 4 * EPI_STAGE_BYTES;
+  static constexpr int BYTES = BAR_OFF + 256;
+  static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment of the base
+  static constexpr uint32_t TMEM_COLS = (2 * BN_MAX < 32) ? 32 : 2 * BN_MAX;
+};
+
+template <int BN_MAX>
+__device__ __forceinline__ GemmUnit unit_at(const GemmArgs& a, int u) {
+  if (a.units != nullptr) return a.units[u];
+  GemmUnit r;
+  const int ft = u % a.dense_ftiles;
+  const int tt = u / a.dense_ftiles;
+  r.a_row = ft * BLOCK_M;
+  r.f0 = r.a_row;
+  r.b_row = tt * BN_MAX;
+  const int mv = min(BLOCK_M, a.dense_feat - r.f0);
+  const int nv = min(BN_MAX, a.dense_tokens - r.b_row);
+  r.nm = nv | (mv << 16);
+  return r;
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16_rn(float v) {
+  __nv_bfloat16 b = __float2bfloat16_rn(v);
+  return *reinterpret_cast<uint16_t*>(&b);
+}
+
+template <int BN_MAX, int STAGES, int BOXN>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_act,
+                   const GemmArgs args) {
+  using S = GemmSmem<BN_MAX, STAGES>;
+  static_assert(BN_MAX % BOXN == 0 && BOXN % 8 == 0, "token box must tile the token block");
+  static_assert(BN_MAX % 16 == 0 && BN_MAX <= 256, "MMA N limit");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&map_w);
+    tma_prefetch_desc(&map_act);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, S::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_units = (args.units != nullptr) ? *args.num_units : args.dense_units;
+  const int nkb = args.num_k_blocks;
+  const uint64_t tmo = args.timeout_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_a = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        const GemmUnit un = unit_at<BN_MAX>(args, u);
+        const int nv = un.nm & 0xFFFF;
+        const int nbox = (nv + BOXN - 1) / BOXN;
+        const uint32_t bytes = A_STAGE_BYTES + nbox * BOXN * BLOCK_K * 2;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, tmo)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * S::STAGE_BYTES;
+          uint8_t* sb = sa + A_STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          tma_load_2d(sa, &map_w, &full[stage], kb * BLOCK_K, un.a_row, pol_w);
+          for (int i = 0; i < nbox; ++i)
+            tma_load_2d(sb + i * BOXN * BLOCK_K * 2, &map_act, &full[stage], kb * BLOCK_K, un.b_row + i * BOXN,
+                        pol_a);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // Give every load still in flight a bounded chance to land before the CTA exits.
+        atomicOr(args.status, DEV_STATUS_TIMEOUT);
+        volatile int never = 0;
+        int s = stage, p = phase;
+        for (int i = 0; i < STAGES && i < issued; ++i) {
+          if (--s < 0) {
+            s = STAGES - 1;
+            p ^= 1;
+          }
+          mbar_wait_bounded(&full[s], p, &never, 100000000ull);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        const GemmUnit un = unit_at<BN_MAX>(args, u);
+        const int nv = un.nm & 0xFFFF;
+        const uint32_t n_mma = (uint32_t)((nv + 15) & ~15);
+        const uint32_t idesc = idesc_bf16_f32(BLOCK_M, n_mma);
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, tmo)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN_MAX);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, tmo)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * S::STAGE_BYTES);
+          const uint64_t da = smem_desc_sw128(sa);
+          const uint64_t db = smem_desc_sw128(sa + A_STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < BLOCK_K / 16; ++k)  // K = 16 per MMA: +32 bytes = +2 in the address field
+            umma_bf16(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) atomicOr(args.status, DEV_STATUS_TIMEOUT);
+      // every MMA this thread issued completes before TMEM is released
+      umma_commit(drain);
+      volatile int never = 0;
+      mbar_wait_bounded(drain, 0, &never, 100000000ull);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    uint8_t* stg = smem + S::EPI_OFF + q * EPI_STAGE_BYTES;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+      const GemmUnit un = unit_at<BN_MAX>(args, u);
+      const int nv = un.nm & 0xFFFF;
+      const int mv = un.nm >> 16;
+      if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, tmo)) {
+        if (lane == 0) atomicOr(args.status, DEV_STATUS_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
+      const int nchunks = (nv + 31) >> 5;
+      const bool feat_ok = (q * 32) < mv;
+      const int f = un.f0 + q * 32;  // first feature of this warp's 32
+      for (int c = 0; c < nchunks; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), r);
+        tmem_ld_wait();
+        if (c == nchunks - 1) {
+          // accumulator fully read by this warp: hand it back to the MMA issuer
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+        const int row0 = un.b_row + c * 32;
+        const int nrows = min(32, nv - c * 32);
+        bool f32_out = (args.epi == EPI_F32) || (args.epi == EPI_ROUTER && un.f0 < args.split_feat);
+        if (args.epi == EPI_ROWSCALE_BF16) {
+          const float mys = (lane < nrows) ? args.row_scale[row0 + lane] : 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * __shfl_sync(0xffffffffu, mys, j));
+        } else if (args.epi == EPI_SQRELU_BF16) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float v = fmaxf(__uint_as_float(r[j]), 0.f);
+            r[j] = __float_as_uint(v * v);
+          }
+        }
+        __syncwarp();
+        if (f32_out) {
+          float* s32 = reinterpret_cast<float*>(stg);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) s32[j * 32 + lane] = __uint_as_float(r[j]);
+          __syncwarp();
+          float* dst = (args.epi == EPI_ROUTER) ? args.out2 : reinterpret_cast<float*>(args.out);
+          const long long ld = (args.epi == EPI_ROUTER) ? args.ld2 : args.ldo;
+          const int col = (args.epi == EPI_ROUTER) ? f : (args.out_col0 + f);
+          if (feat_ok) {
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int j = it * 4 + (lane >> 3);
+              if (j < nrows) {
+                const uint4 v = *reinterpret_cast<const uint4*>(s32 + j * 32 + (lane & 7) * 4);
+                *reinterpret_cast<uint4*>(dst + (long long)(row0 + j) * ld + col + (lane & 7) * 4) = v;
+              }
+            }
+          }
+        } else {
+          uint16_t* s16 = reinterpret_cast<uint16_t*>(stg);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) s16[j * 32 + lane] = f32_to_bf16_rn(__uint_as_float(r[j]));
+          __syncwarp();
+          uint16_t* dst = reinterpret_cast<uint16_t*>(args.out);
+          const int col = (args.epi == EPI_ROUTER) ? (f - args.split_feat) : (args.out_col0 + f);
+          if (feat_ok) {
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int j = it * 8 + (lane >> 2);
+              if (j < nrows) {
+                const uint4 v = *reinterpret_cast<const uint4*>(s16 + j * 32 + (lane & 3) * 8);
+                *reinterpret_cast<uint4*>(dst + (long long)(row0 + j) * args.ldo + col + (lane & 3) * 8) = v;
+              }
+            }
+          }
+        }
+        __syncwarp();
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::TMEM_COLS);
+  }
+}
+
+}  // namespace lmoe

@@ -1,0 +1,590 @@
+// Host side of the LatentMoE layer library: argument checking, workspace, weight preparation,
+// tensor maps and the launch sequence of one forward pass.  Everything on the path runs in the
+// kernels of this directory; the host only validates, enqueues and reports.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/lmoe.h"
+#include "gemm_tc.cuh"
+#include "routing.cuh"
+
+using namespace lmoe;
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool load_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// 2-D bf16 tensor map over rows x cols (row pitch ld elements), 64-element x box_rows tiles,
+// 128-byte swizzle (the layout the MMA descriptors expect).
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The two GEMM shapes: small token tiles with a deep ring (weight streaming at decode sizes) and
+// 256-token tiles (tensor-core bound at prefill sizes).
+enum Variant { V_SMALL = 0, V_LARGE = 1 };
+constexpr int V_BN[2] = {64, 256};
+constexpr int V_STAGES[2] = {8, 4};
+constexpr int V_BOXN[2] = {16, 64};
+
+template <int V>
+struct VT {
+  static constexpr int BN = V_BN[V], ST = V_STAGES[V], BOX = V_BOXN[V];
+  static void* fn() { return reinterpret_cast<void*>(gemm_tc_kernel<BN, ST, BOX>); }
+  static int smem() { return GemmSmem<BN, ST>::ALLOC; }
+};
+
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+struct lmoe_ctx {
+  lmoe_config cfg{};
+  int device = 0;
+  int num_sms = 148;
+  bool loaded = false;
+  bool router_f32 = false;
+  bool fused_router = false;
+  unsigned long long timeout_ns = kDefaultTimeoutNs;
+
+  // weights (library-owned)
+  __nv_bfloat16* w_rd = nullptr;   // [N + l, d]: router rows then W_down rows (bf16 router)
+  float* w_r32 = nullptr;          // [N, d] fp32 router
+  __nv_bfloat16* w_down = nullptr; // [l, d] when not stacked with the router
+  float* b_router = nullptr;       // [N]
+  __nv_bfloat16* w_cat = nullptr;  // [d, l + m_s]: W_up columns then W_s2 columns
+  __nv_bfloat16* ws1 = nullptr;    // [m_s, d]
+  __nv_bfloat16* w1 = nullptr;     // [N * m, l]
+  __nv_bfloat16* w2 = nullptr;     // [N * l, m]
+  CUtensorMap map_rd{}, map_r{}, map_down{}, map_cat{}, map_ws1{}, map_w1{}, map_w2{};
+
+  // workspace
+  float* logits = nullptr;
+  int* idx = nullptr;
+  float* gate = nullptr;
+  int* chunk_counts = nullptr;
+  int* chunk_base = nullptr;
+  int* counts = nullptr;
+  int* offsets = nullptr;
+  int* row_of = nullptr;
+  int* tok_of_row = nullptr;
+  float* gate_of_row = nullptr;
+  __nv_bfloat16* h = nullptr;
+  __nv_bfloat16* h_perm = nullptr;
+  __nv_bfloat16* u = nullptr;
+  __nv_bfloat16* o = nullptr;
+  __nv_bfloat16* zu = nullptr;
+  GemmUnit* units1 = nullptr;
+  GemmUnit* units2 = nullptr;
+  int* num_units = nullptr;  // [2]
+  unsigned* status = nullptr;
+  int max_units1 = 0, max_units2 = 0;
+  CUtensorMap map_hperm[2]{}, map_u[2]{}, map_zu[2]{};
+
+  // x tensor maps, cached by (pointer, T)
+  const void* x_cached = nullptr;
+  int x_cached_T = -1;
+  CUtensorMap map_x[2]{};
+
+  // staging for lmoe_forward_host
+  __nv_bfloat16* x_dev = nullptr;
+  __nv_bfloat16* y_dev = nullptr;
+  int* idx_dev = nullptr;
+  float* gate_dev = nullptr;
+
+  int last_T = 0;
+
+  // stage profiler
+  static constexpr int kProfMax = 1024;
+  bool prof_on = false;
+  int prof_n = 0;
+  int launches = 0;
+  std::vector<cudaEvent_t> prof_ev;  // kProfMax x (LMOE_NUM_STAGES + 1)
+};
+
+namespace {
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    cudaGetDevice(&prev);
+    if (prev != dev) cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+template <typename T>
+bool dalloc(T** p, size_t elems) {
+  *p = nullptr;
+  if (elems == 0) elems = 1;
+  return cudaMalloc(reinterpret_cast<void**>(p), elems * sizeof(T)) == cudaSuccess;
+}
+
+void free_all(lmoe_ctx* c) {
+  void* ptrs[] = {c->w_rd,   c->w_r32,  c->w_down, c->b_router,  c->w_cat,      c->ws1,        c->w1,
+                  c->w2,     c->logits, c->idx,    c->gate,      c->chunk_counts, c->chunk_base, c->counts,
+                  c->offsets, c->row_of, c->tok_of_row, c->gate_of_row, c->h, c->h_perm, c->u,
+                  c->o,      c->zu,     c->units1, c->units2,    c->num_units,  c->status,     c->x_dev,
+                  c->y_dev,  c->idx_dev, c->gate_dev};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+}
+
+int n_chunks_for(int T, int* chunk_tokens) {
+  int ct = (T + 127) / 128;
+  if (ct < 4) ct = 4;
+  *chunk_tokens = ct;
+  return (T + ct - 1) / ct;
+}
+
+lmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA; }
+
+template <int V>
+cudaError_t launch_gemm_v(const CUtensorMap& mw, const CUtensorMap& ma, const GemmArgs& a, int grid,
+                          cudaStream_t s) {
+  gemm_tc_kernel<VT<V>::BN, VT<V>::ST, VT<V>::BOX><<<grid, GEMM_THREADS, VT<V>::smem(), s>>>(mw, ma, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(int v, const CUtensorMap& mw, const CUtensorMap& ma, const GemmArgs& a, int grid,
+                        cudaStream_t s) {
+  return v == V_SMALL ? launch_gemm_v<V_SMALL>(mw, ma, a, grid, s) : launch_gemm_v<V_LARGE>(mw, ma, a, grid, s);
+}
+
+GemmArgs base_args(lmoe_ctx* c, int K) {
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.num_k_blocks = K / BLOCK_K;
+  a.status = c->status;
+  a.timeout_ns = c->timeout_ns;
+  return a;
+}
+
+// Dense GEMM: out[tok, f] = epi(sum_k W[f, k] act[tok, k]) over feat x tokens.
+cudaError_t dense_gemm(lmoe_ctx* c, int v, const CUtensorMap& mw, const CUtensorMap& ma, int feat, int tokens,
+                       int K, int epi, void* out, long long ldo, int col0, float* out2, long long ld2, int split,
+                       cudaStream_t s) {
+  GemmArgs a = base_args(c, K);
+  a.dense_ftiles = (feat + BLOCK_M - 1) / BLOCK_M;
+  a.dense_units = a.dense_ftiles * ((tokens + V_BN[v] - 1) / V_BN[v]);
+  a.dense_feat = feat;
+  a.dense_tokens = tokens;
+  a.epi = epi;
+  a.out = out;
+  a.ldo = ldo;
+  a.out_col0 = col0;
+  a.out2 = out2;
+  a.ld2 = ld2;
+  a.split_feat = split;
+  const int grid = a.dense_units < c->num_sms ? a.dense_units : c->num_sms;
+  return launch_gemm(v, mw, ma, a, grid, s);
+}
+
+cudaError_t grouped_gemm(lmoe_ctx* c, int v, const CUtensorMap& mw, const CUtensorMap& ma, const GemmUnit* units,
+                         const int* num_units, int K, int epi, void* out, long long ldo, const float* row_scale,
+                         cudaStream_t s) {
+  GemmArgs a = base_args(c, K);
+  a.units = units;
+  a.num_units = num_units;
+  a.epi = epi;
+  a.out = out;
+  a.ldo = ldo;
+  a.row_scale = row_scale;
+  return launch_gemm(v, mw, ma, a, c->num_sms, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lmoe_status_string(lmoe_status s) {
+  switch (s) {
+    case LMOE_OK: return "ok";
+    case LMOE_ERR_INVALID_ARG: return "invalid argument";
+    case LMOE_ERR_SHAPE: return "shape out of range";
+    case LMOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LMOE_ERR_OOM: return "device out of memory";
+    case LMOE_ERR_CUDA: return "CUDA error";
+    case LMOE_ERR_NOT_LOADED: return "weights not loaded";
+    case LMOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case LMOE_ERR_DEVICE_INDEX: return "device-side index out of range";
+    case LMOE_ERR_NO_DEVICE: return "no suitable CUDA device";
+  }
+  return "unknown status";
+}
+
+lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
+  if (!cfg || !out) return LMOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  const lmoe_config& g = *cfg;
+  if (g.d <= 0 || g.latent <= 0 || g.n_experts <= 0 || g.top_k <= 0 || g.expert_ffn <= 0 || g.shared_ffn <= 0 ||
+      g.max_tokens <= 0)
+    return LMOE_ERR_INVALID_ARG;
+  if (g.precision != LMOE_PREC_BF16 && g.precision != LMOE_PREC_NVFP4) return LMOE_ERR_INVALID_ARG;
+  if (g.d % 64 || g.latent % 64 || g.expert_ffn % 64 || g.shared_ffn % 64) return LMOE_ERR_UNSUPPORTED;
+  if (g.n_experts > 1024 || g.top_k > 32 || g.top_k > g.n_experts) return LMOE_ERR_UNSUPPORTED;
+  if (g.precision == LMOE_PREC_NVFP4) return LMOE_ERR_UNSUPPORTED;
+  const long long tk = (long long)g.max_tokens * g.top_k;
+  if (tk > 0x7fffffffLL / 2) return LMOE_ERR_UNSUPPORTED;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) return LMOE_ERR_NO_DEVICE;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess || prop.major != 10) return LMOE_ERR_NO_DEVICE;
+  if (!load_encode()) return LMOE_ERR_CUDA;
+  DeviceGuard dg(device);
+
+  lmoe_ctx* c = new lmoe_ctx();
+  c->cfg = g;
+  c->device = device;
+  c->num_sms = prop.multiProcessorCount;
+  const int N = g.n_experts, K = g.top_k, d = g.d, l = g.latent, m = g.expert_ffn, ms = g.shared_ffn;
+  const long long T = g.max_tokens;
+  const int nft1 = (m + BLOCK_M - 1) / BLOCK_M, nft2 = (l + BLOCK_M - 1) / BLOCK_M;
+  c->max_units1 = (int)(nft1 * (N + (tk + V_BN[V_SMALL] - 1) / V_BN[V_SMALL]));
+  c->max_units2 = (int)(nft2 * (N + (tk + V_BN[V_SMALL] - 1) / V_BN[V_SMALL]));
+  bool ok = true;
+  ok = ok && dalloc(&c->logits, T * N) && dalloc(&c->idx, tk) && dalloc(&c->gate, tk);
+  ok = ok && dalloc(&c->chunk_counts, 128LL * N) && dalloc(&c->chunk_base, 128LL * N);
+  ok = ok && dalloc(&c->counts, N) && dalloc(&c->offsets, N + 1);
+  ok = ok && dalloc(&c->row_of, tk) && dalloc(&c->tok_of_row, tk) && dalloc(&c->gate_of_row, tk);
+  ok = ok && dalloc(&c->h, T * l) && dalloc(&c->h_perm, tk * l) && dalloc(&c->u, tk * m) && dalloc(&c->o, tk * l);
+  ok = ok && dalloc(&c->zu, T * (l + ms));
+  ok = ok && dalloc(&c->units1, c->max_units1) && dalloc(&c->units2, c->max_units2) && dalloc(&c->num_units, 2);
+  ok = ok && dalloc(&c->status, 1);
+  if (!ok) {
+    free_all(c);
+    delete c;
+    return LMOE_ERR_OOM;
+  }
+  cudaMemset(c->status, 0, sizeof(unsigned));
+  // rows that no expert writes must still be finite for the MMA (they are masked in the epilogue)
+  cudaMemset(c->h_perm, 0, tk * l * 2);
+  cudaMemset(c->u, 0, tk * m * 2);
+  cudaMemset(c->zu, 0, T * (l + ms) * 2);
+  for (int v = 0; v < 2; ++v) {
+    ok = ok && make_map(&c->map_hperm[v], c->h_perm, tk, l, l, V_BOXN[v]);
+    ok = ok && make_map(&c->map_u[v], c->u, tk, m, m, V_BOXN[v]);
+    ok = ok && make_map(&c->map_zu[v], c->zu, T, l + ms, l + ms, V_BOXN[v]);
+  }
+  ok = ok && cudaFuncSetAttribute(VT<V_SMALL>::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  VT<V_SMALL>::smem()) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(VT<V_LARGE>::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  VT<V_LARGE>::smem()) == cudaSuccess;
+  if (!ok || cudaDeviceSynchronize() != cudaSuccess) {
+    free_all(c);
+    delete c;
+    return LMOE_ERR_CUDA;
+  }
+  (void)d;
+  *out = c;
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream) {
+  if (!c || !w) return LMOE_ERR_INVALID_ARG;
+  if (!w->w_router || !w->w_down || !w->w_up || !w->w1 || !w->w2 || !w->ws1 || !w->ws2) return LMOE_ERR_INVALID_ARG;
+  if (w->dtype != LMOE_DTYPE_BF16 && w->dtype != LMOE_DTYPE_F32) return LMOE_ERR_INVALID_ARG;
+  if (c->cfg.has_router_bias && !w->b_router) return LMOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {w->w_router, w->w_down, w->w_up, w->w1, w->w2, w->ws1, w->ws2};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const lmoe_config& g = c->cfg;
+  const int N = g.n_experts, d = g.d, l = g.latent, m = g.expert_ffn, ms = g.shared_ffn;
+  const int f32 = w->dtype == LMOE_DTYPE_F32;
+
+  // release weights of a previous load
+  void* old[] = {c->w_rd, c->w_r32, c->w_down, c->b_router, c->w_cat, c->ws1, c->w1, c->w2};
+  cudaStreamSynchronize(s);
+  for (void* p : old)
+    if (p) cudaFree(p);
+  c->w_rd = nullptr;
+  c->w_r32 = nullptr;
+  c->w_down = nullptr;
+  c->b_router = nullptr;
+  c->w_cat = nullptr;
+  c->ws1 = c->w1 = c->w2 = nullptr;
+  c->loaded = false;
+
+  c->router_f32 = f32;
+  c->fused_router = !f32 && (N % BLOCK_M == 0);
+  bool ok = true;
+  auto conv = [&](const void* src, long long rows, int cols, long long src_ld, __nv_bfloat16* dst, long long dst_ld,
+                  int col0) {
+    const long long total = rows * cols;
+    int blocks = (int)((total + 255) / 256);
+    if (blocks > 4 * 148 * 8) blocks = 4 * 148 * 8;
+    convert_2d_kernel<<<blocks, 256, 0, s>>>(src, f32, rows, cols, src_ld, dst, dst_ld, col0);
+    return cudaGetLastError() == cudaSuccess;
+  };
+  if (c->router_f32) {
+    ok = ok && dalloc(&c->w_r32, (size_t)N * d) &&
+         cudaMemcpyAsync(c->w_r32, w->w_router, (size_t)N * d * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    ok = ok && dalloc(&c->w_down, (size_t)l * d) && conv(w->w_down, l, d, d, c->w_down, d, 0);
+  } else if (c->fused_router) {
+    ok = ok && dalloc(&c->w_rd, (size_t)(N + l) * d);
+    ok = ok && conv(w->w_router, N, d, d, c->w_rd, d, 0) && conv(w->w_down, l, d, d, c->w_rd + (size_t)N * d, d, 0);
+  } else {
+    ok = ok && dalloc(&c->w_rd, (size_t)N * d) && conv(w->w_router, N, d, d, c->w_rd, d, 0);
+    ok = ok && dalloc(&c->w_down, (size_t)l * d) && conv(w->w_down, l, d, d, c->w_down, d, 0);
+  }
+  if (g.has_router_bias)
+    ok = ok && dalloc(&c->b_router, N) &&
+         cudaMemcpyAsync(c->b_router, w->b_router, (size_t)N * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+  ok = ok && dalloc(&c->w_cat, (size_t)d * (l + ms));
+  ok = ok && conv(w->w_up, d, l, l, c->w_cat, l + ms, 0) && conv(w->ws2, d, ms, ms, c->w_cat, l + ms, l);
+  ok = ok && dalloc(&c->ws1, (size_t)ms * d) && conv(w->ws1, ms, d, d, c->ws1, d, 0);
+  ok = ok && dalloc(&c->w1, (size_t)N * m * l) && conv(w->w1, (long long)N * m, l, l, c->w1, l, 0);
+  ok = ok && dalloc(&c->w2, (size_t)N * l * m) && conv(w->w2, (long long)N * l, m, m, c->w2, m, 0);
+  if (!ok) return LMOE_ERR_OOM;
+  if (c->fused_router) ok = ok && make_map(&c->map_rd, c->w_rd, N + l, d, d, BLOCK_M);
+  if (!c->router_f32 && !c->fused_router) ok = ok && make_map(&c->map_r, c->w_rd, N, d, d, BLOCK_M);
+  if (!c->fused_router) ok = ok && make_map(&c->map_down, c->w_down, l, d, d, BLOCK_M);
+  ok = ok && make_map(&c->map_cat, c->w_cat, d, l + ms, l + ms, BLOCK_M);
+  ok = ok && make_map(&c->map_ws1, c->ws1, ms, d, d, BLOCK_M);
+  ok = ok && make_map(&c->map_w1, c->w1, (uint64_t)N * m, l, l, BLOCK_M);
+  ok = ok && make_map(&c->map_w2, c->w2, (uint64_t)N * l, m, m, BLOCK_M);
+  if (!ok) return LMOE_ERR_CUDA;
+  c->loaded = true;
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32_t* topk_idx, float* topk_gate,
+                         void* stream) {
+  if (!c) return LMOE_ERR_INVALID_ARG;
+  if (T < 0 || T > c->cfg.max_tokens) return LMOE_ERR_SHAPE;
+  if (!c->loaded) return LMOE_ERR_NOT_LOADED;
+  if (T == 0) return LMOE_OK;
+  if (!x || !y) return LMOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || (topk_idx && !aligned16(topk_idx)) || (topk_gate && !aligned16(topk_gate)))
+    return LMOE_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const lmoe_config& g = c->cfg;
+  const int N = g.n_experts, K = g.top_k, d = g.d, l = g.latent, m = g.expert_ffn, ms = g.shared_ffn;
+  const long long TK = (long long)T * K;
+  const long long TKmax = (long long)g.max_tokens * K;
+  const int vd = T <= 512 ? V_SMALL : V_LARGE;
+  const int vg = TK <= 48LL * N ? V_SMALL : V_LARGE;
+
+  if (x != c->x_cached || T != c->x_cached_T) {
+    bool ok = true;
+    for (int v = 0; v < 2; ++v) ok = ok && make_map(&c->map_x[v], x, T, d, d, V_BOXN[v]);
+    if (!ok) return LMOE_ERR_CUDA;
+    c->x_cached = x;
+    c->x_cached_T = T;
+  }
+  int* idx = topk_idx ? topk_idx : c->idx;
+  float* gate = topk_gate ? topk_gate : c->gate;
+  cudaError_t e = cudaSuccess;
+  auto chk = [&](cudaError_t r) {
+    if (e == cudaSuccess) e = r;
+  };
+  const bool prof = c->prof_on && c->prof_n < lmoe_ctx::kProfMax;
+  cudaEvent_t* ev = prof ? &c->prof_ev[(size_t)c->prof_n * (LMOE_NUM_STAGES + 1)] : nullptr;
+  auto mark = [&](int i) {
+    if (prof) chk(cudaEventRecord(ev[i], s));
+  };
+  int launches = 0;
+  mark(0);
+
+  // 1. router logits and the latent h = W_down x
+  if (c->fused_router) {
+    chk(dense_gemm(c, vd, c->map_rd, c->map_x[vd], N + l, T, d, EPI_ROUTER, c->h, l, 0, c->logits, N, N, s));
+    launches += 1;
+  } else {
+    launches += 2;
+    if (c->router_f32) {
+      router_f32_kernel<<<T, 256, d * sizeof(float), s>>>(reinterpret_cast<const __nv_bfloat16*>(x), c->w_r32, d,
+                                                          N, c->logits);
+      chk(cudaGetLastError());
+    } else {
+      chk(dense_gemm(c, vd, c->map_r, c->map_x[vd], N, T, d, EPI_F32, c->logits, N, 0, nullptr, 0, 0, s));
+    }
+    chk(dense_gemm(c, vd, c->map_down, c->map_x[vd], l, T, d, EPI_BF16, c->h, l, 0, nullptr, 0, 0, s));
+  }
+  mark(1);
+  // 2. shared expert, first matrix: zu[:, l:] = sqrelu(W_s1 x)
+  chk(dense_gemm(c, vd, c->map_ws1, c->map_x[vd], ms, T, d, EPI_SQRELU_BF16, c->zu, l + ms, l, nullptr, 0, 0, s));
+  mark(2);
+  // 3. top-K + softmax + per-chunk histogram
+  int ct;
+  const int nch = n_chunks_for(T, &ct);
+  topk_hist_kernel<<<nch, TOPK_WARPS * 32, N * sizeof(int), s>>>(c->logits, c->b_router, T, N, K, ct, idx, gate,
+                                                                 c->chunk_counts);
+  chk(cudaGetLastError());
+  mark(3);
+  // 4. expert offsets and grouped-GEMM unit lists
+  UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1};
+  UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2};
+  scan_units_kernel<<<1, 1024, 0, s>>>(c->chunk_counts, nch, N, c->counts, c->offsets, c->chunk_base, l1, l2,
+                                       c->status);
+  chk(cudaGetLastError());
+  mark(4);
+  // 5. stable grouping and gather of latent rows
+  scatter_gather_kernel<<<nch, SCATTER_WARPS * 32, N * sizeof(int), s>>>(
+      idx, gate, c->chunk_base, T, N, K, ct, c->h, l, c->row_of, c->tok_of_row, c->gate_of_row, c->h_perm,
+      c->status);
+  chk(cudaGetLastError());
+  mark(5);
+  // 6. expert up: u = sqrelu(W1_e h)
+  chk(grouped_gemm(c, vg, c->map_w1, c->map_hperm[vg], c->units1, c->num_units, l, EPI_SQRELU_BF16, c->u, m,
+                   nullptr, s));
+  mark(6);
+  // 7. expert down with the gate folded in: o = g * (W2_e u)
+  chk(grouped_gemm(c, vg, c->map_w2, c->map_u[vg], c->units2, c->num_units + 1, m, EPI_ROWSCALE_BF16, c->o, l,
+                   c->gate_of_row, s));
+  mark(7);
+  // 8. latent combine: zu[:, :l] = sum_k o[row_of[t, k]]
+  {
+    const long long threads = (long long)T * (l / 8);
+    const int blocks = (int)((threads + 255) / 256);
+    combine_kernel<<<blocks, 256, 0, s>>>(c->o, c->row_of, T, K, l, c->zu, l + ms, TKmax, c->status);
+    chk(cudaGetLastError());
+  }
+  mark(8);
+  // 9. y = [z | sqrelu(W_s1 x)] [W_up | W_s2]^T
+  chk(dense_gemm(c, vd, c->map_cat, c->map_zu[vd], d, T, l + ms, EPI_BF16, y, d, 0, nullptr, 0, 0, s));
+  mark(9);
+  launches += 8;
+  c->launches = launches;
+  if (prof) ++c->prof_n;
+  c->last_T = T;
+  (void)TK;
+  return cuda_status(e);
+}
+
+lmoe_status lmoe_forward_host(lmoe_handle c, const void* x_host, int32_t T, void* y_host, int32_t* idx_host,
+                              float* gate_host, void* stream) {
+  if (!c) return LMOE_ERR_INVALID_ARG;
+  if (T < 0 || T > c->cfg.max_tokens) return LMOE_ERR_SHAPE;
+  if (!c->loaded) return LMOE_ERR_NOT_LOADED;
+  if (T == 0) return LMOE_OK;
+  if (!x_host || !y_host) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  const lmoe_config& g = c->cfg;
+  const size_t xb = (size_t)g.max_tokens * g.d * 2, kb = (size_t)g.max_tokens * g.top_k;
+  if (!c->x_dev) {
+    if (!dalloc(&c->x_dev, xb / 2) || !dalloc(&c->y_dev, xb / 2) || !dalloc(&c->idx_dev, kb) ||
+        !dalloc(&c->gate_dev, kb))
+      return LMOE_ERR_OOM;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)T * g.d * 2;
+  if (cudaMemcpyAsync(c->x_dev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return LMOE_ERR_CUDA;
+  lmoe_status st = lmoe_forward(c, c->x_dev, T, c->y_dev, c->idx_dev, c->gate_dev, stream);
+  if (st != LMOE_OK) return st;
+  if (cudaMemcpyAsync(y_host, c->y_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return LMOE_ERR_CUDA;
+  const size_t ib = (size_t)T * g.top_k * 4;
+  if (idx_host && cudaMemcpyAsync(idx_host, c->idx_dev, ib, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return LMOE_ERR_CUDA;
+  if (gate_host && cudaMemcpyAsync(gate_host, c->gate_dev, ib, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return LMOE_ERR_CUDA;
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_get_device_status(lmoe_handle c) {
+  if (!c) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  if (cudaDeviceSynchronize() != cudaSuccess) return LMOE_ERR_CUDA;
+  unsigned st = 0;
+  if (cudaMemcpy(&st, c->status, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return LMOE_ERR_CUDA;
+  cudaMemset(c->status, 0, sizeof(unsigned));
+  if (st & DEV_STATUS_TIMEOUT) return LMOE_ERR_DEVICE_TIMEOUT;
+  if (st & DEV_STATUS_BAD_INDEX) return LMOE_ERR_DEVICE_INDEX;
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_inspect(lmoe_handle c, int32_t which, void** dev_ptr, int64_t* count) {
+  if (!c || !dev_ptr || !count) return LMOE_ERR_INVALID_ARG;
+  const lmoe_config& g = c->cfg;
+  const long long T = c->last_T, TK = T * g.top_k;
+  switch (which) {
+    case LMOE_BUF_LOGITS: *dev_ptr = c->logits; *count = T * g.n_experts; break;
+    case LMOE_BUF_COUNTS: *dev_ptr = c->counts; *count = g.n_experts; break;
+    case LMOE_BUF_OFFSETS: *dev_ptr = c->offsets; *count = g.n_experts + 1; break;
+    case LMOE_BUF_ROW_OF: *dev_ptr = c->row_of; *count = TK; break;
+    case LMOE_BUF_TOK_OF_ROW: *dev_ptr = c->tok_of_row; *count = TK; break;
+    case LMOE_BUF_H: *dev_ptr = c->h; *count = T * g.latent; break;
+    case LMOE_BUF_Z: *dev_ptr = c->zu; *count = T * (g.latent + g.shared_ffn); break;
+    case LMOE_BUF_U: *dev_ptr = c->u; *count = TK * g.expert_ffn; break;
+    default: return LMOE_ERR_INVALID_ARG;
+  }
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_profile(lmoe_handle c, int32_t enable) {
+  if (!c) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  if (enable && c->prof_ev.empty()) {
+    c->prof_ev.resize((size_t)lmoe_ctx::kProfMax * (LMOE_NUM_STAGES + 1));
+    for (auto& e : c->prof_ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return LMOE_ERR_CUDA;
+  }
+  if (enable) c->prof_n = 0;
+  c->prof_on = enable != 0;
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_profile_read(lmoe_handle c, double* stage_ms, int32_t* forwards, int32_t* launches) {
+  if (!c || !stage_ms) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  for (int i = 0; i < LMOE_NUM_STAGES; ++i) stage_ms[i] = 0.0;
+  for (int f = 0; f < c->prof_n; ++f) {
+    cudaEvent_t* ev = &c->prof_ev[(size_t)f * (LMOE_NUM_STAGES + 1)];
+    if (cudaEventSynchronize(ev[LMOE_NUM_STAGES]) != cudaSuccess) return LMOE_ERR_CUDA;
+    for (int i = 0; i < LMOE_NUM_STAGES; ++i) {
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, ev[i], ev[i + 1]) != cudaSuccess) return LMOE_ERR_CUDA;
+      stage_ms[i] += ms;
+    }
+  }
+  if (forwards) *forwards = c->prof_n;
+  if (launches) *launches = c->launches;
+  return LMOE_OK;
+}
+
+void lmoe_destroy(lmoe_handle c) {
+  if (!c) return;
+  {
+    DeviceGuard dg(c->device);
+    cudaDeviceSynchronize();
+    for (auto& e : c->prof_ev) cudaEventDestroy(e);
+    free_all(c);
+  }
+  delete c;
+}
+
+}  // extern "C"

@@ -1,0 +1,344 @@
+// Routing, dispatch grouping and combine kernels of the LatentMoE layer.
+//
+// Router + top-K: the gating network scores every token in the full model dimension d and keeps the
+// K best of N experts ("Nemotron 3 Super" notes, section 3.1 table: top-22 of 512; section 3.2: the
+// gating network stays in dimension d).  The gate is the softmax over the K selected logits.
+//
+// Dispatch: the (token, slot) assignments are grouped by expert with a histogram and an exclusive
+// prefix sum, so that the latent rows h[t] sent to one expert sit contiguously ("the compressed
+// representation is routed to the expanded expert set", section 3.2).  The grouping is stable in
+// (token, slot) order, which makes every map (row_of, tok_of_row) uniquely defined.
+//
+// Combine: z[t] = sum_k o[row_of[t, k]], in slot order, fp32 accumulation (the gate is already
+// folded into o by the second expert GEMM's epilogue).
+#pragma once
+#include <cuda_bf16.h>
+#include "gemm_tc.cuh"
+#include "ptx.cuh"
+
+namespace lmoe {
+
+// ------------------------------------------------------------------------------------------------
+// fp32 router (used when the router weights are kept in fp32): logits[t, e] = x[t, :] . W_r[e, :]
+// one block per token; x row staged in shared memory; one warp per expert, lanes stride over d.
+// ------------------------------------------------------------------------------------------------
+__global__ void router_f32_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ w, int d,
+                                  int n_experts, float* __restrict__ logits) {
+  extern __shared__ float xs[];
+  const int t = blockIdx.x;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) xs[j] = __bfloat162float(x[(long long)t * d + j]);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int e = warp; e < n_experts; e += nw) {
+    const float* we = w + (long long)e * d;
+    float acc = 0.f;
+    for (int j = lane; j < d; j += 32) acc = fmaf(xs[j], we[j], acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) logits[(long long)t * n_experts + e] = acc;
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// top-K + softmax + per-chunk expert histogram.  One block per chunk of `chunk_tokens` tokens, one
+// warp per token.  Each lane keeps its best remaining candidate (value desc, index asc); K rounds
+// of a warp arg-max pick the experts in output order.  Requires K <= 32 and N <= 32 * 32.
+// ------------------------------------------------------------------------------------------------
+constexpr int TOPK_WARPS = 8;
+constexpr int MAX_PER_LANE = 32;  // N <= 1024
+
+__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+__global__ void __launch_bounds__(TOPK_WARPS * 32)
+    topk_hist_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int n_experts,
+                     int k, int chunk_tokens, int* __restrict__ topk_idx, float* __restrict__ topk_gate,
+                     int* __restrict__ chunk_counts) {
+  extern __shared__ int s_counts[];  // [n_experts]
+  for (int e = threadIdx.x; e < n_experts; e += blockDim.x) s_counts[e] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t_begin = blockIdx.x * chunk_tokens;
+  const int t_end = min(T, t_begin + chunk_tokens);
+  const int per_lane = (n_experts + 31) >> 5;
+  for (int t = t_begin + warp; t < t_end; t += TOPK_WARPS) {
+    const float* lrow = logits + (long long)t * n_experts;
+    float v[MAX_PER_LANE];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < MAX_PER_LANE; ++i) {
+      const int e = i * 32 + lane;
+      v[i] = -INFINITY;
+      if (i < per_lane && e < n_experts) v[i] = lrow[e] + (bias ? bias[e] : 0.f);
+    }
+    // local best of this lane
+    auto local_best = [&](float& bv, int& bi) {
+      bv = -INFINITY;
+      bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < MAX_PER_LANE; ++i) {
+        const int e = i * 32 + lane;
+        if (i < per_lane && e < n_experts && !((taken >> i) & 1u) && better(v[i], e, bv, bi)) {
+          bv = v[i];
+          bi = e;
+        }
+      }
+    };
+    float bv;
+    int bi;
+    local_best(bv, bi);
+    float sel_v = 0.f;
+    int sel_i = 0;
+    for (int r = 0; r < k; ++r) {
+      float wv = bv;
+      int wi = bi;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, wv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, wi, o);
+        if (better(ov, oi, wv, wi)) {
+          wv = ov;
+          wi = oi;
+        }
+      }
+      if (lane == r) {
+        sel_v = wv;
+        sel_i = wi;
+      }
+      if ((wi & 31) == lane) {  // the owner lane removes the winner and refreshes its local best
+        taken |= 1u << (wi >> 5);
+        local_best(bv, bi);
+      }
+    }
+    // softmax over the selected logits (lane r holds slot r); the max is slot 0
+    const float vmax = __shfl_sync(0xffffffffu, sel_v, 0);
+    const float ex = (lane < k) ? expf(sel_v - vmax) : 0.f;
+    float sum = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane < k) {
+      topk_idx[(long long)t * k + lane] = sel_i;
+      topk_gate[(long long)t * k + lane] = ex / sum;
+      atomicAdd(&s_counts[sel_i], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n_experts; e += blockDim.x)
+    chunk_counts[(long long)blockIdx.x * n_experts + e] = s_counts[e];
+}
+
+// ------------------------------------------------------------------------------------------------
+// Expert totals, exclusive offsets, per-chunk bases and the grouped-GEMM unit lists.
+// Single block of 1024 threads; thread e owns expert e (N <= 1024).
+// ------------------------------------------------------------------------------------------------
+struct UnitListSpec {
+  GemmUnit* units;     // output list
+  int* num_units;      // output count
+  int feat;            // output features per expert (rows of that expert's weight)
+  int tile_tokens;     // tokens per unit (the GEMM variant's BN_MAX)
+  int max_units;       // capacity
+};
+
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp, int& total) {
+  // s_tmp: 32 ints of shared memory; blockDim.x == 1024
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_tmp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = s_tmp[lane];
+    int ws = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, ws, o);
+      if (lane >= o) ws += y;
+    }
+    s_tmp[lane] = ws - w;  // exclusive prefix of warp totals
+    if (lane == 31) s_tmp[32] = ws;
+  }
+  __syncthreads();
+  const int r = s_tmp[warp] + x - v;
+  total = s_tmp[32];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(1024)
+    scan_units_kernel(const int* __restrict__ chunk_counts, int n_chunks, int n_experts, int* __restrict__ counts,
+                      int* __restrict__ offsets, int* __restrict__ chunk_base, UnitListSpec l1, UnitListSpec l2,
+                      unsigned* status) {
+  __shared__ int s_tmp[33];
+  const int e = threadIdx.x;
+  int c_e = 0;
+  if (e < n_experts)
+    for (int c = 0; c < n_chunks; ++c) c_e += chunk_counts[(long long)c * n_experts + e];
+  int total;
+  const int off = block_exclusive_scan(c_e, s_tmp, total);
+  if (e < n_experts) {
+    counts[e] = c_e;
+    offsets[e] = off;
+    int run = off;
+    for (int c = 0; c < n_chunks; ++c) {
+      chunk_base[(long long)c * n_experts + e] = run;
+      run += chunk_counts[(long long)c * n_experts + e];
+    }
+  }
+  if (e == 0) offsets[n_experts] = total;
+  // unit lists: expert-major, token block next, feature block fastest
+#pragma unroll 1
+  for (int li = 0; li < 2; ++li) {
+    const UnitListSpec& L = li ? l2 : l1;
+    if (L.units == nullptr) continue;
+    const int nft = (L.feat + BLOCK_M - 1) / BLOCK_M;
+    const int ntt = (c_e + L.tile_tokens - 1) / L.tile_tokens;
+    const int nu = (e < n_experts) ? ntt * nft : 0;
+    int nu_total;
+    const int u0 = block_exclusive_scan(nu, s_tmp, nu_total);
+    if (e == 0) {
+      *L.num_units = min(nu_total, L.max_units);
+      if (nu_total > L.max_units) atomicOr(status, DEV_STATUS_BAD_INDEX);
+    }
+    int u = u0;
+    for (int tt = 0; tt < ntt; ++tt) {
+      const int nv = min(L.tile_tokens, c_e - tt * L.tile_tokens);
+      for (int ft = 0; ft < nft; ++ft, ++u) {
+        if (u >= L.max_units) break;
+        GemmUnit g;
+        g.a_row = e * L.feat + ft * BLOCK_M;
+        g.b_row = off + tt * L.tile_tokens;
+        g.f0 = ft * BLOCK_M;
+        g.nm = nv | (min(BLOCK_M, L.feat - ft * BLOCK_M) << 16);
+        L.units[u] = g;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Stable row assignment and the gather of latent rows into expert-grouped order.
+// One block per chunk.  Warp 0 walks the chunk's assignments in (token, slot) order, 32 at a time:
+// lanes holding the same expert are ranked with __match_any_sync, and a per-expert running base
+// (from scan_units_kernel) gives each assignment its row.  Then all warps copy h[t] to h_perm[row].
+// ------------------------------------------------------------------------------------------------
+constexpr int SCATTER_WARPS = 8;
+
+__global__ void __launch_bounds__(SCATTER_WARPS * 32)
+    scatter_gather_kernel(const int* __restrict__ topk_idx, const float* __restrict__ topk_gate,
+                          const int* __restrict__ chunk_base, int T, int n_experts, int k, int chunk_tokens,
+                          const __nv_bfloat16* __restrict__ h, int latent, int* __restrict__ row_of,
+                          int* __restrict__ tok_of_row, float* __restrict__ gate_of_row,
+                          __nv_bfloat16* __restrict__ h_perm, unsigned* status) {
+  extern __shared__ int s_base[];  // [n_experts]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < n_experts; e += blockDim.x) s_base[e] = chunk_base[(long long)blockIdx.x * n_experts + e];
+  __syncthreads();
+  const int t_begin = blockIdx.x * chunk_tokens;
+  const int t_end = min(T, t_begin + chunk_tokens);
+  const long long a_begin = (long long)t_begin * k, a_end = (long long)t_end * k;
+  const long long TK = (long long)T * k;
+  if (warp == 0) {
+    for (long long a0 = a_begin; a0 < a_end; a0 += 32) {
+      const long long a = a0 + lane;
+      const bool act = a < a_end;
+      const unsigned amask = __ballot_sync(0xffffffffu, act);
+      int e = act ? topk_idx[a] : -1 - lane;  // inactive lanes get unique keys
+      const bool e_ok = e >= 0 && e < n_experts;
+      if (act && !e_ok) atomicOr(status, DEV_STATUS_BAD_INDEX);
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int leader = __ffs(peers) - 1;
+      int base = 0;
+      if (act && e_ok) base = s_base[e];
+      __syncwarp();
+      if (act && e_ok && lane == leader) s_base[e] = base + __popc(peers);
+      __syncwarp();
+      if (act && e_ok) {
+        const int row = base + rank;
+        if (row >= 0 && row < TK) {
+          row_of[a] = row;
+          tok_of_row[row] = (int)(a / k);
+          gate_of_row[row] = topk_gate[a];
+        } else {
+          atomicOr(status, DEV_STATUS_BAD_INDEX);
+          row_of[a] = -1;
+        }
+      } else if (act) {
+        row_of[a] = -1;
+      }
+      (void)amask;
+    }
+  }
+  __syncthreads();
+  // gather: 16-byte chunks of each latent row
+  const int vec_per_row = latent / 8;
+  for (long long a = a_begin + warp; a < a_end; a += SCATTER_WARPS) {
+    const int row = row_of[a];
+    if (row < 0) continue;
+    const int t = (int)(a / k);
+    const uint4* src = reinterpret_cast<const uint4*>(h + (long long)t * latent);
+    uint4* dst = reinterpret_cast<uint4*>(h_perm + (long long)row * latent);
+    for (int i = lane; i < vec_per_row; i += 32) dst[i] = src[i];
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// combine: zu[t, 0:latent] = bf16( sum_k o[row_of[t, k], :] ), slot order, fp32 accumulation
+// ------------------------------------------------------------------------------------------------
+__global__ void combine_kernel(const __nv_bfloat16* __restrict__ o, const int* __restrict__ row_of, int T, int k,
+                               int latent, __nv_bfloat16* __restrict__ zu, long long ld_zu, long long n_rows,
+                               unsigned* status) {
+  const int vpr = latent / 8;  // 8 bf16 per thread
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long t = gid / vpr;
+  const int v = (int)(gid % vpr);
+  if (t >= T) return;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < k; ++s) {
+    const int row = row_of[t * k + s];
+    if (row < 0 || row >= n_rows) {
+      atomicOr(status, DEV_STATUS_BAD_INDEX);
+      continue;
+    }
+    const uint4 q = *reinterpret_cast<const uint4*>(o + (long long)row * latent + v * 8);
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(p[i]);
+      acc[2 * i] += f.x;
+      acc[2 * i + 1] += f.y;
+    }
+  }
+  uint4 out;
+  __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&out);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) po[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+  *reinterpret_cast<uint4*>(zu + t * ld_zu + v * 8) = out;
+}
+
+// ------------------------------------------------------------------------------------------------
+// weight preparation: copy or convert a [rows, cols] matrix (bf16 or fp32 source) into a bf16
+// destination with its own row pitch and column offset (used to stack/concatenate weights).
+// ------------------------------------------------------------------------------------------------
+__global__ void convert_2d_kernel(const void* __restrict__ src, int src_is_f32, long long rows, int cols,
+                                  long long src_ld, __nv_bfloat16* __restrict__ dst, long long dst_ld, int dst_col0) {
+  const long long total = rows * cols;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / cols;
+    const int c = (int)(i % cols);
+    __nv_bfloat16 v;
+    if (src_is_f32)
+      v = __float2bfloat16_rn(reinterpret_cast<const float*>(src)[r * src_ld + c]);
+    else
+      v = reinterpret_cast<const __nv_bfloat16*>(src)[r * src_ld + c];
+    dst[r * dst_ld + dst_col0 + c] = v;
+  }
+}
+
+}  // namespace lmoe

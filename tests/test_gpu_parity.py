@@ -1,0 +1,172 @@
+"""Parity of the CUDA layer (through the C ABI) against the fp64 oracle on seeded inputs.
+
+Routing must match bit for bit except on logit near-ties (gap < 1e-5), the dispatch maps must be
+exactly the grouping the oracle derives from the GPU's own routing, and y must be within
+2e-2 x RMS(y) of the oracle (tokens whose routing differs at a near-tie are re-evaluated by the
+oracle with the GPU's routing)."""
+import numpy as np
+import pytest
+import torch
+
+import lmoe_inputs as inp
+from oracle import lmoe_oracle as lo
+from lmoe_testlib import (bf16_to_np, check_routing, check_y, device_weights, host_weights, make_layer,
+                          oracle_weights, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(layer, x_np):
+    x = to_dev(x_np, "bf16")
+    y, idx, gate = layer.forward(x)
+    torch.cuda.synchronize()
+    st = layer.device_status()
+    assert st == 0, f"device status {st}"
+    return bf16_to_np(y), idx.cpu().numpy(), gate.cpu().numpy()
+
+
+def _compare(layer, ow, x_np, k, tokens=None):
+    """Run the layer on x, compare (optionally only `tokens`) with the oracle; returns stats."""
+    y, idx, gate = _run(layer, x_np)
+    x64 = lo.lift(x_np, "bf16")
+    sel = np.arange(x_np.shape[0]) if tokens is None else np.asarray(tokens)
+    ref = lo.forward(ow, x64[sel], k)
+    diff, near = check_routing(idx[sel], gate[sel], ref, k)
+    yref = ref["y"].copy()
+    if diff.any():
+        forced = lo.forward(ow, x64[sel][diff], k, idx=idx[sel][diff])
+        yref[diff] = forced["y"]
+    rel = check_y(y[sel], yref)
+    # router logits of the sampled tokens
+    lg = layer.inspect("logits").cpu().numpy().reshape(x_np.shape[0], -1)[sel]
+    lerr = float(np.abs(lg - (ref["logits"] - (0 if ow.b_router is None else ow.b_router))).max())
+    return {"y": y, "idx": idx, "gate": gate, "rel_err": rel, "logit_err": lerr, "near_ties": int(near.sum()),
+            "routing_diffs": int(diff.sum())}
+
+
+def _check_dispatch(layer, idx, n):
+    counts, offsets, row_of, tok_of_row = lo.dispatch(idx, n)
+    assert np.array_equal(layer.inspect("counts").cpu().numpy(), counts)
+    assert np.array_equal(layer.inspect("offsets").cpu().numpy(), offsets)
+    assert np.array_equal(layer.inspect("row_of").cpu().numpy(), row_of.reshape(-1))
+    assert np.array_equal(layer.inspect("tok_of_row").cpu().numpy(), tok_of_row)
+
+
+# ------------------------------------------------------------------------------------------------ tiny
+@pytest.fixture(scope="module")
+def tiny():
+    wl = inp.workload("tiny")
+    w = inp.make_weights(wl)
+    dev = device_weights(w)
+    layer = make_layer(wl, w, dev, wl.tokens)
+    yield wl, w, layer
+    layer.close()
+
+
+def test_tiny_full_parity(tiny):
+    wl, w, layer = tiny
+    x = inp.make_x(wl)
+    st = _compare(layer, oracle_weights(w, False), x, wl.shape.top_k)
+    assert st["logit_err"] < 1e-5, st["logit_err"]
+    _check_dispatch(layer, st["idx"], wl.shape.n_experts)
+
+
+def test_tiny_latent_h(tiny):
+    wl, w, layer = tiny
+    x = inp.make_x(wl)
+    _run(layer, x)
+    h = bf16_to_np(layer.inspect("h").view(torch.bfloat16)).reshape(wl.tokens, wl.shape.latent)
+    ow = oracle_weights(w, False)
+    href = lo.lift(x, "bf16") @ ow.w_down.T
+    assert np.abs(h - href).max() <= 2 ** -7 * np.abs(href).max()
+
+
+@pytest.mark.parametrize("t", [1, 2, 7, 33, 63])
+def test_tiny_ragged_tokens(tiny, t):
+    wl, w, layer = tiny
+    x = inp.make_x(wl, tokens=t)
+    _compare(layer, oracle_weights(w, False), x, wl.shape.top_k)
+
+
+def test_tiny_deterministic(tiny):
+    wl, w, layer = tiny
+    x = inp.make_x(wl)
+    a = _run(layer, x)
+    b = _run(layer, x)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1]) and np.array_equal(a[2], b[2])
+
+
+def test_zero_tokens_and_too_many(tiny):
+    import latentmoe_expert_layer_b200 as lm
+    wl, w, layer = tiny
+    x = torch.empty((0, wl.shape.d), dtype=torch.bfloat16, device="cuda")
+    y, idx, gate = layer.forward(x)
+    assert y.shape == (0, wl.shape.d)
+    xb = to_dev(inp.make_x(wl), "bf16")
+    big = torch.cat([xb, xb])
+    with pytest.raises(lm.LmoeError) as e:
+        layer.forward(big)
+    assert e.value.code == 2
+
+
+# ------------------------------------------------------------------------------------------------ Super
+@pytest.fixture(scope="module")
+def superlayer():
+    wl = inp.workload("decode")
+    w = host_weights("decode")
+    dev = device_weights(w)
+    layer = make_layer(wl, w, dev, inp.workload("prefill").tokens)
+    yield w, dev, layer
+    layer.close()
+    del dev
+    torch.cuda.empty_cache()
+
+
+def test_decode_full_parity(superlayer):
+    w, _, layer = superlayer
+    wl = inp.workload("decode")
+    st = _compare(layer, oracle_weights(w, False), inp.make_x(wl), wl.shape.top_k)
+    _check_dispatch(layer, st["idx"], wl.shape.n_experts)
+    print(f"decode: rel err {st['rel_err']:.3g}, logit err {st['logit_err']:.3g}, near ties {st['near_ties']}, "
+          f"routing diffs {st['routing_diffs']}")
+
+
+@pytest.mark.parametrize("t", [1, 5, 100, 257, 513])
+def test_super_ragged_tokens(superlayer, t):
+    w, _, layer = superlayer
+    wl = inp.workload("prefill")
+    x = inp.make_x(wl, tokens=t)
+    _compare(layer, oracle_weights(w, False), x, wl.shape.top_k)
+
+
+def test_prefill_sampled_parity_and_full_dispatch(superlayer):
+    w, _, layer = superlayer
+    wl = inp.workload("prefill")
+    x = inp.make_x(wl)
+    rng = np.random.default_rng(0)
+    sample = np.unique(np.concatenate([[0, 1, wl.tokens - 1], rng.choice(wl.tokens, 40, replace=False)]))
+    st = _compare(layer, oracle_weights(w, False), x, wl.shape.top_k, tokens=sample)
+    _check_dispatch(layer, st["idx"], wl.shape.n_experts)
+    print(f"prefill: rel err {st['rel_err']:.3g}, logit err {st['logit_err']:.3g}")
+
+
+@pytest.fixture(scope="module")
+def skewlayer(superlayer):
+    w, dev, _ = superlayer
+    wl = inp.workload("skewed")
+    layer = make_layer(wl, w, dev, wl.tokens)
+    yield layer
+    layer.close()
+
+
+def test_skewed_sampled_parity(skewlayer, superlayer):
+    w, _, _ = superlayer
+    layer = skewlayer
+    wl = inp.workload("skewed")
+    x = inp.make_x(wl)
+    rng = np.random.default_rng(1)
+    sample = np.unique(np.concatenate([[0, wl.tokens - 1], rng.choice(wl.tokens, 40, replace=False)]))
+    st = _compare(layer, oracle_weights(w, True), x, wl.shape.top_k, tokens=sample)
+    _check_dispatch(layer, st["idx"], wl.shape.n_experts)
+    counts = np.bincount(st["idx"].ravel(), minlength=wl.shape.n_experts)
+    assert (counts == 0).sum() >= 32 and counts.max() > 0.1 * wl.tokens
