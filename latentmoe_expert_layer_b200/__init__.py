@@ -88,7 +88,7 @@ class _DevArray:
     """__cuda_array_interface__ view of a library-owned device buffer (for lmoe_inspect)."""
 
     def __init__(self, ptr: int, count: int, typestr: str):
-        self.__cuda_array_interface__ = {"shape": (count,), "typestr": typestr, "data": (ptr, True),
+        self.__cuda_array_interface__ = {"shape": (count,), "typestr": typestr, "data": (ptr, False),
                                          "version": 3, "strides": None}
 
 
