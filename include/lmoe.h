@@ -143,6 +143,32 @@ lmoe_status lmoe_profile(lmoe_handle h, int32_t enable);
 lmoe_status lmoe_profile_read(lmoe_handle h, double* stage_ms /* [LMOE_NUM_STAGES] */, int32_t* forwards,
                               int32_t* launches_per_forward);
 
+/* Routing of T tokens from precomputed router logits WITHOUT allocating device memory.
+ *
+ * The paper has no counterpart; this entry point exists for callers that cannot allocate on their
+ * call path: cudaMalloc may synchronise the device (stalling the caller's other streams), and a
+ * process whose device memory is fully reserved by its own allocator (for example a serving engine
+ * that pre-reserves HBM for its caches) would get an out-of-memory error from it.
+ *
+ * Computes exactly what lmoe_forward's routing stage computes: top-K of (logits + bias) per token
+ * (value desc, lower index first on ties), softmax over the K selected values, and the stable
+ * expert grouping.  All pointers are device pointers owned by the caller, 16-byte aligned:
+ *   logits    [T, N] fp32, read       bias [N] fp32 or NULL, read
+ *   topk_idx  [T, K] int32, written   topk_gate [T, K] fp32, written
+ *   counts    [N] int32, written      offsets [N + 1] int32 (exclusive prefix sum), written
+ *   row_of    [T * K] int32 grouped row of assignment (t, k), written
+ * Limits: 1 <= N <= 1024, 1 <= K <= min(32, N), T * K <= 131072; beyond them the call returns
+ * LMOE_ERR_UNSUPPORTED (N, K) or LMOE_ERR_SHAPE (T), and enqueues nothing.  T = 0 returns LMOE_OK.
+ * Intermediate results live in one 2 MiB array in the library's static device memory, which every
+ * GPU that loads the library holds until the process exits.  That array is shared by every call:
+ * calls that overlap on the GPU (on different streams, or from different host threads) race on it
+ * and must be serialised by the caller.  The first call on a device looks up the array's device
+ * address (once per device, with that device current); make that first call before any stream
+ * capture.  Enqueued on `stream` (the current device's); returns LMOE_ERR_CUDA if a launch fails. */
+lmoe_status lmoe_route_noalloc(const float* logits, const float* bias, int32_t T, int32_t n_experts, int32_t top_k,
+                               int32_t* topk_idx, float* topk_gate, int32_t* counts, int32_t* offsets,
+                               int32_t* row_of, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* lmoe_status_string(lmoe_status s);
 

@@ -12,7 +12,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["LatentMoE", "LmoeError", "lib", "STATUS", "BUF", "SYMBOLS", "STAGES", "library_path"]
+__all__ = ["LatentMoE", "LmoeError", "route_noalloc", "lib", "STATUS", "BUF", "SYMBOLS", "STAGES", "library_path"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "liblmoe.so")
@@ -32,7 +32,8 @@ DTYPE = {torch.bfloat16: 0, torch.float32: 1}
 
 # every extern "C" symbol declared in include/lmoe.h
 SYMBOLS = ("lmoe_create", "lmoe_load_weights", "lmoe_forward", "lmoe_forward_host", "lmoe_get_device_status",
-           "lmoe_inspect", "lmoe_profile", "lmoe_profile_read", "lmoe_status_string", "lmoe_destroy")
+           "lmoe_inspect", "lmoe_profile", "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_status_string",
+           "lmoe_destroy")
 STAGES = ("router", "shared_up", "topk", "grouping", "scatter", "expert_up", "expert_down", "combine", "output")
 
 
@@ -56,12 +57,13 @@ lib.lmoe_get_device_status.argtypes = [_vp]
 lib.lmoe_inspect.argtypes = [_vp, _i32, ctypes.POINTER(_vp), ctypes.POINTER(_i64)]
 lib.lmoe_profile.argtypes = [_vp, _i32]
 lib.lmoe_profile_read.argtypes = [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i32), ctypes.POINTER(_i32)]
+lib.lmoe_route_noalloc.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.lmoe_status_string.argtypes = [ctypes.c_int]
 lib.lmoe_status_string.restype = ctypes.c_char_p
 lib.lmoe_destroy.argtypes = [_vp]
 lib.lmoe_destroy.restype = None
 for _f in ("lmoe_create", "lmoe_load_weights", "lmoe_forward", "lmoe_forward_host", "lmoe_get_device_status",
-           "lmoe_inspect", "lmoe_profile", "lmoe_profile_read"):
+           "lmoe_inspect", "lmoe_profile", "lmoe_profile_read", "lmoe_route_noalloc"):
     getattr(lib, _f).restype = ctypes.c_int
 
 
@@ -94,6 +96,24 @@ class _DevArray:
 
 _BUF_TYPES = {"logits": "<f4", "counts": "<i4", "offsets": "<i4", "row_of": "<i4", "tok_of_row": "<i4",
               "h": "<u2", "z": "<u2", "u": "<u2"}
+
+
+def route_noalloc(logits: torch.Tensor, top_k: int, bias: Optional[torch.Tensor] = None, stream=None):
+    """Routing from precomputed logits [T, N] through lmoe_route_noalloc, which allocates no device
+    memory (for callers that cannot allocate on their call path).  The outputs are allocated here by
+    torch, before the call.  Returns (topk_idx, topk_gate, counts, offsets, row_of)."""
+    t, n = logits.shape
+    dev = logits.device
+    idx = torch.empty((t, top_k), dtype=torch.int32, device=dev)
+    gate = torch.empty((t, top_k), dtype=torch.float32, device=dev)
+    counts = torch.empty((n,), dtype=torch.int32, device=dev)
+    offsets = torch.empty((n + 1,), dtype=torch.int32, device=dev)
+    row_of = torch.empty((t * top_k,), dtype=torch.int32, device=dev)
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    with torch.cuda.device(dev):
+        _check(lib.lmoe_route_noalloc(_ptr(logits), _ptr(bias), t, n, top_k, _ptr(idx), _ptr(gate), _ptr(counts),
+                                      _ptr(offsets), _ptr(row_of), s.cuda_stream), "lmoe_route_noalloc")
+    return idx, gate, counts, offsets, row_of
 
 
 class LatentMoE:

@@ -588,3 +588,74 @@ void lmoe_destroy(lmoe_handle c) {
 }
 
 }  // extern "C"
+// ------------------------------------------------------------------------------------------------
+// Routing without device allocation.  Its scratch (per-chunk expert histograms and bases, and the
+// grouped-row maps the scatter kernel writes) lives in this file-scope device array.  Host code must
+// not pass the array's name to a kernel (on the host it is only a stand-in symbol); the device
+// address is looked up once per device with cudaGetSymbolAddress.
+// ------------------------------------------------------------------------------------------------
+constexpr int kNoAllocMaxExperts = 1024;
+constexpr int kNoAllocMaxChunks = 128;                 // n_chunks_for() never exceeds this
+constexpr long long kNoAllocMaxAssignments = 131072;   // T * K
+constexpr size_t kNoAllocChunkWords = (size_t)kNoAllocMaxExperts * kNoAllocMaxChunks;
+constexpr size_t kNoAllocWords = 2 * kNoAllocChunkWords + 2 * (size_t)kNoAllocMaxAssignments + 64;
+
+static __device__ __align__(256) unsigned int g_noalloc_scratch[kNoAllocWords];
+
+namespace {
+std::mutex g_noalloc_mu;
+constexpr int kNoAllocMaxDevices = 64;
+unsigned int* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up on first use).
+cudaError_t noalloc_scratch(unsigned int** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = static_cast<unsigned int*>(p);
+  }
+  *out = g_noalloc_addr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+extern "C" lmoe_status lmoe_route_noalloc(const float* logits, const float* bias, int32_t T, int32_t n_experts,
+                                          int32_t top_k, int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                                          int32_t* offsets, int32_t* row_of, void* stream) {
+  const int N = n_experts, K = top_k;
+  if (N < 1 || N > kNoAllocMaxExperts || K < 1 || K > 32 || K > N) return LMOE_ERR_UNSUPPORTED;
+  if (T < 0 || (long long)T * K > kNoAllocMaxAssignments) return LMOE_ERR_SHAPE;
+  if (T == 0) return LMOE_OK;
+  if (!logits || !topk_idx || !topk_gate || !counts || !offsets || !row_of) return LMOE_ERR_INVALID_ARG;
+  if (!aligned16(logits) || (bias && !aligned16(bias)) || !aligned16(topk_idx) || !aligned16(topk_gate) ||
+      !aligned16(counts) || !aligned16(offsets) || !aligned16(row_of))
+    return LMOE_ERR_INVALID_ARG;
+  unsigned int* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != cudaSuccess) return LMOE_ERR_CUDA;
+  int* chunk_counts = reinterpret_cast<int*>(scratch);
+  int* chunk_base = chunk_counts + kNoAllocChunkWords;
+  int* tok_of_row = chunk_base + kNoAllocChunkWords;
+  float* gate_of_row = reinterpret_cast<float*>(tok_of_row + kNoAllocMaxAssignments);
+  unsigned* status = reinterpret_cast<unsigned*>(gate_of_row + kNoAllocMaxAssignments);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the status word accumulates with atomicOr, so it must start at zero; every other scratch word
+  // is fully written before it is read
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned), s) != cudaSuccess) return LMOE_ERR_CUDA;
+  int ct;
+  const int nch = n_chunks_for(T, &ct);
+  topk_hist_kernel<<<nch, TOPK_WARPS * 32, N * sizeof(int), s>>>(logits, bias, T, N, K, ct, topk_idx, topk_gate,
+                                                                 chunk_counts);
+  if (cudaGetLastError() != cudaSuccess) return LMOE_ERR_CUDA;
+  UnitListSpec none{nullptr, nullptr, 0, 64, 0};
+  scan_units_kernel<<<1, 1024, 0, s>>>(chunk_counts, nch, N, counts, offsets, chunk_base, none, none, status);
+  if (cudaGetLastError() != cudaSuccess) return LMOE_ERR_CUDA;
+  scatter_gather_kernel<<<nch, SCATTER_WARPS * 32, N * sizeof(int), s>>>(
+      topk_idx, topk_gate, chunk_base, T, N, K, ct, nullptr, 0, row_of, tok_of_row, gate_of_row, nullptr, status);
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}

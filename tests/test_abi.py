@@ -26,7 +26,8 @@ def libmod():
 def test_header_declares_the_boundary():
     assert _declared() == sorted(["lmoe_create", "lmoe_load_weights", "lmoe_forward", "lmoe_forward_host",
                                   "lmoe_get_device_status", "lmoe_inspect", "lmoe_profile",
-                                  "lmoe_profile_read", "lmoe_status_string", "lmoe_destroy"])
+                                  "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_status_string",
+                                  "lmoe_destroy"])
 
 
 def test_library_exports_every_declared_symbol(libmod):
