@@ -34,6 +34,7 @@ import lmoe_inputs as inp  # noqa: E402
 METRIC = "LatentMoE layer tokens/s (Super shape, T=256 & 16K); % of HBM / TC roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DEFAULT_STEPS = {"tiny": 200, "decode": 400, "skewed": 40, "prefill": 20}
+DEFAULT_STEPS["decode_small"] = 400
 
 
 def peaks():
@@ -338,7 +339,7 @@ def main():
     args = ap.parse_args()
     wl = inp.workload(args.workload)
     if args.steps is None:
-        args.steps = DEFAULT_STEPS.get(args.workload.split("_")[0], 20)
+        args.steps = DEFAULT_STEPS.get(args.workload, DEFAULT_STEPS.get(args.workload.split("_")[0], 20))
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

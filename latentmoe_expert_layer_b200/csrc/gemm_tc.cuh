@@ -18,7 +18,10 @@
 //
 // Work units are (weight row block, token block) pairs.  Dense GEMMs enumerate them from the
 // launch arguments; the grouped expert GEMMs read a unit list that the routing kernels built on the
-// device, so no host round trip sits between routing and the experts.
+// device, so no host round trip sits between routing and the experts.  One launch can carry two
+// problems: an optional dense "pre" problem whose units come first, then the main problem.  At
+// decode sizes every problem is a weight stream, so folding a small dense GEMM into an expert launch
+// costs only its bytes instead of a launch that cannot fill the GPU.
 #pragma once
 #include "ptx.cuh"
 
@@ -30,6 +33,7 @@ enum EpiKind : int {
   EPI_SQRELU_BF16 = 2,    // out = bf16(max(acc, 0)^2)
   EPI_ROWSCALE_BF16 = 3,  // out = bf16(acc * row_scale[token row])
   EPI_ROUTER = 4,         // features < split_feat: fp32 to out2; others: bf16 to out (column f - split)
+  EPI_ADD_BF16 = 5,       // out = bf16(acc + addend[token row, f])  (fp32 addend)
 };
 
 // One unit of GEMM work.  a_row: first W row of the tile; b_row: first activation row (also the
@@ -39,17 +43,9 @@ struct GemmUnit {
   int a_row, b_row, f0, nm;
 };
 
-struct GemmArgs {
+// One GEMM problem of a launch: K extent, epilogue, and (for dense problems) the tile grid.
+struct GemmProblem {
   int num_k_blocks;           // K / 64
-  // dense schedule (units == nullptr)
-  int dense_units;            // number of units
-  int dense_ftiles;           // feature tiles
-  int dense_feat;             // output features (rows of W)
-  int dense_tokens;           // tokens (rows of act)
-  // grouped schedule
-  const GemmUnit* units;      // device list
-  const int* num_units;       // device count
-  // epilogue
   int epi;
   void* out;
   long long ldo;              // output row pitch (elements)
@@ -58,11 +54,28 @@ struct GemmArgs {
   long long ld2;
   int split_feat;
   const float* row_scale;     // EPI_ROWSCALE_BF16
+  const float* addend;        // EPI_ADD_BF16
+  long long ld_add;
+  int weights_streamed;       // 1: every weight tile is read by one unit only (L2 evict-first)
+  int dense_ftiles;           // dense: feature tiles
+  int dense_ttiles;           // dense: token tiles (fastest-varying unit index)
+  int dense_feat;             // dense: output features (rows of W)
+  int dense_tokens;           // dense: tokens (rows of act)
+};
+
+struct GemmArgs {
+  GemmProblem prob[2];        // [0] main problem, [1] optional dense pre problem (tensor maps *_1)
+  int n_pre_units;            // units of prob[1], enumerated first
+  int main_dense_units;       // units of prob[0] when it is dense (units == nullptr)
+  const GemmUnit* units;      // prob[0] grouped: device unit list
+  const int* num_units;       // prob[0] grouped: device unit count
+  int* work_counter;          // zero before launch; units are claimed with atomicAdd
   unsigned* status;           // device status word
   unsigned long long timeout_ns;
 };
 
 constexpr int GEMM_THREADS = 192;
+constexpr int UNIT_RING = 4;
 constexpr int BLOCK_M = 128;
 constexpr int BLOCK_K = 64;                 // 64 bf16 = one 128-byte swizzle row
 constexpr int A_STAGE_BYTES = BLOCK_M * BLOCK_K * 2;
@@ -74,24 +87,37 @@ struct GemmSmem {
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
   static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
   static constexpr int BAR_OFF = EPI_OFF + 4 * EPI_STAGE_BYTES;
-  static constexpr int BYTES = BAR_OFF + 256;
+  static constexpr int BYTES = BAR_OFF + 512;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment of the base
   static constexpr uint32_t TMEM_COLS = (2 * BN_MAX < 32) ? 32 : 2 * BN_MAX;
 };
 
 template <int BN_MAX>
-__device__ __forceinline__ GemmUnit unit_at(const GemmArgs& a, int u) {
-  if (a.units != nullptr) return a.units[u];
+__device__ __forceinline__ GemmUnit dense_unit(const GemmProblem& p, int u) {
   GemmUnit r;
-  const int ft = u % a.dense_ftiles;
-  const int tt = u / a.dense_ftiles;
+  // token tiles of one weight tile run on adjacent CTAs, so the weight tile is read from HBM once
+  const int tt = u % p.dense_ttiles;
+  const int ft = u / p.dense_ttiles;
   r.a_row = ft * BLOCK_M;
   r.f0 = r.a_row;
   r.b_row = tt * BN_MAX;
-  const int mv = min(BLOCK_M, a.dense_feat - r.f0);
-  const int nv = min(BN_MAX, a.dense_tokens - r.b_row);
+  const int mv = min(BLOCK_M, p.dense_feat - r.f0);
+  const int nv = min(BN_MAX, p.dense_tokens - r.b_row);
   r.nm = nv | (mv << 16);
   return r;
+}
+
+// Global unit u of the launch: which problem it belongs to, and its tile.
+template <int BN_MAX>
+__device__ __forceinline__ GemmUnit unit_at(const GemmArgs& a, int u, int& pid) {
+  if (u < a.n_pre_units) {
+    pid = 1;
+    return dense_unit<BN_MAX>(a.prob[1], u);
+  }
+  pid = 0;
+  u -= a.n_pre_units;
+  if (a.units != nullptr) return a.units[u];
+  return dense_unit<BN_MAX>(a.prob[0], u);
 }
 
 __device__ __forceinline__ uint16_t f32_to_bf16_rn(float v) {
@@ -101,7 +127,8 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rn(float v) {
 
 template <int BN_MAX, int STAGES, int BOXN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_act,
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap map_w0, const __grid_constant__ CUtensorMap map_act0,
+                   const __grid_constant__ CUtensorMap map_w1, const __grid_constant__ CUtensorMap map_act1,
                    const GemmArgs args) {
   using S = GemmSmem<BN_MAX, STAGES>;
   static_assert(BN_MAX % BOXN == 0 && BOXN % 8 == 0, "token box must tile the token block");
@@ -113,8 +140,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* ufull = drain + 1;              // unit ring: producer -> MMA issuer and epilogue warps
+  uint64_t* uempty = ufull + UNIT_RING;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(uempty + UNIT_RING);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -129,12 +159,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(&tempty[b], 4);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < UNIT_RING; ++i) {
+      mbar_init(&ufull[i], 1);
+      mbar_init(&uempty[i], 5);  // the MMA issuer and the four epilogue warps
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&map_w);
-    tma_prefetch_desc(&map_act);
+    tma_prefetch_desc(&map_w0);
+    tma_prefetch_desc(&map_act0);
+    if (args.n_pre_units > 0) {
+      tma_prefetch_desc(&map_w1);
+      tma_prefetch_desc(&map_act1);
+    }
   }
   if (warp == 1) tmem_alloc(tmem_slot, S::TMEM_COLS);
   tc_fence_before();
@@ -142,21 +180,46 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int num_units = (args.units != nullptr) ? *args.num_units : args.dense_units;
-  const int nkb = args.num_k_blocks;
+  const int num_units = args.n_pre_units + ((args.units != nullptr) ? *args.num_units : args.main_dense_units);
+  // Every role walks the same sequence of units, published by the producer through the unit ring
+  // (a negative entry ends the sequence).
   const uint64_t tmo = args.timeout_ns;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_first = policy_evict_first();
+      const uint64_t pol_normal = policy_evict_normal();
       const uint64_t pol_a = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
-        const GemmUnit un = unit_at<BN_MAX>(args, u);
+      int uslot = 0;
+      uint32_t uphase = 0;
+      // the next unit is claimed one unit ahead, so the atomic's round trip overlaps the loads
+      int u_next = atomicAdd(args.work_counter, 1);
+      while (ok) {
+        if (!mbar_wait_bounded(&uempty[uslot], uphase ^ 1u, abort_flag, tmo)) {
+          ok = false;
+          break;
+        }
+        const int u = u_next < num_units ? u_next : -1;
+        unit_ring[uslot] = u;
+        mbar_arrive(&ufull[uslot]);
+        if (++uslot == UNIT_RING) {
+          uslot = 0;
+          uphase ^= 1u;
+        }
+        if (u < 0) break;
+        u_next = atomicAdd(args.work_counter, 1);
+        int pid;
+        const GemmUnit un = unit_at<BN_MAX>(args, u, pid);
+        const GemmProblem& pr = args.prob[pid];
+        const CUtensorMap* mw = pid ? &map_w1 : &map_w0;
+        const CUtensorMap* ma = pid ? &map_act1 : &map_act0;
+        const uint64_t pol_w = pr.weights_streamed ? pol_first : pol_normal;
+        const int nkb = pr.num_k_blocks;
         const int nv = un.nm & 0xFFFF;
         const int nbox = (nv + BOXN - 1) / BOXN;
         const uint32_t bytes = A_STAGE_BYTES + nbox * BOXN * BLOCK_K * 2;
@@ -168,10 +231,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           uint8_t* sa = smem + stage * S::STAGE_BYTES;
           uint8_t* sb = sa + A_STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d(sa, &map_w, &full[stage], kb * BLOCK_K, un.a_row, pol_w);
+          tma_load_2d(sa, mw, &full[stage], kb * BLOCK_K, un.a_row, pol_w);
           for (int i = 0; i < nbox; ++i)
-            tma_load_2d(sb + i * BOXN * BLOCK_K * 2, &map_act, &full[stage], kb * BLOCK_K, un.b_row + i * BOXN,
-                        pol_a);
+            tma_load_2d(sb + i * BOXN * BLOCK_K * 2, ma, &full[stage], kb * BLOCK_K, un.b_row + i * BOXN, pol_a);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -202,8 +264,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
-        const GemmUnit un = unit_at<BN_MAX>(args, u);
+      int uslot = 0;
+      uint32_t uphase = 0;
+      while (ok) {
+        if (!mbar_wait_bounded(&ufull[uslot], uphase, abort_flag, tmo)) {
+          ok = false;
+          break;
+        }
+        const int u = unit_ring[uslot];
+        mbar_arrive(&uempty[uslot]);
+        if (++uslot == UNIT_RING) {
+          uslot = 0;
+          uphase ^= 1u;
+        }
+        if (u < 0) break;
+        int pid;
+        const GemmUnit un = unit_at<BN_MAX>(args, u, pid);
+        const int nkb = args.prob[pid].num_k_blocks;
         const int nv = un.nm & 0xFFFF;
         const uint32_t n_mma = (uint32_t)((nv + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32(BLOCK_M, n_mma);
@@ -249,8 +326,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     uint8_t* stg = smem + S::EPI_OFF + q * EPI_STAGE_BYTES;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
-      const GemmUnit un = unit_at<BN_MAX>(args, u);
+    int uslot = 0;
+    uint32_t uphase = 0;
+    while (true) {
+      if (!mbar_wait_bounded(&ufull[uslot], uphase, abort_flag, tmo)) {
+        if (lane == 0) atomicOr(args.status, DEV_STATUS_TIMEOUT);
+        break;
+      }
+      const int u = unit_ring[uslot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&uempty[uslot]);
+      if (++uslot == UNIT_RING) {
+        uslot = 0;
+        uphase ^= 1u;
+      }
+      if (u < 0) break;
+      int pid;
+      const GemmUnit un = unit_at<BN_MAX>(args, u, pid);
+      const GemmProblem& pr = args.prob[pid];
       const int nv = un.nm & 0xFFFF;
       const int mv = un.nm >> 16;
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, tmo)) {
@@ -274,12 +367,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         const int row0 = un.b_row + c * 32;
         const int nrows = min(32, nv - c * 32);
-        bool f32_out = (args.epi == EPI_F32) || (args.epi == EPI_ROUTER && un.f0 < args.split_feat);
-        if (args.epi == EPI_ROWSCALE_BF16) {
-          const float mys = (lane < nrows) ? args.row_scale[row0 + lane] : 0.f;
+        bool f32_out = (pr.epi == EPI_F32) || (pr.epi == EPI_ROUTER && un.f0 < pr.split_feat);
+        if (pr.epi == EPI_ROWSCALE_BF16) {
+          const float mys = (lane < nrows) ? pr.row_scale[row0 + lane] : 0.f;
 #pragma unroll
           for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * __shfl_sync(0xffffffffu, mys, j));
-        } else if (args.epi == EPI_SQRELU_BF16) {
+        } else if (pr.epi == EPI_ADD_BF16) {
+          if (feat_ok && q * 32 + lane < mv) {
+            const float* ad = pr.addend + (long long)row0 * pr.ld_add + f + lane;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nrows) r[j] = __float_as_uint(__uint_as_float(r[j]) + ad[(long long)j * pr.ld_add]);
+          }
+        } else if (pr.epi == EPI_SQRELU_BF16) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float v = fmaxf(__uint_as_float(r[j]), 0.f);
@@ -292,9 +392,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) s32[j * 32 + lane] = __uint_as_float(r[j]);
           __syncwarp();
-          float* dst = (args.epi == EPI_ROUTER) ? args.out2 : reinterpret_cast<float*>(args.out);
-          const long long ld = (args.epi == EPI_ROUTER) ? args.ld2 : args.ldo;
-          const int col = (args.epi == EPI_ROUTER) ? f : (args.out_col0 + f);
+          float* dst = (pr.epi == EPI_ROUTER) ? pr.out2 : reinterpret_cast<float*>(pr.out);
+          const long long ld = (pr.epi == EPI_ROUTER) ? pr.ld2 : pr.ldo;
+          const int col = (pr.epi == EPI_ROUTER) ? f : (pr.out_col0 + f);
           if (feat_ok) {
 #pragma unroll
             for (int it = 0; it < 8; ++it) {
@@ -310,15 +410,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) s16[j * 32 + lane] = f32_to_bf16_rn(__uint_as_float(r[j]));
           __syncwarp();
-          uint16_t* dst = reinterpret_cast<uint16_t*>(args.out);
-          const int col = (args.epi == EPI_ROUTER) ? (f - args.split_feat) : (args.out_col0 + f);
+          uint16_t* dst = reinterpret_cast<uint16_t*>(pr.out);
+          const int col = (pr.epi == EPI_ROUTER) ? (f - pr.split_feat) : (pr.out_col0 + f);
           if (feat_ok) {
 #pragma unroll
             for (int it = 0; it < 4; ++it) {
               const int j = it * 8 + (lane >> 2);
               if (j < nrows) {
                 const uint4 v = *reinterpret_cast<const uint4*>(s16 + j * 32 + (lane & 3) * 8);
-                *reinterpret_cast<uint4*>(dst + (long long)(row0 + j) * args.ldo + col + (lane & 3) * 8) = v;
+                *reinterpret_cast<uint4*>(dst + (long long)(row0 + j) * pr.ldo + col + (lane & 3) * 8) = v;
               }
             }
           }

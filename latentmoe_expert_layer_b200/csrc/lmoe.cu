@@ -86,6 +86,7 @@ struct lmoe_ctx {
   __nv_bfloat16* w1 = nullptr;     // [N * m, l]
   __nv_bfloat16* w2 = nullptr;     // [N * l, m]
   CUtensorMap map_rd{}, map_r{}, map_down{}, map_cat{}, map_ws1{}, map_w1{}, map_w2{};
+  CUtensorMap map_wup{}, map_ws2{};  // the W_up and W_s2 column blocks of w_cat
 
   // workspace
   float* logits = nullptr;
@@ -107,8 +108,12 @@ struct lmoe_ctx {
   GemmUnit* units2 = nullptr;
   int* num_units = nullptr;  // [2]
   unsigned* status = nullptr;
+  int* work_counters = nullptr;  // [kCounters] per-launch unit counters, zeroed at the start of a forward
+  static constexpr int kCounters = 8;
   int max_units1 = 0, max_units2 = 0;
   CUtensorMap map_hperm[2]{}, map_u[2]{}, map_zu[2]{};
+  CUtensorMap map_z[2]{}, map_us[2]{};  // the z and u_s column blocks of zu
+  float* y_s = nullptr;                 // [min(T_max, 512), d] fp32: W_s2 u_s at decode sizes
 
   // x tensor maps, cached by (pointer, T)
   const void* x_cached = nullptr;
@@ -156,73 +161,111 @@ void free_all(lmoe_ctx* c) {
                   c->w2,     c->logits, c->idx,    c->gate,      c->chunk_counts, c->chunk_base, c->counts,
                   c->offsets, c->row_of, c->tok_of_row, c->gate_of_row, c->h, c->h_perm, c->u,
                   c->o,      c->zu,     c->units1, c->units2,    c->num_units,  c->status,     c->x_dev,
-                  c->y_dev,  c->idx_dev, c->gate_dev};
+                  c->y_dev,  c->idx_dev, c->gate_dev, c->y_s, c->work_counters};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
 
-int n_chunks_for(int T, int* chunk_tokens) {
-  int ct = (T + 127) / 128;
-  if (ct < 4) ct = 4;
+// Tokens are routed in chunks (one top-K block per chunk); the [N][chunks] histogram must fit the
+// scan kernel's shared memory, so N * chunks <= 32768, and there are at most 128 chunks.
+int n_chunks_for(int T, int N, int* chunk_tokens) {
+  int cap = 32768 / N;
+  if (cap > 128) cap = 128;
+  if (cap < 1) cap = 1;
+  int c = (T + 7) / 8;
+  if (c > cap) c = cap;
+  if (c < 1) c = 1;
+  const int ct = (T + c - 1) / c;
   *chunk_tokens = ct;
   return (T + ct - 1) / ct;
 }
 
+int topk_threads(int chunk_tokens) { return 32 * (chunk_tokens < 32 ? chunk_tokens : 32); }
+
+constexpr int kScanSmemMax = 200 * 1024;
+
 lmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA; }
 
 template <int V>
-cudaError_t launch_gemm_v(const CUtensorMap& mw, const CUtensorMap& ma, const GemmArgs& a, int grid,
-                          cudaStream_t s) {
-  gemm_tc_kernel<VT<V>::BN, VT<V>::ST, VT<V>::BOX><<<grid, GEMM_THREADS, VT<V>::smem(), s>>>(mw, ma, a);
+cudaError_t launch_gemm_v(const CUtensorMap& w0, const CUtensorMap& a0, const CUtensorMap& w1, const CUtensorMap& a1,
+                          const GemmArgs& a, int grid, cudaStream_t s) {
+  gemm_tc_kernel<VT<V>::BN, VT<V>::ST, VT<V>::BOX><<<grid, GEMM_THREADS, VT<V>::smem(), s>>>(w0, a0, w1, a1, a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(int v, const CUtensorMap& mw, const CUtensorMap& ma, const GemmArgs& a, int grid,
-                        cudaStream_t s) {
-  return v == V_SMALL ? launch_gemm_v<V_SMALL>(mw, ma, a, grid, s) : launch_gemm_v<V_LARGE>(mw, ma, a, grid, s);
+// A problem with its epilogue; K in elements (multiple of 64).
+GemmProblem problem(int K, int epi, void* out, long long ldo, int col0 = 0) {
+  GemmProblem p;
+  memset(&p, 0, sizeof(p));
+  p.num_k_blocks = K / BLOCK_K;
+  p.epi = epi;
+  p.out = out;
+  p.ldo = ldo;
+  p.out_col0 = col0;
+  return p;
 }
 
-GemmArgs base_args(lmoe_ctx* c, int K) {
+// Make `p` a dense problem over feat x tokens with the token tile of variant v.
+int set_dense(GemmProblem& p, int v, int feat, int tokens) {
+  p.dense_ftiles = (feat + BLOCK_M - 1) / BLOCK_M;
+  p.dense_ttiles = (tokens + V_BN[v] - 1) / V_BN[v];
+  p.dense_feat = feat;
+  p.dense_tokens = tokens;
+  p.weights_streamed = p.dense_ttiles == 1;
+  return p.dense_ftiles * p.dense_ttiles;
+}
+
+struct GemmLaunch {
+  lmoe_ctx* c;
+  int v;
   GemmArgs a;
-  memset(&a, 0, sizeof(a));
-  a.num_k_blocks = K / BLOCK_K;
-  a.status = c->status;
-  a.timeout_ns = c->timeout_ns;
-  return a;
-}
+  const CUtensorMap *w0 = nullptr, *a0 = nullptr, *w1 = nullptr, *a1 = nullptr;
 
-// Dense GEMM: out[tok, f] = epi(sum_k W[f, k] act[tok, k]) over feat x tokens.
-cudaError_t dense_gemm(lmoe_ctx* c, int v, const CUtensorMap& mw, const CUtensorMap& ma, int feat, int tokens,
-                       int K, int epi, void* out, long long ldo, int col0, float* out2, long long ld2, int split,
-                       cudaStream_t s) {
-  GemmArgs a = base_args(c, K);
-  a.dense_ftiles = (feat + BLOCK_M - 1) / BLOCK_M;
-  a.dense_units = a.dense_ftiles * ((tokens + V_BN[v] - 1) / V_BN[v]);
-  a.dense_feat = feat;
-  a.dense_tokens = tokens;
-  a.epi = epi;
-  a.out = out;
-  a.ldo = ldo;
-  a.out_col0 = col0;
-  a.out2 = out2;
-  a.ld2 = ld2;
-  a.split_feat = split;
-  const int grid = a.dense_units < c->num_sms ? a.dense_units : c->num_sms;
-  return launch_gemm(v, mw, ma, a, grid, s);
-}
-
-cudaError_t grouped_gemm(lmoe_ctx* c, int v, const CUtensorMap& mw, const CUtensorMap& ma, const GemmUnit* units,
-                         const int* num_units, int K, int epi, void* out, long long ldo, const float* row_scale,
-                         cudaStream_t s) {
-  GemmArgs a = base_args(c, K);
-  a.units = units;
-  a.num_units = num_units;
-  a.epi = epi;
-  a.out = out;
-  a.ldo = ldo;
-  a.row_scale = row_scale;
-  return launch_gemm(v, mw, ma, a, c->num_sms, s);
-}
+  GemmLaunch(lmoe_ctx* ctx, int variant, int counter) : c(ctx), v(variant) {
+    memset(&a, 0, sizeof(a));
+    a.status = ctx->status;
+    a.timeout_ns = ctx->timeout_ns;
+    a.work_counter = ctx->work_counters + counter;
+  }
+  // main problem, dense
+  void main_dense(const CUtensorMap& mw, const CUtensorMap& ma, GemmProblem p, int feat, int tokens) {
+    a.main_dense_units = set_dense(p, v, feat, tokens);
+    a.prob[0] = p;
+    w0 = &mw;
+    a0 = &ma;
+  }
+  // main problem, grouped experts (unit list on the device)
+  void main_grouped(const CUtensorMap& mw, const CUtensorMap& ma, GemmProblem p, const GemmUnit* units,
+                    const int* num_units) {
+    p.weights_streamed = v == V_SMALL;  // decode-sized groups: mostly one token tile per expert
+    a.prob[0] = p;
+    a.units = units;
+    a.num_units = num_units;
+    w0 = &mw;
+    a0 = &ma;
+  }
+  // dense pre problem, processed before the main problem's units
+  void pre_dense(const CUtensorMap& mw, const CUtensorMap& ma, GemmProblem p, int feat, int tokens) {
+    a.n_pre_units = set_dense(p, v, feat, tokens);
+    a.prob[1] = p;
+    w1 = &mw;
+    a1 = &ma;
+  }
+  cudaError_t run(cudaStream_t s) {
+    if (!w1) {
+      w1 = w0;
+      a1 = a0;
+    }
+    int grid = c->num_sms;
+    if (a.units == nullptr) {
+      const int total = a.n_pre_units + a.main_dense_units;
+      if (total < grid) grid = total;
+    }
+    if (grid < 1) grid = 1;
+    return v == V_SMALL ? launch_gemm_v<V_SMALL>(*w0, *a0, *w1, *a1, a, grid, s)
+                        : launch_gemm_v<V_LARGE>(*w0, *a0, *w1, *a1, a, grid, s);
+  }
+};
 
 }  // namespace
 
@@ -281,7 +324,8 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   ok = ok && dalloc(&c->h, T * l) && dalloc(&c->h_perm, tk * l) && dalloc(&c->u, tk * m) && dalloc(&c->o, tk * l);
   ok = ok && dalloc(&c->zu, T * (l + ms));
   ok = ok && dalloc(&c->units1, c->max_units1) && dalloc(&c->units2, c->max_units2) && dalloc(&c->num_units, 2);
-  ok = ok && dalloc(&c->status, 1);
+  ok = ok && dalloc(&c->status, 1) && dalloc(&c->work_counters, lmoe_ctx::kCounters);
+  ok = ok && dalloc(&c->y_s, (size_t)(T < 512 ? T : 512) * d);
   if (!ok) {
     free_all(c);
     delete c;
@@ -296,11 +340,15 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
     ok = ok && make_map(&c->map_hperm[v], c->h_perm, tk, l, l, V_BOXN[v]);
     ok = ok && make_map(&c->map_u[v], c->u, tk, m, m, V_BOXN[v]);
     ok = ok && make_map(&c->map_zu[v], c->zu, T, l + ms, l + ms, V_BOXN[v]);
+    ok = ok && make_map(&c->map_z[v], c->zu, T, l, l + ms, V_BOXN[v]);
+    ok = ok && make_map(&c->map_us[v], c->zu + l, T, ms, l + ms, V_BOXN[v]);
   }
   ok = ok && cudaFuncSetAttribute(VT<V_SMALL>::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   VT<V_SMALL>::smem()) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(VT<V_LARGE>::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   VT<V_LARGE>::smem()) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(reinterpret_cast<const void*>(scan_units_kernel),
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kScanSmemMax) == cudaSuccess;
   if (!ok || cudaDeviceSynchronize() != cudaSuccess) {
     free_all(c);
     delete c;
@@ -373,6 +421,8 @@ lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream
   if (!c->router_f32 && !c->fused_router) ok = ok && make_map(&c->map_r, c->w_rd, N, d, d, BLOCK_M);
   if (!c->fused_router) ok = ok && make_map(&c->map_down, c->w_down, l, d, d, BLOCK_M);
   ok = ok && make_map(&c->map_cat, c->w_cat, d, l + ms, l + ms, BLOCK_M);
+  ok = ok && make_map(&c->map_wup, c->w_cat, d, l, l + ms, BLOCK_M);
+  ok = ok && make_map(&c->map_ws2, c->w_cat + l, d, ms, l + ms, BLOCK_M);
   ok = ok && make_map(&c->map_ws1, c->ws1, ms, d, d, BLOCK_M);
   ok = ok && make_map(&c->map_w1, c->w1, (uint64_t)N * m, l, l, BLOCK_M);
   ok = ok && make_map(&c->map_w2, c->w2, (uint64_t)N * l, m, m, BLOCK_M);
@@ -418,54 +468,89 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
     if (prof) chk(cudaEventRecord(ev[i], s));
   };
   int launches = 0;
+  chk(cudaMemsetAsync(c->work_counters, 0, lmoe_ctx::kCounters * sizeof(int), s));
   mark(0);
+
+  // At decode sizes (T <= 512 with decode-sized expert groups) the shared expert's two matrices ride
+  // inside the expert launches as dense pre problems, and the output GEMM only does W_up z + y_s.
+  const bool split = vd == V_SMALL && vg == V_SMALL && c->y_s != nullptr;
 
   // 1. router logits and the latent h = W_down x
   if (c->fused_router) {
-    chk(dense_gemm(c, vd, c->map_rd, c->map_x[vd], N + l, T, d, EPI_ROUTER, c->h, l, 0, c->logits, N, N, s));
+    GemmLaunch g(c, vd, 0);
+    GemmProblem p = problem(d, EPI_ROUTER, c->h, l);
+    p.out2 = c->logits;
+    p.ld2 = N;
+    p.split_feat = N;
+    g.main_dense(c->map_rd, c->map_x[vd], p, N + l, T);
+    chk(g.run(s));
     launches += 1;
   } else {
-    launches += 2;
     if (c->router_f32) {
       router_f32_kernel<<<T, 256, d * sizeof(float), s>>>(reinterpret_cast<const __nv_bfloat16*>(x), c->w_r32, d,
                                                           N, c->logits);
       chk(cudaGetLastError());
     } else {
-      chk(dense_gemm(c, vd, c->map_r, c->map_x[vd], N, T, d, EPI_F32, c->logits, N, 0, nullptr, 0, 0, s));
+      GemmLaunch g(c, vd, 1);
+      g.main_dense(c->map_r, c->map_x[vd], problem(d, EPI_F32, c->logits, N), N, T);
+      chk(g.run(s));
     }
-    chk(dense_gemm(c, vd, c->map_down, c->map_x[vd], l, T, d, EPI_BF16, c->h, l, 0, nullptr, 0, 0, s));
+    GemmLaunch g(c, vd, 2);
+    g.main_dense(c->map_down, c->map_x[vd], problem(d, EPI_BF16, c->h, l), l, T);
+    chk(g.run(s));
+    launches += 2;
   }
   mark(1);
-  // 2. shared expert, first matrix: zu[:, l:] = sqrelu(W_s1 x)
-  chk(dense_gemm(c, vd, c->map_ws1, c->map_x[vd], ms, T, d, EPI_SQRELU_BF16, c->zu, l + ms, l, nullptr, 0, 0, s));
+  // 2. shared expert, first matrix: zu[:, l:] = sqrelu(W_s1 x)   (inside the expert-up launch when split)
+  const GemmProblem shared_up = problem(d, EPI_SQRELU_BF16, c->zu, l + ms, l);
+  if (!split) {
+    GemmLaunch g(c, vd, 3);
+    g.main_dense(c->map_ws1, c->map_x[vd], shared_up, ms, T);
+    chk(g.run(s));
+    launches += 1;
+  }
   mark(2);
   // 3. top-K + softmax + per-chunk histogram
   int ct;
-  const int nch = n_chunks_for(T, &ct);
-  topk_hist_kernel<<<nch, TOPK_WARPS * 32, N * sizeof(int), s>>>(c->logits, c->b_router, T, N, K, ct, idx, gate,
-                                                                 c->chunk_counts);
-  chk(cudaGetLastError());
+  const int nch = n_chunks_for(T, N, &ct);
+  chk(launch_topk_hist(nch, topk_threads(ct), s, c->logits, c->b_router, T, N, K, ct, idx, gate, c->chunk_counts));
   mark(3);
   // 4. expert offsets and grouped-GEMM unit lists
   UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1};
   UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2};
-  scan_units_kernel<<<1, 1024, 0, s>>>(c->chunk_counts, nch, N, c->counts, c->offsets, c->chunk_base, l1, l2,
-                                       c->status);
+  scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(c->chunk_counts, nch, N, c->counts, c->offsets,
+                                                              c->chunk_base, l1, l2, c->status);
   chk(cudaGetLastError());
   mark(4);
-  // 5. stable grouping and gather of latent rows
-  scatter_gather_kernel<<<nch, SCATTER_WARPS * 32, N * sizeof(int), s>>>(
-      idx, gate, c->chunk_base, T, N, K, ct, c->h, l, c->row_of, c->tok_of_row, c->gate_of_row, c->h_perm,
-      c->status);
+  // 5. stable grouping, then the gather of latent rows into grouped order
+  assign_rows_kernel<<<nch, 32, N * sizeof(int), s>>>(idx, gate, c->chunk_base, T, N, K, ct, c->row_of,
+                                                     c->tok_of_row, c->gate_of_row, c->status);
   chk(cudaGetLastError());
+  {
+    long long warps = (TK + GATHER_ROWS - 1) / GATHER_ROWS;
+    long long blocks = (warps + 7) / 8;
+    if (blocks > (long long)c->num_sms * 8) blocks = (long long)c->num_sms * 8;
+    gather_rows_kernel<<<(int)blocks, 256, 0, s>>>(c->h, c->tok_of_row, TK, T, l, c->h_perm, c->status);
+    chk(cudaGetLastError());
+  }
   mark(5);
   // 6. expert up: u = sqrelu(W1_e h)
-  chk(grouped_gemm(c, vg, c->map_w1, c->map_hperm[vg], c->units1, c->num_units, l, EPI_SQRELU_BF16, c->u, m,
-                   nullptr, s));
+  {
+    GemmLaunch g(c, vg, 4);
+    if (split) g.pre_dense(c->map_ws1, c->map_x[vd], shared_up, ms, T);
+    g.main_grouped(c->map_w1, c->map_hperm[vg], problem(l, EPI_SQRELU_BF16, c->u, m), c->units1, c->num_units);
+    chk(g.run(s));
+  }
   mark(6);
-  // 7. expert down with the gate folded in: o = g * (W2_e u)
-  chk(grouped_gemm(c, vg, c->map_w2, c->map_u[vg], c->units2, c->num_units + 1, m, EPI_ROWSCALE_BF16, c->o, l,
-                   c->gate_of_row, s));
+  // 7. expert down with the gate folded in: o = g * (W2_e u); when split, also y_s = W_s2 u_s (fp32)
+  {
+    GemmLaunch g(c, vg, 5);
+    if (split) g.pre_dense(c->map_ws2, c->map_us[vd], problem(ms, EPI_F32, c->y_s, d), d, T);
+    GemmProblem p = problem(m, EPI_ROWSCALE_BF16, c->o, l);
+    p.row_scale = c->gate_of_row;
+    g.main_grouped(c->map_w2, c->map_u[vg], p, c->units2, c->num_units + 1);
+    chk(g.run(s));
+  }
   mark(7);
   // 8. latent combine: zu[:, :l] = sum_k o[row_of[t, k]]
   {
@@ -475,8 +560,19 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
     chk(cudaGetLastError());
   }
   mark(8);
-  // 9. y = [z | sqrelu(W_s1 x)] [W_up | W_s2]^T
-  chk(dense_gemm(c, vd, c->map_cat, c->map_zu[vd], d, T, l + ms, EPI_BF16, y, d, 0, nullptr, 0, 0, s));
+  // 9. y = [z | sqrelu(W_s1 x)] [W_up | W_s2]^T, or y = W_up z + y_s when split
+  {
+    GemmLaunch g(c, vd, 6);
+    if (split) {
+      GemmProblem p = problem(l, EPI_ADD_BF16, y, d);
+      p.addend = c->y_s;
+      p.ld_add = d;
+      g.main_dense(c->map_wup, c->map_z[vd], p, d, T);
+    } else {
+      g.main_dense(c->map_cat, c->map_zu[vd], problem(l + ms, EPI_BF16, y, d), d, T);
+    }
+    chk(g.run(s));
+  }
   mark(9);
   launches += 8;
   c->launches = launches;
@@ -618,6 +714,9 @@ cudaError_t noalloc_scratch(unsigned int** out) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(reinterpret_cast<const void*>(scan_units_kernel),
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kScanSmemMax);
+    if (e != cudaSuccess) return e;
     g_noalloc_addr[dev] = static_cast<unsigned int*>(p);
   }
   *out = g_noalloc_addr[dev];
@@ -648,14 +747,15 @@ extern "C" lmoe_status lmoe_route_noalloc(const float* logits, const float* bias
   // is fully written before it is read
   if (cudaMemsetAsync(status, 0, sizeof(unsigned), s) != cudaSuccess) return LMOE_ERR_CUDA;
   int ct;
-  const int nch = n_chunks_for(T, &ct);
-  topk_hist_kernel<<<nch, TOPK_WARPS * 32, N * sizeof(int), s>>>(logits, bias, T, N, K, ct, topk_idx, topk_gate,
-                                                                 chunk_counts);
-  if (cudaGetLastError() != cudaSuccess) return LMOE_ERR_CUDA;
+  const int nch = n_chunks_for(T, N, &ct);
+  if (launch_topk_hist(nch, topk_threads(ct), s, logits, bias, T, N, K, ct, topk_idx, topk_gate, chunk_counts) !=
+      cudaSuccess)
+    return LMOE_ERR_CUDA;
   UnitListSpec none{nullptr, nullptr, 0, 64, 0};
-  scan_units_kernel<<<1, 1024, 0, s>>>(chunk_counts, nch, N, counts, offsets, chunk_base, none, none, status);
+  scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(chunk_counts, nch, N, counts, offsets, chunk_base,
+                                                              none, none, status);
   if (cudaGetLastError() != cudaSuccess) return LMOE_ERR_CUDA;
-  scatter_gather_kernel<<<nch, SCATTER_WARPS * 32, N * sizeof(int), s>>>(
-      topk_idx, topk_gate, chunk_base, T, N, K, ct, nullptr, 0, row_of, tok_of_row, gate_of_row, nullptr, status);
+  assign_rows_kernel<<<nch, 32, N * sizeof(int), s>>>(topk_idx, topk_gate, chunk_base, T, N, K, ct, row_of,
+                                                     tok_of_row, gate_of_row, status);
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }

@@ -40,59 +40,65 @@ __global__ void router_f32_kernel(const __nv_bfloat16* __restrict__ x, const flo
 }
 
 // ------------------------------------------------------------------------------------------------
-// top-K + softmax + per-chunk expert histogram.  One block per chunk of `chunk_tokens` tokens, one
-// warp per token.  Each lane keeps its best remaining candidate (value desc, index asc); K rounds
-// of a warp arg-max pick the experts in output order.  Requires K <= 32 and N <= 32 * 32.
+// top-K + softmax + per-chunk expert histogram.  One block per chunk of `chunk_tokens` consecutive
+// tokens, one warp per token.  Lane j holds the candidates j, j + 32, ... (P of them); it sorts them
+// once (bitonic network in registers, order: value desc, index asc).  Then K rounds of a warp
+// arg-max over the lanes' current heads pick the experts in output order; only the lane that owned
+// the winner shifts its sorted list by one.  Requires K <= 32 and N <= 32 * P.
 // ------------------------------------------------------------------------------------------------
-constexpr int TOPK_WARPS = 8;
-constexpr int MAX_PER_LANE = 32;  // N <= 1024
-
 __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
 }
 
-__global__ void __launch_bounds__(TOPK_WARPS * 32)
+template <int P>
+__global__ void __launch_bounds__(1024)
     topk_hist_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int n_experts,
                      int k, int chunk_tokens, int* __restrict__ topk_idx, float* __restrict__ topk_gate,
                      int* __restrict__ chunk_counts) {
   extern __shared__ int s_counts[];  // [n_experts]
   for (int e = threadIdx.x; e < n_experts; e += blockDim.x) s_counts[e] = 0;
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   const int t_begin = blockIdx.x * chunk_tokens;
   const int t_end = min(T, t_begin + chunk_tokens);
-  const int per_lane = (n_experts + 31) >> 5;
-  for (int t = t_begin + warp; t < t_end; t += TOPK_WARPS) {
+  for (int t = t_begin + warp; t < t_end; t += nwarps) {
     const float* lrow = logits + (long long)t * n_experts;
-    float v[MAX_PER_LANE];
-    uint32_t taken = 0;
+    float v[P];
+    int ix[P];
 #pragma unroll
-    for (int i = 0; i < MAX_PER_LANE; ++i) {
+    for (int i = 0; i < P; ++i) {
       const int e = i * 32 + lane;
-      v[i] = -INFINITY;
-      if (i < per_lane && e < n_experts) v[i] = lrow[e] + (bias ? bias[e] : 0.f);
+      const bool ok = e < n_experts;
+      v[i] = ok ? lrow[e] + (bias ? bias[e] : 0.f) : -INFINITY;
+      ix[i] = ok ? e : 0x7fffffff;
     }
-    // local best of this lane
-    auto local_best = [&](float& bv, int& bi) {
-      bv = -INFINITY;
-      bi = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < MAX_PER_LANE; ++i) {
-        const int e = i * 32 + lane;
-        if (i < per_lane && e < n_experts && !((taken >> i) & 1u) && better(v[i], e, bv, bi)) {
-          bv = v[i];
-          bi = e;
+    for (int size = 2; size <= P; size <<= 1) {
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+          const int j = i ^ stride;
+          if (j > i) {
+            const bool desc = (i & size) == 0;
+            const bool sw = desc ? better(v[j], ix[j], v[i], ix[i]) : better(v[i], ix[i], v[j], ix[j]);
+            if (sw) {
+              const float tv = v[i];
+              v[i] = v[j];
+              v[j] = tv;
+              const int ti = ix[i];
+              ix[i] = ix[j];
+              ix[j] = ti;
+            }
+          }
         }
       }
-    };
-    float bv;
-    int bi;
-    local_best(bv, bi);
+    }
     float sel_v = 0.f;
     int sel_i = 0;
     for (int r = 0; r < k; ++r) {
-      float wv = bv;
-      int wi = bi;
+      float wv = v[0];
+      int wi = ix[0];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         const float ov = __shfl_xor_sync(0xffffffffu, wv, o);
@@ -106,9 +112,14 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32)
         sel_v = wv;
         sel_i = wi;
       }
-      if ((wi & 31) == lane) {  // the owner lane removes the winner and refreshes its local best
-        taken |= 1u << (wi >> 5);
-        local_best(bv, bi);
+      if (ix[0] == wi) {  // expert ids are unique: this lane owned the winner
+#pragma unroll
+        for (int i = 0; i + 1 < P; ++i) {
+          v[i] = v[i + 1];
+          ix[i] = ix[i + 1];
+        }
+        v[P - 1] = -INFINITY;
+        ix[P - 1] = 0x7fffffff;
       }
     }
     // softmax over the selected logits (lane r holds slot r); the max is slot 0
@@ -124,8 +135,30 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32)
     }
   }
   __syncthreads();
+  // expert-major layout [N][n_chunks]: the scan reads one expert's chunks contiguously
   for (int e = threadIdx.x; e < n_experts; e += blockDim.x)
-    chunk_counts[(long long)blockIdx.x * n_experts + e] = s_counts[e];
+    chunk_counts[(long long)e * gridDim.x + blockIdx.x] = s_counts[e];
+}
+
+// candidates per lane: the next power of two >= ceil(N / 32)
+inline int topk_lane_candidates(int n_experts) {
+  int p = 1;
+  while (32 * p < n_experts) p <<= 1;
+  return p;
+}
+
+inline cudaError_t launch_topk_hist(int n_chunks, int threads, cudaStream_t s, const float* logits, const float* bias,
+                                    int T, int N, int K, int ct, int* idx, float* gate, int* chunk_counts) {
+  const size_t sm = (size_t)N * sizeof(int);
+  switch (topk_lane_candidates(N)) {
+    case 1: topk_hist_kernel<1><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
+    case 2: topk_hist_kernel<2><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
+    case 4: topk_hist_kernel<4><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
+    case 8: topk_hist_kernel<8><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
+    case 16: topk_hist_kernel<16><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
+    default: topk_hist_kernel<32><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
+  }
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -169,28 +202,56 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp, int& tota
   return r;
 }
 
+// Dynamic shared memory of scan_units_kernel: the [N][n_chunks] histogram with rows padded by one
+// word (conflict-free per-expert walks).
+inline size_t scan_smem_bytes(int n_experts, int n_chunks) { return (size_t)n_experts * (n_chunks + 1) * sizeof(int); }
+
 __global__ void __launch_bounds__(1024)
     scan_units_kernel(const int* __restrict__ chunk_counts, int n_chunks, int n_experts, int* __restrict__ counts,
                       int* __restrict__ offsets, int* __restrict__ chunk_base, UnitListSpec l1, UnitListSpec l2,
                       unsigned* status) {
+  // chunk_counts / chunk_base are expert-major: [N][n_chunks]
+  extern __shared__ int s_cc[];  // [N][n_chunks + 1]
   __shared__ int s_tmp[33];
+  const int pitch = n_chunks + 1;
+  const int total_words = n_experts * n_chunks;
+  for (int i = threadIdx.x; i < total_words; i += blockDim.x) {
+    const int e = i / n_chunks, c = i - e * n_chunks;
+    s_cc[e * pitch + c] = chunk_counts[i];
+  }
+  __syncthreads();
   const int e = threadIdx.x;
   int c_e = 0;
   if (e < n_experts)
-    for (int c = 0; c < n_chunks; ++c) c_e += chunk_counts[(long long)c * n_experts + e];
+    for (int c = 0; c < n_chunks; ++c) c_e += s_cc[e * pitch + c];
   int total;
   const int off = block_exclusive_scan(c_e, s_tmp, total);
   if (e < n_experts) {
     counts[e] = c_e;
     offsets[e] = off;
-    int run = off;
+    int run = off;  // chunk bases, in place
     for (int c = 0; c < n_chunks; ++c) {
-      chunk_base[(long long)c * n_experts + e] = run;
-      run += chunk_counts[(long long)c * n_experts + e];
+      const int v = s_cc[e * pitch + c];
+      s_cc[e * pitch + c] = run;
+      run += v;
     }
   }
   if (e == 0) offsets[n_experts] = total;
-  // unit lists: expert-major, token block next, feature block fastest
+  __syncthreads();
+  for (int i = threadIdx.x; i < total_words; i += blockDim.x) {
+    const int ex = i / n_chunks, c = i - ex * n_chunks;
+    chunk_base[i] = s_cc[ex * pitch + c];
+  }
+  // unit lists: expert-major, token block next, feature block fastest.  Consecutive threads write
+  // consecutive units (16-byte stores); a unit finds its expert by binary search over the experts'
+  // first-unit indices.
+  __shared__ int s_u0[1025];
+  __shared__ int s_cnt[1024];
+  __shared__ int s_offs[1024];
+  if (e < n_experts) {
+    s_cnt[e] = c_e;
+    s_offs[e] = off;
+  }
 #pragma unroll 1
   for (int li = 0; li < 2; ++li) {
     const UnitListSpec& L = li ? l2 : l1;
@@ -199,91 +260,115 @@ __global__ void __launch_bounds__(1024)
     const int ntt = (c_e + L.tile_tokens - 1) / L.tile_tokens;
     const int nu = (e < n_experts) ? ntt * nft : 0;
     int nu_total;
-    const int u0 = block_exclusive_scan(nu, s_tmp, nu_total);
+    const int u0 = block_exclusive_scan(nu, s_tmp, nu_total);  // ends with __syncthreads
+    if (e < n_experts) s_u0[e] = u0;
     if (e == 0) {
+      s_u0[n_experts] = nu_total;
       *L.num_units = min(nu_total, L.max_units);
       if (nu_total > L.max_units) atomicOr(status, DEV_STATUS_BAD_INDEX);
     }
-    int u = u0;
-    for (int tt = 0; tt < ntt; ++tt) {
-      const int nv = min(L.tile_tokens, c_e - tt * L.tile_tokens);
-      for (int ft = 0; ft < nft; ++ft, ++u) {
-        if (u >= L.max_units) break;
-        GemmUnit g;
-        g.a_row = e * L.feat + ft * BLOCK_M;
-        g.b_row = off + tt * L.tile_tokens;
-        g.f0 = ft * BLOCK_M;
-        g.nm = nv | (min(BLOCK_M, L.feat - ft * BLOCK_M) << 16);
-        L.units[u] = g;
+    __syncthreads();
+    const int n_write = min(nu_total, L.max_units);
+    for (int u = threadIdx.x; u < n_write; u += blockDim.x) {
+      int lo = 0, hi = n_experts - 1;  // largest expert whose first unit is <= u
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_u0[mid] <= u) lo = mid;
+        else hi = mid - 1;
+      }
+      const int ex = lo;
+      const int local = u - s_u0[ex];
+      const int tt = local / nft, ft = local - tt * nft;
+      const int nv = min(L.tile_tokens, s_cnt[ex] - tt * L.tile_tokens);
+      const int4 g = make_int4(ex * L.feat + ft * BLOCK_M, s_offs[ex] + tt * L.tile_tokens, ft * BLOCK_M,
+                               nv | (min(BLOCK_M, L.feat - ft * BLOCK_M) << 16));
+      *reinterpret_cast<int4*>(&L.units[u]) = g;
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Stable row assignment.  One warp per chunk walks the chunk's assignments in (token, slot) order,
+// 32 at a time: lanes holding the same expert are ranked with __match_any_sync, and a per-expert
+// running base (from scan_units_kernel) gives each assignment its grouped row.
+// ------------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(32)
+    assign_rows_kernel(const int* __restrict__ topk_idx, const float* __restrict__ topk_gate,
+                       const int* __restrict__ chunk_base, int T, int n_experts, int k, int chunk_tokens,
+                       int* __restrict__ row_of, int* __restrict__ tok_of_row, float* __restrict__ gate_of_row,
+                       unsigned* status) {
+  extern __shared__ int s_base[];  // [n_experts]
+  const int lane = threadIdx.x;
+  for (int e = lane; e < n_experts; e += 32) s_base[e] = chunk_base[(long long)e * gridDim.x + blockIdx.x];
+  __syncwarp();
+  const int t_begin = blockIdx.x * chunk_tokens;
+  const int t_end = min(T, t_begin + chunk_tokens);
+  const long long a_begin = (long long)t_begin * k, a_end = (long long)t_end * k;
+  const long long TK = (long long)T * k;
+  for (long long a0 = a_begin; a0 < a_end; a0 += 32) {
+    const long long a = a0 + lane;
+    const bool act = a < a_end;
+    int e = act ? topk_idx[a] : -1 - lane;  // inactive lanes get unique keys
+    const bool e_ok = e >= 0 && e < n_experts;
+    if (act && !e_ok) atomicOr(status, DEV_STATUS_BAD_INDEX);
+    const float g = act ? topk_gate[a] : 0.f;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int leader = __ffs(peers) - 1;
+    int base = 0;
+    if (act && e_ok) base = s_base[e];
+    __syncwarp();
+    if (act && e_ok && lane == leader) s_base[e] = base + __popc(peers);
+    __syncwarp();
+    if (act) {
+      const int row = e_ok ? base + rank : -1;
+      if (row >= 0 && row < TK) {
+        row_of[a] = row;
+        tok_of_row[row] = (int)(a / k);
+        gate_of_row[row] = g;
+      } else {
+        if (e_ok) atomicOr(status, DEV_STATUS_BAD_INDEX);
+        row_of[a] = -1;
       }
     }
   }
 }
 
 // ------------------------------------------------------------------------------------------------
-// Stable row assignment and the gather of latent rows into expert-grouped order.
-// One block per chunk.  Warp 0 walks the chunk's assignments in (token, slot) order, 32 at a time:
-// lanes holding the same expert are ranked with __match_any_sync, and a per-expert running base
-// (from scan_units_kernel) gives each assignment its row.  Then all warps copy h[t] to h_perm[row].
+// Gather of latent rows into expert-grouped order: h_perm[r] = h[tok_of_row[r]].  Grid-stride over
+// groups of 8 grouped rows per warp, so each lane keeps 8 independent 16-byte loads in flight.
 // ------------------------------------------------------------------------------------------------
-constexpr int SCATTER_WARPS = 8;
+constexpr int GATHER_ROWS = 8;
 
-__global__ void __launch_bounds__(SCATTER_WARPS * 32)
-    scatter_gather_kernel(const int* __restrict__ topk_idx, const float* __restrict__ topk_gate,
-                          const int* __restrict__ chunk_base, int T, int n_experts, int k, int chunk_tokens,
-                          const __nv_bfloat16* __restrict__ h, int latent, int* __restrict__ row_of,
-                          int* __restrict__ tok_of_row, float* __restrict__ gate_of_row,
-                          __nv_bfloat16* __restrict__ h_perm, unsigned* status) {
-  extern __shared__ int s_base[];  // [n_experts]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int e = threadIdx.x; e < n_experts; e += blockDim.x) s_base[e] = chunk_base[(long long)blockIdx.x * n_experts + e];
-  __syncthreads();
-  const int t_begin = blockIdx.x * chunk_tokens;
-  const int t_end = min(T, t_begin + chunk_tokens);
-  const long long a_begin = (long long)t_begin * k, a_end = (long long)t_end * k;
-  const long long TK = (long long)T * k;
-  if (warp == 0) {
-    for (long long a0 = a_begin; a0 < a_end; a0 += 32) {
-      const long long a = a0 + lane;
-      const bool act = a < a_end;
-      const unsigned amask = __ballot_sync(0xffffffffu, act);
-      int e = act ? topk_idx[a] : -1 - lane;  // inactive lanes get unique keys
-      const bool e_ok = e >= 0 && e < n_experts;
-      if (act && !e_ok) atomicOr(status, DEV_STATUS_BAD_INDEX);
-      const unsigned peers = __match_any_sync(0xffffffffu, e);
-      const int rank = __popc(peers & ((1u << lane) - 1u));
-      const int leader = __ffs(peers) - 1;
-      int base = 0;
-      if (act && e_ok) base = s_base[e];
-      __syncwarp();
-      if (act && e_ok && lane == leader) s_base[e] = base + __popc(peers);
-      __syncwarp();
-      if (act && e_ok) {
-        const int row = base + rank;
-        if (row >= 0 && row < TK) {
-          row_of[a] = row;
-          tok_of_row[row] = (int)(a / k);
-          gate_of_row[row] = topk_gate[a];
-        } else {
-          atomicOr(status, DEV_STATUS_BAD_INDEX);
-          row_of[a] = -1;
-        }
-      } else if (act) {
-        row_of[a] = -1;
+__global__ void __launch_bounds__(256)
+    gather_rows_kernel(const __nv_bfloat16* __restrict__ h, const int* __restrict__ tok_of_row, long long n_rows,
+                       int T, int latent, __nv_bfloat16* __restrict__ h_perm, unsigned* status) {
+  const int lane = threadIdx.x & 31;
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  const int vpr = latent / 8;
+  for (long long r0 = warp * GATHER_ROWS; r0 < n_rows; r0 += nwarps * GATHER_ROWS) {
+    int tok[GATHER_ROWS];
+#pragma unroll
+    for (int j = 0; j < GATHER_ROWS; ++j) {
+      const long long r = r0 + j;
+      int t = (r < n_rows) ? tok_of_row[r] : -1;
+      if (r < n_rows && (t < 0 || t >= T)) {
+        if (lane == 0) atomicOr(status, DEV_STATUS_BAD_INDEX);
+        t = -1;
       }
-      (void)amask;
+      tok[j] = t;
     }
-  }
-  __syncthreads();
-  // gather: 16-byte chunks of each latent row
-  const int vec_per_row = latent / 8;
-  for (long long a = a_begin + warp; a < a_end; a += SCATTER_WARPS) {
-    const int row = row_of[a];
-    if (row < 0) continue;
-    const int t = (int)(a / k);
-    const uint4* src = reinterpret_cast<const uint4*>(h + (long long)t * latent);
-    uint4* dst = reinterpret_cast<uint4*>(h_perm + (long long)row * latent);
-    for (int i = lane; i < vec_per_row; i += 32) dst[i] = src[i];
+    for (int i = lane; i < vpr; i += 32) {
+      uint4 buf[GATHER_ROWS];
+#pragma unroll
+      for (int j = 0; j < GATHER_ROWS; ++j)
+        if (tok[j] >= 0) buf[j] = reinterpret_cast<const uint4*>(h + (long long)tok[j] * latent)[i];
+#pragma unroll
+      for (int j = 0; j < GATHER_ROWS; ++j)
+        if (tok[j] >= 0) reinterpret_cast<uint4*>(h_perm + (r0 + j) * latent)[i] = buf[j];
+    }
   }
 }
 

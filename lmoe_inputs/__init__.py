@@ -77,6 +77,10 @@ WORKLOADS: Dict[str, Workload] = {
                              description="NVFP4 experts+shared expert, decode batch T=256"),
     "prefill_nvfp4": Workload("prefill_nvfp4", SUPER, 16384, 1, 3, "bf16", "nvfp4",
                               description="NVFP4 experts+shared expert, prefill T=16384"),
+    # profiling case: the decode kernels' regime (~11 tokens per expert, weights streamed once) on a
+    # 128-expert layer, so that a full-metric profiler capture holds ~1.5 GB on the device
+    "decode_small": Workload("decode_small", dataclasses.replace(SUPER, n_experts=128), 64, 1, 2, "bf16", "bf16",
+                             description="Super dims with 128 experts, T=64 (~11 tokens per expert)"),
     "skewed": Workload("skewed", SUPER, 4096, 1, 4, "bf16", "bf16", router_bias=True,
                        description="Super shape T=4096, per-expert router bias giving a capped Zipf(1.2) load"),
 }
