@@ -69,7 +69,8 @@ struct GemmArgs {
   int main_dense_units;       // units of prob[0] when it is dense (units == nullptr)
   const GemmUnit* units;      // prob[0] grouped: device unit list
   const int* num_units;       // prob[0] grouped: device unit count
-  int* work_counter;          // zero before launch; units are claimed with atomicAdd
+  int dynamic;                // 1: units are claimed from work_counter; 0: CTA c takes c, c + grid, ...
+  int* work_counter;          // zero before a dynamic launch
   unsigned* status;           // device status word
   unsigned long long timeout_ns;
 };
@@ -107,7 +108,8 @@ __device__ __forceinline__ GemmUnit dense_unit(const GemmProblem& p, int u) {
   return r;
 }
 
-// Global unit u of the launch: which problem it belongs to, and its tile.
+// Global unit u of the launch: which problem it belongs to, and its tile.  The pre problem's units
+// come first (measured: spreading them through the expert units was slower at decode sizes).
 template <int BN_MAX>
 __device__ __forceinline__ GemmUnit unit_at(const GemmArgs& a, int u, int& pid) {
   if (u < a.n_pre_units) {
@@ -197,8 +199,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       bool ok = true;
       int uslot = 0;
       uint32_t uphase = 0;
-      // the next unit is claimed one unit ahead, so the atomic's round trip overlaps the loads
-      int u_next = atomicAdd(args.work_counter, 1);
+      // dynamic launches claim the next unit one unit ahead, so the atomic's round trip overlaps the
+      // loads; static launches take every gridDim.x-th unit
+      int u_next = args.dynamic ? atomicAdd(args.work_counter, 1) : (int)blockIdx.x;
       while (ok) {
         if (!mbar_wait_bounded(&uempty[uslot], uphase ^ 1u, abort_flag, tmo)) {
           ok = false;
@@ -212,7 +215,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           uphase ^= 1u;
         }
         if (u < 0) break;
-        u_next = atomicAdd(args.work_counter, 1);
+        u_next = args.dynamic ? atomicAdd(args.work_counter, 1) : u_next + (int)gridDim.x;
         int pid;
         const GemmUnit un = unit_at<BN_MAX>(args, u, pid);
         const GemmProblem& pr = args.prob[pid];

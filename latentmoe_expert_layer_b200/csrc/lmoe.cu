@@ -238,6 +238,7 @@ struct GemmLaunch {
   void main_grouped(const CUtensorMap& mw, const CUtensorMap& ma, GemmProblem p, const GemmUnit* units,
                     const int* num_units) {
     p.weights_streamed = v == V_SMALL;  // decode-sized groups: mostly one token tile per expert
+    a.dynamic = v == V_SMALL;           // measured: dynamic claiming helps decode-sized groups only
     a.prob[0] = p;
     a.units = units;
     a.num_units = num_units;
