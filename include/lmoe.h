@@ -54,12 +54,13 @@ typedef enum { LMOE_DTYPE_BF16 = 0, LMOE_DTYPE_F32 = 1 } lmoe_dtype;
 typedef struct {
   int32_t d;           /* model dimension (multiple of 64) */
   int32_t latent;      /* latent dimension l (multiple of 64) */
-  int32_t n_experts;   /* N, 1..1024 */
+  int32_t n_experts;   /* N, a multiple of 16, at most 1024 */
   int32_t top_k;       /* K, 1..min(32, N) */
   int32_t expert_ffn;  /* m, routed expert hidden (multiple of 64) */
   int32_t shared_ffn;  /* m_s, shared expert hidden (multiple of 64) */
   int32_t max_tokens;  /* largest T a forward call may pass; sizes the workspace */
-  int32_t precision;   /* lmoe_precision: NVFP4 quantises routed+shared experts (weights and inputs) */
+  int32_t precision;   /* lmoe_precision: NVFP4 quantises routed+shared experts (weights and inputs);
+                          NVFP4 needs d, latent, expert_ffn and shared_ffn to be multiples of 128 */
   int32_t has_router_bias; /* 1: a per-expert fp32 bias is added to the router logits */
 } lmoe_config;
 
@@ -80,8 +81,8 @@ typedef struct {
 } lmoe_weights;
 
 /* Create a layer on CUDA device `device` and allocate its workspace for cfg->max_tokens tokens.
- * Errors: INVALID_ARG (null), UNSUPPORTED (a dimension not a multiple of 64, N > 1024, K > 32,
- * K > N), NO_DEVICE (device missing or not compute capability 10.0), OOM. */
+ * Errors: INVALID_ARG (null), UNSUPPORTED (a dimension not a multiple of 64, N not a multiple of 16
+ * or above 1024, K > 32, K > N), NO_DEVICE (device missing or not compute capability 10.0), OOM. */
 lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out);
 
 /* Copy (and, for NVFP4, quantise) the weights into library-owned device memory, enqueued on
@@ -104,6 +105,18 @@ lmoe_status lmoe_forward(lmoe_handle h, const void* x, int32_t T, void* y, int32
 lmoe_status lmoe_forward_host(lmoe_handle h, const void* x_host, int32_t T, void* y_host, int32_t* topk_idx_host,
                               float* topk_gate_host, void* stream);
 
+/* Copy one NVFP4-quantised weight matrix back to the host in plain row-major form (synchronous).
+ *   which  0: W1 of expert `index` [m, l]   1: W2 of expert `index` [l, m]
+ *          2: W_s1 [m_s, d]                 3: W_s2 [d, m_s]
+ *   codes_host  [rows, K/2] bytes, element 2i in the low nibble (E2M1: bit 3 sign, bits 0-2
+ *               magnitude index into {0, 0.5, 1, 1.5, 2, 3, 4, 6})
+ *   scales_host [rows, K/16] E4M3 block scales, one per 16 consecutive K elements
+ *   gscale_host fp32 tensor scale; a weight element is code * scale * gscale.
+ * Errors: UNSUPPORTED unless the handle was created with LMOE_PREC_NVFP4; NOT_LOADED; SHAPE for a
+ * bad `which` / `index`. */
+lmoe_status lmoe_export_nvfp4(lmoe_handle h, int32_t which, int32_t index, uint8_t* codes_host,
+                              uint8_t* scales_host, float* gscale_host);
+
 /* Synchronise the handle's device and return the sticky device status raised by any kernel since
  * the last call (DEVICE_TIMEOUT or DEVICE_INDEX), then clear it.  LMOE_OK if none. */
 lmoe_status lmoe_get_device_status(lmoe_handle h);
@@ -118,7 +131,19 @@ typedef enum {
   LMOE_BUF_TOK_OF_ROW = 4, /* int32 [T*K]   token of grouped row r */
   LMOE_BUF_H = 5,          /* bf16 [T, l]   latent h = W_down x */
   LMOE_BUF_Z = 6,          /* bf16 [T, l + m_s] columns 0..l-1: latent sum z; the rest: sqrelu(W_s1 x) */
-  LMOE_BUF_U = 7           /* bf16 [T*K, m] expert hidden activations, grouped rows */
+  LMOE_BUF_U = 7,          /* bf16 [T*K, m] expert hidden activations, grouped rows (bf16 precision) */
+  /* NVFP4 precision only: packed E2M1 codes [rows, K/2] and row-major E4M3 scales
+   * [rows, 16 * ceil(K / 256)] of the quantised activations, and the fp32 shared-expert output */
+  LMOE_BUF_XQ = 8,         /* x codes [T, d/2] */
+  LMOE_BUF_X_SF = 9,       /* x scales */
+  LMOE_BUF_HQ = 10,        /* h codes, grouped rows [T*K, l/2] */
+  LMOE_BUF_H_SF = 11,      /* h scales, grouped rows */
+  LMOE_BUF_UQ = 12,        /* u codes, grouped rows [T*K, m/2] */
+  LMOE_BUF_U_SF = 13,      /* u scales */
+  LMOE_BUF_USQ = 14,       /* u_s codes [T, m_s/2] */
+  LMOE_BUF_US_SF = 15,     /* u_s scales */
+  LMOE_BUF_Y_S = 16,       /* fp32 [T, d]: W_s2 u_s */
+  LMOE_BUF_ACT_SCALE = 17  /* fp32 [2]: tensor scales of x and h in the last forward */
 } lmoe_buffer;
 lmoe_status lmoe_inspect(lmoe_handle h, int32_t which, void** dev_ptr, int64_t* count);
 

@@ -26,14 +26,16 @@ lib = ctypes.CDLL(library_path)
 STATUS = {0: "ok", 1: "invalid argument", 2: "shape out of range", 3: "unsupported configuration",
           4: "device out of memory", 5: "CUDA error", 6: "weights not loaded",
           7: "device-side wait timed out", 8: "device-side index out of range", 9: "no suitable CUDA device"}
-BUF = {"logits": 0, "counts": 1, "offsets": 2, "row_of": 3, "tok_of_row": 4, "h": 5, "z": 6, "u": 7}
+BUF = {"logits": 0, "counts": 1, "offsets": 2, "row_of": 3, "tok_of_row": 4, "h": 5, "z": 6, "u": 7,
+       "xq": 8, "x_sf": 9, "hq": 10, "h_sf": 11, "uq": 12, "u_sf": 13, "usq": 14, "us_sf": 15, "y_s": 16,
+       "act_scale": 17}
 PREC = {"bf16": 0, "nvfp4": 1}
 DTYPE = {torch.bfloat16: 0, torch.float32: 1}
 
 # every extern "C" symbol declared in include/lmoe.h
 SYMBOLS = ("lmoe_create", "lmoe_load_weights", "lmoe_forward", "lmoe_forward_host", "lmoe_get_device_status",
-           "lmoe_inspect", "lmoe_profile", "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_status_string",
-           "lmoe_destroy")
+           "lmoe_inspect", "lmoe_profile", "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_export_nvfp4",
+           "lmoe_status_string", "lmoe_destroy")
 STAGES = ("router", "shared_up", "topk", "grouping", "scatter", "expert_up", "expert_down", "combine", "output")
 
 
@@ -58,12 +60,13 @@ lib.lmoe_inspect.argtypes = [_vp, _i32, ctypes.POINTER(_vp), ctypes.POINTER(_i64
 lib.lmoe_profile.argtypes = [_vp, _i32]
 lib.lmoe_profile_read.argtypes = [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i32), ctypes.POINTER(_i32)]
 lib.lmoe_route_noalloc.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.lmoe_export_nvfp4.argtypes = [_vp, _i32, _i32, _vp, _vp, _vp]
 lib.lmoe_status_string.argtypes = [ctypes.c_int]
 lib.lmoe_status_string.restype = ctypes.c_char_p
 lib.lmoe_destroy.argtypes = [_vp]
 lib.lmoe_destroy.restype = None
 for _f in ("lmoe_create", "lmoe_load_weights", "lmoe_forward", "lmoe_forward_host", "lmoe_get_device_status",
-           "lmoe_inspect", "lmoe_profile", "lmoe_profile_read", "lmoe_route_noalloc"):
+           "lmoe_inspect", "lmoe_profile", "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_export_nvfp4"):
     getattr(lib, _f).restype = ctypes.c_int
 
 
@@ -95,7 +98,8 @@ class _DevArray:
 
 
 _BUF_TYPES = {"logits": "<f4", "counts": "<i4", "offsets": "<i4", "row_of": "<i4", "tok_of_row": "<i4",
-              "h": "<u2", "z": "<u2", "u": "<u2"}
+              "h": "<u2", "z": "<u2", "u": "<u2", "xq": "|u1", "x_sf": "|u1", "hq": "|u1", "h_sf": "|u1",
+              "uq": "|u1", "u_sf": "|u1", "usq": "|u1", "us_sf": "|u1", "y_s": "<f4", "act_scale": "<f4"}
 
 
 def route_noalloc(logits: torch.Tensor, top_k: int, bias: Optional[torch.Tensor] = None, stream=None):
@@ -176,6 +180,20 @@ class LatentMoE:
             return torch.empty(0)
         t = torch.as_tensor(_DevArray(p.value, n.value, _BUF_TYPES[name]), device=self.device)
         return t.clone()
+
+    def export_nvfp4(self, which: int, index: int = 0):
+        """(codes uint8 [rows, K/2], scales uint8 [rows, K/16], tensor scale float) of one quantised
+        weight matrix: which 0 = W1[index], 1 = W2[index], 2 = W_s1, 3 = W_s2."""
+        import numpy as np
+        s = self.shape
+        rows, k = {0: (s.expert_ffn, s.latent), 1: (s.latent, s.expert_ffn), 2: (s.shared_ffn, s.d),
+                   3: (s.d, s.shared_ffn)}[which]
+        codes = np.empty((rows, k // 2), np.uint8)
+        scales = np.empty((rows, k // 16), np.uint8)
+        g = np.empty(1, np.float32)
+        _check(lib.lmoe_export_nvfp4(self._h, which, index, codes.ctypes.data, scales.ctypes.data, g.ctypes.data),
+               "lmoe_export_nvfp4")
+        return codes, scales, np.float32(g[0])
 
     def profile(self, enable: bool) -> None:
         """Start (clearing the record) or stop per-stage CUDA-event timing of forward calls."""

@@ -2,19 +2,25 @@
 //
 //   out[tok, f] = epi( sum_k W[f, k] * act[tok, k] )
 //
-// W (weights, K-major, bf16) is the MMA's A operand: 128 output features per tile fill the
-// M = 128 rows of the tensor core.  The activations (K-major, bf16) are the B operand: up to BN_MAX
-// tokens per tile form N, rounded up to a multiple of 16.  With tokens on N, an expert that holds
-// only ~11 tokens (the T = 256 decode batch spread over 512 experts) costs an N = 16 MMA instead of a
-// 128-row tile that is 90 % padding, and every expert weight byte is streamed exactly once per token
-// tile.
+// W (weights, K-major) is the MMA's A operand: 128 output features per tile fill the M = 128 rows of
+// the tensor core.  The activations (K-major) are the B operand: up to BN_MAX tokens per tile form N,
+// rounded up to a multiple of 16.  With tokens on N, an expert that holds only ~11 tokens (the
+// T = 256 decode batch spread over 512 experts) costs an N = 16 MMA instead of a 128-row tile that is
+// 90 % padding, and every expert weight byte is streamed exactly once per token tile.
+//
+// Two operand formats (template flag FP4):
+//   bf16   kind::f16, 64 elements (128 bytes) of K per pipeline stage
+//   NVFP4  kind::mxf4nvf4 with 16-element E4M3 block scales, 256 E2M1 elements (128 bytes) of K per
+//          stage; weight scales arrive as 512-byte atoms by bulk copy, activation scales are staged
+//          into atoms by the producer warp, and the MMA issuer moves both into TMEM with tcgen05.cp.
+//          The epilogue multiplies by the two fp32 tensor scales.
 //
 // Roles (192 threads):
-//   warp 0      TMA producer: one lane streams W and activation tiles into a STAGES-deep ring
-//   warp 1      MMA issuer: allocates TMEM, one lane issues tcgen05.mma into one of two TMEM
+//   warp 0      producer: streams W and activation tiles (TMA) and scales into a STAGES-deep ring
+//   warp 1      MMA issuer: allocates TMEM, one lane issues tcgen05 MMAs into one of two TMEM
 //               accumulators (double buffered, so the epilogue of tile i overlaps the MMAs of i+1)
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes 32*(w%4)..),
-//               elementwise op, transpose through shared memory, coalesced 16-byte stores
+//               elementwise op, transpose through shared memory, vector stores
 //
 // Work units are (weight row block, token block) pairs.  Dense GEMMs enumerate them from the
 // launch arguments; the grouped expert GEMMs read a unit list that the routing kernels built on the
@@ -23,6 +29,9 @@
 // decode sizes every problem is a weight stream, so folding a small dense GEMM into an expert launch
 // costs only its bytes instead of a launch that cannot fill the GPU.
 #pragma once
+#include <cuda_bf16.h>
+
+#include "nvfp4.cuh"
 #include "ptx.cuh"
 
 namespace lmoe {
@@ -34,21 +43,23 @@ enum EpiKind : int {
   EPI_ROWSCALE_BF16 = 3,  // out = bf16(acc * row_scale[token row])
   EPI_ROUTER = 4,         // features < split_feat: fp32 to out2; others: bf16 to out (column f - split)
   EPI_ADD_BF16 = 5,       // out = bf16(acc + addend[token row, f])  (fp32 addend)
+  EPI_SQRELU_NVFP4 = 6,   // out = NVFP4(max(acc, 0)^2) with tensor scale 1: codes to out, scales to out_sf
 };
 
 // One unit of GEMM work.  a_row: first W row of the tile; b_row: first activation row (also the
 // output row); f0: first output feature (column) of the tile; nm = n_valid | (m_valid << 16) with
-// n_valid tokens (1..BN_MAX) and m_valid features (1..128, a multiple of 32).
+// n_valid tokens (1..BN_MAX) and m_valid features (1..128, a multiple of 16; a multiple of 32 for
+// EPI_SQRELU_NVFP4).
 struct GemmUnit {
   int a_row, b_row, f0, nm;
 };
 
-// One GEMM problem of a launch: K extent, epilogue, and (for dense problems) the tile grid.
+// One GEMM problem of a launch: K extent, epilogue, NVFP4 scales, and (for dense problems) the grid.
 struct GemmProblem {
-  int num_k_blocks;           // K / 64
+  int num_k_blocks;           // pipeline stages along K (64 bf16 or 256 FP4 elements each)
   int epi;
   void* out;
-  long long ldo;              // output row pitch (elements)
+  long long ldo;              // output row pitch (elements; bytes for EPI_SQRELU_NVFP4 codes)
   int out_col0;               // output column offset
   float* out2;                // EPI_ROUTER fp32 destination
   long long ld2;
@@ -56,11 +67,23 @@ struct GemmProblem {
   const float* row_scale;     // EPI_ROWSCALE_BF16
   const float* addend;        // EPI_ADD_BF16
   long long ld_add;
+  uint8_t* out_sf;            // EPI_SQRELU_NVFP4 scales [rows, out_sf_pitch]
+  int out_sf_pitch;
   int weights_streamed;       // 1: every weight tile is read by one unit only (L2 evict-first)
-  int dense_ftiles;           // dense: feature tiles
-  int dense_ttiles;           // dense: token tiles (fastest-varying unit index)
-  int dense_feat;             // dense: output features (rows of W)
-  int dense_tokens;           // dense: tokens (rows of act)
+  // NVFP4 operands
+  const uint8_t* w_sf;        // weight scale atoms
+  int w_atoms_k;              // K atoms per 128-row tile
+  const float* w_gscale;      // per-group weight tensor scale, group = a_row / w_rows_per_g
+  int w_rows_per_g;
+  const uint8_t* act_sf;      // activation scales, row-major [act_rows, act_sf_pitch]
+  int act_sf_pitch;
+  long long act_rows;
+  const float* act_gscale;    // activation tensor scale (device scalar)
+  // dense enumeration
+  int dense_ftiles;           // feature tiles
+  int dense_ttiles;           // token tiles (fastest-varying unit index)
+  int dense_feat;             // output features (rows of W)
+  int dense_tokens;           // tokens (rows of act)
 };
 
 struct GemmArgs {
@@ -78,19 +101,33 @@ struct GemmArgs {
 constexpr int GEMM_THREADS = 192;
 constexpr int UNIT_RING = 4;
 constexpr int BLOCK_M = 128;
-constexpr int BLOCK_K = 64;                 // 64 bf16 = one 128-byte swizzle row
-constexpr int A_STAGE_BYTES = BLOCK_M * BLOCK_K * 2;
+constexpr int BLOCK_K = 64;                 // bf16 elements per stage (one 128-byte swizzle row)
+constexpr int A_STAGE_BYTES = BLOCK_M * 128;
 constexpr int EPI_STAGE_BYTES = 32 * 32 * 4;  // per epilogue warp: 32 tokens x 32 features fp32
+constexpr int SF_ATOM_BYTES = 512;
 
-template <int BN_MAX, int STAGES>
+template <int BN_MAX, int STAGES, bool FP4>
 struct GemmSmem {
-  static constexpr int B_STAGE_BYTES = BN_MAX * BLOCK_K * 2;
-  static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+  static constexpr int NRA = (BN_MAX + 127) / 128;                    // 128-row scale atoms of B
+  static constexpr int B_STAGE_BYTES = BN_MAX * 128;
+  static constexpr int SFA_STAGE_BYTES = FP4 ? 4 * SF_ATOM_BYTES : 0;
+  static constexpr int SFB_STAGE_BYTES = FP4 ? 4 * NRA * SF_ATOM_BYTES : 0;
+  static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES + SFA_STAGE_BYTES + SFB_STAGE_BYTES;
   static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
   static constexpr int BAR_OFF = EPI_OFF + 4 * EPI_STAGE_BYTES;
   static constexpr int BYTES = BAR_OFF + 512;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment of the base
-  static constexpr uint32_t TMEM_COLS = (2 * BN_MAX < 32) ? 32 : 2 * BN_MAX;
+  // TMEM: two fp32 accumulators of BN_MAX columns, then (FP4) the scale columns of one stage:
+  // SFA 4 MMAs x 4 columns, SFB 4 MMAs x NRA x 4 columns
+  static constexpr int SF_COL0 = 2 * BN_MAX;
+  static constexpr int SF_COLS = FP4 ? 16 + 16 * NRA : 0;
+  static constexpr uint32_t TMEM_COLS = (SF_COL0 + SF_COLS <= 32)    ? 32
+                                        : (SF_COL0 + SF_COLS <= 64)  ? 64
+                                        : (SF_COL0 + SF_COLS <= 128) ? 128
+                                        : (SF_COL0 + SF_COLS <= 256) ? 256
+                                                                     : 512;
+  static_assert(SF_COL0 + SF_COLS <= 512, "TMEM holds 512 columns");
+  static_assert(ALLOC <= 232448, "shared memory per CTA");
 };
 
 template <int BN_MAX>
@@ -127,12 +164,12 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rn(float v) {
   return *reinterpret_cast<uint16_t*>(&b);
 }
 
-template <int BN_MAX, int STAGES, int BOXN>
+template <int BN_MAX, int STAGES, int BOXN, bool FP4>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_w0, const __grid_constant__ CUtensorMap map_act0,
                    const __grid_constant__ CUtensorMap map_w1, const __grid_constant__ CUtensorMap map_act1,
                    const GemmArgs args) {
-  using S = GemmSmem<BN_MAX, STAGES>;
+  using S = GemmSmem<BN_MAX, STAGES, FP4>;
   static_assert(BN_MAX % BOXN == 0 && BOXN % 8 == 0, "token box must tile the token block");
   static_assert(BN_MAX % 16 == 0 && BN_MAX <= 256, "MMA N limit");
   extern __shared__ uint8_t smem_raw[];
@@ -153,7 +190,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], FP4 ? 33 : 1);  // FP4: the TMA lane's expect_tx + the 32 scale-staging lanes
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -188,8 +225,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const uint64_t tmo = args.timeout_ns;
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // ------------------------------------------------------------------ producer (whole warp for FP4)
+    if (FP4 || lane == 0) {
       const uint64_t pol_first = policy_evict_first();
       const uint64_t pol_normal = policy_evict_normal();
       const uint64_t pol_a = policy_evict_last();
@@ -201,21 +238,32 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t uphase = 0;
       // dynamic launches claim the next unit one unit ahead, so the atomic's round trip overlaps the
       // loads; static launches take every gridDim.x-th unit
-      int u_next = args.dynamic ? atomicAdd(args.work_counter, 1) : (int)blockIdx.x;
+      int u_next = 0;
+      if (lane == 0) u_next = args.dynamic ? atomicAdd(args.work_counter, 1) : (int)blockIdx.x;
+      // Only lane 0 waits on barriers; for FP4 the other lanes follow its decisions by shuffle.
+      auto wait0 = [&](uint64_t* bar, uint32_t par) -> bool {
+        bool w = true;
+        if (lane == 0) w = mbar_wait_bounded(bar, par, abort_flag, tmo);
+        if (FP4) w = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
+        return w;
+      };
       while (ok) {
-        if (!mbar_wait_bounded(&uempty[uslot], uphase ^ 1u, abort_flag, tmo)) {
+        if (!wait0(&uempty[uslot], uphase ^ 1u)) {
           ok = false;
           break;
         }
-        const int u = u_next < num_units ? u_next : -1;
-        unit_ring[uslot] = u;
-        mbar_arrive(&ufull[uslot]);
+        int u = u_next < num_units ? u_next : -1;
+        if (FP4) u = __shfl_sync(0xffffffffu, u, 0);
+        if (lane == 0) {
+          unit_ring[uslot] = u;
+          mbar_arrive(&ufull[uslot]);
+        }
         if (++uslot == UNIT_RING) {
           uslot = 0;
           uphase ^= 1u;
         }
         if (u < 0) break;
-        u_next = args.dynamic ? atomicAdd(args.work_counter, 1) : u_next + (int)gridDim.x;
+        if (lane == 0) u_next = args.dynamic ? atomicAdd(args.work_counter, 1) : u_next + (int)gridDim.x;
         int pid;
         const GemmUnit un = unit_at<BN_MAX>(args, u, pid);
         const GemmProblem& pr = args.prob[pid];
@@ -225,18 +273,44 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const int nkb = pr.num_k_blocks;
         const int nv = un.nm & 0xFFFF;
         const int nbox = (nv + BOXN - 1) / BOXN;
-        const uint32_t bytes = A_STAGE_BYTES + nbox * BOXN * BLOCK_K * 2;
+        const uint32_t bytes = A_STAGE_BYTES + nbox * BOXN * 128 + S::SFA_STAGE_BYTES;
+        // x coordinate of a stage in the tensor maps: 128 bytes = 64 bf16 elements or 128 FP4 bytes
+        const int kx = FP4 ? 128 : BLOCK_K;
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, tmo)) {
+          if (!wait0(&empty[stage], phase ^ 1u)) {
             ok = false;
             break;
           }
           uint8_t* sa = smem + stage * S::STAGE_BYTES;
           uint8_t* sb = sa + A_STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d(sa, mw, &full[stage], kb * BLOCK_K, un.a_row, pol_w);
-          for (int i = 0; i < nbox; ++i)
-            tma_load_2d(sb + i * BOXN * BLOCK_K * 2, ma, &full[stage], kb * BLOCK_K, un.b_row + i * BOXN, pol_a);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            tma_load_2d(sa, mw, &full[stage], kb * kx, un.a_row, pol_w);
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d(sb + i * BOXN * 128, ma, &full[stage], kb * kx, un.b_row + i * BOXN, pol_a);
+          }
+          if constexpr (FP4) {
+            uint8_t* ssfa = sb + S::B_STAGE_BYTES;
+            uint8_t* ssfb = ssfa + S::SFA_STAGE_BYTES;
+            if (lane == 0)
+              bulk_load(ssfa, pr.w_sf + ((long long)(un.a_row >> 7) * pr.w_atoms_k + kb * 4) * SF_ATOM_BYTES,
+                        S::SFA_STAGE_BYTES, &full[stage]);
+            // activation scales: row j of the token block -> 4 words (one per K atom of this stage)
+            const int n_load = nbox * BOXN;
+            for (int j = lane; j < n_load; j += 32) {
+              const long long row = (long long)un.b_row + j;
+              uint4 w = make_uint4(0u, 0u, 0u, 0u);
+              if (row < pr.act_rows)
+                w = *reinterpret_cast<const uint4*>(pr.act_sf + row * pr.act_sf_pitch + kb * 16);
+              uint8_t* dst = ssfb + (j >> 7) * SF_ATOM_BYTES + (j & 31) * 16 + ((j & 127) >> 5) * 4;
+              *reinterpret_cast<uint32_t*>(dst + 0 * S::NRA * SF_ATOM_BYTES) = w.x;
+              *reinterpret_cast<uint32_t*>(dst + 1 * S::NRA * SF_ATOM_BYTES) = w.y;
+              *reinterpret_cast<uint32_t*>(dst + 2 * S::NRA * SF_ATOM_BYTES) = w.z;
+              *reinterpret_cast<uint32_t*>(dst + 3 * S::NRA * SF_ATOM_BYTES) = w.w;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&full[stage]);
+          }
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -244,7 +318,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
         }
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         // Give every load still in flight a bounded chance to land before the CTA exits.
         atomicOr(args.status, DEV_STATUS_TIMEOUT);
         volatile int never = 0;
@@ -286,7 +360,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const int nkb = args.prob[pid].num_k_blocks;
         const int nv = un.nm & 0xFFFF;
         const uint32_t n_mma = (uint32_t)((nv + 15) & ~15);
-        const uint32_t idesc = idesc_bf16_f32(BLOCK_M, n_mma);
+        const uint32_t idesc = FP4 ? idesc_nvf4(BLOCK_M, n_mma) : idesc_bf16_f32(BLOCK_M, n_mma);
+        const int nra = (int)((n_mma + 127) >> 7);
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, tmo)) {
           ok = false;
           break;
@@ -302,9 +377,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t sa = smem_u32(smem + stage * S::STAGE_BYTES);
           const uint64_t da = smem_desc_sw128(sa);
           const uint64_t db = smem_desc_sw128(sa + A_STAGE_BYTES);
+          if constexpr (FP4) {
+            const uint32_t ssfa = sa + A_STAGE_BYTES + S::B_STAGE_BYTES;
+            const uint32_t ssfb = ssfa + S::SFA_STAGE_BYTES;
+            const uint32_t t_sfa = tmem_base + S::SF_COL0;
+            const uint32_t t_sfb = t_sfa + 16;
 #pragma unroll
-          for (int k = 0; k < BLOCK_K / 16; ++k)  // K = 16 per MMA: +32 bytes = +2 in the address field
-            umma_bf16(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+            for (int k = 0; k < 4; ++k) {
+              tcgen05_cp_32x128b_x4(t_sfa + 4 * k, smem_desc_sf_atom(ssfa + k * SF_ATOM_BYTES));
+              for (int ra = 0; ra < nra; ++ra)
+                tcgen05_cp_32x128b_x4(t_sfb + 4 * (k * nra + ra),
+                                      smem_desc_sf_atom(ssfb + (k * S::NRA + ra) * SF_ATOM_BYTES));
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k)  // K = 64 E2M1 per MMA: +32 bytes = +2 in the address field
+              umma_nvf4(d_tmem, da + 2 * k, db + 2 * k, idesc, t_sfa + 4 * k, t_sfb + 4 * k * nra, (kb | k) != 0);
+          } else {
+#pragma unroll
+            for (int k = 0; k < BLOCK_K / 16; ++k)  // K = 16 bf16 per MMA: +32 bytes = +2 in the address field
+              umma_bf16(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+          }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
@@ -349,6 +441,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const GemmProblem& pr = args.prob[pid];
       const int nv = un.nm & 0xFFFF;
       const int mv = un.nm >> 16;
+      float oscale = 1.0f;
+      if constexpr (FP4) oscale = __ldg(pr.w_gscale + un.a_row / pr.w_rows_per_g) * __ldg(pr.act_gscale);
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, tmo)) {
         if (lane == 0) atomicOr(args.status, DEV_STATUS_TIMEOUT);
         break;
@@ -368,9 +462,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[acc]);
         }
+        if constexpr (FP4) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * oscale);
+        }
         const int row0 = un.b_row + c * 32;
         const int nrows = min(32, nv - c * 32);
-        bool f32_out = (pr.epi == EPI_F32) || (pr.epi == EPI_ROUTER && un.f0 < pr.split_feat);
+        const bool f32_out = (pr.epi == EPI_F32) || (pr.epi == EPI_ROUTER && un.f0 < pr.split_feat);
         if (pr.epi == EPI_ROWSCALE_BF16) {
           const float mys = (lane < nrows) ? pr.row_scale[row0 + lane] : 0.f;
 #pragma unroll
@@ -382,7 +480,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int j = 0; j < 32; ++j)
               if (j < nrows) r[j] = __float_as_uint(__uint_as_float(r[j]) + ad[(long long)j * pr.ld_add]);
           }
-        } else if (pr.epi == EPI_SQRELU_BF16) {
+        } else if (pr.epi == EPI_SQRELU_BF16 || pr.epi == EPI_SQRELU_NVFP4) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float v = fmaxf(__uint_as_float(r[j]), 0.f);
@@ -390,7 +488,32 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
         }
         __syncwarp();
-        if (f32_out) {
+        if (pr.epi == EPI_SQRELU_NVFP4) {
+          // transpose through shared memory (XOR-swizzled columns: conflict-free both ways); lane j then
+          // quantises token j's two 16-feature blocks and writes 16 code bytes and 2 scale bytes
+          float* s32 = reinterpret_cast<float*>(stg);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) s32[j * 32 + (lane ^ j)] = __uint_as_float(r[j]);
+          __syncwarp();
+          if (feat_ok && lane < nrows) {
+            uint32_t cw[4];
+            uint32_t sbs = 0;
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+              float v[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) v[i] = s32[lane * 32 + ((b * 16 + i) ^ lane)];
+              uint32_t cb[2];
+              sbs |= nvfp4_block(v, 1.0f, cb) << (8 * b);
+              cw[2 * b] = cb[0];
+              cw[2 * b + 1] = cb[1];
+            }
+            const long long row = row0 + lane;
+            *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(pr.out) + row * pr.ldo + f / 2) =
+                make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            *reinterpret_cast<uint16_t*>(pr.out_sf + row * pr.out_sf_pitch + f / 16) = (uint16_t)sbs;
+          }
+        } else if (f32_out) {
           float* s32 = reinterpret_cast<float*>(stg);
 #pragma unroll
           for (int j = 0; j < 32; ++j) s32[j * 32 + lane] = __uint_as_float(r[j]);
@@ -398,7 +521,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           float* dst = (pr.epi == EPI_ROUTER) ? pr.out2 : reinterpret_cast<float*>(pr.out);
           const long long ld = (pr.epi == EPI_ROUTER) ? pr.ld2 : pr.ldo;
           const int col = (pr.epi == EPI_ROUTER) ? f : (pr.out_col0 + f);
-          if (feat_ok) {
+          if (feat_ok && q * 32 + (lane & 7) * 4 < mv) {  // this lane's 4 features are valid
 #pragma unroll
             for (int it = 0; it < 8; ++it) {
               const int j = it * 4 + (lane >> 3);
@@ -415,7 +538,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           __syncwarp();
           uint16_t* dst = reinterpret_cast<uint16_t*>(pr.out);
           const int col = (pr.epi == EPI_ROUTER) ? (f - pr.split_feat) : (pr.out_col0 + f);
-          if (feat_ok) {
+          if (feat_ok && q * 32 + (lane & 3) * 8 < mv) {  // this lane's 8 features are valid
 #pragma unroll
             for (int it = 0; it < 4; ++it) {
               const int j = it * 8 + (lane >> 2);

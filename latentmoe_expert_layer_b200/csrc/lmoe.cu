@@ -47,19 +47,34 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
   return r == CUDA_SUCCESS;
 }
 
-// The two GEMM shapes: small token tiles with a deep ring (weight streaming at decode sizes) and
-// 256-token tiles (tensor-core bound at prefill sizes).
-enum Variant { V_SMALL = 0, V_LARGE = 1 };
-constexpr int V_BN[2] = {64, 256};
-constexpr int V_STAGES[2] = {8, 4};
-constexpr int V_BOXN[2] = {16, 64};
+// GEMM shapes: small token tiles with a deep ring (weight streaming at decode sizes) and large token
+// tiles (tensor-core bound at prefill sizes), each in bf16 and in NVFP4.
+enum Variant { V_SMALL = 0, V_LARGE = 1, V_SMALL4 = 2, V_LARGE4 = 3 };
+constexpr int V_BN[4] = {64, 256, 64, 192};
+constexpr int V_STAGES[4] = {8, 4, 7, 4};
+constexpr int V_BOXN[4] = {16, 64, 16, 64};
+constexpr bool V_FP4[4] = {false, false, true, true};
 
 template <int V>
 struct VT {
   static constexpr int BN = V_BN[V], ST = V_STAGES[V], BOX = V_BOXN[V];
-  static void* fn() { return reinterpret_cast<void*>(gemm_tc_kernel<BN, ST, BOX>); }
-  static int smem() { return GemmSmem<BN, ST>::ALLOC; }
+  static constexpr bool F4 = V_FP4[V];
+  static void* fn() { return reinterpret_cast<void*>(gemm_tc_kernel<BN, ST, BOX, F4>); }
+  static int smem() { return GemmSmem<BN, ST, F4>::ALLOC; }
 };
+
+// 2-D byte tensor map (packed NVFP4 codes): rows x cols_bytes, 128-byte x box_rows tiles, 128-byte swizzle.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols_bytes, uint64_t ld_bytes,
+                 uint32_t box_rows) {
+  cuuint64_t dims[2] = {cols_bytes, rows};
+  cuuint64_t strides[1] = {ld_bytes};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
 
@@ -108,8 +123,10 @@ struct lmoe_ctx {
   GemmUnit* units2 = nullptr;
   int* num_units = nullptr;  // [2]
   unsigned* status = nullptr;
-  int* work_counters = nullptr;  // [kCounters] per-launch unit counters, zeroed at the start of a forward
-  static constexpr int kCounters = 8;
+  int* work_counters = nullptr;  // [kCounters] per-launch unit counters and (last two) activation amax
+                                 // bits, all zeroed at the start of a forward
+  static constexpr int kCounters = 10;
+  static constexpr int kAmaxX = 8, kAmaxH = 9;
   int max_units1 = 0, max_units2 = 0;
   CUtensorMap map_hperm[2]{}, map_u[2]{}, map_zu[2]{};
   CUtensorMap map_z[2]{}, map_us[2]{};  // the z and u_s column blocks of zu
@@ -127,6 +144,18 @@ struct lmoe_ctx {
   float* gate_dev = nullptr;
 
   int last_T = 0;
+
+  // NVFP4 (precision == LMOE_PREC_NVFP4): weights, scales, activation buffers
+  bool nvfp4 = false;
+  uint8_t *w1q = nullptr, *w2q = nullptr, *ws1q = nullptr, *ws2q = nullptr;          // codes
+  uint8_t *w1_sf = nullptr, *w2_sf = nullptr, *ws1_sf = nullptr, *ws2_sf = nullptr;  // scale atoms
+  float* wg = nullptr;            // tensor scales: [0, N) W1, [N, 2N) W2, 2N W_s1, 2N + 1 W_s2
+  unsigned* w_amax = nullptr;     // [2N + 2] amax bits used while quantising
+  uint8_t *xq = nullptr, *x_sf = nullptr, *hq = nullptr, *h_sf = nullptr;  // x [T, d]; h grouped [TK, l]
+  uint8_t *uq = nullptr, *u_sf = nullptr, *usq = nullptr, *us_sf = nullptr; // u [TK, m]; u_s [T, m_s]
+  float* act_g = nullptr;         // [0] g_x, [1] g_h, [2] 1.0
+  CUtensorMap map_w1q{}, map_w2q{}, map_ws1q{}, map_ws2q{};
+  CUtensorMap map_xq[4]{}, map_hq[4]{}, map_uq[4]{}, map_usq[4]{};  // indexed by variant (FP4 ones)
 
   // stage profiler
   static constexpr int kProfMax = 1024;
@@ -161,7 +190,10 @@ void free_all(lmoe_ctx* c) {
                   c->w2,     c->logits, c->idx,    c->gate,      c->chunk_counts, c->chunk_base, c->counts,
                   c->offsets, c->row_of, c->tok_of_row, c->gate_of_row, c->h, c->h_perm, c->u,
                   c->o,      c->zu,     c->units1, c->units2,    c->num_units,  c->status,     c->x_dev,
-                  c->y_dev,  c->idx_dev, c->gate_dev, c->y_s, c->work_counters};
+                  c->y_dev,  c->idx_dev, c->gate_dev, c->y_s, c->work_counters,
+                  c->w1q,    c->w2q,    c->ws1q,   c->ws2q,      c->w1_sf,      c->w2_sf,      c->ws1_sf,
+                  c->ws2_sf, c->wg,     c->w_amax, c->xq,        c->x_sf,       c->hq,         c->h_sf,
+                  c->uq,     c->u_sf,   c->usq,    c->us_sf,     c->act_g};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -189,11 +221,11 @@ lmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LMOE_OK : LMO
 template <int V>
 cudaError_t launch_gemm_v(const CUtensorMap& w0, const CUtensorMap& a0, const CUtensorMap& w1, const CUtensorMap& a1,
                           const GemmArgs& a, int grid, cudaStream_t s) {
-  gemm_tc_kernel<VT<V>::BN, VT<V>::ST, VT<V>::BOX><<<grid, GEMM_THREADS, VT<V>::smem(), s>>>(w0, a0, w1, a1, a);
+  gemm_tc_kernel<VT<V>::BN, VT<V>::ST, VT<V>::BOX, VT<V>::F4><<<grid, GEMM_THREADS, VT<V>::smem(), s>>>(w0, a0, w1, a1, a);
   return cudaGetLastError();
 }
 
-// A problem with its epilogue; K in elements (multiple of 64).
+// A bf16 problem with its epilogue; K in elements (multiple of 64).
 GemmProblem problem(int K, int epi, void* out, long long ldo, int col0 = 0) {
   GemmProblem p;
   memset(&p, 0, sizeof(p));
@@ -202,6 +234,26 @@ GemmProblem problem(int K, int epi, void* out, long long ldo, int col0 = 0) {
   p.out = out;
   p.ldo = ldo;
   p.out_col0 = col0;
+  return p;
+}
+
+// An NVFP4 problem: K in elements; weight scale atoms / tensor scales; activation scales.
+GemmProblem problem4(int K, int epi, void* out, long long ldo, const uint8_t* w_sf, const float* w_g,
+                     int w_rows_per_g, const uint8_t* act_sf, long long act_rows, const float* act_g) {
+  GemmProblem p;
+  memset(&p, 0, sizeof(p));
+  p.num_k_blocks = (K + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K;
+  p.epi = epi;
+  p.out = out;
+  p.ldo = ldo;
+  p.w_sf = w_sf;
+  p.w_atoms_k = sf_atoms_k(K);
+  p.w_gscale = w_g;
+  p.w_rows_per_g = w_rows_per_g;
+  p.act_sf = act_sf;
+  p.act_sf_pitch = act_sf_pitch(K);
+  p.act_rows = act_rows;
+  p.act_gscale = act_g;
   return p;
 }
 
@@ -237,8 +289,9 @@ struct GemmLaunch {
   // main problem, grouped experts (unit list on the device)
   void main_grouped(const CUtensorMap& mw, const CUtensorMap& ma, GemmProblem p, const GemmUnit* units,
                     const int* num_units) {
-    p.weights_streamed = v == V_SMALL;  // decode-sized groups: mostly one token tile per expert
-    a.dynamic = v == V_SMALL;           // measured: dynamic claiming helps decode-sized groups only
+    const bool small = v == V_SMALL || v == V_SMALL4;
+    p.weights_streamed = small;  // decode-sized groups: mostly one token tile per expert
+    a.dynamic = small;           // measured: dynamic claiming helps decode-sized groups only
     a.prob[0] = p;
     a.units = units;
     a.num_units = num_units;
@@ -263,10 +316,151 @@ struct GemmLaunch {
       if (total < grid) grid = total;
     }
     if (grid < 1) grid = 1;
-    return v == V_SMALL ? launch_gemm_v<V_SMALL>(*w0, *a0, *w1, *a1, a, grid, s)
-                        : launch_gemm_v<V_LARGE>(*w0, *a0, *w1, *a1, a, grid, s);
+    switch (v) {
+      case V_SMALL: return launch_gemm_v<V_SMALL>(*w0, *a0, *w1, *a1, a, grid, s);
+      case V_LARGE: return launch_gemm_v<V_LARGE>(*w0, *a0, *w1, *a1, a, grid, s);
+      case V_SMALL4: return launch_gemm_v<V_SMALL4>(*w0, *a0, *w1, *a1, a, grid, s);
+      default: return launch_gemm_v<V_LARGE4>(*w0, *a0, *w1, *a1, a, grid, s);
+    }
   }
 };
+
+// NVFP4 forward: router, W_down and W_up in bf16; routed and shared experts as block-scaled FP4 GEMMs.
+template <typename Mark>
+cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, float* gate, cudaStream_t s,
+                          Mark& mark, int& launches) {
+  const lmoe_config& g = c->cfg;
+  const int N = g.n_experts, K = g.top_k, d = g.d, l = g.latent, m = g.expert_ffn, ms = g.shared_ffn;
+  const long long TK = (long long)T * K;
+  const long long TKmax = (long long)g.max_tokens * K;
+  const int vd = T <= 512 ? V_SMALL : V_LARGE;
+  const int vg = TK <= 48LL * N ? V_SMALL4 : V_LARGE4;
+  const bool split = vg == V_SMALL4;  // shared-expert GEMMs ride inside the expert launches
+  unsigned* amax_x = reinterpret_cast<unsigned*>(c->work_counters + lmoe_ctx::kAmaxX);
+  unsigned* amax_h = reinterpret_cast<unsigned*>(c->work_counters + lmoe_ctx::kAmaxH);
+  float* g_x = c->act_g + 0;
+  float* g_h = c->act_g + 1;
+  const float* one = c->act_g + 2;
+  cudaError_t e = cudaSuccess;
+  auto chk = [&](cudaError_t r) {
+    if (e == cudaSuccess) e = r;
+  };
+  auto grid_for = [&](long long work, int per_block) {
+    long long b = (work + per_block - 1) / per_block;
+    if (b > (long long)c->num_sms * 16) b = (long long)c->num_sms * 16;
+    return (int)(b < 1 ? 1 : b);
+  };
+
+  // 1. router logits and h = W_down x (bf16; one stacked GEMM when N is a multiple of 128)
+  if (c->fused_router) {
+    GemmLaunch gl(c, vd, 0);
+    GemmProblem p = problem(d, EPI_ROUTER, c->h, l);
+    p.out2 = c->logits;
+    p.ld2 = N;
+    p.split_feat = N;
+    gl.main_dense(c->map_rd, c->map_x[vd], p, N + l, T);
+    chk(gl.run(s));
+  } else {
+    if (c->router_f32) {
+      router_f32_kernel<<<T, 256, d * sizeof(float), s>>>(reinterpret_cast<const __nv_bfloat16*>(x), c->w_r32, d,
+                                                          N, c->logits);
+      chk(cudaGetLastError());
+    } else {
+      GemmLaunch gl(c, vd, 1);
+      gl.main_dense(c->map_r, c->map_x[vd], problem(d, EPI_F32, c->logits, N), N, T);
+      chk(gl.run(s));
+    }
+    GemmLaunch gl(c, vd, 0);
+    gl.main_dense(c->map_down, c->map_x[vd], problem(d, EPI_BF16, c->h, l), l, T);
+    chk(gl.run(s));
+    ++launches;
+  }
+  mark(1);
+  // 2. quantise x (dynamic tensor scale); amax of h
+  amax_act_kernel<<<grid_for((long long)T * d / 8, 256), 256, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(x), (long long)T * d / 8, amax_x);
+  quant_act_kernel<<<grid_for((long long)T * d / 16, 256), 256, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(x), d, nullptr, T, T, amax_x, c->xq, c->x_sf, g_x, c->status);
+  amax_act_kernel<<<grid_for((long long)T * l / 8, 256), 256, 0, s>>>(c->h, (long long)T * l / 8, amax_h);
+  chk(cudaGetLastError());
+  mark(2);
+  // 3. top-K + softmax + per-chunk histogram
+  int ct;
+  const int nch = n_chunks_for(T, N, &ct);
+  chk(launch_topk_hist(nch, topk_threads(ct), s, c->logits, c->b_router, T, N, K, ct, idx, gate, c->chunk_counts));
+  mark(3);
+  // 4. expert offsets and grouped-GEMM unit lists
+  UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1};
+  UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2};
+  scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(c->chunk_counts, nch, N, c->counts, c->offsets,
+                                                              c->chunk_base, l1, l2, c->status);
+  chk(cudaGetLastError());
+  mark(4);
+  // 5. stable grouping; quantise h rows straight into grouped order
+  assign_rows_kernel<<<nch, 32, N * sizeof(int), s>>>(idx, gate, c->chunk_base, T, N, K, ct, c->row_of,
+                                                     c->tok_of_row, c->gate_of_row, c->status);
+  quant_act_kernel<<<grid_for(TK * l / 16, 256), 256, 0, s>>>(c->h, l, c->tok_of_row, TK, T, amax_h, c->hq, c->h_sf,
+                                                               g_h, c->status);
+  chk(cudaGetLastError());
+  mark(5);
+  // 6. expert up (FP4): u = NVFP4(sqrelu(W1_e h)); shared up u_s = NVFP4(sqrelu(W_s1 x))
+  GemmProblem shared_up =
+      problem4(d, EPI_SQRELU_NVFP4, c->usq, ms / 2, c->ws1_sf, c->wg + 2 * N, ms, c->x_sf, T, g_x);
+  shared_up.out_sf = c->us_sf;
+  shared_up.out_sf_pitch = act_sf_pitch(ms);
+  {
+    GemmLaunch gl(c, vg, 4);
+    if (split) gl.pre_dense(c->map_ws1q, c->map_xq[vg], shared_up, ms, T);
+    GemmProblem p = problem4(l, EPI_SQRELU_NVFP4, c->uq, m / 2, c->w1_sf, c->wg, m, c->h_sf, TK, g_h);
+    p.out_sf = c->u_sf;
+    p.out_sf_pitch = act_sf_pitch(m);
+    gl.main_grouped(c->map_w1q, c->map_hq[vg], p, c->units1, c->num_units);
+    chk(gl.run(s));
+  }
+  if (!split) {
+    GemmLaunch gl(c, vg, 2);
+    gl.main_dense(c->map_ws1q, c->map_xq[vg], shared_up, ms, T);
+    chk(gl.run(s));
+  }
+  mark(6);
+  // 7. expert down (FP4) with the gate folded in: o = g * (W2_e u); y_s = W_s2 u_s (fp32)
+  const GemmProblem shared_down =
+      problem4(ms, EPI_F32, c->y_s, d, c->ws2_sf, c->wg + 2 * N + 1, d, c->us_sf, T, one);
+  {
+    GemmLaunch gl(c, vg, 5);
+    if (split) gl.pre_dense(c->map_ws2q, c->map_usq[vg], shared_down, d, T);
+    GemmProblem p = problem4(m, EPI_ROWSCALE_BF16, c->o, l, c->w2_sf, c->wg + N, l, c->u_sf, TK, one);
+    p.row_scale = c->gate_of_row;
+    gl.main_grouped(c->map_w2q, c->map_uq[vg], p, c->units2, c->num_units + 1);
+    chk(gl.run(s));
+  }
+  if (!split) {
+    GemmLaunch gl(c, vg, 3);
+    gl.main_dense(c->map_ws2q, c->map_usq[vg], shared_down, d, T);
+    chk(gl.run(s));
+  }
+  mark(7);
+  // 8. latent combine: zu[:, :l] = sum_k o[row_of[t, k]]
+  {
+    const long long threads = (long long)T * (l / 8);
+    const int blocks = (int)((threads + 255) / 256);
+    combine_kernel<<<blocks, 256, 0, s>>>(c->o, c->row_of, T, K, l, c->zu, l + ms, TKmax, c->status);
+    chk(cudaGetLastError());
+  }
+  mark(8);
+  // 9. y = W_up z + y_s (bf16 GEMM)
+  {
+    GemmLaunch gl(c, vd, 6);
+    GemmProblem p = problem(l, EPI_ADD_BF16, y, d);
+    p.addend = c->y_s;
+    p.ld_add = d;
+    gl.main_dense(c->map_wup, c->map_z[vd], p, d, T);
+    chk(gl.run(s));
+  }
+  mark(9);
+  launches += 12 + (split ? 0 : 2);
+  return e;
+}
 
 }  // namespace
 
@@ -297,8 +491,10 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
     return LMOE_ERR_INVALID_ARG;
   if (g.precision != LMOE_PREC_BF16 && g.precision != LMOE_PREC_NVFP4) return LMOE_ERR_INVALID_ARG;
   if (g.d % 64 || g.latent % 64 || g.expert_ffn % 64 || g.shared_ffn % 64) return LMOE_ERR_UNSUPPORTED;
-  if (g.n_experts > 1024 || g.top_k > 32 || g.top_k > g.n_experts) return LMOE_ERR_UNSUPPORTED;
-  if (g.precision == LMOE_PREC_NVFP4) return LMOE_ERR_UNSUPPORTED;
+  if (g.n_experts > 1024 || g.n_experts % 16 || g.top_k > 32 || g.top_k > g.n_experts) return LMOE_ERR_UNSUPPORTED;
+  if (g.precision == LMOE_PREC_NVFP4 &&
+      (g.d % 128 || g.latent % 128 || g.expert_ffn % 128 || g.shared_ffn % 128))
+    return LMOE_ERR_UNSUPPORTED;
   const long long tk = (long long)g.max_tokens * g.top_k;
   if (tk > 0x7fffffffLL / 2) return LMOE_ERR_UNSUPPORTED;
   int ndev = 0;
@@ -326,7 +522,16 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   ok = ok && dalloc(&c->zu, T * (l + ms));
   ok = ok && dalloc(&c->units1, c->max_units1) && dalloc(&c->units2, c->max_units2) && dalloc(&c->num_units, 2);
   ok = ok && dalloc(&c->status, 1) && dalloc(&c->work_counters, lmoe_ctx::kCounters);
-  ok = ok && dalloc(&c->y_s, (size_t)(T < 512 ? T : 512) * d);
+  c->nvfp4 = g.precision == LMOE_PREC_NVFP4;
+  // y_s = W_s2 u_s in fp32: needed at decode sizes (bf16) and at every size (NVFP4)
+  ok = ok && dalloc(&c->y_s, (size_t)(c->nvfp4 ? T : (T < 512 ? T : 512)) * d);
+  if (c->nvfp4) {
+    ok = ok && dalloc(&c->xq, T * d / 2) && dalloc(&c->x_sf, T * act_sf_pitch(d));
+    ok = ok && dalloc(&c->hq, tk * l / 2) && dalloc(&c->h_sf, tk * act_sf_pitch(l));
+    ok = ok && dalloc(&c->uq, tk * m / 2) && dalloc(&c->u_sf, tk * act_sf_pitch(m));
+    ok = ok && dalloc(&c->usq, T * ms / 2) && dalloc(&c->us_sf, T * act_sf_pitch(ms));
+    ok = ok && dalloc(&c->act_g, 4);
+  }
   if (!ok) {
     free_all(c);
     delete c;
@@ -348,6 +553,29 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
                                   VT<V_SMALL>::smem()) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(VT<V_LARGE>::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   VT<V_LARGE>::smem()) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(VT<V_SMALL4>::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  VT<V_SMALL4>::smem()) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(VT<V_LARGE4>::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  VT<V_LARGE4>::smem()) == cudaSuccess;
+  if (ok && c->nvfp4) {
+    // scale padding (beyond K / 16) must read as zero; stale rows must hold finite scales
+    cudaMemset(c->x_sf, 0, T * act_sf_pitch(d));
+    cudaMemset(c->h_sf, 0, tk * act_sf_pitch(l));
+    cudaMemset(c->u_sf, 0, tk * act_sf_pitch(m));
+    cudaMemset(c->us_sf, 0, T * act_sf_pitch(ms));
+    cudaMemset(c->xq, 0, T * d / 2);
+    cudaMemset(c->hq, 0, tk * l / 2);
+    cudaMemset(c->uq, 0, tk * m / 2);
+    cudaMemset(c->usq, 0, T * ms / 2);
+    const float one[4] = {1.f, 1.f, 1.f, 1.f};
+    ok = cudaMemcpy(c->act_g, one, sizeof(one), cudaMemcpyHostToDevice) == cudaSuccess;
+    for (int v = V_SMALL4; v <= V_LARGE4; ++v) {
+      ok = ok && make_map_u8(&c->map_xq[v], c->xq, T, d / 2, d / 2, V_BOXN[v]);
+      ok = ok && make_map_u8(&c->map_hq[v], c->hq, tk, l / 2, l / 2, V_BOXN[v]);
+      ok = ok && make_map_u8(&c->map_uq[v], c->uq, tk, m / 2, m / 2, V_BOXN[v]);
+      ok = ok && make_map_u8(&c->map_usq[v], c->usq, T, ms / 2, ms / 2, V_BOXN[v]);
+    }
+  }
   ok = ok && cudaFuncSetAttribute(reinterpret_cast<const void*>(scan_units_kernel),
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kScanSmemMax) == cudaSuccess;
   if (!ok || cudaDeviceSynchronize() != cudaSuccess) {
@@ -375,7 +603,9 @@ lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream
   const int f32 = w->dtype == LMOE_DTYPE_F32;
 
   // release weights of a previous load
-  void* old[] = {c->w_rd, c->w_r32, c->w_down, c->b_router, c->w_cat, c->ws1, c->w1, c->w2};
+  void* old[] = {c->w_rd,  c->w_r32, c->w_down, c->b_router, c->w_cat,  c->ws1,  c->w1,    c->w2,
+                 c->w1q,   c->w2q,   c->ws1q,   c->ws2q,     c->w1_sf,  c->w2_sf, c->ws1_sf, c->ws2_sf,
+                 c->wg,    c->w_amax};
   cudaStreamSynchronize(s);
   for (void* p : old)
     if (p) cudaFree(p);
@@ -385,6 +615,10 @@ lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream
   c->b_router = nullptr;
   c->w_cat = nullptr;
   c->ws1 = c->w1 = c->w2 = nullptr;
+  c->w1q = c->w2q = c->ws1q = c->ws2q = nullptr;
+  c->w1_sf = c->w2_sf = c->ws1_sf = c->ws2_sf = nullptr;
+  c->wg = nullptr;
+  c->w_amax = nullptr;
   c->loaded = false;
 
   c->router_f32 = f32;
@@ -418,15 +652,68 @@ lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream
   ok = ok && dalloc(&c->w1, (size_t)N * m * l) && conv(w->w1, (long long)N * m, l, l, c->w1, l, 0);
   ok = ok && dalloc(&c->w2, (size_t)N * l * m) && conv(w->w2, (long long)N * l, m, m, c->w2, m, 0);
   if (!ok) return LMOE_ERR_OOM;
+  if (c->nvfp4) {
+    // quantise W1, W2, W_s1, W_s2 on the device; keep only codes, scale atoms and tensor scales
+    __nv_bfloat16* ws2_tmp = nullptr;
+    ok = ok && dalloc(&ws2_tmp, (size_t)d * ms) && conv(w->ws2, d, ms, ms, ws2_tmp, ms, 0);
+    auto sf_bytes = [](long long rows, int K) { return (size_t)(rows / 128) * sf_atoms_k(K) * SF_ATOM_BYTES; };
+    ok = ok && dalloc(&c->w1q, (size_t)N * m * l / 2) && dalloc(&c->w1_sf, sf_bytes((long long)N * m, l));
+    ok = ok && dalloc(&c->w2q, (size_t)N * l * m / 2) && dalloc(&c->w2_sf, sf_bytes((long long)N * l, m));
+    ok = ok && dalloc(&c->ws1q, (size_t)ms * d / 2) && dalloc(&c->ws1_sf, sf_bytes(ms, d));
+    ok = ok && dalloc(&c->ws2q, (size_t)d * ms / 2) && dalloc(&c->ws2_sf, sf_bytes(d, ms));
+    ok = ok && dalloc(&c->wg, 2 * N + 2) && dalloc(&c->w_amax, 2 * N + 2);
+    if (!ok) {
+      if (ws2_tmp) cudaFree(ws2_tmp);
+      return LMOE_ERR_OOM;
+    }
+    ok = cudaMemsetAsync(c->w_amax, 0, (2 * N + 2) * sizeof(unsigned), s) == cudaSuccess;
+    ok = ok && cudaMemsetAsync(c->w1_sf, 0, sf_bytes((long long)N * m, l), s) == cudaSuccess;
+    ok = ok && cudaMemsetAsync(c->w2_sf, 0, sf_bytes((long long)N * l, m), s) == cudaSuccess;
+    ok = ok && cudaMemsetAsync(c->ws1_sf, 0, sf_bytes(ms, d), s) == cudaSuccess;
+    ok = ok && cudaMemsetAsync(c->ws2_sf, 0, sf_bytes(d, ms), s) == cudaSuccess;
+    struct Q {
+      const __nv_bfloat16* src;
+      long long rows;
+      int K;
+      long long rows_per_g;
+      int groups;
+      uint8_t* codes;
+      uint8_t* sf;
+      int g0;
+    } qs[4] = {{c->w1, (long long)N * m, l, m, N, c->w1q, c->w1_sf, 0},
+               {c->w2, (long long)N * l, m, l, N, c->w2q, c->w2_sf, N},
+               {c->ws1, ms, d, ms, 1, c->ws1q, c->ws1_sf, 2 * N},
+               {ws2_tmp, d, ms, d, 1, c->ws2q, c->ws2_sf, 2 * N + 1}};
+    for (const Q& q : qs) {
+      amax_groups_kernel<<<dim3(16, q.groups), 256, 0, s>>>(q.src, q.rows_per_g * q.K, c->w_amax + q.g0);
+      const long long blocks_needed = (q.rows * (q.K / 16) + 255) / 256;
+      const int blocks = (int)(blocks_needed < 148LL * 64 ? blocks_needed : 148LL * 64);
+      quant_weight_kernel<<<blocks, 256, 0, s>>>(q.src, q.rows, q.K, q.rows_per_g, c->w_amax + q.g0, q.codes, q.sf,
+                                                 c->wg + q.g0);
+    }
+    ok = ok && cudaGetLastError() == cudaSuccess && cudaStreamSynchronize(s) == cudaSuccess;
+    cudaFree(ws2_tmp);
+    cudaFree(c->w1);
+    cudaFree(c->w2);
+    cudaFree(c->ws1);
+    c->w1 = c->w2 = c->ws1 = nullptr;
+    ok = ok && make_map_u8(&c->map_w1q, c->w1q, (uint64_t)N * m, l / 2, l / 2, BLOCK_M);
+    ok = ok && make_map_u8(&c->map_w2q, c->w2q, (uint64_t)N * l, m / 2, m / 2, BLOCK_M);
+    ok = ok && make_map_u8(&c->map_ws1q, c->ws1q, ms, d / 2, d / 2, BLOCK_M);
+    ok = ok && make_map_u8(&c->map_ws2q, c->ws2q, d, ms / 2, ms / 2, BLOCK_M);
+    if (!ok) return LMOE_ERR_CUDA;
+  }
   if (c->fused_router) ok = ok && make_map(&c->map_rd, c->w_rd, N + l, d, d, BLOCK_M);
   if (!c->router_f32 && !c->fused_router) ok = ok && make_map(&c->map_r, c->w_rd, N, d, d, BLOCK_M);
   if (!c->fused_router) ok = ok && make_map(&c->map_down, c->w_down, l, d, d, BLOCK_M);
   ok = ok && make_map(&c->map_cat, c->w_cat, d, l + ms, l + ms, BLOCK_M);
   ok = ok && make_map(&c->map_wup, c->w_cat, d, l, l + ms, BLOCK_M);
   ok = ok && make_map(&c->map_ws2, c->w_cat + l, d, ms, l + ms, BLOCK_M);
-  ok = ok && make_map(&c->map_ws1, c->ws1, ms, d, d, BLOCK_M);
-  ok = ok && make_map(&c->map_w1, c->w1, (uint64_t)N * m, l, l, BLOCK_M);
-  ok = ok && make_map(&c->map_w2, c->w2, (uint64_t)N * l, m, m, BLOCK_M);
+  if (!c->nvfp4) {
+    ok = ok && make_map(&c->map_ws1, c->ws1, ms, d, d, BLOCK_M);
+    ok = ok && make_map(&c->map_w1, c->w1, (uint64_t)N * m, l, l, BLOCK_M);
+    ok = ok && make_map(&c->map_w2, c->w2, (uint64_t)N * l, m, m, BLOCK_M);
+  }
   if (!ok) return LMOE_ERR_CUDA;
   c->loaded = true;
   return LMOE_OK;
@@ -471,6 +758,14 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   int launches = 0;
   chk(cudaMemsetAsync(c->work_counters, 0, lmoe_ctx::kCounters * sizeof(int), s));
   mark(0);
+  if (c->nvfp4) {
+    const cudaError_t r = forward_nvfp4(c, x, T, y, idx, gate, s, mark, launches);
+    chk(r);
+    c->launches = launches;
+    if (prof) ++c->prof_n;
+    c->last_T = T;
+    return cuda_status(e);
+  }
 
   // At decode sizes (T <= 512 with decode-sized expert groups) the shared expert's two matrices ride
   // inside the expert launches as dense pre problems, and the output GEMM only does W_up z + y_s.
@@ -612,6 +907,47 @@ lmoe_status lmoe_forward_host(lmoe_handle c, const void* x_host, int32_t T, void
   return LMOE_OK;
 }
 
+lmoe_status lmoe_export_nvfp4(lmoe_handle c, int32_t which, int32_t index, uint8_t* codes_host, uint8_t* scales_host,
+                              float* gscale_host) {
+  if (!c || !codes_host || !scales_host || !gscale_host) return LMOE_ERR_INVALID_ARG;
+  if (!c->nvfp4) return LMOE_ERR_UNSUPPORTED;
+  if (!c->loaded) return LMOE_ERR_NOT_LOADED;
+  const lmoe_config& g = c->cfg;
+  const int N = g.n_experts, d = g.d, l = g.latent, m = g.expert_ffn, ms = g.shared_ffn;
+  const uint8_t* codes = nullptr;
+  const uint8_t* atoms = nullptr;
+  long long row0 = 0, rows = 0;
+  int K = 0, gi = 0;
+  switch (which) {
+    case 0:
+      if (index < 0 || index >= N) return LMOE_ERR_SHAPE;
+      codes = c->w1q, atoms = c->w1_sf, row0 = (long long)index * m, rows = m, K = l, gi = index;
+      break;
+    case 1:
+      if (index < 0 || index >= N) return LMOE_ERR_SHAPE;
+      codes = c->w2q, atoms = c->w2_sf, row0 = (long long)index * l, rows = l, K = m, gi = N + index;
+      break;
+    case 2: codes = c->ws1q, atoms = c->ws1_sf, rows = ms, K = d, gi = 2 * N; break;
+    case 3: codes = c->ws2q, atoms = c->ws2_sf, rows = d, K = ms, gi = 2 * N + 1; break;
+    default: return LMOE_ERR_SHAPE;
+  }
+  DeviceGuard dg(c->device);
+  if (cudaDeviceSynchronize() != cudaSuccess) return LMOE_ERR_CUDA;
+  if (cudaMemcpy(codes_host, codes + row0 * (K / 2), (size_t)rows * (K / 2), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LMOE_ERR_CUDA;
+  if (cudaMemcpy(gscale_host, c->wg + gi, sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess) return LMOE_ERR_CUDA;
+  // the matrix's scale atoms are contiguous (its rows start on a 128-row tile)
+  const int atoms_k = sf_atoms_k(K);
+  const size_t atom_bytes = (size_t)(rows / 128) * atoms_k * SF_ATOM_BYTES;
+  std::vector<uint8_t> tmp(atom_bytes);
+  if (cudaMemcpy(tmp.data(), atoms + (row0 / 128) * atoms_k * SF_ATOM_BYTES, atom_bytes, cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return LMOE_ERR_CUDA;
+  for (long long r = 0; r < rows; ++r)
+    for (int kb = 0; kb < K / 16; ++kb) scales_host[r * (K / 16) + kb] = tmp[sf_atom_offset(r, kb, atoms_k)];
+  return LMOE_OK;
+}
+
 lmoe_status lmoe_get_device_status(lmoe_handle c) {
   if (!c) return LMOE_ERR_INVALID_ARG;
   DeviceGuard dg(c->device);
@@ -626,6 +962,7 @@ lmoe_status lmoe_get_device_status(lmoe_handle c) {
 
 lmoe_status lmoe_inspect(lmoe_handle c, int32_t which, void** dev_ptr, int64_t* count) {
   if (!c || !dev_ptr || !count) return LMOE_ERR_INVALID_ARG;
+  if (which >= LMOE_BUF_XQ && !c->nvfp4 && which != LMOE_BUF_Y_S) return LMOE_ERR_UNSUPPORTED;
   const lmoe_config& g = c->cfg;
   const long long T = c->last_T, TK = T * g.top_k;
   switch (which) {
@@ -637,6 +974,16 @@ lmoe_status lmoe_inspect(lmoe_handle c, int32_t which, void** dev_ptr, int64_t* 
     case LMOE_BUF_H: *dev_ptr = c->h; *count = T * g.latent; break;
     case LMOE_BUF_Z: *dev_ptr = c->zu; *count = T * (g.latent + g.shared_ffn); break;
     case LMOE_BUF_U: *dev_ptr = c->u; *count = TK * g.expert_ffn; break;
+    case LMOE_BUF_XQ: *dev_ptr = c->xq; *count = T * g.d / 2; break;
+    case LMOE_BUF_X_SF: *dev_ptr = c->x_sf; *count = T * act_sf_pitch(g.d); break;
+    case LMOE_BUF_HQ: *dev_ptr = c->hq; *count = TK * g.latent / 2; break;
+    case LMOE_BUF_H_SF: *dev_ptr = c->h_sf; *count = TK * act_sf_pitch(g.latent); break;
+    case LMOE_BUF_UQ: *dev_ptr = c->uq; *count = TK * g.expert_ffn / 2; break;
+    case LMOE_BUF_U_SF: *dev_ptr = c->u_sf; *count = TK * act_sf_pitch(g.expert_ffn); break;
+    case LMOE_BUF_USQ: *dev_ptr = c->usq; *count = T * g.shared_ffn / 2; break;
+    case LMOE_BUF_US_SF: *dev_ptr = c->us_sf; *count = T * act_sf_pitch(g.shared_ffn); break;
+    case LMOE_BUF_Y_S: *dev_ptr = c->y_s; *count = T * g.d; break;
+    case LMOE_BUF_ACT_SCALE: *dev_ptr = c->act_g; *count = 2; break;
     default: return LMOE_ERR_INVALID_ARG;
   }
   return LMOE_OK;

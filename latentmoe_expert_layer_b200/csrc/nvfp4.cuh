@@ -1,0 +1,212 @@
+// NVFP4 quantisation: E2M1 elements in 16-element blocks along the reduction dimension, one E4M3
+// scale per block, one fp32 scale per tensor.  The pages name the two-level scheme (a per-tensor
+// global scale and per-block fine scales: "Nemotron 3 Super" notes, section 3.6; E2M1 data with E4M3
+// block scales: "Nemotron 3 Ultra" summary) but fix neither block size nor rounding.  This library
+// uses 16-element blocks and round-to-nearest-even with saturation, every decision in fp32:
+//
+//   g   = amax(tensor) / 2688            (2688 = 6 * 448; an all-zero tensor gets g = 1)
+//   s   = E4M3_rne_sat( amax(block) / (6 g) )
+//   q_i = E2M1_rne_sat( v_i / (s g) )     (s decoded to fp32 first; s == 0 gives q_i = sign only)
+//
+// Layouts
+//   codes   row-major [rows, K/2] bytes, element 2i in the low nibble, 2i+1 in the high nibble
+//   weight scales: 512-byte atoms, one per (128 rows, 64 K) tile; inside an atom the scale of row r
+//           (0..127) and K-block s (0..3) sits at byte (r % 32) * 16 + (r / 32) * 4 + s, which is the
+//           layout tcgen05.cp (32x128b, replicated to the 4 lane quadrants) turns into the TMEM scale
+//           columns the block-scaled MMA reads.  Atoms are ordered [row tile][K atom], K atoms padded
+//           to a multiple of 4 (one 256-element pipeline stage) with zero scales.
+//   activation scales: row-major [rows, pitch] bytes, pitch = 16 * ceil(K / 256), zero padded.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include "ptx.cuh"
+
+namespace lmoe {
+
+constexpr float NVFP4_TENSOR_DIV = 2688.0f;  // E2M1 max (6) times E4M3 max (448)
+constexpr int NVFP4_STAGE_K = 256;           // FP4 elements per 128-byte smem row
+
+// E2M1 code of r: magnitude rounded to {0, .5, 1, 1.5, 2, 3, 4, 6} (nearest, ties to the even
+// code, saturating at 6); bit 3 carries the sign of r.
+__device__ __forceinline__ uint32_t e2m1_code(float r) {
+  const float a = fabsf(r);
+  uint32_t c;
+  if (a <= 0.25f) c = 0u;
+  else if (a < 0.75f) c = 1u;
+  else if (a <= 1.25f) c = 2u;
+  else if (a < 1.75f) c = 3u;
+  else if (a <= 2.5f) c = 4u;
+  else if (a < 3.5f) c = 5u;
+  else if (a <= 5.0f) c = 6u;
+  else c = 7u;
+  return c | ((__float_as_uint(r) >> 28) & 8u);
+}
+
+__device__ __forceinline__ uint32_t e4m3_rne_sat(float s) {
+  return (uint32_t)__nv_cvt_float_to_fp8(s, __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+  const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)b, __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+__device__ __forceinline__ float tensor_scale_from_amax(float amax) {
+  return amax > 0.f ? __fdiv_rn(amax, NVFP4_TENSOR_DIV) : 1.0f;
+}
+
+// Quantise one 16-element block with tensor scale g.  Returns the E4M3 scale byte; writes the 8
+// packed code bytes (element 2i low nibble) into codes[0..1] (two 32-bit words).
+__device__ __forceinline__ uint32_t nvfp4_block(const float (&v)[16], float g, uint32_t (&codes)[2]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const float den6 = __fmul_rn(6.0f, g);
+  const uint32_t sb = e4m3_rne_sat(__fdiv_rn(amax, den6));
+  const float den = __fmul_rn(e4m3_to_f32(sb), g);
+  codes[0] = codes[1] = 0u;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t c = den > 0.f ? e2m1_code(__fdiv_rn(v[i], den)) : ((__float_as_uint(v[i]) >> 28) & 8u);
+    codes[i >> 3] |= c << (4 * (i & 7));
+  }
+  return sb;
+}
+
+// Byte offset of the scale of (row r, 16-element block kb) inside a weight-scale atom array with
+// `atoms_k` K atoms per 128-row tile.
+__host__ __device__ __forceinline__ long long sf_atom_offset(long long r, int kb, int atoms_k) {
+  return ((r >> 7) * atoms_k + (kb >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (kb & 3);
+}
+
+__host__ __device__ __forceinline__ int sf_atoms_k(int K) { return ((K + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K) * 4; }
+__host__ __device__ __forceinline__ int act_sf_pitch(int K) { return ((K + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K) * 16; }
+
+// ------------------------------------------------------------------------------------------------
+// amax of contiguous groups (one weight matrix each): amax_bits[blockIdx.y] = max |w| over the
+// group's group_elems bf16 values (fp32 bits; non-negative floats order like unsigned ints).
+// ------------------------------------------------------------------------------------------------
+__global__ void amax_groups_kernel(const __nv_bfloat16* __restrict__ w, long long group_elems,
+                                   unsigned* __restrict__ amax_bits) {
+  const uint4* base = reinterpret_cast<const uint4*>(w + (long long)blockIdx.y * group_elems);
+  const long long n8 = group_elems / 8;
+  float m = 0.f;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    const uint4 q = base[i];
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(p[j]);
+      m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0 && m > 0.f) atomicMax(&amax_bits[blockIdx.y], __float_as_uint(m));
+}
+
+// ------------------------------------------------------------------------------------------------
+// Weight quantiser: one thread per 16-element block.  Writes codes [rows, K/2], scales into atoms,
+// and (thread 0 of each group) the group's fp32 tensor scale.
+// ------------------------------------------------------------------------------------------------
+__global__ void quant_weight_kernel(const __nv_bfloat16* __restrict__ w, long long rows, int K, long long rows_per_group,
+                                   const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes,
+                                   uint8_t* __restrict__ sf_atoms, float* __restrict__ g_out) {
+  const int nb = K / 16;
+  const long long total = rows * nb;
+  const int atoms_k = sf_atoms_k(K);
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / nb;
+    const int kb = (int)(i - r * nb);
+    const long long grp = r / rows_per_group;
+    const float g = tensor_scale_from_amax(__uint_as_float(amax_bits[grp]));
+    const uint4* src = reinterpret_cast<const uint4*>(w + r * K + kb * 16);
+    float v[16];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint4 q = src[h];
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(p[j]);
+        v[h * 8 + 2 * j] = f.x;
+        v[h * 8 + 2 * j + 1] = f.y;
+      }
+    }
+    uint32_t c[2];
+    const uint32_t sb = nvfp4_block(v, g, c);
+    *reinterpret_cast<uint2*>(codes + r * (K / 2) + kb * 8) = make_uint2(c[0], c[1]);
+    sf_atoms[sf_atom_offset(r, kb, atoms_k)] = (uint8_t)sb;
+    if (kb == 0 && r % rows_per_group == 0) g_out[grp] = g;
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Activation amax: amax_bits[0] = max |a| over a bf16 [rows, K] tensor.
+// ------------------------------------------------------------------------------------------------
+__global__ void amax_act_kernel(const __nv_bfloat16* __restrict__ a, long long n_vec8, unsigned* __restrict__ amax_bits) {
+  float m = 0.f;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec8;
+       i += (long long)gridDim.x * blockDim.x) {
+    const uint4 q = reinterpret_cast<const uint4*>(a)[i];
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(p[j]);
+      m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0 && m > 0.f) atomicMax(amax_bits, __float_as_uint(m));
+}
+
+// ------------------------------------------------------------------------------------------------
+// Activation quantiser with optional row gather: dst row r takes source row (src_rows ? src_rows[r]
+// : r).  One thread per 16-element block; tensor scale from amax_bits[0].  Also writes g to *g_out.
+// ------------------------------------------------------------------------------------------------
+__global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, const int* __restrict__ src_rows,
+                                 long long n_rows, int n_src_rows, const unsigned* __restrict__ amax_bits,
+                                 uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ g_out,
+                                 unsigned* status) {
+  const int nb = K / 16;
+  const int pitch = act_sf_pitch(K);
+  const float g = tensor_scale_from_amax(__uint_as_float(amax_bits[0]));
+  if (blockIdx.x == 0 && threadIdx.x == 0 && g_out) *g_out = g;
+  const long long total = n_rows * nb;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / nb;
+    const int kb = (int)(i - r * nb);
+    long long sr = r;
+    if (src_rows) {
+      sr = src_rows[r];
+      if (sr < 0 || sr >= n_src_rows) {
+        atomicOr(status, DEV_STATUS_BAD_INDEX);
+        continue;
+      }
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(a + sr * K + kb * 16);
+    float v[16];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint4 q = src[h];
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(p[j]);
+        v[h * 8 + 2 * j] = f.x;
+        v[h * 8 + 2 * j + 1] = f.y;
+      }
+    }
+    uint32_t c[2];
+    const uint32_t sb = nvfp4_block(v, g, c);
+    *reinterpret_cast<uint2*>(codes + r * (K / 2) + kb * 8) = make_uint2(c[0], c[1]);
+    sf[r * pitch + kb] = (uint8_t)sb;
+  }
+}
+
+}  // namespace lmoe

@@ -146,6 +146,59 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D[tmem] (+)= (A * SFA) * (B * SFB)^T, kind::mxf4nvf4 with 16-element blocks: A and B are packed
+// E2M1 in shared memory, the E4M3 block scales SFA / SFB are in TMEM (see tcgen05_cp_32x128b_x4).
+__device__ __forceinline__ void umma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copy a 32-row x 128-bit shared-memory block (rows 16 bytes apart) into 4 consecutive TMEM columns
+// of lanes 0..31, replicated into the other three lane quadrants.
+__device__ __forceinline__ void tcgen05_cp_32x128b_x4(uint32_t dst_tmem, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(dst_tmem), "l"(src_desc) : "memory");
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte block without swizzle (8-row core matrices of 128
+// contiguous bytes, 128 bytes apart).  Used as the tcgen05.cp source of one scale atom.
+__device__ __forceinline__ uint64_t smem_desc_sf_atom(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;   // leading byte offset (one core matrix wide: unused)
+  d |= static_cast<uint64_t>(128u >> 4) << 32;   // stride byte offset: next 8 rows
+  d |= static_cast<uint64_t>(1) << 46;           // descriptor version (sm_100)
+  return d;                                      // swizzle mode 0: none
+}
+
+// Instruction descriptor, kind::mxf4nvf4: E2M1 A and B (K-major), UE4M3 scales, M x N, K = 64.
+__host__ __device__ constexpr uint32_t idesc_nvf4(uint32_t m, uint32_t n) {
+  return (1u << 7)            // A format: E2M1
+         | (1u << 10)         // B format: E2M1
+         | ((n >> 3) << 17)   // N / 8
+         | ((m >> 4) << 24);  // M / 16   (bit 23 = 0: E4M3 scales; bit 31 = 0: K = 64)
+}
+
+// Bulk copy (no tensor map) of `bytes` (multiple of 16, 16-byte aligned) into shared memory.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Order this thread's generic-proxy shared-memory writes before later async-proxy reads
+// (TMA, tcgen05.cp, tcgen05.mma) of the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Arrive (once) on an mbarrier when every previously issued tcgen05.mma of this thread completes.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(

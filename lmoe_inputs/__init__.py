@@ -81,6 +81,12 @@ WORKLOADS: Dict[str, Workload] = {
     # 128-expert layer, so that a full-metric profiler capture holds ~1.5 GB on the device
     "decode_small": Workload("decode_small", dataclasses.replace(SUPER, n_experts=128), 64, 1, 2, "bf16", "bf16",
                              description="Super dims with 128 experts, T=64 (~11 tokens per expert)"),
+    # small NVFP4 layers: several 128-row tiles, a ragged 256-element K stage (m = 384), both the
+    # decode-sized (~10 tokens per expert) and the prefill-sized (~256 per expert) GEMM shapes
+    "nvfp4_tiny": Workload("nvfp4_tiny", LayerShape(512, 256, 16, 4, 384, 512), 40, 7, 8, "bf16", "nvfp4",
+                           description="NVFP4 layer d=512 l=256 N=16 K=4 m=384 m_s=512, T=40"),
+    "nvfp4_mid": Workload("nvfp4_mid", LayerShape(512, 256, 16, 4, 384, 512), 1024, 7, 9, "bf16", "nvfp4",
+                          description="NVFP4 layer d=512 l=256 N=16 K=4 m=384 m_s=512, T=1024"),
     "skewed": Workload("skewed", SUPER, 4096, 1, 4, "bf16", "bf16", router_bias=True,
                        description="Super shape T=4096, per-expert router bias giving a capped Zipf(1.2) load"),
 }

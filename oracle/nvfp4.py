@@ -31,7 +31,7 @@ from . import lmoe_oracle as lo
 
 __all__ = [
     "E2M1_VALUES", "e2m1_encode", "e2m1_decode", "e4m3_encode", "e4m3_decode", "tensor_scale",
-    "quantize", "dequantize", "qdq", "forward_nvfp4",
+    "quantize", "dequantize", "qdq", "bf16_round", "forward_nvfp4",
 ]
 
 E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
@@ -137,6 +137,14 @@ def dequantize(codes: np.ndarray, scales: np.ndarray, g) -> np.ndarray:
     return (v * s * float(g)).reshape(rows, cols)
 
 
+def bf16_round(a: np.ndarray) -> np.ndarray:
+    """Round to the nearest bfloat16 (ties to even), via float32; returns float64 values."""
+    f = np.ascontiguousarray(np.asarray(a, dtype=np.float64).astype(np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16 << 16
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
 def qdq(a: np.ndarray, g: Optional[np.float32] = None) -> np.ndarray:
     """Quantise then dequantise (float64 result)."""
     c, s, gg = quantize(a, g)
@@ -148,13 +156,16 @@ def forward_nvfp4(w: "lo.OracleWeights", x: np.ndarray, k: int, idx: Optional[np
     """Layer forward with NVFP4 routed and shared experts (weights and activations); router,
     W_down and W_up stay at the device's bf16 values.
 
+    W_down is a BF16 layer in this variant, so the latent h it produces is a BF16 tensor: h is
+    rounded to bf16 (nearest even) before it is quantised for the experts.
+
     g_x / g_h: per-call activation scales.  They depend on the whole call's x / h, so a caller that
     evaluates a sample of tokens passes the full batch's values."""
     logits = lo.router_logits(x, w.w_router, w.b_router)
     if idx is None:
         idx = lo.topk(logits, k)
     gate = lo.softmax_gates(logits, idx)
-    h = x @ w.w_down.T
+    h = bf16_round(x @ w.w_down.T)
     if g_x is None:
         g_x = tensor_scale(x.astype(np.float32))
     if g_h is None:

@@ -12,7 +12,7 @@ HEADER = os.path.join(ROOT, "include", "lmoe.h")
 def _declared():
     txt = open(HEADER).read()
     txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
-    return sorted(set(re.findall(r"\b(lmoe_[a-z_]+)\s*\(", txt)))
+    return sorted(set(re.findall(r"\b(lmoe_[a-z0-9_]+)\s*\(", txt)))
 
 
 @pytest.fixture(scope="module")
@@ -26,14 +26,15 @@ def libmod():
 def test_header_declares_the_boundary():
     assert _declared() == sorted(["lmoe_create", "lmoe_load_weights", "lmoe_forward", "lmoe_forward_host",
                                   "lmoe_get_device_status", "lmoe_inspect", "lmoe_profile",
-                                  "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_status_string",
+                                  "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_export_nvfp4",
+                                  "lmoe_status_string",
                                   "lmoe_destroy"])
 
 
 def test_library_exports_every_declared_symbol(libmod):
     out = subprocess.run(["nm", "-D", "--defined-only", libmod.library_path], capture_output=True, text=True,
                          check=True).stdout
-    exported = set(re.findall(r"\bT (lmoe_[a-z_]+)\b", out))
+    exported = set(re.findall(r"\bT (lmoe_[a-z0-9_]+)\b", out))
     missing = set(_declared()) - exported
     assert not missing, missing
     assert set(libmod.SYMBOLS) == set(_declared())

@@ -367,6 +367,14 @@ def test_rne_ties_and_saturation():
     assert sb2[0, 0] == 0x38 and nv.e2m1_decode(c2)[0, :2].tolist() == [6.0, -3.0]
 
 
+def test_oracle_bf16_round_against_ml_dtypes():
+    ml = pytest.importorskip("ml_dtypes")
+    r = np.concatenate([np.random.default_rng(24).standard_normal(20000) * 7,
+                        [1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 0.0, 1e-30]])
+    ref = r.astype(np.float32).astype(ml.bfloat16).astype(np.float64)
+    assert np.array_equal(nv.bf16_round(r), ref)
+
+
 def test_zero_block_and_zero_tensor():
     v = np.zeros((2, 32), np.float32)
     v[1, 16:] = np.linspace(-1, 1, 16)
