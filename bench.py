@@ -34,7 +34,8 @@ import lmoe_inputs as inp  # noqa: E402
 METRIC = "LatentMoE layer tokens/s (Super shape, T=256 & 16K); % of HBM / TC roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DEFAULT_STEPS = {"tiny": 200, "decode": 400, "skewed": 40, "prefill": 20}
-DEFAULT_STEPS["decode_small"] = 400
+DEFAULT_STEPS.update({"decode_small": 400, "decode_nvfp4": 400, "prefill_nvfp4": 20, "nvfp4_tiny": 200,
+                      "nvfp4_mid": 100})
 
 
 def peaks():
@@ -99,19 +100,24 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------------------ helpers
 def algorithmic_work(wl, counts: np.ndarray):
-    """Bytes and FLOPs one forward must move / compute, from the actual routing (counts per expert)."""
+    """Bytes and FLOPs one forward must move / compute, from the actual routing (counts per expert).
+
+    bf16 weights: 2 bytes per element.  NVFP4 weights and activations: 0.5 byte per element plus one
+    E4M3 scale byte per 16 elements (router, W_down and W_up stay bf16 in the NVFP4 variant)."""
     s = wl.shape
     d, l, n, k, m, ms = s.d, s.latent, s.n_experts, s.top_k, s.expert_ffn, s.shared_ffn
     t = wl.tokens
     tk = t * k
     touched = int((counts > 0).sum())
-    w_exp = touched * m * l * 2                                  # bf16 bytes of one expert matrix set (W1 or W2)
-    up = {"bytes": w_exp + tk * l * 2 + tk * m * 2, "flops": 2 * tk * m * l}
-    down = {"bytes": w_exp + tk * m * 2 + tk * l * 2 + tk * 4, "flops": 2 * tk * m * l}
-    layer_bytes = (2 * w_exp + (n + l) * d * 2 + ms * d * 2 + d * (l + ms) * 2 + 2 * t * d * 2 + tk * 8)
+    fp4 = wl.precision == "nvfp4"
+    eb = (lambda elems: elems * 0.5 + elems / 16) if fp4 else (lambda elems: elems * 2)
+    w_exp = touched * eb(m * l)                     # one expert matrix set (W1 or W2) of the touched experts
+    up = {"bytes": w_exp + eb(tk * l) + eb(tk * m), "flops": 2 * tk * m * l}
+    down = {"bytes": w_exp + eb(tk * m) + tk * l * 2 + tk * 4, "flops": 2 * tk * m * l}
+    layer_bytes = (2 * w_exp + (n + l) * d * 2 + eb(ms * d) + eb(d * ms) + d * l * 2 + 2 * t * d * 2 + tk * 8)
     layer_flops = 2 * t * ((n + l) * d + ms * d + d * (l + ms)) + 4 * tk * m * l
-    return {"expert_up": up, "expert_down": down, "layer": {"bytes": layer_bytes, "flops": layer_flops},
-            "touched_experts": touched}
+    return {"expert_up": up, "expert_down": down, "layer": {"bytes": int(layer_bytes), "flops": layer_flops},
+            "touched_experts": touched, "expert_weight_bytes": int(2 * w_exp)}
 
 
 def make_device_layer(wl, device):
@@ -132,6 +138,12 @@ def make_device_layer(wl, device):
     return layer, w
 
 
+def _oracle_forward(wl):
+    from oracle import lmoe_oracle as lo
+    from oracle import nvfp4 as nv
+    return nv.forward_nvfp4 if wl.precision == "nvfp4" else lo.forward
+
+
 def cpu_baseline(wl, w, budget_s: float = 20.0):
     """The fp64 oracle, as it stands, on a bounded token sample of the same workload."""
     from oracle import lmoe_oracle as lo
@@ -142,10 +154,11 @@ def cpu_baseline(wl, w, budget_s: float = 20.0):
         cores = os.cpu_count()
     ow = lo.OracleWeights(w)
     x = lo.lift(inp.make_x(wl), "bf16")
+    fwd = _oracle_forward(wl)
     done, t0, sample = 0, time.perf_counter(), 0
     while time.perf_counter() - t0 < budget_s and done < wl.tokens:
         n = min(4, wl.tokens - done)
-        lo.forward(ow, x[done:done + n], wl.shape.top_k)
+        fwd(ow, x[done:done + n], wl.shape.top_k)
         done += n
     el = time.perf_counter() - t0
     return {"value": done / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -168,9 +181,11 @@ def run_reference(args, wl, rank):
     per_step = 1 if wl.shape.n_experts > 64 else wl.tokens   # bounded sample per step
     pos = 0
 
+    fwd = _oracle_forward(wl)
+
     def step():
         nonlocal pos
-        lo.forward(ow, x[pos:pos + per_step], wl.shape.top_k)
+        fwd(ow, x[pos:pos + per_step], wl.shape.top_k)
         pos = (pos + per_step) % max(1, wl.tokens - per_step + 1)
 
     for _ in range(args.warmup):
@@ -285,15 +300,19 @@ def run_ours(args, wl, rank, world):
         else:
             ach = unit_work["flops"] / (per_launch_ms * 1e-3) / 1e12
             p = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+            src = pk_kind + " bf16 (sustained)"
+            if wl.precision == "nvfp4":  # no measured FP4 peak: bf16 measured x the nominal 4x FP4/BF16 ratio
+                p *= 4.0
+                src = pk_kind + " bf16 (sustained) x nominal FP4/BF16 ratio 4"
             roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": p, "unit": "TFLOP/s",
                     "frac": ach / p, "traffic": None, "algorithmic_flops": unit_work["flops"],
-                    "launch_ms": per_launch_ms, "peak_source": pk_kind + " (sustained)"}
+                    "launch_ms": per_launch_ms, "peak_source": src}
     step_ms = ms_max / args.steps
     lay = work["layer"]
     layer_roof = {"bytes_per_step": lay["bytes"], "flops_per_step": lay["flops"],
                   "hbm_frac": lay["bytes"] / (step_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
-                  "tc_frac": lay["flops"] / (step_ms * 1e-3) / 1e12 / pk.get("bf16_tflops_sustained",
-                                                                               pk["bf16_tflops"])}
+                  "tc_frac_of_bf16_peak": lay["flops"] / (step_ms * 1e-3) / 1e12 /
+                  pk.get("bf16_tflops_sustained", pk["bf16_tflops"])}
     line = {
         "metric": METRIC,
         "value": world * t * args.steps / (ms_max * 1e-3),
@@ -305,14 +324,15 @@ def run_ours(args, wl, rank, world):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic: seeded N(0,1/fan_in) weights, N(0,1) x, bf16",
+        "dtype": "nvfp4+bf16" if wl.precision == "nvfp4" else "bf16",
+        "data": "synthetic: seeded N(0,1/fan_in) weights, N(0,1) x, bf16" +
+                (" (experts and shared expert quantised to NVFP4 on the device)" if wl.precision == "nvfp4" else ""),
         "config": {"workload": wl.name, "tokens": t, "d": wl.shape.d, "latent": wl.shape.latent,
                    "experts": wl.shape.n_experts, "top_k": wl.shape.top_k, "expert_ffn": wl.shape.expert_ffn,
                    "shared_ffn": wl.shape.shared_ffn, "precision": wl.precision,
                    "parallelism": f"{world} independent replica(s)",
                    "l2": "inputs larger than L2: every step streams all touched expert weights "
-                         f"({work['touched_experts']} experts, {2 * work['touched_experts'] * wl.shape.expert_ffn * wl.shape.latent * 2 / 1e9:.2f} GB)"},
+                         f"({work['touched_experts']} experts, {work['expert_weight_bytes'] / 1e9:.2f} GB)"},
         "roofline": roof,
         "layer_roofline": layer_roof,
         "stages_ms_per_step": {k: v / max(1, recorded) for k, v in stage_ms.items()},

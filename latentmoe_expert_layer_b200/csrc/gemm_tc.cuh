@@ -49,9 +49,10 @@ enum EpiKind : int {
 // One unit of GEMM work.  a_row: first W row of the tile; b_row: first activation row (also the
 // output row); f0: first output feature (column) of the tile; nm = n_valid | (m_valid << 16) with
 // n_valid tokens (1..BN_MAX) and m_valid features (1..128, a multiple of 16; a multiple of 32 for
-// EPI_SQRELU_NVFP4).
+// EPI_SQRELU_NVFP4); tile: token-tile id (NVFP4 activation scales are stored per token tile).
 struct GemmUnit {
   int a_row, b_row, f0, nm;
+  int tile, pad0, pad1, pad2;
 };
 
 // One GEMM problem of a launch: K extent, epilogue, NVFP4 scales, and (for dense problems) the grid.
@@ -67,17 +68,16 @@ struct GemmProblem {
   const float* row_scale;     // EPI_ROWSCALE_BF16
   const float* addend;        // EPI_ADD_BF16
   long long ld_add;
-  uint8_t* out_sf;            // EPI_SQRELU_NVFP4 scales [rows, out_sf_pitch]
-  int out_sf_pitch;
+  uint8_t* out_sf;            // EPI_SQRELU_NVFP4 scales, tile-local atoms (act_sf_offset)
+  int out_sf_stages;          // 256-element stages of the output's K
   int weights_streamed;       // 1: every weight tile is read by one unit only (L2 evict-first)
   // NVFP4 operands
   const uint8_t* w_sf;        // weight scale atoms
   int w_atoms_k;              // K atoms per 128-row tile
   const float* w_gscale;      // per-group weight tensor scale, group = a_row / w_rows_per_g
   int w_rows_per_g;
-  const uint8_t* act_sf;      // activation scales, row-major [act_rows, act_sf_pitch]
-  int act_sf_pitch;
-  long long act_rows;
+  const uint8_t* act_sf;      // activation scales, tile-local atoms (act_sf_offset)
+  int act_sf_stages;          // 256-element stages of the activations' K
   const float* act_gscale;    // activation tensor scale (device scalar)
   // dense enumeration
   int dense_ftiles;           // feature tiles
@@ -117,16 +117,19 @@ struct GemmSmem {
   static constexpr int BAR_OFF = EPI_OFF + 4 * EPI_STAGE_BYTES;
   static constexpr int BYTES = BAR_OFF + 512;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment of the base
-  // TMEM: two fp32 accumulators of BN_MAX columns, then (FP4) the scale columns of one stage:
-  // SFA 4 MMAs x 4 columns, SFB 4 MMAs x NRA x 4 columns
+  // TMEM: two fp32 accumulators of BN_MAX columns, then (FP4) SF_SLOTS rotating slots of scale
+  // columns, one stage each (SFA 4 MMAs x 4 columns, SFB 4 MMAs x NRA x 4 columns).  Every MMA's scale
+  // address is 4-column aligned (the block-scaled MMA faults on a misaligned scale address).
   static constexpr int SF_COL0 = 2 * BN_MAX;
   static constexpr int SF_COLS = FP4 ? 16 + 16 * NRA : 0;
-  static constexpr uint32_t TMEM_COLS = (SF_COL0 + SF_COLS <= 32)    ? 32
-                                        : (SF_COL0 + SF_COLS <= 64)  ? 64
-                                        : (SF_COL0 + SF_COLS <= 128) ? 128
-                                        : (SF_COL0 + SF_COLS <= 256) ? 256
-                                                                     : 512;
-  static_assert(SF_COL0 + SF_COLS <= 512, "TMEM holds 512 columns");
+  static constexpr int SF_SLOTS = !FP4 ? 1 : ((512 - SF_COL0) / SF_COLS >= 4 ? 4 : (512 - SF_COL0) / SF_COLS);
+  static constexpr int TMEM_NEED = SF_COL0 + SF_SLOTS * SF_COLS;
+  static constexpr uint32_t TMEM_COLS = (TMEM_NEED <= 32)    ? 32
+                                        : (TMEM_NEED <= 64)  ? 64
+                                        : (TMEM_NEED <= 128) ? 128
+                                        : (TMEM_NEED <= 256) ? 256
+                                                             : 512;
+  static_assert(TMEM_NEED <= 512 && SF_SLOTS >= 1, "TMEM holds 512 columns");
   static_assert(ALLOC <= 232448, "shared memory per CTA");
 };
 
@@ -142,6 +145,7 @@ __device__ __forceinline__ GemmUnit dense_unit(const GemmProblem& p, int u) {
   const int mv = min(BLOCK_M, p.dense_feat - r.f0);
   const int nv = min(BN_MAX, p.dense_tokens - r.b_row);
   r.nm = nv | (mv << 16);
+  r.tile = tt;
   return r;
 }
 
@@ -190,7 +194,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], FP4 ? 33 : 1);  // FP4: the TMA lane's expect_tx + the 32 scale-staging lanes
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -225,8 +229,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const uint64_t tmo = args.timeout_ns;
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ producer (whole warp for FP4)
-    if (FP4 || lane == 0) {
+    // ------------------------------------------------------------------ producer (one lane)
+    if (lane == 0) {
       const uint64_t pol_first = policy_evict_first();
       const uint64_t pol_normal = policy_evict_normal();
       const uint64_t pol_a = policy_evict_last();
@@ -238,32 +242,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t uphase = 0;
       // dynamic launches claim the next unit one unit ahead, so the atomic's round trip overlaps the
       // loads; static launches take every gridDim.x-th unit
-      int u_next = 0;
-      if (lane == 0) u_next = args.dynamic ? atomicAdd(args.work_counter, 1) : (int)blockIdx.x;
-      // Only lane 0 waits on barriers; for FP4 the other lanes follow its decisions by shuffle.
-      auto wait0 = [&](uint64_t* bar, uint32_t par) -> bool {
-        bool w = true;
-        if (lane == 0) w = mbar_wait_bounded(bar, par, abort_flag, tmo);
-        if (FP4) w = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
-        return w;
-      };
+      int u_next = args.dynamic ? atomicAdd(args.work_counter, 1) : (int)blockIdx.x;
+      auto wait0 = [&](uint64_t* bar, uint32_t par) -> bool { return mbar_wait_bounded(bar, par, abort_flag, tmo); };
       while (ok) {
         if (!wait0(&uempty[uslot], uphase ^ 1u)) {
           ok = false;
           break;
         }
-        int u = u_next < num_units ? u_next : -1;
-        if (FP4) u = __shfl_sync(0xffffffffu, u, 0);
-        if (lane == 0) {
-          unit_ring[uslot] = u;
-          mbar_arrive(&ufull[uslot]);
-        }
+        const int u = u_next < num_units ? u_next : -1;
+        unit_ring[uslot] = u;
+        mbar_arrive(&ufull[uslot]);
         if (++uslot == UNIT_RING) {
           uslot = 0;
           uphase ^= 1u;
         }
         if (u < 0) break;
-        if (lane == 0) u_next = args.dynamic ? atomicAdd(args.work_counter, 1) : u_next + (int)gridDim.x;
+        u_next = args.dynamic ? atomicAdd(args.work_counter, 1) : u_next + (int)gridDim.x;
         int pid;
         const GemmUnit un = unit_at<BN_MAX>(args, u, pid);
         const GemmProblem& pr = args.prob[pid];
@@ -273,7 +267,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const int nkb = pr.num_k_blocks;
         const int nv = un.nm & 0xFFFF;
         const int nbox = (nv + BOXN - 1) / BOXN;
-        const uint32_t bytes = A_STAGE_BYTES + nbox * BOXN * 128 + S::SFA_STAGE_BYTES;
+        const uint32_t bytes = A_STAGE_BYTES + nbox * BOXN * 128 + S::SFA_STAGE_BYTES + S::SFB_STAGE_BYTES;
         // x coordinate of a stage in the tensor maps: 128 bytes = 64 bf16 elements or 128 FP4 bytes
         const int kx = FP4 ? 128 : BLOCK_K;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -283,33 +277,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
           uint8_t* sa = smem + stage * S::STAGE_BYTES;
           uint8_t* sb = sa + A_STAGE_BYTES;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&full[stage], bytes);
-            tma_load_2d(sa, mw, &full[stage], kb * kx, un.a_row, pol_w);
-            for (int i = 0; i < nbox; ++i)
-              tma_load_2d(sb + i * BOXN * 128, ma, &full[stage], kb * kx, un.b_row + i * BOXN, pol_a);
-          }
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          tma_load_2d(sa, mw, &full[stage], kb * kx, un.a_row, pol_w);
+          for (int i = 0; i < nbox; ++i)
+            tma_load_2d(sb + i * BOXN * 128, ma, &full[stage], kb * kx, un.b_row + i * BOXN, pol_a);
           if constexpr (FP4) {
             uint8_t* ssfa = sb + S::B_STAGE_BYTES;
             uint8_t* ssfb = ssfa + S::SFA_STAGE_BYTES;
-            if (lane == 0)
-              bulk_load(ssfa, pr.w_sf + ((long long)(un.a_row >> 7) * pr.w_atoms_k + kb * 4) * SF_ATOM_BYTES,
-                        S::SFA_STAGE_BYTES, &full[stage]);
-            // activation scales: row j of the token block -> 4 words (one per K atom of this stage)
-            const int n_load = nbox * BOXN;
-            for (int j = lane; j < n_load; j += 32) {
-              const long long row = (long long)un.b_row + j;
-              uint4 w = make_uint4(0u, 0u, 0u, 0u);
-              if (row < pr.act_rows)
-                w = *reinterpret_cast<const uint4*>(pr.act_sf + row * pr.act_sf_pitch + kb * 16);
-              uint8_t* dst = ssfb + (j >> 7) * SF_ATOM_BYTES + (j & 31) * 16 + ((j & 127) >> 5) * 4;
-              *reinterpret_cast<uint32_t*>(dst + 0 * S::NRA * SF_ATOM_BYTES) = w.x;
-              *reinterpret_cast<uint32_t*>(dst + 1 * S::NRA * SF_ATOM_BYTES) = w.y;
-              *reinterpret_cast<uint32_t*>(dst + 2 * S::NRA * SF_ATOM_BYTES) = w.z;
-              *reinterpret_cast<uint32_t*>(dst + 3 * S::NRA * SF_ATOM_BYTES) = w.w;
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&full[stage]);
+            bulk_load(ssfa, pr.w_sf + ((long long)(un.a_row >> 7) * pr.w_atoms_k + kb * 4) * SF_ATOM_BYTES,
+                      S::SFA_STAGE_BYTES, &full[stage]);
+            bulk_load(ssfb, pr.act_sf + ((long long)un.tile * pr.act_sf_stages + kb) * S::SFB_STAGE_BYTES,
+                      S::SFB_STAGE_BYTES, &full[stage]);
           }
           ++issued;
           if (++stage == STAGES) {
@@ -318,7 +296,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
         }
       }
-      if (!ok && lane == 0) {
+      if (!ok) {
         // Give every load still in flight a bounded chance to land before the CTA exits.
         atomicOr(args.status, DEV_STATUS_TIMEOUT);
         volatile int never = 0;
@@ -336,6 +314,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      int sf_slot = 0;
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -380,8 +359,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           if constexpr (FP4) {
             const uint32_t ssfa = sa + A_STAGE_BYTES + S::B_STAGE_BYTES;
             const uint32_t ssfb = ssfa + S::SFA_STAGE_BYTES;
-            const uint32_t t_sfa = tmem_base + S::SF_COL0;
+            const uint32_t t_sfa = tmem_base + S::SF_COL0 + (uint32_t)(sf_slot * S::SF_COLS);
             const uint32_t t_sfb = t_sfa + 16;
+            if (++sf_slot == S::SF_SLOTS) sf_slot = 0;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               tcgen05_cp_32x128b_x4(t_sfa + 4 * k, smem_desc_sf_atom(ssfa + k * SF_ATOM_BYTES));
@@ -504,14 +484,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
               for (int i = 0; i < 16; ++i) v[i] = s32[lane * 32 + ((b * 16 + i) ^ lane)];
               uint32_t cb[2];
-              sbs |= nvfp4_block(v, 1.0f, cb) << (8 * b);
+              sbs |= nvfp4_block_fast(v, 1.0f, cb) << (8 * b);
               cw[2 * b] = cb[0];
               cw[2 * b + 1] = cb[1];
             }
             const long long row = row0 + lane;
             *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(pr.out) + row * pr.ldo + f / 2) =
                 make_uint4(cw[0], cw[1], cw[2], cw[3]);
-            *reinterpret_cast<uint16_t*>(pr.out_sf + row * pr.out_sf_pitch + f / 16) = (uint16_t)sbs;
+            // the two blocks are adjacent bytes of one atom row (f is a multiple of 32)
+            *reinterpret_cast<uint16_t*>(
+                pr.out_sf + act_sf_offset(un.tile, c * 32 + lane, f / 16, pr.out_sf_stages, S::NRA)) =
+                (uint16_t)sbs;
           }
         } else if (f32_out) {
           float* s32 = reinterpret_cast<float*>(stg);

@@ -154,8 +154,28 @@ struct lmoe_ctx {
   uint8_t *xq = nullptr, *x_sf = nullptr, *hq = nullptr, *h_sf = nullptr;  // x [T, d]; h grouped [TK, l]
   uint8_t *uq = nullptr, *u_sf = nullptr, *usq = nullptr, *us_sf = nullptr; // u [TK, m]; u_s [T, m_s]
   float* act_g = nullptr;         // [0] g_x, [1] g_h, [2] 1.0
+  int* tile0 = nullptr;           // [N + 1] first token tile of each expert (NVFP4 scale tiles)
   CUtensorMap map_w1q{}, map_w2q{}, map_ws1q{}, map_ws2q{};
   CUtensorMap map_xq[4]{}, map_hq[4]{}, map_uq[4]{}, map_usq[4]{};  // indexed by variant (FP4 ones)
+
+  // Bytes of tile-local activation scales for K-extent K, large enough for either FP4 variant:
+  // tiles x stages x 4 K atoms x row atoms x 512.  Dense tensors tile T_max tokens; grouped ones have
+  // at most N + T_max*K / tile_tokens tiles.
+  size_t sf_bytes_tiles(long long tiles_small, long long tiles_large, int K) const {
+    const long long st = (K + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K;
+    const long long a = tiles_small * st * 4 * ((V_BN[V_SMALL4] + 127) / 128) * 512;
+    const long long b = tiles_large * st * 4 * ((V_BN[V_LARGE4] + 127) / 128) * 512;
+    return (size_t)(a > b ? a : b);
+  }
+  size_t sf_bytes_dense(int K) const {
+    const long long T = cfg.max_tokens;
+    return sf_bytes_tiles((T + V_BN[V_SMALL4] - 1) / V_BN[V_SMALL4], (T + V_BN[V_LARGE4] - 1) / V_BN[V_LARGE4], K);
+  }
+  size_t sf_bytes_grouped(int K) const {
+    const long long tk = (long long)cfg.max_tokens * cfg.top_k, n = cfg.n_experts;
+    return sf_bytes_tiles(n + (tk + V_BN[V_SMALL4] - 1) / V_BN[V_SMALL4], n + (tk + V_BN[V_LARGE4] - 1) / V_BN[V_LARGE4],
+                          K);
+  }
 
   // stage profiler
   static constexpr int kProfMax = 1024;
@@ -193,7 +213,7 @@ void free_all(lmoe_ctx* c) {
                   c->y_dev,  c->idx_dev, c->gate_dev, c->y_s, c->work_counters,
                   c->w1q,    c->w2q,    c->ws1q,   c->ws2q,      c->w1_sf,      c->w2_sf,      c->ws1_sf,
                   c->ws2_sf, c->wg,     c->w_amax, c->xq,        c->x_sf,       c->hq,         c->h_sf,
-                  c->uq,     c->u_sf,   c->usq,    c->us_sf,     c->act_g};
+                  c->uq,     c->u_sf,   c->usq,    c->us_sf,     c->act_g,      c->tile0};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -239,7 +259,7 @@ GemmProblem problem(int K, int epi, void* out, long long ldo, int col0 = 0) {
 
 // An NVFP4 problem: K in elements; weight scale atoms / tensor scales; activation scales.
 GemmProblem problem4(int K, int epi, void* out, long long ldo, const uint8_t* w_sf, const float* w_g,
-                     int w_rows_per_g, const uint8_t* act_sf, long long act_rows, const float* act_g) {
+                     int w_rows_per_g, const uint8_t* act_sf, const float* act_g) {
   GemmProblem p;
   memset(&p, 0, sizeof(p));
   p.num_k_blocks = (K + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K;
@@ -251,8 +271,7 @@ GemmProblem problem4(int K, int epi, void* out, long long ldo, const uint8_t* w_
   p.w_gscale = w_g;
   p.w_rows_per_g = w_rows_per_g;
   p.act_sf = act_sf;
-  p.act_sf_pitch = act_sf_pitch(K);
-  p.act_rows = act_rows;
+  p.act_sf_stages = p.num_k_blocks;
   p.act_gscale = act_g;
   return p;
 }
@@ -379,8 +398,10 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
   // 2. quantise x (dynamic tensor scale); amax of h
   amax_act_kernel<<<grid_for((long long)T * d / 8, 256), 256, 0, s>>>(
       reinterpret_cast<const __nv_bfloat16*>(x), (long long)T * d / 8, amax_x);
+  const int nra = (V_BN[vg] + 127) / 128;  // scale row atoms per token tile of the FP4 variant
   quant_act_kernel<<<grid_for((long long)T * d / 16, 256), 256, 0, s>>>(
-      reinterpret_cast<const __nv_bfloat16*>(x), d, nullptr, T, T, amax_x, c->xq, c->x_sf, g_x, c->status);
+      reinterpret_cast<const __nv_bfloat16*>(x), d, nullptr, T, T, nullptr, nullptr, N, V_BN[vg], nra, amax_x, c->xq,
+      c->x_sf, g_x, c->status);
   amax_act_kernel<<<grid_for((long long)T * l / 8, 256), 256, 0, s>>>(c->h, (long long)T * l / 8, amax_h);
   chk(cudaGetLastError());
   mark(2);
@@ -393,27 +414,27 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
   UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1};
   UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2};
   scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(c->chunk_counts, nch, N, c->counts, c->offsets,
-                                                              c->chunk_base, l1, l2, c->status);
+                                                              c->chunk_base, l1, l2, c->tile0, c->status);
   chk(cudaGetLastError());
   mark(4);
   // 5. stable grouping; quantise h rows straight into grouped order
   assign_rows_kernel<<<nch, 32, N * sizeof(int), s>>>(idx, gate, c->chunk_base, T, N, K, ct, c->row_of,
                                                      c->tok_of_row, c->gate_of_row, c->status);
-  quant_act_kernel<<<grid_for(TK * l / 16, 256), 256, 0, s>>>(c->h, l, c->tok_of_row, TK, T, amax_h, c->hq, c->h_sf,
-                                                               g_h, c->status);
+  quant_act_kernel<<<grid_for(TK * l / 16, 256), 256, 0, s>>>(c->h, l, c->tok_of_row, TK, T, c->offsets, c->tile0,
+                                                               N, V_BN[vg], nra, amax_h, c->hq, c->h_sf, g_h,
+                                                               c->status);
   chk(cudaGetLastError());
   mark(5);
   // 6. expert up (FP4): u = NVFP4(sqrelu(W1_e h)); shared up u_s = NVFP4(sqrelu(W_s1 x))
-  GemmProblem shared_up =
-      problem4(d, EPI_SQRELU_NVFP4, c->usq, ms / 2, c->ws1_sf, c->wg + 2 * N, ms, c->x_sf, T, g_x);
+  GemmProblem shared_up = problem4(d, EPI_SQRELU_NVFP4, c->usq, ms / 2, c->ws1_sf, c->wg + 2 * N, ms, c->x_sf, g_x);
   shared_up.out_sf = c->us_sf;
-  shared_up.out_sf_pitch = act_sf_pitch(ms);
+  shared_up.out_sf_stages = (ms + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K;
   {
     GemmLaunch gl(c, vg, 4);
     if (split) gl.pre_dense(c->map_ws1q, c->map_xq[vg], shared_up, ms, T);
-    GemmProblem p = problem4(l, EPI_SQRELU_NVFP4, c->uq, m / 2, c->w1_sf, c->wg, m, c->h_sf, TK, g_h);
+    GemmProblem p = problem4(l, EPI_SQRELU_NVFP4, c->uq, m / 2, c->w1_sf, c->wg, m, c->h_sf, g_h);
     p.out_sf = c->u_sf;
-    p.out_sf_pitch = act_sf_pitch(m);
+    p.out_sf_stages = (m + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K;
     gl.main_grouped(c->map_w1q, c->map_hq[vg], p, c->units1, c->num_units);
     chk(gl.run(s));
   }
@@ -424,12 +445,11 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
   }
   mark(6);
   // 7. expert down (FP4) with the gate folded in: o = g * (W2_e u); y_s = W_s2 u_s (fp32)
-  const GemmProblem shared_down =
-      problem4(ms, EPI_F32, c->y_s, d, c->ws2_sf, c->wg + 2 * N + 1, d, c->us_sf, T, one);
+  const GemmProblem shared_down = problem4(ms, EPI_F32, c->y_s, d, c->ws2_sf, c->wg + 2 * N + 1, d, c->us_sf, one);
   {
     GemmLaunch gl(c, vg, 5);
     if (split) gl.pre_dense(c->map_ws2q, c->map_usq[vg], shared_down, d, T);
-    GemmProblem p = problem4(m, EPI_ROWSCALE_BF16, c->o, l, c->w2_sf, c->wg + N, l, c->u_sf, TK, one);
+    GemmProblem p = problem4(m, EPI_ROWSCALE_BF16, c->o, l, c->w2_sf, c->wg + N, l, c->u_sf, one);
     p.row_scale = c->gate_of_row;
     gl.main_grouped(c->map_w2q, c->map_uq[vg], p, c->units2, c->num_units + 1);
     chk(gl.run(s));
@@ -526,11 +546,11 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   // y_s = W_s2 u_s in fp32: needed at decode sizes (bf16) and at every size (NVFP4)
   ok = ok && dalloc(&c->y_s, (size_t)(c->nvfp4 ? T : (T < 512 ? T : 512)) * d);
   if (c->nvfp4) {
-    ok = ok && dalloc(&c->xq, T * d / 2) && dalloc(&c->x_sf, T * act_sf_pitch(d));
-    ok = ok && dalloc(&c->hq, tk * l / 2) && dalloc(&c->h_sf, tk * act_sf_pitch(l));
-    ok = ok && dalloc(&c->uq, tk * m / 2) && dalloc(&c->u_sf, tk * act_sf_pitch(m));
-    ok = ok && dalloc(&c->usq, T * ms / 2) && dalloc(&c->us_sf, T * act_sf_pitch(ms));
-    ok = ok && dalloc(&c->act_g, 4);
+    ok = ok && dalloc(&c->xq, T * d / 2) && dalloc(&c->x_sf, c->sf_bytes_dense(d));
+    ok = ok && dalloc(&c->hq, tk * l / 2) && dalloc(&c->h_sf, c->sf_bytes_grouped(l));
+    ok = ok && dalloc(&c->uq, tk * m / 2) && dalloc(&c->u_sf, c->sf_bytes_grouped(m));
+    ok = ok && dalloc(&c->usq, T * ms / 2) && dalloc(&c->us_sf, c->sf_bytes_dense(ms));
+    ok = ok && dalloc(&c->act_g, 4) && dalloc(&c->tile0, N + 1);
   }
   if (!ok) {
     free_all(c);
@@ -559,10 +579,10 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
                                   VT<V_LARGE4>::smem()) == cudaSuccess;
   if (ok && c->nvfp4) {
     // scale padding (beyond K / 16) must read as zero; stale rows must hold finite scales
-    cudaMemset(c->x_sf, 0, T * act_sf_pitch(d));
-    cudaMemset(c->h_sf, 0, tk * act_sf_pitch(l));
-    cudaMemset(c->u_sf, 0, tk * act_sf_pitch(m));
-    cudaMemset(c->us_sf, 0, T * act_sf_pitch(ms));
+    cudaMemset(c->x_sf, 0, c->sf_bytes_dense(d));
+    cudaMemset(c->h_sf, 0, c->sf_bytes_grouped(l));
+    cudaMemset(c->u_sf, 0, c->sf_bytes_grouped(m));
+    cudaMemset(c->us_sf, 0, c->sf_bytes_dense(ms));
     cudaMemset(c->xq, 0, T * d / 2);
     cudaMemset(c->hq, 0, tk * l / 2);
     cudaMemset(c->uq, 0, tk * m / 2);
@@ -815,7 +835,7 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1};
   UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2};
   scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(c->chunk_counts, nch, N, c->counts, c->offsets,
-                                                              c->chunk_base, l1, l2, c->status);
+                                                              c->chunk_base, l1, l2, nullptr, c->status);
   chk(cudaGetLastError());
   mark(4);
   // 5. stable grouping, then the gather of latent rows into grouped order
@@ -975,13 +995,13 @@ lmoe_status lmoe_inspect(lmoe_handle c, int32_t which, void** dev_ptr, int64_t* 
     case LMOE_BUF_Z: *dev_ptr = c->zu; *count = T * (g.latent + g.shared_ffn); break;
     case LMOE_BUF_U: *dev_ptr = c->u; *count = TK * g.expert_ffn; break;
     case LMOE_BUF_XQ: *dev_ptr = c->xq; *count = T * g.d / 2; break;
-    case LMOE_BUF_X_SF: *dev_ptr = c->x_sf; *count = T * act_sf_pitch(g.d); break;
+    case LMOE_BUF_X_SF: *dev_ptr = c->x_sf; *count = (int64_t)c->sf_bytes_dense(g.d); break;
     case LMOE_BUF_HQ: *dev_ptr = c->hq; *count = TK * g.latent / 2; break;
-    case LMOE_BUF_H_SF: *dev_ptr = c->h_sf; *count = TK * act_sf_pitch(g.latent); break;
+    case LMOE_BUF_H_SF: *dev_ptr = c->h_sf; *count = (int64_t)c->sf_bytes_grouped(g.latent); break;
     case LMOE_BUF_UQ: *dev_ptr = c->uq; *count = TK * g.expert_ffn / 2; break;
-    case LMOE_BUF_U_SF: *dev_ptr = c->u_sf; *count = TK * act_sf_pitch(g.expert_ffn); break;
+    case LMOE_BUF_U_SF: *dev_ptr = c->u_sf; *count = (int64_t)c->sf_bytes_grouped(g.expert_ffn); break;
     case LMOE_BUF_USQ: *dev_ptr = c->usq; *count = T * g.shared_ffn / 2; break;
-    case LMOE_BUF_US_SF: *dev_ptr = c->us_sf; *count = T * act_sf_pitch(g.shared_ffn); break;
+    case LMOE_BUF_US_SF: *dev_ptr = c->us_sf; *count = (int64_t)c->sf_bytes_dense(g.shared_ffn); break;
     case LMOE_BUF_Y_S: *dev_ptr = c->y_s; *count = T * g.d; break;
     case LMOE_BUF_ACT_SCALE: *dev_ptr = c->act_g; *count = 2; break;
     default: return LMOE_ERR_INVALID_ARG;
@@ -1101,7 +1121,7 @@ extern "C" lmoe_status lmoe_route_noalloc(const float* logits, const float* bias
     return LMOE_ERR_CUDA;
   UnitListSpec none{nullptr, nullptr, 0, 64, 0};
   scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(chunk_counts, nch, N, counts, offsets, chunk_base,
-                                                              none, none, status);
+                                                              none, none, nullptr, status);
   if (cudaGetLastError() != cudaSuccess) return LMOE_ERR_CUDA;
   assign_rows_kernel<<<nch, 32, N * sizeof(int), s>>>(topk_idx, topk_gate, chunk_base, T, N, K, ct, row_of,
                                                      tok_of_row, gate_of_row, status);

@@ -15,7 +15,8 @@
 //           layout tcgen05.cp (32x128b, replicated to the 4 lane quadrants) turns into the TMEM scale
 //           columns the block-scaled MMA reads.  Atoms are ordered [row tile][K atom], K atoms padded
 //           to a multiple of 4 (one 256-element pipeline stage) with zero scales.
-//   activation scales: row-major [rows, pitch] bytes, pitch = 16 * ceil(K / 256), zero padded.
+//   activation scales: tile-local atoms (see act_sf_offset), so that one token tile's scales for one
+//           pipeline stage are a single contiguous copy.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -73,6 +74,81 @@ __device__ __forceinline__ uint32_t nvfp4_block(const float (&v)[16], float g, u
     codes[i >> 3] |= c << (4 * (i & 7));
   }
   return sb;
+}
+
+// Eight E2M1 codes (element 2i in the low nibble) of v[i] * rcp, rounded to nearest even and
+// saturated by the hardware conversion.
+__device__ __forceinline__ uint32_t e2m1x8_scaled(const float* v, float rcp) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(__fmul_rn(v[0], rcp)), "f"(__fmul_rn(v[1], rcp)), "f"(__fmul_rn(v[2], rcp)), "f"(__fmul_rn(v[3], rcp)),
+        "f"(__fmul_rn(v[4], rcp)), "f"(__fmul_rn(v[5], rcp)), "f"(__fmul_rn(v[6], rcp)), "f"(__fmul_rn(v[7], rcp)));
+  return r;
+}
+
+// Eight E2M1 codes of r[0..7] (already divided by the block scale), hardware conversion: round to
+// nearest even, saturating at 6.
+__device__ __forceinline__ uint32_t e2m1x8(const float* r) {
+  uint32_t o;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(o)
+      : "f"(r[0]), "f"(r[1]), "f"(r[2]), "f"(r[3]), "f"(r[4]), "f"(r[5]), "f"(r[6]), "f"(r[7]));
+  return o;
+}
+
+// Quantiser for bf16 activations (x, h): the oracle's decisions exactly (IEEE division of each
+// element by the decoded block scale, then round-to-nearest-even).  bf16 inputs hit exact E2M1
+// rounding ties often enough that a reciprocal multiply would land beside them; the rounding itself
+// is the hardware conversion.  A zero block scale gives zero codes.
+__device__ __forceinline__ uint32_t nvfp4_block_exact(const float (&v)[16], float g, uint32_t (&codes)[2]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t sb = e4m3_rne_sat(__fdiv_rn(amax, __fmul_rn(6.0f, g)));
+  const float den = __fmul_rn(e4m3_to_f32(sb), g);
+  float r[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) r[i] = den > 0.f ? __fdiv_rn(v[i], den) : 0.f;
+  codes[0] = e2m1x8(r);
+  codes[1] = e2m1x8(r + 8);
+  return sb;
+}
+
+// Activation block quantiser for fp32 accumulator outputs (u, u_s in the GEMM epilogue): same scale
+// rule, elements scaled by the fp32 reciprocal of the block scale (one multiply and half a conversion
+// per element).  fp32 accumulator values essentially never sit on an E2M1 rounding tie.
+__device__ __forceinline__ uint32_t nvfp4_block_fast(const float (&v)[16], float g, uint32_t (&codes)[2]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t sb = e4m3_rne_sat(__fdiv_rn(amax, __fmul_rn(6.0f, g)));
+  const float den = __fmul_rn(e4m3_to_f32(sb), g);
+  const float rcp = den > 0.f ? __frcp_rn(den) : 0.f;
+  codes[0] = e2m1x8_scaled(v, rcp);
+  codes[1] = e2m1x8_scaled(v + 8, rcp);
+  return sb;
+}
+
+// Activation scales live in tile-local atoms, so that the GEMM fetches one token tile's scales for one
+// pipeline stage with a single bulk copy: for token tile `tile` (nra = ceil(tile tokens / 128) row
+// atoms) and stage `st` (256 K elements = 4 K atoms of 64), the 4 * nra atoms are contiguous, K-atom
+// major: atom (ka, ra) at ((tile * stages + st) * 4 + ka) * nra + ra.  Inside an atom the layout is the
+// weight atoms' one.  Each K atom's scales must start on a 4-column-aligned TMEM address for the
+// block-scaled MMA, hence one atom (one tcgen05.cp) per K atom and 128 tokens even for short tiles.
+__host__ __device__ __forceinline__ long long act_sf_offset(long long tile, int j, int kb16, int stages, int nra) {
+  const int st = kb16 >> 4, ka = (kb16 >> 2) & 3, s = kb16 & 3;
+  return (((tile * stages + st) * 4 + ka) * nra + (j >> 7)) * 512 + (j & 31) * 16 + ((j & 127) >> 5) * 4 + s;
 }
 
 // Byte offset of the scale of (row r, 16-element block kb) inside a weight-scale atom array with
@@ -165,15 +241,20 @@ __global__ void amax_act_kernel(const __nv_bfloat16* __restrict__ a, long long n
 }
 
 // ------------------------------------------------------------------------------------------------
-// Activation quantiser with optional row gather: dst row r takes source row (src_rows ? src_rows[r]
-// : r).  One thread per 16-element block; tensor scale from amax_bits[0].  Also writes g to *g_out.
+// Activation quantiser.  Output row r (0..n_rows) reads source row (src_rows ? src_rows[r] : r) and
+// is written as codes [n_rows, K/2] plus scales in tile-local atoms.  Token tiles: dense mode
+// (offsets == nullptr) tile = r / tile_rows; grouped mode the tiles restart at each expert's first
+// row: expert e = the one with offsets[e] <= r < offsets[e + 1], tile = tile0[e] + (r - offsets[e])
+// / tile_rows.  One thread per 16-element block; tensor scale from amax_bits[0], also written to
+// *g_out.
 // ------------------------------------------------------------------------------------------------
 __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, const int* __restrict__ src_rows,
-                                 long long n_rows, int n_src_rows, const unsigned* __restrict__ amax_bits,
-                                 uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ g_out,
-                                 unsigned* status) {
+                                 long long n_rows, int n_src_rows, const int* __restrict__ offsets,
+                                 const int* __restrict__ tile0, int n_experts, int tile_rows, int nra,
+                                 const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes,
+                                 uint8_t* __restrict__ sf, float* __restrict__ g_out, unsigned* status) {
   const int nb = K / 16;
-  const int pitch = act_sf_pitch(K);
+  const int stages = (K + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K;
   const float g = tensor_scale_from_amax(__uint_as_float(amax_bits[0]));
   if (blockIdx.x == 0 && threadIdx.x == 0 && g_out) *g_out = g;
   const long long total = n_rows * nb;
@@ -189,6 +270,22 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, con
         continue;
       }
     }
+    long long tile;
+    int j;  // row within the tile
+    if (offsets) {
+      int lo = 0, hi = n_experts - 1;  // largest expert whose first row is <= r
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offsets[mid] <= r) lo = mid;
+        else hi = mid - 1;
+      }
+      const int local = (int)(r - offsets[lo]);
+      tile = tile0[lo] + local / tile_rows;
+      j = local % tile_rows;
+    } else {
+      tile = r / tile_rows;
+      j = (int)(r % tile_rows);
+    }
     const uint4* src = reinterpret_cast<const uint4*>(a + sr * K + kb * 16);
     float v[16];
 #pragma unroll
@@ -196,16 +293,16 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, con
       const uint4 q = src[h];
       const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(p[j]);
-        v[h * 8 + 2 * j] = f.x;
-        v[h * 8 + 2 * j + 1] = f.y;
+      for (int t = 0; t < 4; ++t) {
+        const float2 f = __bfloat1622float2(p[t]);
+        v[h * 8 + 2 * t] = f.x;
+        v[h * 8 + 2 * t + 1] = f.y;
       }
     }
     uint32_t c[2];
-    const uint32_t sb = nvfp4_block(v, g, c);
+    const uint32_t sb = nvfp4_block_exact(v, g, c);
     *reinterpret_cast<uint2*>(codes + r * (K / 2) + kb * 8) = make_uint2(c[0], c[1]);
-    sf[r * pitch + kb] = (uint8_t)sb;
+    sf[act_sf_offset(tile, j, kb, stages, nra)] = (uint8_t)sb;
   }
 }
 

@@ -209,7 +209,7 @@ inline size_t scan_smem_bytes(int n_experts, int n_chunks) { return (size_t)n_ex
 __global__ void __launch_bounds__(1024)
     scan_units_kernel(const int* __restrict__ chunk_counts, int n_chunks, int n_experts, int* __restrict__ counts,
                       int* __restrict__ offsets, int* __restrict__ chunk_base, UnitListSpec l1, UnitListSpec l2,
-                      unsigned* status) {
+                      int* __restrict__ tile0, unsigned* status) {
   // chunk_counts / chunk_base are expert-major: [N][n_chunks]
   extern __shared__ int s_cc[];  // [N][n_chunks + 1]
   __shared__ int s_tmp[33];
@@ -244,14 +244,21 @@ __global__ void __launch_bounds__(1024)
   }
   // unit lists: expert-major, token block next, feature block fastest.  Consecutive threads write
   // consecutive units (16-byte stores); a unit finds its expert by binary search over the experts'
-  // first-unit indices.
+  // first-unit indices.  Token tiles are numbered expert-major: expert e owns tiles tile0[e] ...
   __shared__ int s_u0[1025];
   __shared__ int s_cnt[1024];
   __shared__ int s_offs[1024];
+  __shared__ int s_t0[1024];
+  const int tile_tokens = l1.units ? l1.tile_tokens : 64;
+  int n_tiles;
+  const int t0 = block_exclusive_scan((e < n_experts) ? (c_e + tile_tokens - 1) / tile_tokens : 0, s_tmp, n_tiles);
   if (e < n_experts) {
     s_cnt[e] = c_e;
     s_offs[e] = off;
+    s_t0[e] = t0;
+    if (tile0) tile0[e] = t0;
   }
+  if (e == 0 && tile0) tile0[n_experts] = n_tiles;
 #pragma unroll 1
   for (int li = 0; li < 2; ++li) {
     const UnitListSpec& L = li ? l2 : l1;
@@ -282,7 +289,9 @@ __global__ void __launch_bounds__(1024)
       const int nv = min(L.tile_tokens, s_cnt[ex] - tt * L.tile_tokens);
       const int4 g = make_int4(ex * L.feat + ft * BLOCK_M, s_offs[ex] + tt * L.tile_tokens, ft * BLOCK_M,
                                nv | (min(BLOCK_M, L.feat - ft * BLOCK_M) << 16));
-      *reinterpret_cast<int4*>(&L.units[u]) = g;
+      int4* dst = reinterpret_cast<int4*>(&L.units[u]);
+      dst[0] = g;
+      dst[1] = make_int4(s_t0[ex] + tt, 0, 0, 0);
     }
     __syncthreads();
   }
