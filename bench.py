@@ -165,6 +165,25 @@ def cpu_baseline(wl, w, budget_s: float = 20.0):
             "sample": f"first {done} of the {wl.tokens} tokens, fp64 numpy oracle, {el:.1f} s"}
 
 
+# ------------------------------------------------------------------------------------------ ranks
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest of every rank's `value` (a device-timed duration): the job's time is its slowest
+    replica's.  Every rank calls this at the same point; one all-reduce, none at world == 1."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, tokens: int, steps: int, ms: float) -> float:
+    """Tokens every replica processed in `steps` steps of `tokens` tokens, over the max-over-ranks
+    time `ms`."""
+    return world * tokens * steps / (ms * 1e-3)
+
+
 # ------------------------------------------------------------------------------------------ arms
 def run_reference(args, wl, rank):
     if rank != 0:
@@ -250,11 +269,7 @@ def run_ours(args, wl, rank, world):
     stage_ms, recorded, launches = layer.profile_read()
     if layer.device_status() != 0:
         raise RuntimeError("device status not clean after the timed region")
-    ms_max = ms
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_max = float(tt.item())
+    ms_max = max_over_ranks(ms, world, device)
 
     # ---- end to end through the host-buffer entry point ----
     xh = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -271,11 +286,7 @@ def run_ours(args, wl, rank, world):
         layer.forward_host(xh, yh, ih, gh)
     e1.record(stream)
     torch.cuda.synchronize(device)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
 
     if rank != 0:
         layer.close()
@@ -315,7 +326,7 @@ def run_ours(args, wl, rank, world):
                   pk.get("bf16_tflops_sustained", pk["bf16_tflops"])}
     line = {
         "metric": METRIC,
-        "value": world * t * args.steps / (ms_max * 1e-3),
+        "value": whole_job_tokens_per_s(world, t, args.steps, ms_max),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -336,7 +347,7 @@ def run_ours(args, wl, rank, world):
         "roofline": roof,
         "layer_roofline": layer_roof,
         "stages_ms_per_step": {k: v / max(1, recorded) for k, v in stage_ms.items()},
-        "e2e": {"value": world * t * e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_tokens_per_s(world, t, e2e_steps, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": t * wl.shape.d * 2,
                 "d2h_bytes_per_step": t * wl.shape.d * 2 + t * wl.shape.top_k * 8, "steps": e2e_steps},
         "gpu_launches": launches * args.steps,

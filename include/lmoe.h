@@ -194,6 +194,14 @@ lmoe_status lmoe_route_noalloc(const float* logits, const float* bias, int32_t T
                                int32_t* topk_idx, float* topk_gate, int32_t* counts, int32_t* offsets,
                                int32_t* row_of, void* stream);
 
+/* Failure-detection self-test.  Enqueues on `stream` one kernel that waits, with the bounded
+ * mbarrier wait that every pipelined kernel of the library uses, on a barrier that nothing ever
+ * arrives on.  After `limit_ns` nanoseconds (clamped to 1 us .. 2 s) the wait gives up, the kernel
+ * records a timeout in the handle's device status word and returns, leaving the context usable; the
+ * next lmoe_get_device_status then returns LMOE_ERR_DEVICE_TIMEOUT (and clears the word).
+ * Returns LMOE_ERR_CUDA if the launch fails. */
+lmoe_status lmoe_selftest_wait_timeout(lmoe_handle h, uint64_t limit_ns, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* lmoe_status_string(lmoe_status s);
 

@@ -35,7 +35,7 @@ DTYPE = {torch.bfloat16: 0, torch.float32: 1}
 # every extern "C" symbol declared in include/lmoe.h
 SYMBOLS = ("lmoe_create", "lmoe_load_weights", "lmoe_forward", "lmoe_forward_host", "lmoe_get_device_status",
            "lmoe_inspect", "lmoe_profile", "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_export_nvfp4",
-           "lmoe_status_string", "lmoe_destroy")
+           "lmoe_selftest_wait_timeout", "lmoe_status_string", "lmoe_destroy")
 STAGES = ("router", "shared_up", "topk", "grouping", "scatter", "expert_up", "expert_down", "combine", "output")
 
 
@@ -61,12 +61,14 @@ lib.lmoe_profile.argtypes = [_vp, _i32]
 lib.lmoe_profile_read.argtypes = [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i32), ctypes.POINTER(_i32)]
 lib.lmoe_route_noalloc.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.lmoe_export_nvfp4.argtypes = [_vp, _i32, _i32, _vp, _vp, _vp]
+lib.lmoe_selftest_wait_timeout.argtypes = [_vp, ctypes.c_uint64, _vp]
 lib.lmoe_status_string.argtypes = [ctypes.c_int]
 lib.lmoe_status_string.restype = ctypes.c_char_p
 lib.lmoe_destroy.argtypes = [_vp]
 lib.lmoe_destroy.restype = None
 for _f in ("lmoe_create", "lmoe_load_weights", "lmoe_forward", "lmoe_forward_host", "lmoe_get_device_status",
-           "lmoe_inspect", "lmoe_profile", "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_export_nvfp4"):
+           "lmoe_inspect", "lmoe_profile", "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_export_nvfp4",
+           "lmoe_selftest_wait_timeout"):
     getattr(lib, _f).restype = ctypes.c_int
 
 
@@ -172,6 +174,11 @@ class LatentMoE:
 
     def device_status(self) -> int:
         return lib.lmoe_get_device_status(self._h)
+
+    def selftest_wait_timeout(self, limit_ns: int, stream=None) -> None:
+        """Enqueue a kernel whose bounded wait never completes (see lmoe_selftest_wait_timeout)."""
+        _check(lib.lmoe_selftest_wait_timeout(self._h, int(limit_ns), self._stream(stream)),
+               "lmoe_selftest_wait_timeout")
 
     def inspect(self, name: str) -> torch.Tensor:
         p, n = _vp(), _i64()

@@ -79,6 +79,8 @@ struct GemmProblem {
   const uint8_t* act_sf;      // activation scales, tile-local atoms (act_sf_offset)
   int act_sf_stages;          // 256-element stages of the activations' K
   const float* act_gscale;    // activation tensor scale (device scalar)
+  int sfb_resident;           // 1: a token tile's activation scales for the whole K are loaded once
+                              // and stay in TMEM while consecutive units use the same tile
   // dense enumeration
   int dense_ftiles;           // feature tiles
   int dense_ttiles;           // token tiles (fastest-varying unit index)
@@ -92,7 +94,8 @@ struct GemmArgs {
   int main_dense_units;       // units of prob[0] when it is dense (units == nullptr)
   const GemmUnit* units;      // prob[0] grouped: device unit list
   const int* num_units;       // prob[0] grouped: device unit count
-  int dynamic;                // 1: units are claimed from work_counter; 0: CTA c takes c, c + grid, ...
+  int dynamic;                // 1: claims come from work_counter; 0: CTA c takes claims c, c + grid, ...
+  int chunk;                  // main-problem units per claim (>= 1); every pre unit is a claim of its own
   int* work_counter;          // zero before a dynamic launch
   unsigned* status;           // device status word
   unsigned long long timeout_ns;
@@ -106,7 +109,10 @@ constexpr int A_STAGE_BYTES = BLOCK_M * 128;
 constexpr int EPI_STAGE_BYTES = 32 * 32 * 4;  // per epilogue warp: 32 tokens x 32 features fp32
 constexpr int SF_ATOM_BYTES = 512;
 
-template <int BN_MAX, int STAGES, bool FP4>
+// RES_STAGES > 0 (FP4): room for the activation scales of one token tile over up to RES_STAGES
+// K stages, kept in TMEM across consecutive units of that tile (problems with sfb_resident): the
+// tile's first unit loads and copies them stage by stage, its later units reuse them.
+template <int BN_MAX, int STAGES, bool FP4, int ACC_SPLIT, int RES_STAGES>
 struct GemmSmem {
   static constexpr int NRA = (BN_MAX + 127) / 128;                    // 128-row scale atoms of B
   static constexpr int B_STAGE_BYTES = BN_MAX * 128;
@@ -117,13 +123,25 @@ struct GemmSmem {
   static constexpr int BAR_OFF = EPI_OFF + 4 * EPI_STAGE_BYTES;
   static constexpr int BYTES = BAR_OFF + 512;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment of the base
-  // TMEM: two fp32 accumulators of BN_MAX columns, then (FP4) SF_SLOTS rotating slots of scale
-  // columns, one stage each (SFA 4 MMAs x 4 columns, SFB 4 MMAs x NRA x 4 columns).  Every MMA's scale
-  // address is 4-column aligned (the block-scaled MMA faults on a misaligned scale address).
-  static constexpr int SF_COL0 = 2 * BN_MAX;
-  static constexpr int SF_COLS = FP4 ? 16 + 16 * NRA : 0;
-  static constexpr int SF_SLOTS = !FP4 ? 1 : ((512 - SF_COL0) / SF_COLS >= 4 ? 4 : (512 - SF_COL0) / SF_COLS);
-  static constexpr int TMEM_NEED = SF_COL0 + SF_SLOTS * SF_COLS;
+  // TMEM: two accumulator buffers (double buffering), each ACC_SPLIT partial fp32 accumulators of
+  // BN_MAX columns; then (FP4) SF_SLOTS rotating slots of weight scales (SFA: 4 MMAs x 4 columns per
+  // stage), then the activation scales (SFB): either SF_SLOTS rotating per-stage slots (4 MMAs x NRA
+  // x 4 columns) or one resident tile of up to RES_STAGES stages, sharing the same columns.  Every
+  // MMA's scale address is 4-column aligned (the block-scaled MMA faults on a misaligned scale
+  // address).
+  static constexpr int ACC_COLS = ACC_SPLIT * BN_MAX;
+  static constexpr int SF_COL0 = 2 * ACC_COLS;
+  static constexpr int sf_need(int slots) {
+    return 16 * slots + 16 * NRA * (RES_STAGES > slots ? RES_STAGES : slots);
+  }
+  static constexpr int SF_SLOTS = !FP4 ? 1
+                                  : SF_COL0 + sf_need(4) <= 512 ? 4
+                                  : SF_COL0 + sf_need(3) <= 512 ? 3
+                                  : SF_COL0 + sf_need(2) <= 512 ? 2
+                                                                : 1;
+  static constexpr int SFA_COL0 = SF_COL0;
+  static constexpr int SFB_COL0 = SF_COL0 + 16 * SF_SLOTS;
+  static constexpr int TMEM_NEED = SF_COL0 + (FP4 ? sf_need(SF_SLOTS) : 0);
   static constexpr uint32_t TMEM_COLS = (TMEM_NEED <= 32)    ? 32
                                         : (TMEM_NEED <= 64)  ? 64
                                         : (TMEM_NEED <= 128) ? 128
@@ -168,12 +186,15 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rn(float v) {
   return *reinterpret_cast<uint16_t*>(&b);
 }
 
-template <int BN_MAX, int STAGES, int BOXN, bool FP4>
+// ACC_SPLIT > 1: consecutive MMAs of a tile rotate over ACC_SPLIT independent partial accumulators,
+// summed by the epilogue.  With few tokens (N = 16..64) one MMA is far shorter than the tensor pipe's
+// latency, and MMAs chained on one accumulator would each wait for the previous one.
+template <int BN_MAX, int STAGES, int BOXN, bool FP4, int ACC_SPLIT, int RES_STAGES>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_w0, const __grid_constant__ CUtensorMap map_act0,
                    const __grid_constant__ CUtensorMap map_w1, const __grid_constant__ CUtensorMap map_act1,
                    const GemmArgs args) {
-  using S = GemmSmem<BN_MAX, STAGES, FP4>;
+  using S = GemmSmem<BN_MAX, STAGES, FP4, ACC_SPLIT, RES_STAGES>;
   static_assert(BN_MAX % BOXN == 0 && BOXN % 8 == 0, "token box must tile the token block");
   static_assert(BN_MAX % 16 == 0 && BN_MAX <= 256, "MMA N limit");
   extern __shared__ uint8_t smem_raw[];
@@ -240,9 +261,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       bool ok = true;
       int uslot = 0;
       uint32_t uphase = 0;
-      // dynamic launches claim the next unit one unit ahead, so the atomic's round trip overlaps the
-      // loads; static launches take every gridDim.x-th unit
-      int u_next = args.dynamic ? atomicAdd(args.work_counter, 1) : (int)blockIdx.x;
+      // Work is handed out in claims: claim c < n_pre is pre unit c; later claims cover `chunk`
+      // consecutive main units each (consecutive main units share a token tile, feature tiles
+      // fastest).  Dynamic launches take the next claim from work_counter one unit ahead, so the
+      // atomic's round trip overlaps the loads; static launches take claims c, c + grid, ...
+      const int n_pre = args.n_pre_units;
+      const int chunk = args.chunk > 0 ? args.chunk : 1;
+      const int n_claims = n_pre + (num_units - n_pre + chunk - 1) / chunk;
+      int claim = args.dynamic ? atomicAdd(args.work_counter, 1) : (int)blockIdx.x;
+      int u_next = num_units, u_end = num_units;
+      auto open_claim = [&]() {
+        if (claim < n_claims) {
+          u_next = claim < n_pre ? claim : n_pre + (claim - n_pre) * chunk;
+          u_end = claim < n_pre ? claim + 1 : min(num_units, u_next + chunk);
+        } else {
+          u_next = u_end = num_units;
+        }
+      };
+      open_claim();
+      int res_key = -1;  // (token tile, problem) whose activation scales are resident in TMEM
       auto wait0 = [&](uint64_t* bar, uint32_t par) -> bool { return mbar_wait_bounded(bar, par, abort_flag, tmo); };
       while (ok) {
         if (!wait0(&uempty[uslot], uphase ^ 1u)) {
@@ -257,7 +294,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           uphase ^= 1u;
         }
         if (u < 0) break;
-        u_next = args.dynamic ? atomicAdd(args.work_counter, 1) : u_next + (int)gridDim.x;
+        if (++u_next >= u_end) {
+          claim = args.dynamic ? atomicAdd(args.work_counter, 1) : claim + (int)gridDim.x;
+          open_claim();
+        }
         int pid;
         const GemmUnit un = unit_at<BN_MAX>(args, u, pid);
         const GemmProblem& pr = args.prob[pid];
@@ -267,7 +307,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const int nkb = pr.num_k_blocks;
         const int nv = un.nm & 0xFFFF;
         const int nbox = (nv + BOXN - 1) / BOXN;
-        const uint32_t bytes = A_STAGE_BYTES + nbox * BOXN * 128 + S::SFA_STAGE_BYTES + S::SFB_STAGE_BYTES;
+        // activation scales are loaded unless the previous unit left this tile's resident in TMEM
+        bool fill = true;
+        if constexpr (FP4 && RES_STAGES > 0) {
+          const bool res = pr.sfb_resident != 0 && nkb <= RES_STAGES;
+          const int key = (un.tile << 1) | pid;
+          fill = !res || key != res_key;
+          res_key = res ? key : -1;
+        }
+        const uint32_t bytes = A_STAGE_BYTES + nbox * BOXN * 128 + S::SFA_STAGE_BYTES + (fill ? S::SFB_STAGE_BYTES : 0);
         // x coordinate of a stage in the tensor maps: 128 bytes = 64 bf16 elements or 128 FP4 bytes
         const int kx = FP4 ? 128 : BLOCK_K;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -286,8 +334,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint8_t* ssfb = ssfa + S::SFA_STAGE_BYTES;
             bulk_load(ssfa, pr.w_sf + ((long long)(un.a_row >> 7) * pr.w_atoms_k + kb * 4) * SF_ATOM_BYTES,
                       S::SFA_STAGE_BYTES, &full[stage]);
-            bulk_load(ssfb, pr.act_sf + ((long long)un.tile * pr.act_sf_stages + kb) * S::SFB_STAGE_BYTES,
-                      S::SFB_STAGE_BYTES, &full[stage]);
+            if (fill)
+              bulk_load(ssfb, pr.act_sf + ((long long)un.tile * pr.act_sf_stages + kb) * S::SFB_STAGE_BYTES,
+                        S::SFB_STAGE_BYTES, &full[stage]);
           }
           ++issued;
           if (++stage == STAGES) {
@@ -322,6 +371,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       bool ok = true;
       int uslot = 0;
       uint32_t uphase = 0;
+      int res_key = -1;
       while (ok) {
         if (!mbar_wait_bounded(&ufull[uslot], uphase, abort_flag, tmo)) {
           ok = false;
@@ -341,12 +391,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const uint32_t n_mma = (uint32_t)((nv + 15) & ~15);
         const uint32_t idesc = FP4 ? idesc_nvf4(BLOCK_M, n_mma) : idesc_bf16_f32(BLOCK_M, n_mma);
         const int nra = (int)((n_mma + 127) >> 7);
+        // res: this unit's activation scales live in the resident columns (filled by the tile's first
+        // unit, whose copies the tensor pipe runs after the previous tile's MMAs)
+        bool res = false, fill = true;
+        if constexpr (FP4 && RES_STAGES > 0) {
+          res = args.prob[pid].sfb_resident != 0 && nkb <= RES_STAGES;
+          const int key = (un.tile << 1) | pid;
+          fill = !res || key != res_key;
+          res_key = res ? key : -1;
+        }
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, tmo)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN_MAX);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S::ACC_COLS);
+        int mma_i = 0;  // MMA index within the tile: partial accumulator mma_i % ACC_SPLIT
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, tmo)) {
             ok = false;
@@ -359,23 +419,35 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           if constexpr (FP4) {
             const uint32_t ssfa = sa + A_STAGE_BYTES + S::B_STAGE_BYTES;
             const uint32_t ssfb = ssfa + S::SFA_STAGE_BYTES;
-            const uint32_t t_sfa = tmem_base + S::SF_COL0 + (uint32_t)(sf_slot * S::SF_COLS);
-            const uint32_t t_sfb = t_sfa + 16;
+            const uint32_t t_sfa = tmem_base + S::SFA_COL0 + (uint32_t)(sf_slot * 16);
+            // activation scales of MMA k of this stage: t_sfb + 4 * k * sfb_pitch
+            uint32_t t_sfb;
+            int sfb_pitch;
+            if (res) {
+              t_sfb = tmem_base + S::SFB_COL0 + (uint32_t)(16 * kb * S::NRA);
+              sfb_pitch = S::NRA;
+            } else {
+              t_sfb = tmem_base + S::SFB_COL0 + (uint32_t)(sf_slot * 16 * S::NRA);
+              sfb_pitch = nra;
+            }
             if (++sf_slot == S::SF_SLOTS) sf_slot = 0;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               tcgen05_cp_32x128b_x4(t_sfa + 4 * k, smem_desc_sf_atom(ssfa + k * SF_ATOM_BYTES));
-              for (int ra = 0; ra < nra; ++ra)
-                tcgen05_cp_32x128b_x4(t_sfb + 4 * (k * nra + ra),
-                                      smem_desc_sf_atom(ssfb + (k * S::NRA + ra) * SF_ATOM_BYTES));
+              if (fill)
+                for (int ra = 0; ra < nra; ++ra)
+                  tcgen05_cp_32x128b_x4(t_sfb + 4 * (k * sfb_pitch + ra),
+                                        smem_desc_sf_atom(ssfb + (k * S::NRA + ra) * SF_ATOM_BYTES));
             }
 #pragma unroll
-            for (int k = 0; k < 4; ++k)  // K = 64 E2M1 per MMA: +32 bytes = +2 in the address field
-              umma_nvf4(d_tmem, da + 2 * k, db + 2 * k, idesc, t_sfa + 4 * k, t_sfb + 4 * k * nra, (kb | k) != 0);
+            for (int k = 0; k < 4; ++k, ++mma_i)  // K = 64 E2M1 per MMA: +32 bytes = +2 in the address field
+              umma_nvf4(d_tmem + (uint32_t)((mma_i % ACC_SPLIT) * BN_MAX), da + 2 * k, db + 2 * k, idesc, t_sfa + 4 * k,
+                        t_sfb + 4 * k * sfb_pitch, mma_i >= ACC_SPLIT);
           } else {
 #pragma unroll
-            for (int k = 0; k < BLOCK_K / 16; ++k)  // K = 16 bf16 per MMA: +32 bytes = +2 in the address field
-              umma_bf16(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+            for (int k = 0; k < BLOCK_K / 16; ++k, ++mma_i)  // K = 16 bf16 per MMA: +32 bytes = +2 in the address field
+              umma_bf16(d_tmem + (uint32_t)((mma_i % ACC_SPLIT) * BN_MAX), da + 2 * k, db + 2 * k, idesc,
+                        mma_i >= ACC_SPLIT);
           }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
@@ -404,7 +476,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     int uslot = 0;
     uint32_t uphase = 0;
     while (true) {
-      if (!mbar_wait_bounded(&ufull[uslot], uphase, abort_flag, tmo)) {
+      // every wait's outcome is made warp-uniform: the lanes go on to warp-collective TMEM loads
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&ufull[uslot], uphase, abort_flag, tmo))) {
         if (lane == 0) atomicOr(args.status, DEV_STATUS_TIMEOUT);
         break;
       }
@@ -423,12 +496,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int mv = un.nm >> 16;
       float oscale = 1.0f;
       if constexpr (FP4) oscale = __ldg(pr.w_gscale + un.a_row / pr.w_rows_per_g) * __ldg(pr.act_gscale);
-      if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, tmo)) {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, tmo))) {
         if (lane == 0) atomicOr(args.status, DEV_STATUS_TIMEOUT);
         break;
       }
       tc_fence_after();
-      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * S::ACC_COLS);
+      // partial accumulators that received at least one MMA (every tile has >= 4 MMAs)
+      const int n_part = min(ACC_SPLIT, pr.num_k_blocks * 4);
       const int nchunks = (nv + 31) >> 5;
       const bool feat_ok = (q * 32) < mv;
       const int f = un.f0 + q * 32;  // first feature of this warp's 32
@@ -436,6 +511,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         uint32_t r[32];
         tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), r);
         tmem_ld_wait();
+        for (int pp = 1; pp < n_part; ++pp) {
+          uint32_t r2[32];
+          tmem_ld_32x32b_x32(tbase + (uint32_t)(pp * BN_MAX + c * 32), r2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(r2[j]));
+        }
         if (c == nchunks - 1) {
           // accumulator fully read by this warp: hand it back to the MMA issuer
           tc_fence_before();

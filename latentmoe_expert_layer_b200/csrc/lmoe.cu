@@ -54,13 +54,16 @@ constexpr int V_BN[4] = {64, 256, 64, 192};
 constexpr int V_STAGES[4] = {8, 4, 7, 4};
 constexpr int V_BOXN[4] = {16, 64, 16, 64};
 constexpr bool V_FP4[4] = {false, false, true, true};
+constexpr int V_ACC_SPLIT[4] = {4, 1, 2, 1};  // decode-sized tiles rotate over independent accumulators
+// K stages of one token tile's activation scales that fit resident in TMEM (0: per-stage copies)
+constexpr int V_RES[4] = {0, 0, 12, 0};
 
 template <int V>
 struct VT {
-  static constexpr int BN = V_BN[V], ST = V_STAGES[V], BOX = V_BOXN[V];
+  static constexpr int BN = V_BN[V], ST = V_STAGES[V], BOX = V_BOXN[V], AS = V_ACC_SPLIT[V], RS = V_RES[V];
   static constexpr bool F4 = V_FP4[V];
-  static void* fn() { return reinterpret_cast<void*>(gemm_tc_kernel<BN, ST, BOX, F4>); }
-  static int smem() { return GemmSmem<BN, ST, F4>::ALLOC; }
+  static void* fn() { return reinterpret_cast<void*>(gemm_tc_kernel<BN, ST, BOX, F4, AS, RS>); }
+  static int smem() { return GemmSmem<BN, ST, F4, AS, RS>::ALLOC; }
 };
 
 // 2-D byte tensor map (packed NVFP4 codes): rows x cols_bytes, 128-byte x box_rows tiles, 128-byte swizzle.
@@ -241,7 +244,8 @@ lmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LMOE_OK : LMO
 template <int V>
 cudaError_t launch_gemm_v(const CUtensorMap& w0, const CUtensorMap& a0, const CUtensorMap& w1, const CUtensorMap& a1,
                           const GemmArgs& a, int grid, cudaStream_t s) {
-  gemm_tc_kernel<VT<V>::BN, VT<V>::ST, VT<V>::BOX, VT<V>::F4><<<grid, GEMM_THREADS, VT<V>::smem(), s>>>(w0, a0, w1, a1, a);
+  gemm_tc_kernel<VT<V>::BN, VT<V>::ST, VT<V>::BOX, VT<V>::F4, VT<V>::AS, VT<V>::RS>
+      <<<grid, GEMM_THREADS, VT<V>::smem(), s>>>(w0, a0, w1, a1, a);
   return cudaGetLastError();
 }
 
@@ -297,6 +301,7 @@ struct GemmLaunch {
     a.status = ctx->status;
     a.timeout_ns = ctx->timeout_ns;
     a.work_counter = ctx->work_counters + counter;
+    a.chunk = 1;
   }
   // main problem, dense
   void main_dense(const CUtensorMap& mw, const CUtensorMap& ma, GemmProblem p, int feat, int tokens) {
@@ -306,11 +311,28 @@ struct GemmLaunch {
     a0 = &ma;
   }
   // main problem, grouped experts (unit list on the device)
+  // feat: output features of every expert (units per token tile = ceil(feat / 128));
+  // max_tiles: upper bound on the token tiles of the launch
   void main_grouped(const CUtensorMap& mw, const CUtensorMap& ma, GemmProblem p, const GemmUnit* units,
-                    const int* num_units) {
+                    const int* num_units, int feat, long long max_tiles) {
     const bool small = v == V_SMALL || v == V_SMALL4;
     p.weights_streamed = small;  // decode-sized groups: mostly one token tile per expert
     a.dynamic = small;           // measured: dynamic claiming helps decode-sized groups only
+    if (V_FP4[v] && p.num_k_blocks <= V_RES[v]) {
+      // A token tile's activation scales stay in TMEM while a claim's units use that tile.  A claim
+      // is a divisor of the tile's feature-tile count (claims never straddle two tiles), as large
+      // as leaves every CTA about 6 claims to balance the load with.
+      p.sfb_resident = 1;
+      const int nft = (feat + BLOCK_M - 1) / BLOCK_M;
+      const long long cap = max_tiles * nft / (6LL * c->num_sms);
+      int ch = 1;
+      for (int cand = nft; cand >= 1; --cand)
+        if (nft % cand == 0 && cand <= cap) {
+          ch = cand;
+          break;
+        }
+      a.chunk = ch;
+    }
     a.prob[0] = p;
     a.units = units;
     a.num_units = num_units;
@@ -355,6 +377,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
   const int vd = T <= 512 ? V_SMALL : V_LARGE;
   const int vg = TK <= 48LL * N ? V_SMALL4 : V_LARGE4;
   const bool split = vg == V_SMALL4;  // shared-expert GEMMs ride inside the expert launches
+  const long long max_tiles4 = N + (TK + V_BN[vg] - 1) / V_BN[vg];  // token tiles of the expert launches
   unsigned* amax_x = reinterpret_cast<unsigned*>(c->work_counters + lmoe_ctx::kAmaxX);
   unsigned* amax_h = reinterpret_cast<unsigned*>(c->work_counters + lmoe_ctx::kAmaxH);
   float* g_x = c->act_g + 0;
@@ -435,7 +458,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
     GemmProblem p = problem4(l, EPI_SQRELU_NVFP4, c->uq, m / 2, c->w1_sf, c->wg, m, c->h_sf, g_h);
     p.out_sf = c->u_sf;
     p.out_sf_stages = (m + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K;
-    gl.main_grouped(c->map_w1q, c->map_hq[vg], p, c->units1, c->num_units);
+    gl.main_grouped(c->map_w1q, c->map_hq[vg], p, c->units1, c->num_units, m, max_tiles4);
     chk(gl.run(s));
   }
   if (!split) {
@@ -451,7 +474,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
     if (split) gl.pre_dense(c->map_ws2q, c->map_usq[vg], shared_down, d, T);
     GemmProblem p = problem4(m, EPI_ROWSCALE_BF16, c->o, l, c->w2_sf, c->wg + N, l, c->u_sf, one);
     p.row_scale = c->gate_of_row;
-    gl.main_grouped(c->map_w2q, c->map_uq[vg], p, c->units2, c->num_units + 1);
+    gl.main_grouped(c->map_w2q, c->map_uq[vg], p, c->units2, c->num_units + 1, l, max_tiles4);
     chk(gl.run(s));
   }
   if (!split) {
@@ -854,7 +877,8 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   {
     GemmLaunch g(c, vg, 4);
     if (split) g.pre_dense(c->map_ws1, c->map_x[vd], shared_up, ms, T);
-    g.main_grouped(c->map_w1, c->map_hperm[vg], problem(l, EPI_SQRELU_BF16, c->u, m), c->units1, c->num_units);
+    g.main_grouped(c->map_w1, c->map_hperm[vg], problem(l, EPI_SQRELU_BF16, c->u, m), c->units1, c->num_units, m,
+                   0);
     chk(g.run(s));
   }
   mark(6);
@@ -864,7 +888,7 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
     if (split) g.pre_dense(c->map_ws2, c->map_us[vd], problem(ms, EPI_F32, c->y_s, d), d, T);
     GemmProblem p = problem(m, EPI_ROWSCALE_BF16, c->o, l);
     p.row_scale = c->gate_of_row;
-    g.main_grouped(c->map_w2, c->map_u[vg], p, c->units2, c->num_units + 1);
+    g.main_grouped(c->map_w2, c->map_u[vg], p, c->units2, c->num_units + 1, l, 0);
     chk(g.run(s));
   }
   mark(7);
@@ -966,6 +990,27 @@ lmoe_status lmoe_export_nvfp4(lmoe_handle c, int32_t which, int32_t index, uint8
   for (long long r = 0; r < rows; ++r)
     for (int kb = 0; kb < K / 16; ++kb) scales_host[r * (K / 16) + kb] = tmp[sf_atom_offset(r, kb, atoms_k)];
   return LMOE_OK;
+}
+
+// One thread waits on a shared-memory mbarrier whose single expected arrival never comes.
+__global__ void wait_timeout_probe_kernel(unsigned* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, &abort_flag, limit_ns)) atomicOr(status, DEV_STATUS_TIMEOUT);
+}
+
+lmoe_status lmoe_selftest_wait_timeout(lmoe_handle c, uint64_t limit_ns, void* stream) {
+  if (!c) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  const unsigned long long lim = std::min<uint64_t>(std::max<uint64_t>(limit_ns, 1000ull), 2000000000ull);
+  wait_timeout_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(c->status, lim);
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
 
 lmoe_status lmoe_get_device_status(lmoe_handle c) {

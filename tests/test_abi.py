@@ -27,7 +27,7 @@ def test_header_declares_the_boundary():
     assert _declared() == sorted(["lmoe_create", "lmoe_load_weights", "lmoe_forward", "lmoe_forward_host",
                                   "lmoe_get_device_status", "lmoe_inspect", "lmoe_profile",
                                   "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_export_nvfp4",
-                                  "lmoe_status_string",
+                                  "lmoe_selftest_wait_timeout", "lmoe_status_string",
                                   "lmoe_destroy"])
 
 

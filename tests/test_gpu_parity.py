@@ -170,3 +170,19 @@ def test_skewed_sampled_parity(skewlayer, superlayer):
     _check_dispatch(layer, st["idx"], wl.shape.n_experts)
     counts = np.bincount(st["idx"].ravel(), minlength=wl.shape.n_experts)
     assert (counts == 0).sum() >= 32 and counts.max() > 0.1 * wl.tokens
+
+
+def test_wait_timeout_reported_and_context_survives(tiny):
+    """Failure detection without a fault: a kernel waits, bounded, on a barrier nothing arrives on.
+    The timeout reaches the host as LMOE_ERR_DEVICE_TIMEOUT, the status word is cleared by reading
+    it, and the context still runs the layer with unchanged results."""
+    wl, w, layer = tiny
+    x = inp.make_x(wl)
+    before = _run(layer, x)
+    layer.selftest_wait_timeout(2_000_000)  # 2 ms
+    torch.cuda.synchronize()
+    assert layer.device_status() == 7
+    assert layer.device_status() == 0
+    after = _run(layer, x)
+    for a, b in zip(before, after):
+        assert np.array_equal(a, b)
