@@ -537,10 +537,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * __shfl_sync(0xffffffffu, mys, j));
         } else if (pr.epi == EPI_ADD_BF16) {
           if (feat_ok && q * 32 + lane < mv) {
+            // all 32 loads (one coalesced 128-byte row segment each) are in flight before the
+            // first add, so the chunk pays one memory latency rather than 32
             const float* ad = pr.addend + (long long)row0 * pr.ld_add + f + lane;
+            float av[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nrows) r[j] = __float_as_uint(__uint_as_float(r[j]) + ad[(long long)j * pr.ld_add]);
+            for (int j = 0; j < 32; ++j) av[j] = __ldg(ad + (long long)(j < nrows ? j : 0) * pr.ld_add);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) + av[j]);
           }
         } else if (pr.epi == EPI_SQRELU_BF16 || pr.epi == EPI_SQRELU_NVFP4) {
 #pragma unroll
