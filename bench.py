@@ -35,7 +35,7 @@ METRIC = "LatentMoE layer tokens/s (Super shape, T=256 & 16K); % of HBM / TC roo
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DEFAULT_STEPS = {"tiny": 200, "decode": 400, "skewed": 40, "prefill": 20}
 DEFAULT_STEPS.update({"decode_small": 400, "decode_nvfp4": 400, "prefill_nvfp4": 20, "nvfp4_tiny": 200,
-                      "nvfp4_mid": 100})
+                      "nvfp4_mid": 100, "ultra_decode": 200, "ultra_decode_nvfp4": 200, "ultra_prefill": 10})
 
 
 def peaks():

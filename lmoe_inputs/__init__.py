@@ -28,7 +28,7 @@ from typing import Dict, Optional
 import numpy as np
 
 __all__ = [
-    "LayerShape", "Workload", "WORKLOADS", "workload", "f32_to_bf16_bits", "bf16_bits_to_f32",
+    "LayerShape", "SUPER", "ULTRA", "Workload", "WORKLOADS", "workload", "f32_to_bf16_bits", "bf16_bits_to_f32",
     "LayerWeights", "make_weights", "make_router", "make_x", "expert_weight", "skewed_router_bias",
 ]
 
@@ -50,6 +50,10 @@ class LayerShape:
 
 
 SUPER = LayerShape(d=4096, latent=1024, n_experts=512, top_k=22, expert_ffn=2688, shared_ffn=5376)
+# Ultra-width experts: 512 experts, top-22, expert hidden 5120, shared-expert intermediate 10240
+# ("Nemotron 3 Ultra" summary, core method).  That page gives neither the model dimension nor the
+# latent dimension, so Super's d = 4096 and l = 1024 are kept.
+ULTRA = LayerShape(d=4096, latent=1024, n_experts=512, top_k=22, expert_ffn=5120, shared_ffn=10240)
 TINY = LayerShape(d=256, latent=64, n_experts=16, top_k=4, expert_ffn=128, shared_ffn=256)
 
 
@@ -87,6 +91,12 @@ WORKLOADS: Dict[str, Workload] = {
                            description="NVFP4 layer d=512 l=256 N=16 K=4 m=384 m_s=512, T=40"),
     "nvfp4_mid": Workload("nvfp4_mid", LayerShape(512, 256, 16, 4, 384, 512), 1024, 7, 9, "bf16", "nvfp4",
                           description="NVFP4 layer d=512 l=256 N=16 K=4 m=384 m_s=512, T=1024"),
+    "ultra_decode": Workload("ultra_decode", ULTRA, 256, 5, 2, "bf16", "bf16",
+                             description="Ultra-width experts (m=5120, m_s=10240; d=4096, l=1024), decode T=256"),
+    "ultra_decode_nvfp4": Workload("ultra_decode_nvfp4", ULTRA, 256, 5, 2, "bf16", "nvfp4",
+                                   description="NVFP4 Ultra-width experts, decode T=256"),
+    "ultra_prefill": Workload("ultra_prefill", ULTRA, 16384, 5, 3, "bf16", "bf16",
+                              description="Ultra-width experts, prefill T=16384"),
     "skewed": Workload("skewed", SUPER, 4096, 1, 4, "bf16", "bf16", router_bias=True,
                        description="Super shape T=4096, per-expert router bias giving a capped Zipf(1.2) load"),
 }

@@ -9,9 +9,11 @@ import torch
 
 import lmoe_inputs as inp
 from oracle import lmoe_oracle as lo
+from oracle import nvfp4 as nv
 
 NEAR_TIE_EPS = 1e-5       # logit gap below which routing may legitimately differ
 Y_TOL_BF16 = 2e-2         # max |y_gpu - y_oracle| <= Y_TOL * RMS(y_oracle)
+Y_TOL_NVFP4 = 5e-2        # the same against the oracle's NVFP4 forward
 GATE_TOL = 1e-5           # |g_gpu - g_oracle| on tokens routed identically
 
 
@@ -76,3 +78,78 @@ def check_y(y_gpu: np.ndarray, y_ref: np.ndarray, tol: float = Y_TOL_BF16) -> fl
     err = float(np.abs(y_gpu - y_ref).max())
     assert err <= tol * rms, f"max |y - y_ref| = {err:.4g} > {tol} * RMS {rms:.4g}"
     return err / rms
+
+
+# ------------------------------------------------------------------------------------------------
+# running the layer and comparing with the oracle
+# ------------------------------------------------------------------------------------------------
+def run_layer(layer, x_np):
+    """Forward on x (bf16 bits); returns y (float64), idx, gate as numpy; asserts a clean status."""
+    x = to_dev(x_np, "bf16")
+    y, idx, gate = layer.forward(x)
+    torch.cuda.synchronize()
+    st = layer.device_status()
+    assert st == 0, f"device status {st}"
+    return bf16_to_np(y), idx.cpu().numpy(), gate.cpu().numpy()
+
+
+def compare_bf16(layer, ow, x_np, k, tokens=None):
+    """Run the layer on x, compare (optionally only `tokens`) with the oracle; returns stats."""
+    y, idx, gate = run_layer(layer, x_np)
+    x64 = lo.lift(x_np, "bf16")
+    sel = np.arange(x_np.shape[0]) if tokens is None else np.asarray(tokens)
+    ref = lo.forward(ow, x64[sel], k)
+    diff, near = check_routing(idx[sel], gate[sel], ref, k)
+    yref = ref["y"].copy()
+    if diff.any():
+        forced = lo.forward(ow, x64[sel][diff], k, idx=idx[sel][diff])
+        yref[diff] = forced["y"]
+    rel = check_y(y[sel], yref)
+    # router logits of the sampled tokens
+    lg = layer.inspect("logits").cpu().numpy().reshape(x_np.shape[0], -1)[sel]
+    lerr = float(np.abs(lg - (ref["logits"] - (0 if ow.b_router is None else ow.b_router))).max())
+    return {"y": y, "idx": idx, "gate": gate, "rel_err": rel, "logit_err": lerr, "near_ties": int(near.sum()),
+            "routing_diffs": int(diff.sum())}
+
+
+def check_dispatch(layer, idx, n):
+    """The device's grouping maps equal the oracle's grouping of the device's own routing."""
+    counts, offsets, row_of, tok_of_row = lo.dispatch(idx, n)
+    assert np.array_equal(layer.inspect("counts").cpu().numpy(), counts)
+    assert np.array_equal(layer.inspect("offsets").cpu().numpy(), offsets)
+    assert np.array_equal(layer.inspect("row_of").cpu().numpy(), row_of.reshape(-1))
+    assert np.array_equal(layer.inspect("tok_of_row").cpu().numpy(), tok_of_row)
+
+
+def pack_codes(codes):
+    """One E2M1 code per byte -> two per byte, element 2i in the low nibble."""
+    return (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+
+
+def check_weight_bytes(layer, w, which, index, quantize=None):
+    """The device's quantised weight (codes, block scales, tensor scale) equals the oracle's bytes."""
+    quantize = quantize or nv.quantize
+    src = {0: lambda: w.w1[index], 1: lambda: w.w2[index], 2: lambda: w.ws1, 3: lambda: w.ws2}[which]()
+    ref_c, ref_s, ref_g = quantize(inp.bf16_bits_to_f32(src))
+    codes, scales, g = layer.export_nvfp4(which, index)
+    assert g == ref_g, (which, index, g, ref_g)
+    assert np.array_equal(scales, ref_s), (which, index, np.argwhere(scales != ref_s)[:5])
+    assert np.array_equal(codes, pack_codes(ref_c)), (which, index, np.argwhere(codes != pack_codes(ref_c))[:5])
+
+
+def compare_nvfp4(layer, w, x_np, k, tokens=None, weight_quantize=None):
+    """NVFP4 layer against the oracle's NVFP4 forward; returns max|err| / RMS(y)."""
+    y, idx, gate = run_layer(layer, x_np)
+    ow = oracle_weights(w, False)
+    x64 = lo.lift(x_np, "bf16")
+    # the per-call activation scales come from the whole batch (oracle's own x and bf16 h)
+    g_x = nv.tensor_scale(x64.astype(np.float32))
+    g_h = nv.tensor_scale(nv.bf16_round(x64 @ ow.w_down.T).astype(np.float32))
+    sel = np.arange(x_np.shape[0]) if tokens is None else np.asarray(tokens)
+    kw = {} if weight_quantize is None else {"weight_quantize": weight_quantize}
+    ref = nv.forward_nvfp4(ow, x64[sel], k, g_x=g_x, g_h=g_h, **kw)
+    diff, near = check_routing(idx[sel], gate[sel], ref, k)
+    yref = ref["y"].copy()
+    if diff.any():
+        yref[diff] = nv.forward_nvfp4(ow, x64[sel][diff], k, idx=idx[sel][diff], g_x=g_x, g_h=g_h, **kw)["y"]
+    return check_y(y[sel], yref, Y_TOL_NVFP4)

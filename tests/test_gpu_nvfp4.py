@@ -11,48 +11,15 @@ import torch
 import lmoe_inputs as inp
 from oracle import lmoe_oracle as lo
 from oracle import nvfp4 as nv
-from lmoe_testlib import (bf16_to_np, check_routing, check_y, device_weights, host_weights, make_layer,
-                          oracle_weights, to_dev)
+from lmoe_testlib import (check_weight_bytes, compare_nvfp4, device_weights, host_weights, make_layer,
+                          pack_codes)
 
 pytestmark = pytest.mark.gpu
-Y_TOL_NVFP4 = 5e-2
 
 
-def _pack(codes):
-    return (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
-
-
-def _check_weight_bytes(layer, w, which, index):
-    src = {0: lambda: w.w1[index], 1: lambda: w.w2[index], 2: lambda: w.ws1, 3: lambda: w.ws2}[which]()
-    ref_c, ref_s, ref_g = nv.quantize(inp.bf16_bits_to_f32(src))
-    codes, scales, g = layer.export_nvfp4(which, index)
-    assert g == ref_g, (which, index, g, ref_g)
-    assert np.array_equal(scales, ref_s), (which, index, np.argwhere(scales != ref_s)[:5])
-    assert np.array_equal(codes, _pack(ref_c)), (which, index, np.argwhere(codes != _pack(ref_c))[:5])
-
-
-def _run(layer, x_np):
-    x = to_dev(x_np, "bf16")
-    y, idx, gate = layer.forward(x)
-    torch.cuda.synchronize()
-    assert layer.device_status() == 0
-    return bf16_to_np(y), idx.cpu().numpy(), gate.cpu().numpy()
-
-
-def _compare_nvfp4(layer, w, x_np, k, tokens=None):
-    y, idx, gate = _run(layer, x_np)
-    ow = oracle_weights(w, False)
-    x64 = lo.lift(x_np, "bf16")
-    # the per-call activation scales come from the whole batch (oracle's own x and bf16 h)
-    g_x = nv.tensor_scale(x64.astype(np.float32))
-    g_h = nv.tensor_scale(nv.bf16_round(x64 @ ow.w_down.T).astype(np.float32))
-    sel = np.arange(x_np.shape[0]) if tokens is None else np.asarray(tokens)
-    ref = nv.forward_nvfp4(ow, x64[sel], k, g_x=g_x, g_h=g_h)
-    diff, near = check_routing(idx[sel], gate[sel], ref, k)
-    yref = ref["y"].copy()
-    if diff.any():
-        yref[diff] = nv.forward_nvfp4(ow, x64[sel][diff], k, idx=idx[sel][diff], g_x=g_x, g_h=g_h)["y"]
-    return check_y(y[sel], yref, Y_TOL_NVFP4)
+_pack = pack_codes
+_check_weight_bytes = check_weight_bytes
+_compare_nvfp4 = compare_nvfp4
 
 
 @pytest.fixture(scope="module")

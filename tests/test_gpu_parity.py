@@ -10,46 +10,15 @@ import torch
 
 import lmoe_inputs as inp
 from oracle import lmoe_oracle as lo
-from lmoe_testlib import (bf16_to_np, check_routing, check_y, device_weights, host_weights, make_layer,
-                          oracle_weights, to_dev)
+from lmoe_testlib import (bf16_to_np, check_dispatch, compare_bf16, device_weights, host_weights, make_layer,
+                          oracle_weights, run_layer, to_dev)
 
 pytestmark = pytest.mark.gpu
 
 
-def _run(layer, x_np):
-    x = to_dev(x_np, "bf16")
-    y, idx, gate = layer.forward(x)
-    torch.cuda.synchronize()
-    st = layer.device_status()
-    assert st == 0, f"device status {st}"
-    return bf16_to_np(y), idx.cpu().numpy(), gate.cpu().numpy()
-
-
-def _compare(layer, ow, x_np, k, tokens=None):
-    """Run the layer on x, compare (optionally only `tokens`) with the oracle; returns stats."""
-    y, idx, gate = _run(layer, x_np)
-    x64 = lo.lift(x_np, "bf16")
-    sel = np.arange(x_np.shape[0]) if tokens is None else np.asarray(tokens)
-    ref = lo.forward(ow, x64[sel], k)
-    diff, near = check_routing(idx[sel], gate[sel], ref, k)
-    yref = ref["y"].copy()
-    if diff.any():
-        forced = lo.forward(ow, x64[sel][diff], k, idx=idx[sel][diff])
-        yref[diff] = forced["y"]
-    rel = check_y(y[sel], yref)
-    # router logits of the sampled tokens
-    lg = layer.inspect("logits").cpu().numpy().reshape(x_np.shape[0], -1)[sel]
-    lerr = float(np.abs(lg - (ref["logits"] - (0 if ow.b_router is None else ow.b_router))).max())
-    return {"y": y, "idx": idx, "gate": gate, "rel_err": rel, "logit_err": lerr, "near_ties": int(near.sum()),
-            "routing_diffs": int(diff.sum())}
-
-
-def _check_dispatch(layer, idx, n):
-    counts, offsets, row_of, tok_of_row = lo.dispatch(idx, n)
-    assert np.array_equal(layer.inspect("counts").cpu().numpy(), counts)
-    assert np.array_equal(layer.inspect("offsets").cpu().numpy(), offsets)
-    assert np.array_equal(layer.inspect("row_of").cpu().numpy(), row_of.reshape(-1))
-    assert np.array_equal(layer.inspect("tok_of_row").cpu().numpy(), tok_of_row)
+_run = run_layer
+_compare = compare_bf16
+_check_dispatch = check_dispatch
 
 
 # ------------------------------------------------------------------------------------------------ tiny
