@@ -62,7 +62,16 @@ typedef struct {
   int32_t precision;   /* lmoe_precision: NVFP4 quantises routed+shared experts (weights and inputs);
                           NVFP4 needs d, latent, expert_ffn and shared_ffn to be multiples of 128 */
   int32_t has_router_bias; /* 1: a per-expert fp32 bias is added to the router logits */
+  int32_t weight_scale;    /* NVFP4 weight block scales (lmoe_weight_scale); ignored for bf16 */
 } lmoe_config;
+
+/* How the NVFP4 quantiser picks a weight block's E4M3 scale.  AMAX: s = E4M3(amax_block / (6 g)).
+ * MSE: the per-block MSE weight quantiser that the "Nemotron 3 Super" notes (section 4.2, the NVFP4
+ * quantisation ablation) name but do not define, read here as: among the AMAX scale (code c0), the
+ * next larger E4M3 value and the six next smaller ones (codes c0, c0+1, c0-1 .. c0-6, kept in
+ * 1..0x7E), the first, in that order, with the strictly smallest fp32 sum of squared block
+ * reconstruction errors.  Activations always use AMAX. */
+typedef enum { LMOE_WSCALE_AMAX = 0, LMOE_WSCALE_MSE = 1 } lmoe_weight_scale;
 
 /* Device pointers to the caller's weights, all of element type `dtype`, row-major [out, in].
  * With LMOE_DTYPE_F32 the router stays fp32 (scored with fp32 FMAs) and every other matrix is

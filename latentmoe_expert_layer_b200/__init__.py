@@ -30,6 +30,7 @@ BUF = {"logits": 0, "counts": 1, "offsets": 2, "row_of": 3, "tok_of_row": 4, "h"
        "xq": 8, "x_sf": 9, "hq": 10, "h_sf": 11, "uq": 12, "u_sf": 13, "usq": 14, "us_sf": 15, "y_s": 16,
        "act_scale": 17}
 PREC = {"bf16": 0, "nvfp4": 1}
+WSCALE = {"amax": 0, "mse": 1}
 DTYPE = {torch.bfloat16: 0, torch.float32: 1}
 
 # every extern "C" symbol declared in include/lmoe.h
@@ -41,7 +42,7 @@ STAGES = ("router", "shared_up", "topk", "grouping", "scatter", "expert_up", "ex
 
 class _Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("d", "latent", "n_experts", "top_k", "expert_ffn", "shared_ffn",
-                                             "max_tokens", "precision", "has_router_bias")]
+                                             "max_tokens", "precision", "has_router_bias", "weight_scale")]
 
 
 class _Weights(ctypes.Structure):
@@ -126,12 +127,13 @@ class LatentMoE:
     """One LatentMoE layer on one GPU.
 
     shape: object with d, latent, n_experts, top_k, expert_ffn, shared_ffn attributes.
+    weight_scale: NVFP4 weight block scales, "amax" or "mse" (lmoe_weight_scale).
     """
 
     def __init__(self, shape, max_tokens: int, precision: str = "bf16", router_bias: bool = False,
-                 device: int = 0):
+                 device: int = 0, weight_scale: str = "amax"):
         cfg = _Config(shape.d, shape.latent, shape.n_experts, shape.top_k, shape.expert_ffn, shape.shared_ffn,
-                      max_tokens, PREC[precision], int(router_bias))
+                      max_tokens, PREC[precision], int(router_bias), WSCALE[weight_scale])
         h = _vp()
         _check(lib.lmoe_create(ctypes.byref(cfg), device, ctypes.byref(h)), "lmoe_create")
         self._h = h

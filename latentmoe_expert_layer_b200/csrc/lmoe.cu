@@ -533,6 +533,7 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
       g.max_tokens <= 0)
     return LMOE_ERR_INVALID_ARG;
   if (g.precision != LMOE_PREC_BF16 && g.precision != LMOE_PREC_NVFP4) return LMOE_ERR_INVALID_ARG;
+  if (g.weight_scale != LMOE_WSCALE_AMAX && g.weight_scale != LMOE_WSCALE_MSE) return LMOE_ERR_INVALID_ARG;
   if (g.d % 64 || g.latent % 64 || g.expert_ffn % 64 || g.shared_ffn % 64) return LMOE_ERR_UNSUPPORTED;
   if (g.n_experts > 1024 || g.n_experts % 16 || g.top_k > 32 || g.top_k > g.n_experts) return LMOE_ERR_UNSUPPORTED;
   if (g.precision == LMOE_PREC_NVFP4 &&
@@ -732,7 +733,7 @@ lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream
       const long long blocks_needed = (q.rows * (q.K / 16) + 255) / 256;
       const int blocks = (int)(blocks_needed < 148LL * 64 ? blocks_needed : 148LL * 64);
       quant_weight_kernel<<<blocks, 256, 0, s>>>(q.src, q.rows, q.K, q.rows_per_g, c->w_amax + q.g0, q.codes, q.sf,
-                                                 c->wg + q.g0);
+                                                 c->wg + q.g0, c->cfg.weight_scale == LMOE_WSCALE_MSE);
     }
     ok = ok && cudaGetLastError() == cudaSuccess && cudaStreamSynchronize(s) == cudaSuccess;
     cudaFree(ws2_tmp);

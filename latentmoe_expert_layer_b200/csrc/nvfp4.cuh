@@ -76,6 +76,57 @@ __device__ __forceinline__ uint32_t nvfp4_block(const float (&v)[16], float g, u
   return sb;
 }
 
+// Signed value of a 4-bit E2M1 code.
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  const uint32_t m = c & 7u;
+  const float a = m < 4u ? 0.5f * (float)m : (m == 4u ? 2.0f : m == 5u ? 3.0f : m == 6u ? 4.0f : 6.0f);
+  return (c & 8u) ? -a : a;
+}
+
+// Sum of squared reconstruction errors of a block under block scale s (decoded E4M3) and tensor
+// scale g: every step rounded to fp32 on its own (no fused multiply-add), elements in order.
+__device__ __forceinline__ float nvfp4_block_sq_error(const float (&v)[16], float s, float g) {
+  const float den = __fmul_rn(s, g);
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float q = den > 0.f ? e2m1_value(e2m1_code(__fdiv_rn(v[i], den))) : 0.f;
+    const float e = __fsub_rn(v[i], __fmul_rn(__fmul_rn(q, s), g));
+    acc = __fadd_rn(acc, __fmul_rn(e, e));
+  }
+  return acc;
+}
+
+// nvfp4_block with the block scale searched for the smallest squared error: candidates c0 (the
+// amax rule), c0 + 1, c0 - 1 .. c0 - 6 (inside the positive finite codes 1..0x7E); the first
+// strict minimum wins.
+__device__ __forceinline__ uint32_t nvfp4_block_mse(const float (&v)[16], float g, uint32_t (&codes)[2]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t c0 = e4m3_rne_sat(__fdiv_rn(amax, __fmul_rn(6.0f, g)));
+  uint32_t best = c0;
+  float best_e = nvfp4_block_sq_error(v, e4m3_to_f32(c0), g);
+#pragma unroll 1
+  for (int t = 0; t < 7; ++t) {
+    const int c = (int)c0 + (t == 0 ? 1 : -t);
+    if (c < 1 || c > 0x7E) continue;
+    const float e = nvfp4_block_sq_error(v, e4m3_to_f32((uint32_t)c), g);
+    if (e < best_e) {
+      best_e = e;
+      best = (uint32_t)c;
+    }
+  }
+  const float den = __fmul_rn(e4m3_to_f32(best), g);
+  codes[0] = codes[1] = 0u;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t c = den > 0.f ? e2m1_code(__fdiv_rn(v[i], den)) : ((__float_as_uint(v[i]) >> 28) & 8u);
+    codes[i >> 3] |= c << (4 * (i & 7));
+  }
+  return best;
+}
+
 // Eight E2M1 codes (element 2i in the low nibble) of v[i] * rcp, rounded to nearest even and
 // saturated by the hardware conversion.
 __device__ __forceinline__ uint32_t e2m1x8_scaled(const float* v, float rcp) {
@@ -185,11 +236,11 @@ __global__ void amax_groups_kernel(const __nv_bfloat16* __restrict__ w, long lon
 
 // ------------------------------------------------------------------------------------------------
 // Weight quantiser: one thread per 16-element block.  Writes codes [rows, K/2], scales into atoms,
-// and (thread 0 of each group) the group's fp32 tensor scale.
+// and (thread 0 of each group) the group's fp32 tensor scale.  mse: block scales by nvfp4_block_mse.
 // ------------------------------------------------------------------------------------------------
 __global__ void quant_weight_kernel(const __nv_bfloat16* __restrict__ w, long long rows, int K, long long rows_per_group,
                                    const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes,
-                                   uint8_t* __restrict__ sf_atoms, float* __restrict__ g_out) {
+                                   uint8_t* __restrict__ sf_atoms, float* __restrict__ g_out, int mse) {
   const int nb = K / 16;
   const long long total = rows * nb;
   const int atoms_k = sf_atoms_k(K);
@@ -213,7 +264,7 @@ __global__ void quant_weight_kernel(const __nv_bfloat16* __restrict__ w, long lo
       }
     }
     uint32_t c[2];
-    const uint32_t sb = nvfp4_block(v, g, c);
+    const uint32_t sb = mse ? nvfp4_block_mse(v, g, c) : nvfp4_block(v, g, c);
     *reinterpret_cast<uint2*>(codes + r * (K / 2) + kb * 8) = make_uint2(c[0], c[1]);
     sf_atoms[sf_atom_offset(r, kb, atoms_k)] = (uint8_t)sb;
     if (kb == 0 && r % rows_per_group == 0) g_out[grp] = g;

@@ -17,9 +17,10 @@ Scale rules (all decisions in float32, the precision the kernels use):
   element        q   = E2M1_rne_sat( v / (s * g) )  (s decoded back to float32 first; s == 0
                                                     gives q = 0)
   dequantised    v'  = q * s * g                     (exact)
-Weights (W1_e, W2_e, W_s1, W_s2) get one g per matrix per expert.  Activations: x and h get a
-dynamic g from the amax of the whole call's tensor; u and u_s (produced inside a GEMM epilogue,
-before any tensor-wide amax exists) use the static g = 1.
+Weights (W1_e, W2_e, W_s1, W_s2) get one g per matrix per expert; optionally (quantize_mse) a
+weight block's scale is searched around s for the smallest squared reconstruction error.
+Activations: x and h get a dynamic g from the amax of the whole call's tensor; u and u_s (produced
+inside a GEMM epilogue, before any tensor-wide amax exists) use the static g = 1.
 """
 from __future__ import annotations
 
@@ -31,7 +32,8 @@ from . import lmoe_oracle as lo
 
 __all__ = [
     "E2M1_VALUES", "e2m1_encode", "e2m1_decode", "e4m3_encode", "e4m3_decode", "tensor_scale",
-    "quantize", "dequantize", "qdq", "bf16_round", "forward_nvfp4",
+    "quantize", "quantize_mse", "mse_candidates", "block_sq_error", "dequantize", "qdq", "bf16_round",
+    "forward_nvfp4",
 ]
 
 E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
@@ -130,6 +132,85 @@ def quantize(a: np.ndarray, g: Optional[np.float32] = None):
     return codes, s_b, g
 
 
+MSE_DOWN = 6   # candidate block scales below the amax-derived one
+MSE_UP = 1     # candidate block scales above it
+
+
+def mse_candidates(c0: int):
+    """E4M3 codes tried for a block whose amax-derived scale code is c0, in evaluation order:
+    c0 first, then c0 + 1, then c0 - 1 ... c0 - 6, kept inside the positive finite codes 1..0x7E
+    (code 0 is tried only as c0 itself)."""
+    out = [c0]
+    for c in [c0 + k for k in range(1, MSE_UP + 1)] + [c0 - k for k in range(1, MSE_DOWN + 1)]:
+        if 1 <= c <= 0x7E and c not in out:
+            out.append(c)
+    return out
+
+
+def block_sq_error(blk: np.ndarray, s_code: int, g: np.float32) -> np.float32:
+    """Sum of squared reconstruction errors of one 16-element block (float32 values) under E4M3
+    block scale code s_code, every operation in float32 in element order:
+        den = s * g;  q_i = E2M1(v_i / den);  d_i = (q_i * s) * g;  e_i = v_i - d_i;  acc += e_i * e_i."""
+    s = F32(e4m3_decode(np.array([s_code], np.uint8))[0])
+    den = F32(s * F32(g))
+    blk = np.asarray(blk, np.float32)
+    if den > 0:
+        q = e2m1_decode(e2m1_encode((blk / den).astype(np.float32))).astype(np.float32)
+    else:
+        q = np.zeros_like(blk)
+    d = ((q * s).astype(np.float32) * F32(g)).astype(np.float32)
+    e = (blk - d).astype(np.float32)
+    acc = F32(0)
+    for i in range(blk.shape[0]):
+        acc = F32(acc + F32(e[i] * e[i]))
+    return acc
+
+
+def quantize_mse(a: np.ndarray, g: Optional[np.float32] = None):
+    """Like quantize(), with each block's E4M3 scale chosen by a small search ("Nemotron 3 Super"
+    notes, section 4.2, name a per-block-MSE weight quantiser without defining it; this library's
+    reading): among mse_candidates(c0) of the amax-derived scale c0, the first one (in that order)
+    with the strictly smallest block_sq_error.  Codes are then quantize()'s rule with that scale."""
+    a = np.asarray(a, dtype=np.float32)
+    rows, cols = a.shape
+    if cols % BLOCK:
+        raise ValueError("reduction dimension must be a multiple of 16")
+    _, s0, g = quantize(a, g)
+    blk = a.reshape(rows, cols // BLOCK, BLOCK)
+    # block_sq_error for every block at once, one candidate offset at a time (same float32 steps
+    # and element order; offsets in mse_candidates' order, so the first strict minimum wins)
+    c0 = s0.astype(np.int64)
+    best_c = c0.copy()
+    best_e = None
+    for k in [0] + list(range(1, MSE_UP + 1)) + [-j for j in range(1, MSE_DOWN + 1)]:
+        c = c0 + k
+        valid = np.ones_like(c, dtype=bool) if k == 0 else (c >= 1) & (c <= 0x7E)
+        cc = np.clip(c, 0, 0x7E).astype(np.uint8)
+        s = e4m3_decode(cc).astype(np.float32)
+        den = (s * g).astype(np.float32)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            r_ = np.where(den[..., None] > 0, blk / den[..., None], F32(0)).astype(np.float32)
+        q = np.where(den[..., None] > 0, e2m1_decode(e2m1_encode(r_)), 0.0).astype(np.float32)
+        d = ((q * s[..., None]).astype(np.float32) * g).astype(np.float32)
+        e = (blk - d).astype(np.float32)
+        acc = np.zeros(c0.shape, np.float32)
+        for i in range(BLOCK):
+            acc = (acc + (e[..., i] * e[..., i]).astype(np.float32)).astype(np.float32)
+        if best_e is None:
+            best_e = acc
+            continue
+        better = valid & (acc < best_e)
+        best_c = np.where(better, c, best_c)
+        best_e = np.where(better, acc, best_e)
+    s_b = best_c.astype(np.uint8)
+    s_dec = e4m3_decode(s_b).astype(np.float32)
+    den = (s_dec * g).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r_ = np.where(den[..., None] > 0, blk / den[..., None], F32(0)).astype(np.float32)
+    r_ = np.where(den[..., None] > 0, r_, np.copysign(F32(0), blk)).astype(np.float32)
+    return e2m1_encode(r_).reshape(rows, cols), s_b, g
+
+
 def dequantize(codes: np.ndarray, scales: np.ndarray, g) -> np.ndarray:
     rows, cols = codes.shape
     v = e2m1_decode(codes).reshape(rows, cols // BLOCK, BLOCK)
@@ -145,14 +226,14 @@ def bf16_round(a: np.ndarray) -> np.ndarray:
     return u.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
-def qdq(a: np.ndarray, g: Optional[np.float32] = None) -> np.ndarray:
-    """Quantise then dequantise (float64 result)."""
-    c, s, gg = quantize(a, g)
+def qdq(a: np.ndarray, g: Optional[np.float32] = None, quantizer=None) -> np.ndarray:
+    """Quantise (quantize(), or the given quantizer) then dequantise (float64 result)."""
+    c, s, gg = (quantizer or quantize)(a, g)
     return dequantize(c, s, gg)
 
 
 def forward_nvfp4(w: "lo.OracleWeights", x: np.ndarray, k: int, idx: Optional[np.ndarray] = None,
-                  g_x: Optional[np.float32] = None, g_h: Optional[np.float32] = None):
+                  g_x: Optional[np.float32] = None, g_h: Optional[np.float32] = None, weight_quantize=None):
     """Layer forward with NVFP4 routed and shared experts (weights and activations); router,
     W_down and W_up stay at the device's bf16 values.
 
@@ -160,7 +241,9 @@ def forward_nvfp4(w: "lo.OracleWeights", x: np.ndarray, k: int, idx: Optional[np
     rounded to bf16 (nearest even) before it is quantised for the experts.
 
     g_x / g_h: per-call activation scales.  They depend on the whole call's x / h, so a caller that
-    evaluates a sample of tokens passes the full batch's values."""
+    evaluates a sample of tokens passes the full batch's values.
+    weight_quantize: the weights' quantiser (quantize, the default, or quantize_mse)."""
+    wq = weight_quantize or quantize
     logits = lo.router_logits(x, w.w_router, w.b_router)
     if idx is None:
         idx = lo.topk(logits, k)
@@ -178,13 +261,13 @@ def forward_nvfp4(w: "lo.OracleWeights", x: np.ndarray, k: int, idx: Optional[np
         tt, kk = np.nonzero(idx == e)
         if tt.size == 0:
             continue
-        w1 = qdq(w.w1(e).astype(np.float32))
-        w2 = qdq(w.w2(e).astype(np.float32))
+        w1 = qdq(w.w1(e).astype(np.float32), quantizer=wq)
+        w2 = qdq(w.w2(e).astype(np.float32), quantizer=wq)
         u = lo.sqrelu(hq[tt] @ w1.T)
         o = qdq(u.astype(np.float32), one) @ w2.T
         z[tt] += gate[tt, kk][:, None] * o
-    ws1 = qdq(w.ws1.astype(np.float32))
-    ws2 = qdq(w.ws2.astype(np.float32))
+    ws1 = qdq(w.ws1.astype(np.float32), quantizer=wq)
+    ws2 = qdq(w.ws2.astype(np.float32), quantizer=wq)
     us = lo.sqrelu(xq @ ws1.T)
     s = qdq(us.astype(np.float32), one) @ ws2.T
     y = z @ w.w_up.T + s

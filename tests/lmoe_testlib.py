@@ -39,10 +39,11 @@ def device_weights(w: inp.LayerWeights) -> dict:
     return d
 
 
-def make_layer(wl: inp.Workload, w: inp.LayerWeights, dev: dict, max_tokens: int, router_bias=None):
+def make_layer(wl: inp.Workload, w: inp.LayerWeights, dev: dict, max_tokens: int, router_bias=None,
+               weight_scale: str = "amax"):
     import latentmoe_expert_layer_b200 as lm
     rb = wl.router_bias if router_bias is None else router_bias
-    layer = lm.LatentMoE(wl.shape, max_tokens, precision=wl.precision, router_bias=rb)
+    layer = lm.LatentMoE(wl.shape, max_tokens, precision=wl.precision, router_bias=rb, weight_scale=weight_scale)
     b = None
     if rb:
         b = to_dev(inp.skewed_router_bias(), "f32")

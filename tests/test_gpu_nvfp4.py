@@ -89,3 +89,58 @@ def test_nvfp4_prefill_sampled_parity(super4):
     wl = inp.workload("prefill_nvfp4")
     rel = _compare_nvfp4(layer, w, inp.make_x(wl), wl.shape.top_k, tokens=[0, 9000, wl.tokens - 1])
     print(f"nvfp4 prefill: max|err|/RMS {rel:.3g}")
+
+
+# ------------------------------------------------------------------------------------------------
+# per-block MSE weight scales (lmoe_config.weight_scale = LMOE_WSCALE_MSE)
+# ------------------------------------------------------------------------------------------------
+@pytest.fixture(scope="module")
+def tiny4_mse():
+    wl = inp.workload("nvfp4_tiny")
+    w = host_weights("nvfp4_tiny")
+    layer = make_layer(wl, w, device_weights(w), inp.workload("nvfp4_mid").tokens, weight_scale="mse")
+    yield wl, w, layer
+    layer.close()
+
+
+def test_nvfp4_mse_weight_bytes_small(tiny4_mse):
+    wl, w, layer = tiny4_mse
+    for e in range(wl.shape.n_experts):
+        check_weight_bytes(layer, w, 0, e, quantize=nv.quantize_mse)
+        check_weight_bytes(layer, w, 1, e, quantize=nv.quantize_mse)
+    check_weight_bytes(layer, w, 2, 0, quantize=nv.quantize_mse)
+    check_weight_bytes(layer, w, 3, 0, quantize=nv.quantize_mse)
+
+
+def test_nvfp4_mse_parity_small(tiny4_mse):
+    wl, w, layer = tiny4_mse
+    compare_nvfp4(layer, w, inp.make_x(wl), wl.shape.top_k, weight_quantize=nv.quantize_mse)
+    mid = inp.workload("nvfp4_mid")
+    compare_nvfp4(layer, w, inp.make_x(mid), mid.shape.top_k, weight_quantize=nv.quantize_mse)
+
+
+def test_nvfp4_mse_lowers_weight_error_small(tiny4_mse):
+    """The searched scales reconstruct the weights more closely than the amax rule."""
+    _, w, layer = tiny4_mse
+    src = inp.bf16_bits_to_f32(w.w1[0])
+    codes, scales, g = layer.export_nvfp4(0, 0)
+    full = np.empty((codes.shape[0], codes.shape[1] * 2), np.uint8)
+    full[:, 0::2], full[:, 1::2] = codes & 15, codes >> 4
+    e_mse = ((nv.dequantize(full, scales, g) - src) ** 2).sum()
+    e_amax = ((nv.qdq(src) - src) ** 2).sum()
+    assert e_mse < e_amax
+
+
+def test_nvfp4_mse_super_sampled(super4):
+    wl, w, _ = super4
+    layer = make_layer(wl, w, device_weights(w), wl.tokens, weight_scale="mse")
+    try:
+        for e in (0, 511):
+            check_weight_bytes(layer, w, 0, e, quantize=nv.quantize_mse)
+            check_weight_bytes(layer, w, 1, e, quantize=nv.quantize_mse)
+        rel = compare_nvfp4(layer, w, inp.make_x(wl), wl.shape.top_k, tokens=[255],
+                            weight_quantize=nv.quantize_mse)
+        print(f"nvfp4 mse decode: max|err|/RMS {rel:.3g}")
+    finally:
+        layer.close()
+        torch.cuda.empty_cache()

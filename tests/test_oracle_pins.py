@@ -409,6 +409,109 @@ def test_qdq_idempotent_and_error_bound():
 
 
 # ------------------------------------------------------------------------------------------------
+# per-block MSE weight scales
+# ------------------------------------------------------------------------------------------------
+_E2M1_GRID = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def _e4m3_value(code):
+    """E4M3 value from its bit fields (bias 7; exponent field 0 is subnormal), written out here."""
+    e, m = code >> 3, code & 7
+    return m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7)
+
+
+def _e2m1_round(r):
+    """Nearest E2M1 magnitude to |r| (ties to the even index, above 6 saturates), by scanning."""
+    a = min(abs(r), 6.0)
+    best = None
+    for i, gv in enumerate(_E2M1_GRID):
+        dist = abs(a - gv)
+        if best is None or dist < best[0] or (dist == best[0] and i % 2 == 0):
+            best = (dist, i, gv)
+    return math.copysign(best[2], r)
+
+
+def _bruteforce_choice(blk, g):
+    """Scale code with the smallest float64 squared error over the window c0+1, c0, c0-1..c0-6,
+    plus every candidate's error (quotients v / (s*g) taken in float32 as the method defines)."""
+    g32 = np.float32(g)
+    c0 = int(nv.e4m3_encode(np.array([np.float32(np.max(np.abs(blk)) / np.float32(6 * g32))]))[0])
+    errs = {}
+    for c in range(max(c0 - 6, 1 if c0 > 0 else 0), min(c0 + 1, 0x7E) + 1):
+        s = _e4m3_value(c)
+        den = np.float32(np.float32(s) * g32)
+        q = [_e2m1_round(float(np.float32(np.float32(v) / den))) if den > 0 else 0.0 for v in blk]
+        errs[c] = sum((float(v) - qi * s * float(g32)) ** 2 for v, qi in zip(blk, q))
+    return min(errs, key=lambda c: (errs[c], c != c0)), errs
+
+
+def test_mse_choice_matches_bruteforce_argmin():
+    rng = np.random.default_rng(31)
+    # heavy tails make clipping the block's largest element worthwhile in some blocks
+    a = (rng.standard_t(3, size=(24, 256)) * 0.02).astype(np.float32)
+    g = nv.tensor_scale(a)
+    _, sb, _ = nv.quantize_mse(a, g)
+    blk = a.reshape(24, 16, 16)
+    changed = close = 0
+    for r in range(24):
+        for b in range(16):
+            c, errs = _bruteforce_choice(blk[r, b], g)
+            got = int(sb[r, b])
+            if got != c:
+                # only where the float32 and float64 error sums order two candidates differently
+                assert abs(errs[got] - errs[c]) <= 1e-5 * max(errs[c], 1e-30), (r, b, got, c, errs)
+                close += 1
+            changed += got != nv.quantize(blk[r, b][None, :], g)[1][0, 0]
+    assert changed > 0 and close <= 2
+
+
+def test_mse_hand_block_prefers_a_smaller_scale():
+    # g = 1.  Squared block errors by hand: s = 1.125: 0.5625 + 15 * 0.015625 = 0.796875;
+    # s = 1 (the amax rule; the fifteen 1.25 ties round to 1): 15 * 0.0625 = 0.9375;
+    # s = 0.9375: 6 saturates to 5.625 and 1.25 / 0.9375 = 1.33 goes to 1.5 (1.40625):
+    #   0.140625 + 15 * 0.0244140625 = 0.5068359375;  s = 0.875: 0.5625 + 15 * 0.00390625 = 0.62109375;
+    # smaller scales clip the 6 harder.
+    blk = np.array([[6.0] + [1.25] * 15], np.float32)
+    c_amax = int(nv.quantize(blk, np.float32(1))[1][0, 0])
+    codes, sb, _ = nv.quantize_mse(blk, np.float32(1))
+    assert _e4m3_value(c_amax) == 1.0 and _e4m3_value(int(sb[0, 0])) == 0.9375
+    deq = nv.dequantize(codes, sb, np.float32(1))
+    assert ((deq - blk) ** 2).sum() == 0.5068359375
+
+
+def test_mse_keeps_exactly_representable_blocks():
+    rng = np.random.default_rng(32)
+    g = np.float32(2.0 ** -7)                           # a power of two keeps q * s * g exact
+    for code in (0x08, 0x30, 0x38, 0x50, 0x7E):
+        s = _e4m3_value(code)
+        vals = rng.choice(_E2M1_GRID, size=16) * rng.choice([-1.0, 1.0], size=16)
+        vals[0] = 6.0                                   # the block amax pins the amax scale to s
+        blk = (vals * s * float(g)).astype(np.float32)[None, :]
+        codes, sb, _ = nv.quantize_mse(blk, g)
+        assert int(sb[0, 0]) == int(nv.quantize(blk, g)[1][0, 0])
+        assert np.array_equal(nv.dequantize(codes, sb, g), blk.astype(np.float64))
+
+
+def test_mse_candidate_window_edges():
+    assert nv.mse_candidates(0x38) == [0x38, 0x39, 0x37, 0x36, 0x35, 0x34, 0x33, 0x32]
+    assert nv.mse_candidates(0x7E) == [0x7E, 0x7D, 0x7C, 0x7B, 0x7A, 0x79, 0x78]
+    assert nv.mse_candidates(3) == [3, 4, 2, 1]
+    assert nv.mse_candidates(0) == [0, 1]
+
+
+def test_mse_never_worse_than_amax_and_lower_on_average():
+    rng = np.random.default_rng(33)
+    a = (rng.standard_normal((64, 512)) / math.sqrt(512)).astype(np.float32)
+    g = nv.tensor_scale(a)
+    c0, s0, _ = nv.quantize(a, g)
+    c1, s1, _ = nv.quantize_mse(a, g)
+    e0 = ((nv.dequantize(c0, s0, g) - a) ** 2).reshape(64, 32, 16).sum(-1)
+    e1 = ((nv.dequantize(c1, s1, g) - a) ** 2).reshape(64, 32, 16).sum(-1)
+    assert np.all(e1 <= e0 * (1 + 1e-6) + 1e-30)
+    assert e1.sum() < 0.9 * e0.sum()
+
+
+# ------------------------------------------------------------------------------------------------
 # shapes and workloads
 # ------------------------------------------------------------------------------------------------
 def test_super_shape_matches_architecture_table():
