@@ -35,7 +35,8 @@ METRIC = "LatentMoE layer tokens/s (Super shape, T=256 & 16K); % of HBM / TC roo
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DEFAULT_STEPS = {"tiny": 200, "decode": 400, "skewed": 40, "prefill": 20}
 DEFAULT_STEPS.update({"decode_small": 400, "decode_nvfp4": 400, "prefill_nvfp4": 20, "nvfp4_tiny": 200,
-                      "nvfp4_mid": 100, "ultra_decode": 200, "ultra_decode_nvfp4": 200, "ultra_prefill": 10})
+                      "nvfp4_mid": 100, "ultra_decode": 200, "ultra_decode_nvfp4": 200, "ultra_prefill": 10,
+                      "standard_decode": 400, "standard_prefill": 20})
 
 
 def peaks():
@@ -106,16 +107,17 @@ def algorithmic_work(wl, counts: np.ndarray):
     E4M3 scale byte per 16 elements (router, W_down and W_up stay bf16 in the NVFP4 variant)."""
     s = wl.shape
     d, l, n, k, m, ms = s.d, s.latent, s.n_experts, s.top_k, s.expert_ffn, s.shared_ffn
+    le = s.expert_in        # the experts' input width: l, or d for a standard MoE (l = 0)
     t = wl.tokens
     tk = t * k
     touched = int((counts > 0).sum())
     fp4 = wl.precision == "nvfp4"
     eb = (lambda elems: elems * 0.5 + elems / 16) if fp4 else (lambda elems: elems * 2)
-    w_exp = touched * eb(m * l)                     # one expert matrix set (W1 or W2) of the touched experts
-    up = {"bytes": w_exp + eb(tk * l) + eb(tk * m), "flops": 2 * tk * m * l}
-    down = {"bytes": w_exp + eb(tk * m) + tk * l * 2 + tk * 4, "flops": 2 * tk * m * l}
+    w_exp = touched * eb(m * le)                    # one expert matrix set (W1 or W2) of the touched experts
+    up = {"bytes": w_exp + eb(tk * le) + eb(tk * m), "flops": 2 * tk * m * le}
+    down = {"bytes": w_exp + eb(tk * m) + tk * le * 2 + tk * 4, "flops": 2 * tk * m * le}
     layer_bytes = (2 * w_exp + (n + l) * d * 2 + eb(ms * d) + eb(d * ms) + d * l * 2 + 2 * t * d * 2 + tk * 8)
-    layer_flops = 2 * t * ((n + l) * d + ms * d + d * (l + ms)) + 4 * tk * m * l
+    layer_flops = 2 * t * ((n + l) * d + ms * d + d * (l + ms)) + 4 * tk * m * le
     return {"expert_up": up, "expert_down": down, "layer": {"bytes": int(layer_bytes), "flops": layer_flops},
             "touched_experts": touched, "expert_weight_bytes": int(2 * w_exp)}
 
@@ -128,6 +130,8 @@ def make_device_layer(wl, device):
     to = lambda a: (torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
                     if w.dtype == "bf16" else torch.from_numpy(np.ascontiguousarray(a))).to(device)
     dev = {k: to(getattr(w, k)) for k in ("w_router", "w_down", "w_up", "w1", "w2", "ws1", "ws2")}
+    if wl.shape.latent == 0:          # a standard MoE has no projections
+        dev["w_down"] = dev["w_up"] = None
     b = torch.from_numpy(w.b_router).to(device) if w.b_router is not None else None
     layer = lm.LatentMoE(wl.shape, wl.tokens, precision=wl.precision, router_bias=wl.router_bias,
                          device=device.index)

@@ -53,7 +53,10 @@ typedef enum { LMOE_DTYPE_BF16 = 0, LMOE_DTYPE_F32 = 1 } lmoe_dtype;
 
 typedef struct {
   int32_t d;           /* model dimension (multiple of 64) */
-  int32_t latent;      /* latent dimension l (multiple of 64) */
+  int32_t latent;      /* latent dimension l (multiple of 64), or 0 for the standard MoE that LatentMoE
+                          replaces ("Nemotron 3 Super" notes, section 3.2): experts d -> m -> d on x
+                          itself, no W_down / W_up, y = sum_k g_k W2 sqrelu(W1 x) + shared expert
+                          (bf16 precision only) */
   int32_t n_experts;   /* N, a multiple of 16, at most 1024 */
   int32_t top_k;       /* K, 1..min(32, N) */
   int32_t expert_ffn;  /* m, routed expert hidden (multiple of 64) */
@@ -80,10 +83,10 @@ typedef enum { LMOE_WSCALE_AMAX = 0, LMOE_WSCALE_MSE = 1 } lmoe_weight_scale;
 typedef struct {
   const void* w_router;  /* [N, d] */
   const float* b_router; /* [N] fp32, or NULL (required iff has_router_bias) */
-  const void* w_down;    /* [l, d]   (W_down) */
-  const void* w_up;      /* [d, l]   (W_up) */
-  const void* w1;        /* [N, m, l] expert up matrices */
-  const void* w2;        /* [N, l, m] expert down matrices */
+  const void* w_down;    /* [l, d]   (W_down); NULL for a standard MoE (latent == 0), else required */
+  const void* w_up;      /* [d, l]   (W_up); NULL for a standard MoE, else required */
+  const void* w1;        /* [N, m, l] expert up matrices ([N, m, d] for a standard MoE) */
+  const void* w2;        /* [N, l, m] expert down matrices ([N, d, m] for a standard MoE) */
   const void* ws1;       /* [m_s, d] shared expert */
   const void* ws2;       /* [d, m_s] shared expert */
   int32_t dtype;         /* lmoe_dtype */
@@ -138,7 +141,7 @@ typedef enum {
   LMOE_BUF_OFFSETS = 2,    /* int32 [N+1]   exclusive prefix sum of counts */
   LMOE_BUF_ROW_OF = 3,     /* int32 [T*K]   grouped row of assignment (t, k) */
   LMOE_BUF_TOK_OF_ROW = 4, /* int32 [T*K]   token of grouped row r */
-  LMOE_BUF_H = 5,          /* bf16 [T, l]   latent h = W_down x */
+  LMOE_BUF_H = 5,          /* bf16 [T, l]   latent h = W_down x (UNSUPPORTED for a standard MoE) */
   LMOE_BUF_Z = 6,          /* bf16 [T, l + m_s] columns 0..l-1: latent sum z; the rest: sqrelu(W_s1 x) */
   LMOE_BUF_U = 7,          /* bf16 [T*K, m] expert hidden activations, grouped rows (bf16 precision) */
   /* NVFP4 precision only: packed E2M1 codes [rows, K/2] and row-major E4M3 scales

@@ -142,8 +142,9 @@ class LatentMoE:
         self.device = torch.device("cuda", device)
 
     def load_weights(self, w_router, w_down, w_up, w1, w2, ws1, ws2, b_router=None, stream=None) -> None:
+        # a standard MoE (latent == 0) passes w_down = w_up = None
         ts = (w_router, w_down, w_up, w1, w2, ws1, ws2)
-        dt = {t.dtype for t in ts}
+        dt = {t.dtype for t in ts if t is not None}
         if len(dt) != 1 or next(iter(dt)) not in DTYPE:
             raise ValueError("all weight matrices must share one dtype, bf16 or fp32")
         w = _Weights(_ptr(w_router), _ptr(b_router), _ptr(w_down), _ptr(w_up), _ptr(w1), _ptr(w2), _ptr(ws1),

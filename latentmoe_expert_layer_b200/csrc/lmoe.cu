@@ -92,6 +92,8 @@ struct lmoe_ctx {
   bool loaded = false;
   bool router_f32 = false;
   bool fused_router = false;
+  bool standard = false;  // latent == 0: a standard MoE, experts d -> m -> d, no W_down / W_up
+  int le = 0;             // width the routed experts work in: latent, or d for a standard MoE
   unsigned long long timeout_ns = kDefaultTimeoutNs;
 
   // weights (library-owned)
@@ -529,9 +531,10 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   if (!cfg || !out) return LMOE_ERR_INVALID_ARG;
   *out = nullptr;
   const lmoe_config& g = *cfg;
-  if (g.d <= 0 || g.latent <= 0 || g.n_experts <= 0 || g.top_k <= 0 || g.expert_ffn <= 0 || g.shared_ffn <= 0 ||
+  if (g.d <= 0 || g.latent < 0 || g.n_experts <= 0 || g.top_k <= 0 || g.expert_ffn <= 0 || g.shared_ffn <= 0 ||
       g.max_tokens <= 0)
     return LMOE_ERR_INVALID_ARG;
+  if (g.latent == 0 && g.precision != LMOE_PREC_BF16) return LMOE_ERR_UNSUPPORTED;
   if (g.precision != LMOE_PREC_BF16 && g.precision != LMOE_PREC_NVFP4) return LMOE_ERR_INVALID_ARG;
   if (g.weight_scale != LMOE_WSCALE_AMAX && g.weight_scale != LMOE_WSCALE_MSE) return LMOE_ERR_INVALID_ARG;
   if (g.d % 64 || g.latent % 64 || g.expert_ffn % 64 || g.shared_ffn % 64) return LMOE_ERR_UNSUPPORTED;
@@ -554,7 +557,10 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   c->num_sms = prop.multiProcessorCount;
   const int N = g.n_experts, K = g.top_k, d = g.d, l = g.latent, m = g.expert_ffn, ms = g.shared_ffn;
   const long long T = g.max_tokens;
-  const int nft1 = (m + BLOCK_M - 1) / BLOCK_M, nft2 = (l + BLOCK_M - 1) / BLOCK_M;
+  c->standard = l == 0;
+  const int le = c->standard ? d : l;
+  c->le = le;
+  const int nft1 = (m + BLOCK_M - 1) / BLOCK_M, nft2 = (le + BLOCK_M - 1) / BLOCK_M;
   c->max_units1 = (int)(nft1 * (N + (tk + V_BN[V_SMALL] - 1) / V_BN[V_SMALL]));
   c->max_units2 = (int)(nft2 * (N + (tk + V_BN[V_SMALL] - 1) / V_BN[V_SMALL]));
   bool ok = true;
@@ -562,13 +568,14 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   ok = ok && dalloc(&c->chunk_counts, 128LL * N) && dalloc(&c->chunk_base, 128LL * N);
   ok = ok && dalloc(&c->counts, N) && dalloc(&c->offsets, N + 1);
   ok = ok && dalloc(&c->row_of, tk) && dalloc(&c->tok_of_row, tk) && dalloc(&c->gate_of_row, tk);
-  ok = ok && dalloc(&c->h, T * l) && dalloc(&c->h_perm, tk * l) && dalloc(&c->u, tk * m) && dalloc(&c->o, tk * l);
+  if (!c->standard) ok = ok && dalloc(&c->h, T * l);
+  ok = ok && dalloc(&c->h_perm, tk * le) && dalloc(&c->u, tk * m) && dalloc(&c->o, tk * le);
   ok = ok && dalloc(&c->zu, T * (l + ms));
   ok = ok && dalloc(&c->units1, c->max_units1) && dalloc(&c->units2, c->max_units2) && dalloc(&c->num_units, 2);
   ok = ok && dalloc(&c->status, 1) && dalloc(&c->work_counters, lmoe_ctx::kCounters);
   c->nvfp4 = g.precision == LMOE_PREC_NVFP4;
-  // y_s = W_s2 u_s in fp32: needed at decode sizes (bf16) and at every size (NVFP4)
-  ok = ok && dalloc(&c->y_s, (size_t)(c->nvfp4 ? T : (T < 512 ? T : 512)) * d);
+  // y_s = W_s2 u_s in fp32: needed at decode sizes (bf16) and at every size (NVFP4, standard MoE)
+  ok = ok && dalloc(&c->y_s, (size_t)(c->nvfp4 || c->standard ? T : (T < 512 ? T : 512)) * d);
   if (c->nvfp4) {
     ok = ok && dalloc(&c->xq, T * d / 2) && dalloc(&c->x_sf, c->sf_bytes_dense(d));
     ok = ok && dalloc(&c->hq, tk * l / 2) && dalloc(&c->h_sf, c->sf_bytes_grouped(l));
@@ -583,14 +590,14 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   }
   cudaMemset(c->status, 0, sizeof(unsigned));
   // rows that no expert writes must still be finite for the MMA (they are masked in the epilogue)
-  cudaMemset(c->h_perm, 0, tk * l * 2);
+  cudaMemset(c->h_perm, 0, tk * le * 2);
   cudaMemset(c->u, 0, tk * m * 2);
   cudaMemset(c->zu, 0, T * (l + ms) * 2);
   for (int v = 0; v < 2; ++v) {
-    ok = ok && make_map(&c->map_hperm[v], c->h_perm, tk, l, l, V_BOXN[v]);
+    ok = ok && make_map(&c->map_hperm[v], c->h_perm, tk, le, le, V_BOXN[v]);
     ok = ok && make_map(&c->map_u[v], c->u, tk, m, m, V_BOXN[v]);
     ok = ok && make_map(&c->map_zu[v], c->zu, T, l + ms, l + ms, V_BOXN[v]);
-    ok = ok && make_map(&c->map_z[v], c->zu, T, l, l + ms, V_BOXN[v]);
+    if (!c->standard) ok = ok && make_map(&c->map_z[v], c->zu, T, l, l + ms, V_BOXN[v]);
     ok = ok && make_map(&c->map_us[v], c->zu + l, T, ms, l + ms, V_BOXN[v]);
   }
   ok = ok && cudaFuncSetAttribute(VT<V_SMALL>::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -634,16 +641,19 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
 
 lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream) {
   if (!c || !w) return LMOE_ERR_INVALID_ARG;
-  if (!w->w_router || !w->w_down || !w->w_up || !w->w1 || !w->w2 || !w->ws1 || !w->ws2) return LMOE_ERR_INVALID_ARG;
+  if (!w->w_router || !w->w1 || !w->w2 || !w->ws1 || !w->ws2) return LMOE_ERR_INVALID_ARG;
+  // a standard MoE has no projections; a LatentMoE layer needs both
+  if (c->standard ? (w->w_down || w->w_up) : (!w->w_down || !w->w_up)) return LMOE_ERR_INVALID_ARG;
   if (w->dtype != LMOE_DTYPE_BF16 && w->dtype != LMOE_DTYPE_F32) return LMOE_ERR_INVALID_ARG;
   if (c->cfg.has_router_bias && !w->b_router) return LMOE_ERR_INVALID_ARG;
   const void* ptrs[] = {w->w_router, w->w_down, w->w_up, w->w1, w->w2, w->ws1, w->ws2};
   for (const void* p : ptrs)
-    if (!aligned16(p)) return LMOE_ERR_INVALID_ARG;
+    if (p && !aligned16(p)) return LMOE_ERR_INVALID_ARG;
   DeviceGuard dg(c->device);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const lmoe_config& g = c->cfg;
   const int N = g.n_experts, d = g.d, l = g.latent, m = g.expert_ffn, ms = g.shared_ffn;
+  const int le = c->le;
   const int f32 = w->dtype == LMOE_DTYPE_F32;
 
   // release weights of a previous load
@@ -666,7 +676,7 @@ lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream
   c->loaded = false;
 
   c->router_f32 = f32;
-  c->fused_router = !f32 && (N % BLOCK_M == 0);
+  c->fused_router = !f32 && (N % BLOCK_M == 0) && !c->standard;
   bool ok = true;
   auto conv = [&](const void* src, long long rows, int cols, long long src_ld, __nv_bfloat16* dst, long long dst_ld,
                   int col0) {
@@ -679,22 +689,23 @@ lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream
   if (c->router_f32) {
     ok = ok && dalloc(&c->w_r32, (size_t)N * d) &&
          cudaMemcpyAsync(c->w_r32, w->w_router, (size_t)N * d * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
-    ok = ok && dalloc(&c->w_down, (size_t)l * d) && conv(w->w_down, l, d, d, c->w_down, d, 0);
+    if (!c->standard) ok = ok && dalloc(&c->w_down, (size_t)l * d) && conv(w->w_down, l, d, d, c->w_down, d, 0);
   } else if (c->fused_router) {
     ok = ok && dalloc(&c->w_rd, (size_t)(N + l) * d);
     ok = ok && conv(w->w_router, N, d, d, c->w_rd, d, 0) && conv(w->w_down, l, d, d, c->w_rd + (size_t)N * d, d, 0);
   } else {
     ok = ok && dalloc(&c->w_rd, (size_t)N * d) && conv(w->w_router, N, d, d, c->w_rd, d, 0);
-    ok = ok && dalloc(&c->w_down, (size_t)l * d) && conv(w->w_down, l, d, d, c->w_down, d, 0);
+    if (!c->standard) ok = ok && dalloc(&c->w_down, (size_t)l * d) && conv(w->w_down, l, d, d, c->w_down, d, 0);
   }
   if (g.has_router_bias)
     ok = ok && dalloc(&c->b_router, N) &&
          cudaMemcpyAsync(c->b_router, w->b_router, (size_t)N * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
   ok = ok && dalloc(&c->w_cat, (size_t)d * (l + ms));
-  ok = ok && conv(w->w_up, d, l, l, c->w_cat, l + ms, 0) && conv(w->ws2, d, ms, ms, c->w_cat, l + ms, l);
+  if (!c->standard) ok = ok && conv(w->w_up, d, l, l, c->w_cat, l + ms, 0);
+  ok = ok && conv(w->ws2, d, ms, ms, c->w_cat, l + ms, l);
   ok = ok && dalloc(&c->ws1, (size_t)ms * d) && conv(w->ws1, ms, d, d, c->ws1, d, 0);
-  ok = ok && dalloc(&c->w1, (size_t)N * m * l) && conv(w->w1, (long long)N * m, l, l, c->w1, l, 0);
-  ok = ok && dalloc(&c->w2, (size_t)N * l * m) && conv(w->w2, (long long)N * l, m, m, c->w2, m, 0);
+  ok = ok && dalloc(&c->w1, (size_t)N * m * le) && conv(w->w1, (long long)N * m, le, le, c->w1, le, 0);
+  ok = ok && dalloc(&c->w2, (size_t)N * le * m) && conv(w->w2, (long long)N * le, m, m, c->w2, m, 0);
   if (!ok) return LMOE_ERR_OOM;
   if (c->nvfp4) {
     // quantise W1, W2, W_s1, W_s2 on the device; keep only codes, scale atoms and tensor scales
@@ -749,14 +760,14 @@ lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream
   }
   if (c->fused_router) ok = ok && make_map(&c->map_rd, c->w_rd, N + l, d, d, BLOCK_M);
   if (!c->router_f32 && !c->fused_router) ok = ok && make_map(&c->map_r, c->w_rd, N, d, d, BLOCK_M);
-  if (!c->fused_router) ok = ok && make_map(&c->map_down, c->w_down, l, d, d, BLOCK_M);
+  if (!c->fused_router && !c->standard) ok = ok && make_map(&c->map_down, c->w_down, l, d, d, BLOCK_M);
   ok = ok && make_map(&c->map_cat, c->w_cat, d, l + ms, l + ms, BLOCK_M);
-  ok = ok && make_map(&c->map_wup, c->w_cat, d, l, l + ms, BLOCK_M);
+  if (!c->standard) ok = ok && make_map(&c->map_wup, c->w_cat, d, l, l + ms, BLOCK_M);
   ok = ok && make_map(&c->map_ws2, c->w_cat + l, d, ms, l + ms, BLOCK_M);
   if (!c->nvfp4) {
     ok = ok && make_map(&c->map_ws1, c->ws1, ms, d, d, BLOCK_M);
-    ok = ok && make_map(&c->map_w1, c->w1, (uint64_t)N * m, l, l, BLOCK_M);
-    ok = ok && make_map(&c->map_w2, c->w2, (uint64_t)N * l, m, m, BLOCK_M);
+    ok = ok && make_map(&c->map_w1, c->w1, (uint64_t)N * m, le, le, BLOCK_M);
+    ok = ok && make_map(&c->map_w2, c->w2, (uint64_t)N * le, m, m, BLOCK_M);
   }
   if (!ok) return LMOE_ERR_CUDA;
   c->loaded = true;
@@ -776,6 +787,7 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const lmoe_config& g = c->cfg;
   const int N = g.n_experts, K = g.top_k, d = g.d, l = g.latent, m = g.expert_ffn, ms = g.shared_ffn;
+  const int le = c->le;  // expert input / output width: l, or d for a standard MoE
   const long long TK = (long long)T * K;
   const long long TKmax = (long long)g.max_tokens * K;
   const int vd = T <= 512 ? V_SMALL : V_LARGE;
@@ -835,10 +847,13 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
       g.main_dense(c->map_r, c->map_x[vd], problem(d, EPI_F32, c->logits, N), N, T);
       chk(g.run(s));
     }
-    GemmLaunch g(c, vd, 2);
-    g.main_dense(c->map_down, c->map_x[vd], problem(d, EPI_BF16, c->h, l), l, T);
-    chk(g.run(s));
-    launches += 2;
+    launches += 1;
+    if (!c->standard) {
+      GemmLaunch g(c, vd, 2);
+      g.main_dense(c->map_down, c->map_x[vd], problem(d, EPI_BF16, c->h, l), l, T);
+      chk(g.run(s));
+      launches += 1;
+    }
   }
   mark(1);
   // 2. shared expert, first matrix: zu[:, l:] = sqrelu(W_s1 x)   (inside the expert-up launch when split)
@@ -857,7 +872,7 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   mark(3);
   // 4. expert offsets and grouped-GEMM unit lists
   UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1};
-  UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2};
+  UnitListSpec l2{c->units2, c->num_units + 1, le, V_BN[vg], c->max_units2};
   scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(c->chunk_counts, nch, N, c->counts, c->offsets,
                                                               c->chunk_base, l1, l2, nullptr, c->status);
   chk(cudaGetLastError());
@@ -870,7 +885,9 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
     long long warps = (TK + GATHER_ROWS - 1) / GATHER_ROWS;
     long long blocks = (warps + 7) / 8;
     if (blocks > (long long)c->num_sms * 8) blocks = (long long)c->num_sms * 8;
-    gather_rows_kernel<<<(int)blocks, 256, 0, s>>>(c->h, c->tok_of_row, TK, T, l, c->h_perm, c->status);
+    // a standard MoE's experts read x itself
+    const __nv_bfloat16* src = c->standard ? reinterpret_cast<const __nv_bfloat16*>(x) : c->h;
+    gather_rows_kernel<<<(int)blocks, 256, 0, s>>>(src, c->tok_of_row, TK, T, le, c->h_perm, c->status);
     chk(cudaGetLastError());
   }
   mark(5);
@@ -878,7 +895,7 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   {
     GemmLaunch g(c, vg, 4);
     if (split) g.pre_dense(c->map_ws1, c->map_x[vd], shared_up, ms, T);
-    g.main_grouped(c->map_w1, c->map_hperm[vg], problem(l, EPI_SQRELU_BF16, c->u, m), c->units1, c->num_units, m,
+    g.main_grouped(c->map_w1, c->map_hperm[vg], problem(le, EPI_SQRELU_BF16, c->u, m), c->units1, c->num_units, m,
                    0);
     chk(g.run(s));
   }
@@ -887,20 +904,40 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   {
     GemmLaunch g(c, vg, 5);
     if (split) g.pre_dense(c->map_ws2, c->map_us[vd], problem(ms, EPI_F32, c->y_s, d), d, T);
-    GemmProblem p = problem(m, EPI_ROWSCALE_BF16, c->o, l);
+    GemmProblem p = problem(m, EPI_ROWSCALE_BF16, c->o, le);
     p.row_scale = c->gate_of_row;
-    g.main_grouped(c->map_w2, c->map_u[vg], p, c->units2, c->num_units + 1, l, 0);
+    g.main_grouped(c->map_w2, c->map_u[vg], p, c->units2, c->num_units + 1, le, 0);
     chk(g.run(s));
   }
+  if (c->standard && !split) {
+    // a standard MoE adds the shared expert after the combine: y_s = W_s2 u_s (fp32)
+    GemmLaunch g(c, vd, 6);
+    g.main_dense(c->map_ws2, c->map_us[vd], problem(ms, EPI_F32, c->y_s, d), d, T);
+    chk(g.run(s));
+    launches += 1;
+  }
   mark(7);
-  // 8. latent combine: zu[:, :l] = sum_k o[row_of[t, k]]
+  // 8. latent combine: zu[:, :l] = sum_k o[row_of[t, k]]; a standard MoE's combine writes
+  //    y = sum_k o[row_of[t, k]] + y_s and the layer ends here
   {
-    const long long threads = (long long)T * (l / 8);
+    const long long threads = (long long)T * (le / 8);
     const int blocks = (int)((threads + 255) / 256);
-    combine_kernel<<<blocks, 256, 0, s>>>(c->o, c->row_of, T, K, l, c->zu, l + ms, TKmax, c->status);
+    if (c->standard)
+      combine_kernel<<<blocks, 256, 0, s>>>(c->o, c->row_of, T, K, d, reinterpret_cast<__nv_bfloat16*>(y), d, TKmax,
+                                           c->status, c->y_s, d);
+    else
+      combine_kernel<<<blocks, 256, 0, s>>>(c->o, c->row_of, T, K, l, c->zu, l + ms, TKmax, c->status);
     chk(cudaGetLastError());
   }
   mark(8);
+  if (c->standard) {
+    mark(9);
+    launches += 7;
+    c->launches = launches;
+    if (prof) ++c->prof_n;
+    c->last_T = T;
+    return cuda_status(e);
+  }
   // 9. y = [z | sqrelu(W_s1 x)] [W_up | W_s2]^T, or y = W_up z + y_s when split
   {
     GemmLaunch g(c, vd, 6);
@@ -1037,7 +1074,11 @@ lmoe_status lmoe_inspect(lmoe_handle c, int32_t which, void** dev_ptr, int64_t* 
     case LMOE_BUF_OFFSETS: *dev_ptr = c->offsets; *count = g.n_experts + 1; break;
     case LMOE_BUF_ROW_OF: *dev_ptr = c->row_of; *count = TK; break;
     case LMOE_BUF_TOK_OF_ROW: *dev_ptr = c->tok_of_row; *count = TK; break;
-    case LMOE_BUF_H: *dev_ptr = c->h; *count = T * g.latent; break;
+    case LMOE_BUF_H:
+      if (c->standard) return LMOE_ERR_UNSUPPORTED;
+      *dev_ptr = c->h;
+      *count = T * g.latent;
+      break;
     case LMOE_BUF_Z: *dev_ptr = c->zu; *count = T * (g.latent + g.shared_ffn); break;
     case LMOE_BUF_U: *dev_ptr = c->u; *count = TK * g.expert_ffn; break;
     case LMOE_BUF_XQ: *dev_ptr = c->xq; *count = T * g.d / 2; break;

@@ -382,11 +382,12 @@ __global__ void __launch_bounds__(256)
 }
 
 // ------------------------------------------------------------------------------------------------
-// combine: zu[t, 0:latent] = bf16( sum_k o[row_of[t, k], :] ), slot order, fp32 accumulation
+// combine: zu[t, 0:latent] = bf16( sum_k o[row_of[t, k], :] (+ add[t, :]) ), slot order, fp32
+// accumulation; the fp32 addend (a standard MoE's shared-expert output) is added last
 // ------------------------------------------------------------------------------------------------
 __global__ void combine_kernel(const __nv_bfloat16* __restrict__ o, const int* __restrict__ row_of, int T, int k,
                                int latent, __nv_bfloat16* __restrict__ zu, long long ld_zu, long long n_rows,
-                               unsigned* status) {
+                               unsigned* status, const float* __restrict__ add = nullptr, long long ld_add = 0) {
   const int vpr = latent / 8;  // 8 bf16 per thread
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long t = gid / vpr;
@@ -407,6 +408,18 @@ __global__ void combine_kernel(const __nv_bfloat16* __restrict__ o, const int* _
       acc[2 * i] += f.x;
       acc[2 * i + 1] += f.y;
     }
+  }
+  if (add != nullptr) {
+    const float4* pa = reinterpret_cast<const float4*>(add + t * ld_add + v * 8);
+    const float4 a0 = pa[0], a1 = pa[1];
+    acc[0] += a0.x;
+    acc[1] += a0.y;
+    acc[2] += a0.z;
+    acc[3] += a0.w;
+    acc[4] += a1.x;
+    acc[5] += a1.y;
+    acc[6] += a1.z;
+    acc[7] += a1.w;
   }
   uint4 out;
   __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&out);

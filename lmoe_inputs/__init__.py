@@ -28,7 +28,7 @@ from typing import Dict, Optional
 import numpy as np
 
 __all__ = [
-    "LayerShape", "SUPER", "ULTRA", "Workload", "WORKLOADS", "workload", "f32_to_bf16_bits", "bf16_bits_to_f32",
+    "LayerShape", "SUPER", "ULTRA", "STANDARD", "Workload", "WORKLOADS", "workload", "f32_to_bf16_bits", "bf16_bits_to_f32",
     "LayerWeights", "make_weights", "make_router", "make_x", "expert_weight", "skewed_router_bias",
 ]
 
@@ -43,9 +43,14 @@ class LayerShape:
     shared_ffn: int   # m_s (shared expert hidden)
 
     @property
+    def expert_in(self) -> int:
+        """Width the routed experts work in: l, or d for a standard MoE (latent = 0)."""
+        return self.latent if self.latent else self.d
+
+    @property
     def params(self) -> int:
         s = self
-        return (s.n_experts * s.d + 2 * s.latent * s.d + 2 * s.n_experts * s.expert_ffn * s.latent
+        return (s.n_experts * s.d + 2 * s.latent * s.d + 2 * s.n_experts * s.expert_ffn * s.expert_in
                 + 2 * s.d * s.shared_ffn)
 
 
@@ -54,6 +59,10 @@ SUPER = LayerShape(d=4096, latent=1024, n_experts=512, top_k=22, expert_ffn=2688
 # ("Nemotron 3 Ultra" summary, core method).  That page gives neither the model dimension nor the
 # latent dimension, so Super's d = 4096 and l = 1024 are kept.
 ULTRA = LayerShape(d=4096, latent=1024, n_experts=512, top_k=22, expert_ffn=5120, shared_ffn=10240)
+# The standard MoE with the Super layer's budget: LatentMoE turns N, K into N' = N d / l and
+# K' = K d / l ("Nemotron 3 Super" notes, section 3.2), so N = 512 * 1024 / 4096 = 128 experts and
+# K = 22 / 4 = 5.5, rounded to 6; experts d -> m -> d with no W_down / W_up (latent = 0).
+STANDARD = LayerShape(d=4096, latent=0, n_experts=128, top_k=6, expert_ffn=2688, shared_ffn=5376)
 TINY = LayerShape(d=256, latent=64, n_experts=16, top_k=4, expert_ffn=128, shared_ffn=256)
 
 
@@ -97,6 +106,11 @@ WORKLOADS: Dict[str, Workload] = {
                                    description="NVFP4 Ultra-width experts, decode T=256"),
     "ultra_prefill": Workload("ultra_prefill", ULTRA, 16384, 5, 3, "bf16", "bf16",
                               description="Ultra-width experts, prefill T=16384"),
+    "standard_decode": Workload("standard_decode", STANDARD, 256, 6, 2, "bf16", "bf16",
+                                description="standard MoE of the Super budget (N=128, K=6, experts d->m->d, "
+                                            "no W_down/W_up), decode T=256"),
+    "standard_prefill": Workload("standard_prefill", STANDARD, 16384, 6, 3, "bf16", "bf16",
+                                 description="standard MoE of the Super budget, prefill T=16384"),
     "skewed": Workload("skewed", SUPER, 4096, 1, 4, "bf16", "bf16", router_bias=True,
                        description="Super shape T=4096, per-expert router bias giving a capped Zipf(1.2) load"),
 }
@@ -147,9 +161,9 @@ def expert_weight(wl: Workload, which: str, e: int) -> np.ndarray:
     s = wl.shape
     ss = _streams(wl.weight_seed)[which].spawn(s.n_experts)[e]
     if which == "w1":
-        return _finish(_normal(ss, (s.expert_ffn, s.latent), 1.0 / np.sqrt(s.latent)), wl.weight_dtype)
+        return _finish(_normal(ss, (s.expert_ffn, s.expert_in), 1.0 / np.sqrt(s.expert_in)), wl.weight_dtype)
     if which == "w2":
-        return _finish(_normal(ss, (s.latent, s.expert_ffn), 1.0 / np.sqrt(s.expert_ffn)), wl.weight_dtype)
+        return _finish(_normal(ss, (s.expert_in, s.expert_ffn), 1.0 / np.sqrt(s.expert_ffn)), wl.weight_dtype)
     raise ValueError(which)
 
 
@@ -158,10 +172,10 @@ class LayerWeights:
     """All weights of one layer in the device dtype.  bf16 tensors are uint16 bit patterns."""
     w_router: np.ndarray   # [N, d]
     b_router: Optional[np.ndarray]  # [N] float32 or None
-    w_down: np.ndarray     # [l, d]
-    w_up: np.ndarray       # [d, l]
-    w1: np.ndarray         # [N, m, l]
-    w2: np.ndarray         # [N, l, m]
+    w_down: np.ndarray     # [l, d]   ([0, d] for a standard MoE)
+    w_up: np.ndarray       # [d, l]   ([d, 0] for a standard MoE)
+    w1: np.ndarray         # [N, m, l] ([N, m, d] for a standard MoE)
+    w2: np.ndarray         # [N, l, m] ([N, d, m] for a standard MoE)
     ws1: np.ndarray        # [m_s, d]
     ws2: np.ndarray        # [d, m_s]
     dtype: str             # "f32" or "bf16"
@@ -175,13 +189,13 @@ def make_weights(wl: Workload, threads: Optional[int] = None, experts: bool = Tr
     # the router keeps fp32 in the tiny (fp32) workload, bf16 otherwise
     w_router = f("w_router", (s.n_experts, s.d), s.d)
     w_down = f("w_down", (s.latent, s.d), s.d)
-    w_up = f("w_up", (s.d, s.latent), s.latent)
+    w_up = f("w_up", (s.d, s.latent), s.latent) if s.latent else w_down.reshape(s.d, 0)
     ws1 = f("ws1", (s.shared_ffn, s.d), s.d)
     ws2 = f("ws2", (s.d, s.shared_ffn), s.shared_ffn)
     dt = np.float32 if wl.weight_dtype == "f32" else np.uint16
     n = s.n_experts if experts else 0
-    w1 = np.empty((n, s.expert_ffn, s.latent), dtype=dt)
-    w2 = np.empty((n, s.latent, s.expert_ffn), dtype=dt)
+    w1 = np.empty((n, s.expert_ffn, s.expert_in), dtype=dt)
+    w2 = np.empty((n, s.expert_in, s.expert_ffn), dtype=dt)
     if n:
         threads = threads or min(32, os.cpu_count() or 1)
 

@@ -21,6 +21,8 @@ What it computes, per token t (x in R^d), written out plainly:
                                                                          ReLU, non-gated, no bias)
   6. output            y = W_up z + W_s2 sqrelu(W_s1 x),  W_up in R^{d x l} (section 3.2; the shared
                                                                          expert runs in full d)
+  A layer given without W_down and W_up is the standard MoE of the same section: h = x and
+  y = z + W_s2 sqrelu(W_s1 x).
 
 Everything is float64 numpy; weights arrive as the exact values the device consumes (bf16 bit
 patterns or float32) and are lifted losslessly.  Per-expert work loops over experts, lifting one
@@ -148,12 +150,17 @@ def forward(w: OracleWeights, x: np.ndarray, k: int, idx: Optional[np.ndarray] =
     idx    optional forced routing [T, K] (used to re-evaluate tokens whose GPU routing differs at a
            near-tie); gates are then the softmax of the oracle's own logits at those experts.
     Returns dict with y [T, d], idx [T, K], gate [T, K], logits [T, N], h [T, l], z [T, l].
+
+    A layer without W_down / W_up (w.w_down with zero rows) is the standard MoE these replace
+    ("Nemotron 3 Super" notes, section 3.2): the experts run on x itself (d -> m -> d) and
+    y = z + W_s2 sqrelu(W_s1 x).
     """
     logits = router_logits(x, w.w_router, w.b_router)
     if idx is None:
         idx = topk(logits, k)
     gate = softmax_gates(logits, idx)
-    h = x @ w.w_down.T
+    standard = w.w_down.shape[0] == 0
+    h = x if standard else x @ w.w_down.T
     z = np.zeros_like(h)
     for e in range(w.n_experts):
         tt, kk = np.nonzero(idx == e)
@@ -164,5 +171,5 @@ def forward(w: OracleWeights, x: np.ndarray, k: int, idx: Optional[np.ndarray] =
         # each token selects an expert at most once, so tt has no repeats
         z[tt] += gate[tt, kk][:, None] * o
     s = sqrelu(x @ w.ws1.T) @ w.ws2.T
-    y = z @ w.w_up.T + s
+    y = (z if standard else z @ w.w_up.T) + s
     return {"y": y, "idx": idx, "gate": gate, "logits": logits, "h": h, "z": z}

@@ -34,7 +34,8 @@ def host_weights(weight_seed_workload: str) -> inp.LayerWeights:
 
 def device_weights(w: inp.LayerWeights) -> dict:
     dt = w.dtype
-    d = {k: to_dev(getattr(w, k), dt) for k in ("w_router", "w_down", "w_up", "w1", "w2", "ws1", "ws2")}
+    d = {k: to_dev(getattr(w, k), dt) if getattr(w, k).size else None
+         for k in ("w_router", "w_down", "w_up", "w1", "w2", "ws1", "ws2")}
     d["b_router"] = None if w.b_router is None else to_dev(w.b_router, "f32")
     return d
 

@@ -4,6 +4,8 @@ Routing must match bit for bit except on logit near-ties (gap < 1e-5), the dispa
 exactly the grouping the oracle derives from the GPU's own routing, and y must be within
 2e-2 x RMS(y) of the oracle (tokens whose routing differs at a near-tie are re-evaluated by the
 oracle with the GPU's routing)."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -155,3 +157,51 @@ def test_wait_timeout_reported_and_context_survives(tiny):
     after = _run(layer, x)
     for a, b in zip(before, after):
         assert np.array_equal(a, b)
+
+
+# ------------------------------------------------------------------------------------------------ standard MoE
+@pytest.fixture(scope="module")
+def stdlayer():
+    """The standard MoE of the Super budget (latent = 0: N = 128, K = 6, experts d -> m -> d)."""
+    wl = inp.workload("standard_decode")
+    w = inp.make_weights(wl)
+    layer = make_layer(wl, w, device_weights(w), inp.workload("standard_prefill").tokens)
+    torch.cuda.empty_cache()
+    yield w, layer
+    layer.close()
+    torch.cuda.empty_cache()
+
+
+def test_standard_decode_parity_and_dispatch(stdlayer):
+    w, layer = stdlayer
+    wl = inp.workload("standard_decode")
+    st = _compare(layer, oracle_weights(w, False), inp.make_x(wl), wl.shape.top_k)
+    _check_dispatch(layer, st["idx"], wl.shape.n_experts)
+    print(f"standard decode: rel err {st['rel_err']:.3g}, logit err {st['logit_err']:.3g}")
+
+
+@pytest.mark.parametrize("t", [3, 600])
+def test_standard_ragged_tokens(stdlayer, t):
+    w, layer = stdlayer
+    wl = inp.workload("standard_prefill")
+    _compare(layer, oracle_weights(w, False), inp.make_x(wl, tokens=t), wl.shape.top_k,
+             tokens=np.unique([0, t // 2, t - 1]))
+
+
+def test_standard_prefill_sampled_parity(stdlayer):
+    w, layer = stdlayer
+    wl = inp.workload("standard_prefill")
+    st = _compare(layer, oracle_weights(w, False), inp.make_x(wl), wl.shape.top_k, tokens=[0, 8191, wl.tokens - 1])
+    _check_dispatch(layer, st["idx"], wl.shape.n_experts)
+
+
+def test_standard_rejects_projections_and_nvfp4():
+    import latentmoe_expert_layer_b200 as lm
+    with pytest.raises(RuntimeError):
+        lm.LatentMoE(inp.STANDARD, 16, precision="nvfp4")
+    w = inp.make_weights(inp.workload("tiny"))
+    layer = lm.LatentMoE(dataclasses.replace(inp.TINY, latent=0), 16)
+    dev = device_weights(w)
+    with pytest.raises(RuntimeError):     # W_down / W_up given to a layer without projections
+        layer.load_weights(dev["w_router"], dev["w_down"], dev["w_up"], dev["w1"], dev["w2"], dev["ws1"], dev["ws2"])
+    layer.close()

@@ -204,6 +204,42 @@ def test_identity_projections_equal_standard_moe():
         assert np.allclose(out["y"][t], ref, rtol=1e-12, atol=1e-12)
 
 
+def test_standard_moe_without_projections():
+    """A layer given without W_down / W_up (zero-row arrays) runs its experts on x: it equals the
+    per-token loop of the standard MoE and the l = d layer with identity projections."""
+    rng = np.random.default_rng(15)
+    d, n, k = 6, 7, 3
+    W = _W(rng, d=d, l=d, n=n, m=5, ms=4)
+    x = rng.standard_normal((9, d))
+    W.w_down, W.w_up = np.eye(d), np.eye(d)
+    ident = lo.forward(W, x, k)["y"]
+    W.w_down, W.w_up = np.zeros((0, d)), np.zeros((d, 0))
+    out = lo.forward(W, x, k)
+    assert np.allclose(out["y"], ident, rtol=1e-13, atol=1e-13)
+    for t in range(x.shape[0]):
+        logit = W.w_router @ x[t]
+        sel = sorted(range(n), key=lambda e: (-logit[e], e))[:k]
+        w = np.exp(logit[sel] - logit[sel].max())
+        w /= w.sum()
+        ref = sum(w[i] * (W.w2(e) @ (np.maximum(W.w1(e) @ x[t], 0) ** 2)) for i, e in enumerate(sel))
+        ref = ref + W.ws2 @ (np.maximum(W.ws1 @ x[t], 0) ** 2)
+        assert np.allclose(out["y"][t], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_standard_budget_matches_the_latent_layer():
+    """N = N' l / d and K = K' l / d (rounded up): the standard layer holds the Super layer's
+    expert parameters and about its active expert weights per token."""
+    sup, std = inp.SUPER, inp.STANDARD
+    assert std.n_experts == sup.n_experts * sup.latent // sup.d
+    assert std.top_k == math.ceil(sup.top_k * sup.latent / sup.d)
+    e_sup = sup.n_experts * 2 * sup.expert_ffn * sup.latent
+    e_std = std.n_experts * 2 * std.expert_ffn * std.d
+    assert e_sup == e_std
+    act_sup = sup.top_k * 2 * sup.expert_ffn * sup.latent + 2 * sup.latent * sup.d
+    act_std = std.top_k * 2 * std.expert_ffn * std.d
+    assert abs(act_std / act_sup - 1) < 0.1
+
+
 def test_latent_sum_equals_sum_of_up_projections():
     """W_up is linear: up-projecting the latent sum equals summing the up-projected expert outputs."""
     rng = np.random.default_rng(15)
