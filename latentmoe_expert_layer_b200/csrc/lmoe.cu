@@ -159,7 +159,8 @@ struct lmoe_ctx {
   uint8_t *xq = nullptr, *x_sf = nullptr, *hq = nullptr, *h_sf = nullptr;  // x [T, d]; h grouped [TK, l]
   uint8_t *uq = nullptr, *u_sf = nullptr, *usq = nullptr, *us_sf = nullptr; // u [TK, m]; u_s [T, m_s]
   float* act_g = nullptr;         // [0] g_x, [1] g_h, [2] 1.0
-  int* tile0 = nullptr;           // [N + 1] first token tile of each expert (NVFP4 scale tiles)
+  int* tile0 = nullptr;           // [N + 1] first token tile of each expert
+  int* unit_u0 = nullptr;         // [2][N + 1] first unit of each expert in the two unit lists
   CUtensorMap map_w1q{}, map_w2q{}, map_ws1q{}, map_ws2q{};
   CUtensorMap map_xq[4]{}, map_hq[4]{}, map_uq[4]{}, map_usq[4]{};  // indexed by variant (FP4 ones)
 
@@ -218,7 +219,7 @@ void free_all(lmoe_ctx* c) {
                   c->y_dev,  c->idx_dev, c->gate_dev, c->y_s, c->work_counters,
                   c->w1q,    c->w2q,    c->ws1q,   c->ws2q,      c->w1_sf,      c->w2_sf,      c->ws1_sf,
                   c->ws2_sf, c->wg,     c->w_amax, c->xq,        c->x_sf,       c->hq,         c->h_sf,
-                  c->uq,     c->u_sf,   c->usq,    c->us_sf,     c->act_g,      c->tile0};
+                  c->uq,     c->u_sf,   c->usq,    c->us_sf,     c->act_g,      c->tile0,      c->unit_u0};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -368,6 +369,15 @@ struct GemmLaunch {
   }
 };
 
+// The two grouped-GEMM unit lists from the scan's first units: one unit per thread.
+cudaError_t launch_build_units(const lmoe_ctx* c, cudaStream_t s, const UnitListSpec& l1, const UnitListSpec& l2) {
+  const long long cap = (long long)c->max_units1 + c->max_units2;
+  long long blocks = (cap + 255) / 256;
+  if (blocks > 4LL * c->num_sms) blocks = 4LL * c->num_sms;
+  build_units_kernel<<<(int)blocks, 256, 0, s>>>(c->counts, c->offsets, c->tile0, c->cfg.n_experts, l1, l2);
+  return cudaGetLastError();
+}
+
 // NVFP4 forward: router, W_down and W_up in bf16; routed and shared experts as block-scaled FP4 GEMMs.
 template <typename Mark>
 cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, float* gate, cudaStream_t s,
@@ -436,11 +446,12 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
   chk(launch_topk_hist(nch, topk_threads(ct), s, c->logits, c->b_router, T, N, K, ct, idx, gate, c->chunk_counts));
   mark(3);
   // 4. expert offsets and grouped-GEMM unit lists
-  UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1};
-  UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2};
+  UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1, c->unit_u0};
+  UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2, c->unit_u0 + N + 1};
   scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(c->chunk_counts, nch, N, c->counts, c->offsets,
                                                               c->chunk_base, l1, l2, c->tile0, c->status);
   chk(cudaGetLastError());
+  chk(launch_build_units(c, s, l1, l2));
   mark(4);
   // 5. stable grouping; quantise h rows straight into grouped order
   assign_rows_kernel<<<nch, 32, N * sizeof(int), s>>>(idx, gate, c->chunk_base, T, N, K, ct, c->row_of,
@@ -486,12 +497,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
   }
   mark(7);
   // 8. latent combine: zu[:, :l] = sum_k o[row_of[t, k]]
-  {
-    const long long threads = (long long)T * (l / 8);
-    const int blocks = (int)((threads + 255) / 256);
-    combine_kernel<<<blocks, 256, 0, s>>>(c->o, c->row_of, T, K, l, c->zu, l + ms, TKmax, c->status);
-    chk(cudaGetLastError());
-  }
+  chk(launch_combine(c->num_sms, s, c->o, c->row_of, T, K, l, c->zu, l + ms, TKmax, c->status));
   mark(8);
   // 9. y = W_up z + y_s (bf16 GEMM)
   {
@@ -503,7 +509,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
     chk(gl.run(s));
   }
   mark(9);
-  launches += 12 + (split ? 0 : 2);
+  launches += 13 + (split ? 0 : 2);
   return e;
 }
 
@@ -573,6 +579,7 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   ok = ok && dalloc(&c->zu, T * (l + ms));
   ok = ok && dalloc(&c->units1, c->max_units1) && dalloc(&c->units2, c->max_units2) && dalloc(&c->num_units, 2);
   ok = ok && dalloc(&c->status, 1) && dalloc(&c->work_counters, lmoe_ctx::kCounters);
+  ok = ok && dalloc(&c->tile0, N + 1) && dalloc(&c->unit_u0, 2 * (N + 1));
   c->nvfp4 = g.precision == LMOE_PREC_NVFP4;
   // y_s = W_s2 u_s in fp32: needed at decode sizes (bf16) and at every size (NVFP4, standard MoE)
   ok = ok && dalloc(&c->y_s, (size_t)(c->nvfp4 || c->standard ? T : (T < 512 ? T : 512)) * d);
@@ -581,7 +588,7 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
     ok = ok && dalloc(&c->hq, tk * l / 2) && dalloc(&c->h_sf, c->sf_bytes_grouped(l));
     ok = ok && dalloc(&c->uq, tk * m / 2) && dalloc(&c->u_sf, c->sf_bytes_grouped(m));
     ok = ok && dalloc(&c->usq, T * ms / 2) && dalloc(&c->us_sf, c->sf_bytes_dense(ms));
-    ok = ok && dalloc(&c->act_g, 4) && dalloc(&c->tile0, N + 1);
+    ok = ok && dalloc(&c->act_g, 4);
   }
   if (!ok) {
     free_all(c);
@@ -871,11 +878,12 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   chk(launch_topk_hist(nch, topk_threads(ct), s, c->logits, c->b_router, T, N, K, ct, idx, gate, c->chunk_counts));
   mark(3);
   // 4. expert offsets and grouped-GEMM unit lists
-  UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1};
-  UnitListSpec l2{c->units2, c->num_units + 1, le, V_BN[vg], c->max_units2};
+  UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1, c->unit_u0};
+  UnitListSpec l2{c->units2, c->num_units + 1, le, V_BN[vg], c->max_units2, c->unit_u0 + N + 1};
   scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(c->chunk_counts, nch, N, c->counts, c->offsets,
-                                                              c->chunk_base, l1, l2, nullptr, c->status);
+                                                              c->chunk_base, l1, l2, c->tile0, c->status);
   chk(cudaGetLastError());
+  chk(launch_build_units(c, s, l1, l2));
   mark(4);
   // 5. stable grouping, then the gather of latent rows into grouped order
   assign_rows_kernel<<<nch, 32, N * sizeof(int), s>>>(idx, gate, c->chunk_base, T, N, K, ct, c->row_of,
@@ -919,20 +927,15 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   mark(7);
   // 8. latent combine: zu[:, :l] = sum_k o[row_of[t, k]]; a standard MoE's combine writes
   //    y = sum_k o[row_of[t, k]] + y_s and the layer ends here
-  {
-    const long long threads = (long long)T * (le / 8);
-    const int blocks = (int)((threads + 255) / 256);
-    if (c->standard)
-      combine_kernel<<<blocks, 256, 0, s>>>(c->o, c->row_of, T, K, d, reinterpret_cast<__nv_bfloat16*>(y), d, TKmax,
-                                           c->status, c->y_s, d);
-    else
-      combine_kernel<<<blocks, 256, 0, s>>>(c->o, c->row_of, T, K, l, c->zu, l + ms, TKmax, c->status);
-    chk(cudaGetLastError());
-  }
+  if (c->standard)
+    chk(launch_combine(c->num_sms, s, c->o, c->row_of, T, K, d, reinterpret_cast<__nv_bfloat16*>(y), d, TKmax,
+                       c->status, c->y_s, d));
+  else
+    chk(launch_combine(c->num_sms, s, c->o, c->row_of, T, K, l, c->zu, l + ms, TKmax, c->status));
   mark(8);
   if (c->standard) {
     mark(9);
-    launches += 7;
+    launches += 8;
     c->launches = launches;
     if (prof) ++c->prof_n;
     c->last_T = T;
@@ -952,7 +955,7 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
     chk(g.run(s));
   }
   mark(9);
-  launches += 8;
+  launches += 9;
   c->launches = launches;
   if (prof) ++c->prof_n;
   c->last_T = T;
@@ -1206,7 +1209,7 @@ extern "C" lmoe_status lmoe_route_noalloc(const float* logits, const float* bias
   if (launch_topk_hist(nch, topk_threads(ct), s, logits, bias, T, N, K, ct, topk_idx, topk_gate, chunk_counts) !=
       cudaSuccess)
     return LMOE_ERR_CUDA;
-  UnitListSpec none{nullptr, nullptr, 0, 64, 0};
+  UnitListSpec none{nullptr, nullptr, 0, 64, 0, nullptr};
   scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(chunk_counts, nch, N, counts, offsets, chunk_base,
                                                               none, none, nullptr, status);
   if (cudaGetLastError() != cudaSuccess) return LMOE_ERR_CUDA;

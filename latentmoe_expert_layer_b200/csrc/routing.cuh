@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(1024)
     topk_hist_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int n_experts,
                      int k, int chunk_tokens, int* __restrict__ topk_idx, float* __restrict__ topk_gate,
                      int* __restrict__ chunk_counts) {
-  extern __shared__ int s_counts[];  // [n_experts]
+  extern __shared__ int s_counts[];  // [n_experts], then per warp 32 keys + 32 indices
   for (int e = threadIdx.x; e < n_experts; e += blockDim.x) s_counts[e] = 0;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
@@ -63,65 +63,72 @@ __global__ void __launch_bounds__(1024)
   const int t_end = min(T, t_begin + chunk_tokens);
   for (int t = t_begin + warp; t < t_end; t += nwarps) {
     const float* lrow = logits + (long long)t * n_experts;
-    float v[P];
-    int ix[P];
+    // order-preserving keys: a larger logit has a larger key, -0 and +0 share one; padding is 0
+    uint32_t key[P];
 #pragma unroll
     for (int i = 0; i < P; ++i) {
       const int e = i * 32 + lane;
-      const bool ok = e < n_experts;
-      v[i] = ok ? lrow[e] + (bias ? bias[e] : 0.f) : -INFINITY;
-      ix[i] = ok ? e : 0x7fffffff;
+      if (e < n_experts) {
+        const uint32_t u = __float_as_uint(__fadd_rn(lrow[e] + (bias ? bias[e] : 0.f), 0.f));
+        key[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+      } else {
+        key[i] = 0u;
+      }
     }
+    // the K-th largest key X: the largest value with at least K keys >= X, built bit by bit
+    uint32_t X = 0u;
+#pragma unroll 1
+    for (int b = 31; b >= 0; --b) {
+      const uint32_t Y = X | (1u << b);
+      int cnt = 0;
 #pragma unroll
-    for (int size = 2; size <= P; size <<= 1) {
+      for (int i = 0; i < P; ++i) cnt += key[i] >= Y;
+      if (__reduce_add_sync(0xffffffffu, cnt) >= k) X = Y;
+    }
+    // selected: every key above X, then the lowest expert indices among the keys equal to X
+    int above = 0;
+#pragma unroll
+    for (int i = 0; i < P; ++i) above += key[i] > X;
+    const int need = k - __reduce_add_sync(0xffffffffu, above);
+    const unsigned lt = (1u << lane) - 1u;
+    int tie_base = 0, pos_base = 0;
+    uint32_t* s_key = reinterpret_cast<uint32_t*>(s_counts + n_experts) + warp * 64;
+    int* s_idx = reinterpret_cast<int*>(s_key + 32);
+#pragma unroll
+    for (int i = 0; i < P; ++i) {
+      const unsigned tie = __ballot_sync(0xffffffffu, key[i] == X);
+      const bool sel = key[i] > X || (key[i] == X && tie_base + __popc(tie & lt) < need);
+      tie_base += __popc(tie);
+      const unsigned sb = __ballot_sync(0xffffffffu, sel);
+      if (sel) {
+        const int pos = pos_base + __popc(sb & lt);
+        s_key[pos] = key[i];
+        s_idx[pos] = i * 32 + lane;
+      }
+      pos_base += __popc(sb);
+    }
+    __syncwarp();
+    uint32_t mk = lane < k ? s_key[lane] : 0u;
+    int mi = lane < k ? s_idx[lane] : 0x7fffffff;
+    __syncwarp();
+    // bitonic sort of the K selections over the warp: key descending, then index ascending
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
 #pragma unroll
       for (int stride = size >> 1; stride > 0; stride >>= 1) {
-#pragma unroll
-        for (int i = 0; i < P; ++i) {
-          const int j = i ^ stride;
-          if (j > i) {
-            const bool desc = (i & size) == 0;
-            const bool sw = desc ? better(v[j], ix[j], v[i], ix[i]) : better(v[i], ix[i], v[j], ix[j]);
-            if (sw) {
-              const float tv = v[i];
-              v[i] = v[j];
-              v[j] = tv;
-              const int ti = ix[i];
-              ix[i] = ix[j];
-              ix[j] = ti;
-            }
-          }
+        const uint32_t ok = __shfl_xor_sync(0xffffffffu, mk, stride);
+        const int oi = __shfl_xor_sync(0xffffffffu, mi, stride);
+        const bool other_better = ok > mk || (ok == mk && oi < mi);
+        const bool keep_better = ((lane & stride) == 0) == ((lane & size) == 0);
+        if (keep_better == other_better) {
+          mk = ok;
+          mi = oi;
         }
       }
     }
-    float sel_v = 0.f;
-    int sel_i = 0;
-    for (int r = 0; r < k; ++r) {
-      float wv = v[0];
-      int wi = ix[0];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, wv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, wi, o);
-        if (better(ov, oi, wv, wi)) {
-          wv = ov;
-          wi = oi;
-        }
-      }
-      if (lane == r) {
-        sel_v = wv;
-        sel_i = wi;
-      }
-      if (ix[0] == wi) {  // expert ids are unique: this lane owned the winner
-#pragma unroll
-        for (int i = 0; i + 1 < P; ++i) {
-          v[i] = v[i + 1];
-          ix[i] = ix[i + 1];
-        }
-        v[P - 1] = -INFINITY;
-        ix[P - 1] = 0x7fffffff;
-      }
-    }
+    const uint32_t ub = (mk & 0x80000000u) ? (mk & 0x7fffffffu) : ~mk;
+    const float sel_v = __uint_as_float(ub);
+    const int sel_i = mi;
     // softmax over the selected logits (lane r holds slot r); the max is slot 0
     const float vmax = __shfl_sync(0xffffffffu, sel_v, 0);
     const float ex = (lane < k) ? expf(sel_v - vmax) : 0.f;
@@ -149,7 +156,7 @@ inline int topk_lane_candidates(int n_experts) {
 
 inline cudaError_t launch_topk_hist(int n_chunks, int threads, cudaStream_t s, const float* logits, const float* bias,
                                     int T, int N, int K, int ct, int* idx, float* gate, int* chunk_counts) {
-  const size_t sm = (size_t)N * sizeof(int);
+  const size_t sm = (size_t)N * sizeof(int) + (size_t)(threads / 32) * 64 * sizeof(int);
   switch (topk_lane_candidates(N)) {
     case 1: topk_hist_kernel<1><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
     case 2: topk_hist_kernel<2><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
@@ -171,6 +178,7 @@ struct UnitListSpec {
   int feat;            // output features per expert (rows of that expert's weight)
   int tile_tokens;     // tokens per unit (the GEMM variant's BN_MAX)
   int max_units;       // capacity
+  int* u0;             // [N + 1] first unit of each expert, then the total (written by the scan)
 };
 
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp, int& total) {
@@ -215,9 +223,22 @@ __global__ void __launch_bounds__(1024)
   __shared__ int s_tmp[33];
   const int pitch = n_chunks + 1;
   const int total_words = n_experts * n_chunks;
-  for (int i = threadIdx.x; i < total_words; i += blockDim.x) {
-    const int e = i / n_chunks, c = i - e * n_chunks;
-    s_cc[e * pitch + c] = chunk_counts[i];
+  // 8 loads in flight per thread at a time (a plain loop waits for each before the next)
+  for (int i0 = threadIdx.x; i0 < total_words; i0 += 8 * blockDim.x) {
+    int vals[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = i0 + j * blockDim.x;
+      vals[j] = i < total_words ? chunk_counts[i] : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = i0 + j * blockDim.x;
+      if (i < total_words) {
+        const int e = i / n_chunks, c = i - e * n_chunks;
+        s_cc[e * pitch + c] = vals[j];
+      }
+    }
   }
   __syncthreads();
   const int e = threadIdx.x;
@@ -242,22 +263,13 @@ __global__ void __launch_bounds__(1024)
     const int ex = i / n_chunks, c = i - ex * n_chunks;
     chunk_base[i] = s_cc[ex * pitch + c];
   }
-  // unit lists: expert-major, token block next, feature block fastest.  Consecutive threads write
-  // consecutive units (16-byte stores); a unit finds its expert by binary search over the experts'
-  // first-unit indices.  Token tiles are numbered expert-major: expert e owns tiles tile0[e] ...
-  __shared__ int s_u0[1025];
-  __shared__ int s_cnt[1024];
-  __shared__ int s_offs[1024];
-  __shared__ int s_t0[1024];
+  // unit lists (written by build_units_kernel): expert-major, token block next, feature block
+  // fastest; here only each expert's first unit.  Token tiles are numbered expert-major: expert e
+  // owns tiles tile0[e] ...
   const int tile_tokens = l1.units ? l1.tile_tokens : 64;
   int n_tiles;
   const int t0 = block_exclusive_scan((e < n_experts) ? (c_e + tile_tokens - 1) / tile_tokens : 0, s_tmp, n_tiles);
-  if (e < n_experts) {
-    s_cnt[e] = c_e;
-    s_offs[e] = off;
-    s_t0[e] = t0;
-    if (tile0) tile0[e] = t0;
-  }
+  if (e < n_experts && tile0) tile0[e] = t0;
   if (e == 0 && tile0) tile0[n_experts] = n_tiles;
 #pragma unroll 1
   for (int li = 0; li < 2; ++li) {
@@ -268,32 +280,46 @@ __global__ void __launch_bounds__(1024)
     const int nu = (e < n_experts) ? ntt * nft : 0;
     int nu_total;
     const int u0 = block_exclusive_scan(nu, s_tmp, nu_total);  // ends with __syncthreads
-    if (e < n_experts) s_u0[e] = u0;
+    if (e < n_experts) L.u0[e] = u0;
     if (e == 0) {
-      s_u0[n_experts] = nu_total;
+      L.u0[n_experts] = nu_total;
       *L.num_units = min(nu_total, L.max_units);
       if (nu_total > L.max_units) atomicOr(status, DEV_STATUS_BAD_INDEX);
     }
-    __syncthreads();
-    const int n_write = min(nu_total, L.max_units);
-    for (int u = threadIdx.x; u < n_write; u += blockDim.x) {
-      int lo = 0, hi = n_experts - 1;  // largest expert whose first unit is <= u
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_u0[mid] <= u) lo = mid;
-        else hi = mid - 1;
-      }
-      const int ex = lo;
-      const int local = u - s_u0[ex];
-      const int tt = local / nft, ft = local - tt * nft;
-      const int nv = min(L.tile_tokens, s_cnt[ex] - tt * L.tile_tokens);
-      const int4 g = make_int4(ex * L.feat + ft * BLOCK_M, s_offs[ex] + tt * L.tile_tokens, ft * BLOCK_M,
-                               nv | (min(BLOCK_M, L.feat - ft * BLOCK_M) << 16));
-      int4* dst = reinterpret_cast<int4*>(&L.units[u]);
-      dst[0] = g;
-      dst[1] = make_int4(s_t0[ex] + tt, 0, 0, 0);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Grouped-GEMM unit lists from the scan's per-expert first units, one unit per thread over the
+// whole grid: a unit finds its expert by binary search over the first-unit indices (the largest
+// expert whose first unit is <= u, which skips experts without units).
+// ------------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    build_units_kernel(const int* __restrict__ counts, const int* __restrict__ offsets,
+                       const int* __restrict__ tile0, int n_experts, UnitListSpec l1, UnitListSpec l2) {
+  const int n1 = l1.units ? *l1.num_units : 0;
+  const int n2 = l2.units ? *l2.num_units : 0;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n1 + n2; i += stride) {
+    const bool second = i >= n1;
+    const UnitListSpec& L = second ? l2 : l1;
+    const int u = (int)(second ? i - n1 : i);
+    int lo = 0, hi = n_experts - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(L.u0 + mid) <= u) lo = mid;
+      else hi = mid - 1;
     }
-    __syncthreads();
+    const int ex = lo;
+    const int nft = (L.feat + BLOCK_M - 1) / BLOCK_M;
+    const int local = u - __ldg(L.u0 + ex);
+    const int tt = local / nft, ft = local - tt * nft;
+    const int nv = min(L.tile_tokens, __ldg(counts + ex) - tt * L.tile_tokens);
+    const int4 g = make_int4(ex * L.feat + ft * BLOCK_M, __ldg(offsets + ex) + tt * L.tile_tokens, ft * BLOCK_M,
+                             nv | (min(BLOCK_M, L.feat - ft * BLOCK_M) << 16));
+    int4* dst = reinterpret_cast<int4*>(&L.units[u]);
+    dst[0] = g;
+    dst[1] = make_int4(__ldg(tile0 + ex) + tt, 0, 0, 0);
   }
 }
 
@@ -309,19 +335,37 @@ __global__ void __launch_bounds__(32)
                        unsigned* status) {
   extern __shared__ int s_base[];  // [n_experts]
   const int lane = threadIdx.x;
-  for (int e = lane; e < n_experts; e += 32) s_base[e] = chunk_base[(long long)e * gridDim.x + blockIdx.x];
+  // chunk bases, 8 loads in flight per lane at a time
+  for (int e0 = lane; e0 < n_experts; e0 += 8 * 32) {
+    int vals[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = e0 + 32 * j;
+      vals[j] = e < n_experts ? chunk_base[(long long)e * gridDim.x + blockIdx.x] : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (e0 + 32 * j < n_experts) s_base[e0 + 32 * j] = vals[j];
+  }
   __syncwarp();
   const int t_begin = blockIdx.x * chunk_tokens;
   const int t_end = min(T, t_begin + chunk_tokens);
   const long long a_begin = (long long)t_begin * k, a_end = (long long)t_end * k;
   const long long TK = (long long)T * k;
+  // the next round's expert ids and gates are loaded while this round is ranked
+  int e_next = (a_begin + lane < a_end) ? topk_idx[a_begin + lane] : 0;
+  float g_next = (a_begin + lane < a_end) ? topk_gate[a_begin + lane] : 0.f;
   for (long long a0 = a_begin; a0 < a_end; a0 += 32) {
     const long long a = a0 + lane;
     const bool act = a < a_end;
-    int e = act ? topk_idx[a] : -1 - lane;  // inactive lanes get unique keys
+    int e = act ? e_next : -1 - lane;  // inactive lanes get unique keys
+    const float g = act ? g_next : 0.f;
+    if (a + 32 < a_end) {
+      e_next = topk_idx[a + 32];
+      g_next = topk_gate[a + 32];
+    }
     const bool e_ok = e >= 0 && e < n_experts;
     if (act && !e_ok) atomicOr(status, DEV_STATUS_BAD_INDEX);
-    const float g = act ? topk_gate[a] : 0.f;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & ((1u << lane) - 1u));
     const int leader = __ffs(peers) - 1;
@@ -385,22 +429,20 @@ __global__ void __launch_bounds__(256)
 // combine: zu[t, 0:latent] = bf16( sum_k o[row_of[t, k], :] (+ add[t, :]) ), slot order, fp32
 // accumulation; the fp32 addend (a standard MoE's shared-expert output) is added last
 // ------------------------------------------------------------------------------------------------
+// BATCH: every row index, then the rows 8 at a time, are in flight together (k <= 32): few memory
+// latencies per token, for small grids that cannot hide latency with many threads; otherwise one row
+// at a time with fewer registers, for occupancy.  Both sum in slot order.
+template <bool BATCH>
 __global__ void combine_kernel(const __nv_bfloat16* __restrict__ o, const int* __restrict__ row_of, int T, int k,
                                int latent, __nv_bfloat16* __restrict__ zu, long long ld_zu, long long n_rows,
-                               unsigned* status, const float* __restrict__ add = nullptr, long long ld_add = 0) {
+                               unsigned* status, const float* __restrict__ add, long long ld_add) {
   const int vpr = latent / 8;  // 8 bf16 per thread
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long t = gid / vpr;
   const int v = (int)(gid % vpr);
   if (t >= T) return;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < k; ++s) {
-    const int row = row_of[t * k + s];
-    if (row < 0 || row >= n_rows) {
-      atomicOr(status, DEV_STATUS_BAD_INDEX);
-      continue;
-    }
-    const uint4 q = *reinterpret_cast<const uint4*>(o + (long long)row * latent + v * 8);
+  auto add_row = [&](const uint4& q) {
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -408,6 +450,36 @@ __global__ void combine_kernel(const __nv_bfloat16* __restrict__ o, const int* _
       acc[2 * i] += f.x;
       acc[2 * i + 1] += f.y;
     }
+  };
+  if constexpr (!BATCH) {
+    for (int s = 0; s < k; ++s) {
+      const int row = row_of[t * k + s];
+      if (row < 0 || row >= n_rows) {
+        atomicOr(status, DEV_STATUS_BAD_INDEX);
+        continue;
+      }
+      add_row(*reinterpret_cast<const uint4*>(o + (long long)row * latent + v * 8));
+    }
+  } else {
+  int rows[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) rows[j] = j < k ? row_of[t * k + j] : -1;
+#pragma unroll
+  for (int s0 = 0; s0 < 32; s0 += 8) {
+    if (s0 >= k) break;
+    uint4 q[8];
+    bool okq[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int row = rows[s0 + j];
+      okq[j] = s0 + j < k && row >= 0 && row < n_rows;
+      if (s0 + j < k && !okq[j]) atomicOr(status, DEV_STATUS_BAD_INDEX);
+      if (okq[j]) q[j] = *reinterpret_cast<const uint4*>(o + (long long)row * latent + v * 8);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (okq[j]) add_row(q[j]);
+  }
   }
   if (add != nullptr) {
     const float4* pa = reinterpret_cast<const float4*>(add + t * ld_add + v * 8);
@@ -431,6 +503,20 @@ __global__ void combine_kernel(const __nv_bfloat16* __restrict__ o, const int* _
 // ------------------------------------------------------------------------------------------------
 // weight preparation: copy or convert a [rows, cols] matrix (bf16 or fp32 source) into a bf16
 // destination with its own row pitch and column offset (used to stack/concatenate weights).
+// combine over T tokens of `latent` columns: the batched variant while the grid is below ~8 warps
+// per SM
+inline cudaError_t launch_combine(int num_sms, cudaStream_t s, const __nv_bfloat16* o, const int* row_of, int T,
+                                  int k, int latent, __nv_bfloat16* out, long long ld_out, long long n_rows,
+                                  unsigned* status, const float* add = nullptr, long long ld_add = 0) {
+  const long long threads = (long long)T * (latent / 8);
+  const int blocks = (int)((threads + 255) / 256);
+  if (threads <= (long long)num_sms * 256)
+    combine_kernel<true><<<blocks, 256, 0, s>>>(o, row_of, T, k, latent, out, ld_out, n_rows, status, add, ld_add);
+  else
+    combine_kernel<false><<<blocks, 256, 0, s>>>(o, row_of, T, k, latent, out, ld_out, n_rows, status, add, ld_add);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------------------------------------
 __global__ void convert_2d_kernel(const void* __restrict__ src, int src_is_f32, long long rows, int cols,
                                   long long src_ld, __nv_bfloat16* __restrict__ dst, long long dst_ld, int dst_col0) {
