@@ -52,7 +52,7 @@ enum EpiKind : int {
 // EPI_SQRELU_NVFP4); tile: token-tile id (NVFP4 activation scales are stored per token tile).
 struct GemmUnit {
   int a_row, b_row, f0, nm;
-  int tile, pad0, pad1, pad2;
+  int tile, kslice, pad1, pad2;  // kslice: K slice of a split dense unit (0 otherwise)
 };
 
 // One GEMM problem of a launch: K extent, epilogue, NVFP4 scales, and (for dense problems) the grid.
@@ -86,6 +86,10 @@ struct GemmProblem {
   int dense_ttiles;           // token tiles (fastest-varying unit index)
   int dense_feat;             // output features (rows of W)
   int dense_tokens;           // tokens (rows of act)
+  // split K (dense bf16 problems with EPI_F32): k_splits slices of the K blocks, slice s writes its
+  // fp32 partial at out + s * split_stride; the caller sums the slices
+  int k_splits;
+  long long split_stride;
 };
 
 struct GemmArgs {
@@ -154,7 +158,12 @@ struct GemmSmem {
 template <int BN_MAX>
 __device__ __forceinline__ GemmUnit dense_unit(const GemmProblem& p, int u) {
   GemmUnit r;
-  // token tiles of one weight tile run on adjacent CTAs, so the weight tile is read from HBM once
+  // K slices outermost; token tiles of one weight tile run on adjacent CTAs, so the weight tile is
+  // read from HBM once
+  const int per_slice = p.dense_ftiles * p.dense_ttiles;
+  const int ks = p.k_splits > 1 ? u / per_slice : 0;
+  u -= ks * per_slice;
+  r.kslice = ks;
   const int tt = u % p.dense_ttiles;
   const int ft = u / p.dense_ttiles;
   r.a_row = ft * BLOCK_M;
@@ -165,6 +174,18 @@ __device__ __forceinline__ GemmUnit dense_unit(const GemmProblem& p, int u) {
   r.nm = nv | (mv << 16);
   r.tile = tt;
   return r;
+}
+
+// K blocks [kb0, kb1) of a unit: all of them, or its slice of a split problem.
+__device__ __forceinline__ void unit_k_range(const GemmProblem& p, const GemmUnit& un, int& kb0, int& kb1) {
+  if (p.k_splits > 1) {
+    const int per = (p.num_k_blocks + p.k_splits - 1) / p.k_splits;
+    kb0 = un.kslice * per;
+    kb1 = min(p.num_k_blocks, kb0 + per);
+  } else {
+    kb0 = 0;
+    kb1 = p.num_k_blocks;
+  }
 }
 
 // Global unit u of the launch: which problem it belongs to, and its tile.  The pre problem's units
@@ -318,7 +339,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const uint32_t bytes = A_STAGE_BYTES + nbox * BOXN * 128 + S::SFA_STAGE_BYTES + (fill ? S::SFB_STAGE_BYTES : 0);
         // x coordinate of a stage in the tensor maps: 128 bytes = 64 bf16 elements or 128 FP4 bytes
         const int kx = FP4 ? 128 : BLOCK_K;
-        for (int kb = 0; kb < nkb; ++kb) {
+        int kb0, kb1;
+        unit_k_range(pr, un, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait0(&empty[stage], phase ^ 1u)) {
             ok = false;
             break;
@@ -407,7 +430,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S::ACC_COLS);
         int mma_i = 0;  // MMA index within the tile: partial accumulator mma_i % ACC_SPLIT
-        for (int kb = 0; kb < nkb; ++kb) {
+        int kb0, kb1;
+        unit_k_range(args.prob[pid], un, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, tmo)) {
             ok = false;
             break;
@@ -503,7 +528,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * S::ACC_COLS);
       // partial accumulators that received at least one MMA (every tile has >= 4 MMAs)
-      const int n_part = min(ACC_SPLIT, pr.num_k_blocks * 4);
+      int ekb0, ekb1;
+      unit_k_range(pr, un, ekb0, ekb1);
+      const int n_part = min(ACC_SPLIT, (ekb1 - ekb0) * 4);
       const int nchunks = (nv + 31) >> 5;
       const bool feat_ok = (q * 32) < mv;
       const int f = un.f0 + q * 32;  // first feature of this warp's 32
@@ -587,7 +614,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) s32[j * 32 + lane] = __uint_as_float(r[j]);
           __syncwarp();
-          float* dst = (pr.epi == EPI_ROUTER) ? pr.out2 : reinterpret_cast<float*>(pr.out);
+          float* dst = (pr.epi == EPI_ROUTER) ? pr.out2
+                                              : reinterpret_cast<float*>(pr.out) + un.kslice * pr.split_stride;
           const long long ld = (pr.epi == EPI_ROUTER) ? pr.ld2 : pr.ldo;
           const int col = (pr.epi == EPI_ROUTER) ? f : (pr.out_col0 + f);
           if (feat_ok && q * 32 + (lane & 7) * 4 < mv) {  // this lane's 4 features are valid

@@ -161,6 +161,9 @@ struct lmoe_ctx {
   float* act_g = nullptr;         // [0] g_x, [1] g_h, [2] 1.0
   int* tile0 = nullptr;           // [N + 1] first token tile of each expert
   int* unit_u0 = nullptr;         // [2][N + 1] first unit of each expert in the two unit lists
+  // split-K router (decode sizes): fp32 slice partials [slices][T][N + l], T <= kSplitRows
+  float* router_part = nullptr;
+  static constexpr int kSplitRows = 512, kMaxSplits = 8;
   CUtensorMap map_w1q{}, map_w2q{}, map_ws1q{}, map_ws2q{};
   CUtensorMap map_xq[4]{}, map_hq[4]{}, map_uq[4]{}, map_usq[4]{};  // indexed by variant (FP4 ones)
 
@@ -219,7 +222,8 @@ void free_all(lmoe_ctx* c) {
                   c->y_dev,  c->idx_dev, c->gate_dev, c->y_s, c->work_counters,
                   c->w1q,    c->w2q,    c->ws1q,   c->ws2q,      c->w1_sf,      c->w2_sf,      c->ws1_sf,
                   c->ws2_sf, c->wg,     c->w_amax, c->xq,        c->x_sf,       c->hq,         c->h_sf,
-                  c->uq,     c->u_sf,   c->usq,    c->us_sf,     c->act_g,      c->tile0,      c->unit_u0};
+                  c->uq,     c->u_sf,   c->usq,    c->us_sf,     c->act_g,      c->tile0,      c->unit_u0,
+                  c->router_part};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -290,7 +294,7 @@ int set_dense(GemmProblem& p, int v, int feat, int tokens) {
   p.dense_feat = feat;
   p.dense_tokens = tokens;
   p.weights_streamed = p.dense_ttiles == 1;
-  return p.dense_ftiles * p.dense_ttiles;
+  return p.dense_ftiles * p.dense_ttiles * (p.k_splits > 1 ? p.k_splits : 1);
 }
 
 struct GemmLaunch {
@@ -369,6 +373,39 @@ struct GemmLaunch {
   }
 };
 
+// K slices for the stacked router + W_down GEMM: at decode sizes its feature x token tiles cover
+// few SMs, and one SM streams only ~1/148 of HBM bandwidth; slicing K fills the GPU.  1 = no split.
+int router_splits(const lmoe_ctx* c, int T) {
+  const lmoe_config& g = c->cfg;
+  if (!c->fused_router || !c->router_part || T > lmoe_ctx::kSplitRows) return 1;
+  const int units = ((g.n_experts + g.latent + BLOCK_M - 1) / BLOCK_M) * ((T + V_BN[V_SMALL] - 1) / V_BN[V_SMALL]);
+  const int nkb = g.d / BLOCK_K;
+  int ks = c->num_sms / units;
+  if (ks > lmoe_ctx::kMaxSplits) ks = lmoe_ctx::kMaxSplits;
+  if (ks > nkb) ks = nkb;
+  if (ks < 2) return 1;
+  const int per = (nkb + ks - 1) / ks;
+  return (nkb + per - 1) / per;  // no empty slice
+}
+
+// The stacked router + W_down GEMM as K slices, then the slice sum into logits (fp32) and h (bf16).
+cudaError_t router_split_k(lmoe_ctx* c, int T, int ks, cudaStream_t s) {
+  const lmoe_config& g = c->cfg;
+  const int N = g.n_experts, l = g.latent;
+  GemmLaunch gl(c, V_SMALL, 0);
+  GemmProblem p = problem(g.d, EPI_F32, c->router_part, N + l);
+  p.k_splits = ks;
+  p.split_stride = (long long)T * (N + l);
+  gl.main_dense(c->map_rd, c->map_x[V_SMALL], p, N + l, T);
+  cudaError_t e = gl.run(s);
+  if (e != cudaSuccess) return e;
+  const long long work = (long long)T * (N + l) / 4;
+  long long blocks = (work + 255) / 256;
+  if (blocks > 4LL * c->num_sms) blocks = 4LL * c->num_sms;
+  split_reduce_kernel<<<(int)blocks, 256, 0, s>>>(c->router_part, ks, p.split_stride, T, N, l, c->logits, c->h);
+  return cudaGetLastError();
+}
+
 // The two grouped-GEMM unit lists from the scan's first units: one unit per thread.
 cudaError_t launch_build_units(const lmoe_ctx* c, cudaStream_t s, const UnitListSpec& l1, const UnitListSpec& l2) {
   const long long cap = (long long)c->max_units1 + c->max_units2;
@@ -406,7 +443,11 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
   };
 
   // 1. router logits and h = W_down x (bf16; one stacked GEMM when N is a multiple of 128)
-  if (c->fused_router) {
+  const int rks = router_splits(c, T);
+  if (rks > 1) {
+    chk(router_split_k(c, T, rks, s));
+    ++launches;
+  } else if (c->fused_router) {
     GemmLaunch gl(c, vd, 0);
     GemmProblem p = problem(d, EPI_ROUTER, c->h, l);
     p.out2 = c->logits;
@@ -580,6 +621,9 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   ok = ok && dalloc(&c->units1, c->max_units1) && dalloc(&c->units2, c->max_units2) && dalloc(&c->num_units, 2);
   ok = ok && dalloc(&c->status, 1) && dalloc(&c->work_counters, lmoe_ctx::kCounters);
   ok = ok && dalloc(&c->tile0, N + 1) && dalloc(&c->unit_u0, 2 * (N + 1));
+  if (l > 0)
+    ok = ok && dalloc(&c->router_part, (size_t)lmoe_ctx::kMaxSplits * (T < lmoe_ctx::kSplitRows ? T : lmoe_ctx::kSplitRows) *
+                                           (N + l));
   c->nvfp4 = g.precision == LMOE_PREC_NVFP4;
   // y_s = W_s2 u_s in fp32: needed at decode sizes (bf16) and at every size (NVFP4, standard MoE)
   ok = ok && dalloc(&c->y_s, (size_t)(c->nvfp4 || c->standard ? T : (T < 512 ? T : 512)) * d);
@@ -835,7 +879,11 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   const bool split = vd == V_SMALL && vg == V_SMALL && c->y_s != nullptr;
 
   // 1. router logits and the latent h = W_down x
-  if (c->fused_router) {
+  const int rks = router_splits(c, T);
+  if (rks > 1) {
+    chk(router_split_k(c, T, rks, s));
+    launches += 2;
+  } else if (c->fused_router) {
     GemmLaunch g(c, vd, 0);
     GemmProblem p = problem(d, EPI_ROUTER, c->h, l);
     p.out2 = c->logits;

@@ -503,6 +503,40 @@ __global__ void combine_kernel(const __nv_bfloat16* __restrict__ o, const int* _
 // ------------------------------------------------------------------------------------------------
 // weight preparation: copy or convert a [rows, cols] matrix (bf16 or fp32 source) into a bf16
 // destination with its own row pitch and column offset (used to stack/concatenate weights).
+// Sum of a split-K router GEMM's slices (fixed slice order): part[s] is [T, n_logits + n_h] fp32;
+// columns < n_logits go to the fp32 logits, the rest to bf16 h.  One thread per 4 columns
+// (n_logits is a multiple of 16, so a group never straddles the two outputs).
+__global__ void __launch_bounds__(256)
+    split_reduce_kernel(const float* __restrict__ part, int n_slices, long long slice_stride, int T, int n_logits,
+                        int n_h, float* __restrict__ logits, __nv_bfloat16* __restrict__ h) {
+  const int W = n_logits + n_h;
+  const int vpr = W / 4;
+  const long long total = (long long)T * vpr;
+  for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < total;
+       g += (long long)gridDim.x * blockDim.x) {
+    const long long t = g / vpr;
+    const int col = (int)(g - t * vpr) * 4;
+    const float* src = part + t * W + col;
+    float4 a = *reinterpret_cast<const float4*>(src);
+    for (int sl = 1; sl < n_slices; ++sl) {
+      const float4 b = *reinterpret_cast<const float4*>(src + sl * slice_stride);
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    if (col < n_logits) {
+      *reinterpret_cast<float4*>(logits + t * n_logits + col) = a;
+    } else {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(h + t * n_h + (col - n_logits)) = pk;
+    }
+  }
+}
+
 // combine over T tokens of `latent` columns: the batched variant while the grid is below ~8 warps
 // per SM
 inline cudaError_t launch_combine(int num_sms, cudaStream_t s, const __nv_bfloat16* o, const int* row_of, int T,
