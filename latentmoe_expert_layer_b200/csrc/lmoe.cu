@@ -157,6 +157,7 @@ struct lmoe_ctx {
   float* wg = nullptr;            // tensor scales: [0, N) W1, [N, 2N) W2, 2N W_s1, 2N + 1 W_s2
   unsigned* w_amax = nullptr;     // [2N + 2] amax bits used while quantising
   uint8_t *xq = nullptr, *x_sf = nullptr, *hq = nullptr, *h_sf = nullptr;  // x [T, d]; h grouped [TK, l]
+  uint8_t *hq_tok = nullptr, *h_sf_tok = nullptr;  // h per token [T, l/2] codes, [T, l/16] plain scales
   uint8_t *uq = nullptr, *u_sf = nullptr, *usq = nullptr, *us_sf = nullptr; // u [TK, m]; u_s [T, m_s]
   float* act_g = nullptr;         // [0] g_x, [1] g_h, [2] 1.0
   int* tile0 = nullptr;           // [N + 1] first token tile of each expert
@@ -222,6 +223,7 @@ void free_all(lmoe_ctx* c) {
                   c->y_dev,  c->idx_dev, c->gate_dev, c->y_s, c->work_counters,
                   c->w1q,    c->w2q,    c->ws1q,   c->ws2q,      c->w1_sf,      c->w2_sf,      c->ws1_sf,
                   c->ws2_sf, c->wg,     c->w_amax, c->xq,        c->x_sf,       c->hq,         c->h_sf,
+                  c->hq_tok, c->h_sf_tok,
                   c->uq,     c->u_sf,   c->usq,    c->us_sf,     c->act_g,      c->tile0,      c->unit_u0,
                   c->router_part};
   for (void* p : ptrs)
@@ -373,6 +375,9 @@ struct GemmLaunch {
   }
 };
 
+// warps per token chunk of the stable row assignment (each ranks a contiguous part of the chunk)
+constexpr int kAssignWarps = 8;
+
 // K slices for the stacked router + W_down GEMM: at decode sizes its feature x token tiles cover
 // few SMs, and one SM streams only ~1/148 of HBM bandwidth; slicing K fills the GPU.  1 = no split.
 int router_splits(const lmoe_ctx* c, int T) {
@@ -494,12 +499,19 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
   chk(cudaGetLastError());
   chk(launch_build_units(c, s, l1, l2));
   mark(4);
-  // 5. stable grouping; quantise h rows straight into grouped order
-  assign_rows_kernel<<<nch, 32, N * sizeof(int), s>>>(idx, gate, c->chunk_base, T, N, K, ct, c->row_of,
-                                                     c->tok_of_row, c->gate_of_row, c->status);
-  quant_act_kernel<<<grid_for(TK * l / 16, 256), 256, 0, s>>>(c->h, l, c->tok_of_row, TK, T, c->offsets, c->tile0,
-                                                               N, V_BN[vg], nra, amax_h, c->hq, c->h_sf, g_h,
-                                                               c->status);
+  // 5. stable grouping; h quantised once per token, then its rows copied into grouped order with
+  //    their scales in the expert GEMM's tile-local atoms
+  assign_rows_kernel<<<nch, 32 * kAssignWarps, kAssignWarps * N * sizeof(int), s>>>(
+      idx, gate, c->chunk_base, T, N, K, ct, c->row_of, c->tok_of_row, c->gate_of_row, c->status);
+  quant_act_kernel<<<grid_for((long long)T * l / 16, 256), 256, 0, s>>>(c->h, l, nullptr, T, T, nullptr, nullptr, N,
+                                                                         V_BN[vg], 0, amax_h, c->hq_tok, c->h_sf_tok,
+                                                                         g_h, c->status);
+  {
+    long long blocks = (TK + 7) / 8;  // one warp per row
+    if (blocks > 16LL * c->num_sms) blocks = 16LL * c->num_sms;
+    gather_act_q_kernel<<<(int)blocks, 256, 0, s>>>(c->hq_tok, c->h_sf_tok, l, c->tok_of_row, TK, T, c->offsets,
+                                                     c->tile0, N, V_BN[vg], nra, c->hq, c->h_sf, c->status);
+  }
   chk(cudaGetLastError());
   mark(5);
   // 6. expert up (FP4): u = NVFP4(sqrelu(W1_e h)); shared up u_s = NVFP4(sqrelu(W_s1 x))
@@ -550,7 +562,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
     chk(gl.run(s));
   }
   mark(9);
-  launches += 13 + (split ? 0 : 2);
+  launches += 14 + (split ? 0 : 2);
   return e;
 }
 
@@ -630,6 +642,7 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   if (c->nvfp4) {
     ok = ok && dalloc(&c->xq, T * d / 2) && dalloc(&c->x_sf, c->sf_bytes_dense(d));
     ok = ok && dalloc(&c->hq, tk * l / 2) && dalloc(&c->h_sf, c->sf_bytes_grouped(l));
+    ok = ok && dalloc(&c->hq_tok, T * l / 2) && dalloc(&c->h_sf_tok, T * l / 16);
     ok = ok && dalloc(&c->uq, tk * m / 2) && dalloc(&c->u_sf, c->sf_bytes_grouped(m));
     ok = ok && dalloc(&c->usq, T * ms / 2) && dalloc(&c->us_sf, c->sf_bytes_dense(ms));
     ok = ok && dalloc(&c->act_g, 4);
@@ -934,8 +947,8 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   chk(launch_build_units(c, s, l1, l2));
   mark(4);
   // 5. stable grouping, then the gather of latent rows into grouped order
-  assign_rows_kernel<<<nch, 32, N * sizeof(int), s>>>(idx, gate, c->chunk_base, T, N, K, ct, c->row_of,
-                                                     c->tok_of_row, c->gate_of_row, c->status);
+  assign_rows_kernel<<<nch, 32 * kAssignWarps, kAssignWarps * N * sizeof(int), s>>>(
+      idx, gate, c->chunk_base, T, N, K, ct, c->row_of, c->tok_of_row, c->gate_of_row, c->status);
   chk(cudaGetLastError());
   {
     long long warps = (TK + GATHER_ROWS - 1) / GATHER_ROWS;

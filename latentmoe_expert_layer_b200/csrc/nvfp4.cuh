@@ -296,8 +296,8 @@ __global__ void amax_act_kernel(const __nv_bfloat16* __restrict__ a, long long n
 // is written as codes [n_rows, K/2] plus scales in tile-local atoms.  Token tiles: dense mode
 // (offsets == nullptr) tile = r / tile_rows; grouped mode the tiles restart at each expert's first
 // row: expert e = the one with offsets[e] <= r < offsets[e + 1], tile = tile0[e] + (r - offsets[e])
-// / tile_rows.  One thread per 16-element block; tensor scale from amax_bits[0], also written to
-// *g_out.
+// / tile_rows.  nra == 0: scales in plain row-major bytes [n_rows, K/16] instead of atoms.  One
+// thread per 16-element block; tensor scale from amax_bits[0], also written to *g_out.
 // ------------------------------------------------------------------------------------------------
 __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, const int* __restrict__ src_rows,
                                  long long n_rows, int n_src_rows, const int* __restrict__ offsets,
@@ -353,7 +353,48 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, con
     uint32_t c[2];
     const uint32_t sb = nvfp4_block_exact(v, g, c);
     *reinterpret_cast<uint2*>(codes + r * (K / 2) + kb * 8) = make_uint2(c[0], c[1]);
-    sf[act_sf_offset(tile, j, kb, stages, nra)] = (uint8_t)sb;
+    if (nra > 0) sf[act_sf_offset(tile, j, kb, stages, nra)] = (uint8_t)sb;
+    else sf[r * nb + kb] = (uint8_t)sb;  // plain row-major scales
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Grouped copy of per-token NVFP4 rows: grouped row r gets the codes of token tok_of_row[r]
+// (quantised once per token: a row's codes and block scales depend only on its values and the
+// tensor scale) and its block scales go into the consuming GEMM's tile-local atoms.  One warp per
+// row; K is a multiple of 128, so a row is a whole number of 512-byte code chunks and 4-byte scale
+// groups, and the four scales of one K atom of a row are four adjacent bytes of the atom.
+// ------------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    gather_act_q_kernel(const uint8_t* __restrict__ codes_tok, const uint8_t* __restrict__ sf_tok, int K,
+                        const int* __restrict__ tok_of_row, long long n_rows, int n_tok,
+                        const int* __restrict__ offsets, const int* __restrict__ tile0, int n_experts, int tile_rows,
+                        int nra, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, unsigned* status) {
+  const int lane = threadIdx.x & 31;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  const int row_bytes = K / 2, nb = K / 16;
+  const int stages = (K + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K;
+  for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < n_rows; r += nwarps) {
+    const int t = tok_of_row[r];
+    if (t < 0 || t >= n_tok) {
+      if (lane == 0) atomicOr(status, DEV_STATUS_BAD_INDEX);
+      continue;
+    }
+    int lo = 0, hi = n_experts - 1;  // largest expert whose first row is <= r
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(offsets + mid) <= r) lo = mid;
+      else hi = mid - 1;
+    }
+    const int local = (int)(r - __ldg(offsets + lo));
+    const long long tile = __ldg(tile0 + lo) + local / tile_rows;
+    const int j = local % tile_rows;
+    for (int c = lane * 16; c < row_bytes; c += 32 * 16)
+      *reinterpret_cast<uint4*>(codes + r * row_bytes + c) =
+          *reinterpret_cast<const uint4*>(codes_tok + (long long)t * row_bytes + c);
+    for (int q = lane; q < nb / 4; q += 32)
+      *reinterpret_cast<uint32_t*>(sf + act_sf_offset(tile, j, 4 * q, stages, nra)) =
+          *reinterpret_cast<const uint32_t*>(sf_tok + (long long)t * nb + 4 * q);
   }
 }
 

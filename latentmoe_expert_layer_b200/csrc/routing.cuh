@@ -328,39 +328,53 @@ __global__ void __launch_bounds__(256)
 // 32 at a time: lanes holding the same expert are ranked with __match_any_sync, and a per-expert
 // running base (from scan_units_kernel) gives each assignment its grouped row.
 // ------------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(32)
+__global__ void __launch_bounds__(256)
     assign_rows_kernel(const int* __restrict__ topk_idx, const float* __restrict__ topk_gate,
                        const int* __restrict__ chunk_base, int T, int n_experts, int k, int chunk_tokens,
                        int* __restrict__ row_of, int* __restrict__ tok_of_row, float* __restrict__ gate_of_row,
                        unsigned* status) {
-  extern __shared__ int s_base[];  // [n_experts]
-  const int lane = threadIdx.x;
-  // chunk bases, 8 loads in flight per lane at a time
-  for (int e0 = lane; e0 < n_experts; e0 += 8 * 32) {
-    int vals[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = e0 + 32 * j;
-      vals[j] = e < n_experts ? chunk_base[(long long)e * gridDim.x + blockIdx.x] : 0;
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (e0 + 32 * j < n_experts) s_base[e0 + 32 * j] = vals[j];
-  }
-  __syncwarp();
+  extern __shared__ int s_hist[];  // [W][n_experts]: per warp, then per-warp running bases
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, W = blockDim.x >> 5;
+  for (int i = threadIdx.x; i < W * n_experts; i += blockDim.x) s_hist[i] = 0;
   const int t_begin = blockIdx.x * chunk_tokens;
   const int t_end = min(T, t_begin + chunk_tokens);
   const long long a_begin = (long long)t_begin * k, a_end = (long long)t_end * k;
   const long long TK = (long long)T * k;
-  // the next round's expert ids and gates are loaded while this round is ranked
-  int e_next = (a_begin + lane < a_end) ? topk_idx[a_begin + lane] : 0;
-  float g_next = (a_begin + lane < a_end) ? topk_gate[a_begin + lane] : 0.f;
-  for (long long a0 = a_begin; a0 < a_end; a0 += 32) {
+  // warp w walks the w-th contiguous sub-range of the chunk's assignments, in (token, slot) order
+  const long long per = (a_end - a_begin + W - 1) / W;
+  const long long s_begin = min(a_end, a_begin + warp * per), s_end = min(a_end, s_begin + per);
+  int* my = s_hist + warp * n_experts;
+  __syncthreads();
+  // 1. per-warp expert counts (the leader of each group of equal experts adds the group's size)
+  for (long long a0 = s_begin; a0 < s_end; a0 += 32) {
     const long long a = a0 + lane;
-    const bool act = a < a_end;
-    int e = act ? e_next : -1 - lane;  // inactive lanes get unique keys
+    const int e = a < s_end ? topk_idx[a] : -1 - lane;
+    const bool e_ok = e >= 0 && e < n_experts;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e_ok && lane == __ffs(peers) - 1) my[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // 2. per-warp bases: the chunk's base for the expert plus the counts of the earlier warps
+  for (int e = threadIdx.x; e < n_experts; e += blockDim.x) {
+    int run = chunk_base[(long long)e * gridDim.x + blockIdx.x];
+    for (int w = 0; w < W; ++w) {
+      const int v = s_hist[w * n_experts + e];
+      s_hist[w * n_experts + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  // 3. ranks: lanes holding the same expert are ranked with __match_any_sync on top of the warp's
+  //    running base; the next round's ids and gates load while this round is ranked
+  int e_next = (s_begin + lane < s_end) ? topk_idx[s_begin + lane] : 0;
+  float g_next = (s_begin + lane < s_end) ? topk_gate[s_begin + lane] : 0.f;
+  for (long long a0 = s_begin; a0 < s_end; a0 += 32) {
+    const long long a = a0 + lane;
+    const bool act = a < s_end;
+    const int e = act ? e_next : -1 - lane;  // inactive lanes get unique keys
     const float g = act ? g_next : 0.f;
-    if (a + 32 < a_end) {
+    if (a + 32 < s_end) {
       e_next = topk_idx[a + 32];
       g_next = topk_gate[a + 32];
     }
@@ -370,9 +384,9 @@ __global__ void __launch_bounds__(32)
     const int rank = __popc(peers & ((1u << lane) - 1u));
     const int leader = __ffs(peers) - 1;
     int base = 0;
-    if (act && e_ok) base = s_base[e];
+    if (act && e_ok) base = my[e];
     __syncwarp();
-    if (act && e_ok && lane == leader) s_base[e] = base + __popc(peers);
+    if (act && e_ok && lane == leader) my[e] = base + __popc(peers);
     __syncwarp();
     if (act) {
       const int row = e_ok ? base + rank : -1;
