@@ -244,7 +244,12 @@ int n_chunks_for(int T, int N, int* chunk_tokens) {
   return (T + ct - 1) / ct;
 }
 
-int topk_threads(int chunk_tokens) { return 32 * (chunk_tokens < 32 ? chunk_tokens : 32); }
+// blocks per token chunk of the top-K kernel: chunks of more than 32 tokens are split so that a
+// warp selects for about one token (the chunk count is capped by the scan's shared memory)
+int topk_parts(int chunk_tokens) {
+  int p = chunk_tokens / 32;
+  return p < 1 ? 1 : (p > 16 ? 16 : p);
+}
 
 constexpr int kScanSmemMax = 200 * 1024;
 
@@ -489,7 +494,11 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
   // 3. top-K + softmax + per-chunk histogram
   int ct;
   const int nch = n_chunks_for(T, N, &ct);
-  chk(launch_topk_hist(nch, topk_threads(ct), s, c->logits, c->b_router, T, N, K, ct, idx, gate, c->chunk_counts));
+  {
+    const int parts = topk_parts(ct);
+    if (parts > 1) chk(cudaMemsetAsync(c->chunk_counts, 0, (size_t)N * nch * sizeof(int), s));
+    chk(launch_topk_hist(nch, parts, s, c->logits, c->b_router, T, N, K, ct, idx, gate, c->chunk_counts));
+  }
   mark(3);
   // 4. expert offsets and grouped-GEMM unit lists
   UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1, c->unit_u0};
@@ -936,7 +945,11 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   // 3. top-K + softmax + per-chunk histogram
   int ct;
   const int nch = n_chunks_for(T, N, &ct);
-  chk(launch_topk_hist(nch, topk_threads(ct), s, c->logits, c->b_router, T, N, K, ct, idx, gate, c->chunk_counts));
+  {
+    const int parts = topk_parts(ct);
+    if (parts > 1) chk(cudaMemsetAsync(c->chunk_counts, 0, (size_t)N * nch * sizeof(int), s));
+    chk(launch_topk_hist(nch, parts, s, c->logits, c->b_router, T, N, K, ct, idx, gate, c->chunk_counts));
+  }
   mark(3);
   // 4. expert offsets and grouped-GEMM unit lists
   UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1, c->unit_u0};
@@ -1267,7 +1280,7 @@ extern "C" lmoe_status lmoe_route_noalloc(const float* logits, const float* bias
   if (cudaMemsetAsync(status, 0, sizeof(unsigned), s) != cudaSuccess) return LMOE_ERR_CUDA;
   int ct;
   const int nch = n_chunks_for(T, N, &ct);
-  if (launch_topk_hist(nch, topk_threads(ct), s, logits, bias, T, N, K, ct, topk_idx, topk_gate, chunk_counts) !=
+  if (launch_topk_hist(nch, 1, s, logits, bias, T, N, K, ct, topk_idx, topk_gate, chunk_counts) !=
       cudaSuccess)
     return LMOE_ERR_CUDA;
   UnitListSpec none{nullptr, nullptr, 0, 64, 0, nullptr};

@@ -53,14 +53,18 @@ __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
 template <int P>
 __global__ void __launch_bounds__(1024)
     topk_hist_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int n_experts,
-                     int k, int chunk_tokens, int* __restrict__ topk_idx, float* __restrict__ topk_gate,
+                     int k, int chunk_tokens, int parts, int* __restrict__ topk_idx, float* __restrict__ topk_gate,
                      int* __restrict__ chunk_counts) {
   extern __shared__ int s_counts[];  // [n_experts], then per warp 32 keys + 32 indices
   for (int e = threadIdx.x; e < n_experts; e += blockDim.x) s_counts[e] = 0;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  const int t_begin = blockIdx.x * chunk_tokens;
-  const int t_end = min(T, t_begin + chunk_tokens);
+  // `parts` blocks share a chunk: block b takes part (b mod parts) of chunk (b / parts)
+  const int chunk = blockIdx.x / parts, part = blockIdx.x - chunk * parts;
+  const int n_chunks = gridDim.x / parts;
+  const int sub = (chunk_tokens + parts - 1) / parts;
+  const int t_begin = chunk * chunk_tokens + part * sub;
+  const int t_end = min(min(T, (chunk + 1) * chunk_tokens), t_begin + sub);
   for (int t = t_begin + warp; t < t_end; t += nwarps) {
     const float* lrow = logits + (long long)t * n_experts;
     // order-preserving keys: a larger logit has a larger key, -0 and +0 share one; padding is 0
@@ -75,15 +79,23 @@ __global__ void __launch_bounds__(1024)
         key[i] = 0u;
       }
     }
-    // the K-th largest key X: the largest value with at least K keys >= X, built bit by bit
+    // the K-th largest key X: the largest value with at least K keys >= X, built two bits at a
+    // time (three independent warp-wide counts per step)
     uint32_t X = 0u;
 #pragma unroll 1
-    for (int b = 31; b >= 0; --b) {
-      const uint32_t Y = X | (1u << b);
-      int cnt = 0;
+    for (int b = 30; b >= 0; b -= 2) {
+      const uint32_t Y1 = X | (1u << b), Y2 = X | (2u << b), Y3 = X | (3u << b);
+      int c1 = 0, c2 = 0, c3 = 0;
 #pragma unroll
-      for (int i = 0; i < P; ++i) cnt += key[i] >= Y;
-      if (__reduce_add_sync(0xffffffffu, cnt) >= k) X = Y;
+      for (int i = 0; i < P; ++i) {
+        c1 += key[i] >= Y1;
+        c2 += key[i] >= Y2;
+        c3 += key[i] >= Y3;
+      }
+      c1 = __reduce_add_sync(0xffffffffu, c1);
+      c2 = __reduce_add_sync(0xffffffffu, c2);
+      c3 = __reduce_add_sync(0xffffffffu, c3);
+      X = c3 >= k ? Y3 : c2 >= k ? Y2 : c1 >= k ? Y1 : X;
     }
     // selected: every key above X, then the lowest expert indices among the keys equal to X
     int above = 0;
@@ -142,9 +154,13 @@ __global__ void __launch_bounds__(1024)
     }
   }
   __syncthreads();
-  // expert-major layout [N][n_chunks]: the scan reads one expert's chunks contiguously
-  for (int e = threadIdx.x; e < n_experts; e += blockDim.x)
-    chunk_counts[(long long)e * gridDim.x + blockIdx.x] = s_counts[e];
+  // expert-major layout [N][n_chunks]: the scan reads one expert's chunks contiguously; blocks that
+  // share a chunk add into a zeroed histogram
+  for (int e = threadIdx.x; e < n_experts; e += blockDim.x) {
+    int* dst = chunk_counts + (long long)e * n_chunks + chunk;
+    if (parts == 1) *dst = s_counts[e];
+    else if (s_counts[e]) atomicAdd(dst, s_counts[e]);
+  }
 }
 
 // candidates per lane: the next power of two >= ceil(N / 32)
@@ -154,17 +170,25 @@ inline int topk_lane_candidates(int n_experts) {
   return p;
 }
 
-inline cudaError_t launch_topk_hist(int n_chunks, int threads, cudaStream_t s, const float* logits, const float* bias,
+// parts > 1: blocks per chunk (the caller zeroes chunk_counts first); threads per block from the
+// tokens each block takes
+inline cudaError_t launch_topk_hist(int n_chunks, int parts, cudaStream_t s, const float* logits, const float* bias,
                                     int T, int N, int K, int ct, int* idx, float* gate, int* chunk_counts) {
+  const int sub = (ct + parts - 1) / parts;
+  const int threads = 32 * (sub < 32 ? sub : 32);
   const size_t sm = (size_t)N * sizeof(int) + (size_t)(threads / 32) * 64 * sizeof(int);
+  const int grid = n_chunks * parts;
+#define LMOE_TOPK(PP) \
+  topk_hist_kernel<PP><<<grid, threads, sm, s>>>(logits, bias, T, N, K, ct, parts, idx, gate, chunk_counts)
   switch (topk_lane_candidates(N)) {
-    case 1: topk_hist_kernel<1><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
-    case 2: topk_hist_kernel<2><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
-    case 4: topk_hist_kernel<4><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
-    case 8: topk_hist_kernel<8><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
-    case 16: topk_hist_kernel<16><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
-    default: topk_hist_kernel<32><<<n_chunks, threads, sm, s>>>(logits, bias, T, N, K, ct, idx, gate, chunk_counts); break;
+    case 1: LMOE_TOPK(1); break;
+    case 2: LMOE_TOPK(2); break;
+    case 4: LMOE_TOPK(4); break;
+    case 8: LMOE_TOPK(8); break;
+    case 16: LMOE_TOPK(16); break;
+    default: LMOE_TOPK(32); break;
   }
+#undef LMOE_TOPK
   return cudaGetLastError();
 }
 
