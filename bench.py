@@ -37,7 +37,31 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 DEFAULT_STEPS = {"tiny": 200, "decode": 400, "skewed": 40, "prefill": 20}
 DEFAULT_STEPS.update({"decode_small": 400, "decode_nvfp4": 400, "prefill_nvfp4": 20, "nvfp4_tiny": 200,
                       "nvfp4_mid": 100, "ultra_decode": 200, "ultra_decode_nvfp4": 200, "ultra_prefill": 10,
-                      "standard_decode": 400, "standard_prefill": 20})
+                      "standard_decode": 400, "standard_prefill": 20, "prefill_small": 20})
+
+
+# DRAM traffic per launch of the expert GEMMs over their algorithmic bytes (dram__bytes_read.sum +
+# dram__bytes_write.sum from ncu section captures, summarised under profiles/): the decode NVFP4
+# capture is the full workload; the bf16 ones are smaller cases of the same regime (Super dims with
+# 128 experts: T = 64 for decode, T = 4096 for prefill), scaled to a launch by its algorithmic
+# bytes, which grow with the units processed.  Valid only while the GEMM's sources are the ones
+# captured (TRAFFIC_SOURCES_SHA256); otherwise the roofline reports no traffic.
+TRAFFIC_RATIO = {
+    ("bf16", "decode", "expert_up"): 0.998, ("bf16", "decode", "expert_down"): 1.002,
+    ("nvfp4", "decode", "expert_up"): 1.040, ("nvfp4", "decode", "expert_down"): 1.119,
+    ("bf16", "prefill", "expert_up"): 0.987, ("bf16", "prefill", "expert_down"): 1.008,
+}
+TRAFFIC_SOURCES = ("gemm_tc.cuh", "ptx.cuh", "nvfp4.cuh", "lmoe.cu")
+TRAFFIC_SOURCES_SHA256 = "60bc4c0ef1e0f155c59701185d66cc95d66e7ab037e55d7a86961a917628ce5d"
+
+
+def gemm_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "latentmoe_expert_layer_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
 
 
 def peaks():
@@ -117,6 +141,15 @@ def algorithmic_work(wl, counts: np.ndarray):
     w_exp = touched * eb(m * le)                    # one expert matrix set (W1 or W2) of the touched experts
     up = {"bytes": w_exp + eb(tk * le) + eb(tk * m), "flops": 2 * tk * m * le}
     down = {"bytes": w_exp + eb(tk * m) + tk * le * 2 + tk * 4, "flops": 2 * tk * m * le}
+    # At decode sizes the library folds the shared expert into the two expert launches (its first
+    # matrix into the up launch, its second, writing fp32 y_s, into the down launch); their bytes
+    # and FLOPs are then part of those launches.  Same condition as the library's split path.
+    folded = tk <= 48 * n and (fp4 or t <= 512)
+    if folded:
+        up["bytes"] += eb(ms * d) + eb(t * d) + eb(t * ms)
+        up["flops"] += 2 * t * ms * d
+        down["bytes"] += eb(d * ms) + eb(t * ms) + t * d * 4
+        down["flops"] += 2 * t * d * ms
     layer_bytes = (2 * w_exp + (n + l) * d * 2 + eb(ms * d) + eb(d * ms) + d * l * 2 + 2 * t * d * 2 + tk * 8)
     layer_flops = 2 * t * ((n + l) * d + ms * d + d * (l + ms)) + 4 * tk * m * le
     return {"expert_up": up, "expert_down": down, "layer": {"bytes": int(layer_bytes), "flops": layer_flops},
@@ -321,10 +354,14 @@ def run_ours(args, wl, rank, world):
         unit_work = None
     roof = None
     if unit_work is not None:
+        ratio = TRAFFIC_RATIO.get((wl.precision, "decode" if decode_like else "prefill", dom))
+        traffic = None
+        if ratio is not None and gemm_sources_sha256() == TRAFFIC_SOURCES_SHA256:
+            traffic = ratio * unit_work["bytes"]
         if decode_like:
             ach = unit_work["bytes"] / (per_launch_ms * 1e-3) / 1e9
             roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": ach / pk["hbm_gbs"], "traffic": None, "algorithmic_bytes": unit_work["bytes"],
+                    "frac": ach / pk["hbm_gbs"], "traffic": traffic, "algorithmic_bytes": unit_work["bytes"],
                     "launch_ms": per_launch_ms, "peak_source": pk_kind}
         else:
             ach = unit_work["flops"] / (per_launch_ms * 1e-3) / 1e12
@@ -334,7 +371,8 @@ def run_ours(args, wl, rank, world):
                 p *= 4.0
                 src = pk_kind + " bf16 (sustained) x nominal FP4/BF16 ratio 4"
             roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": p, "unit": "TFLOP/s",
-                    "frac": ach / p, "traffic": None, "algorithmic_flops": unit_work["flops"],
+                    "frac": ach / p, "traffic": traffic, "algorithmic_flops": unit_work["flops"],
+                    "algorithmic_bytes": unit_work["bytes"],
                     "launch_ms": per_launch_ms, "peak_source": src}
     step_ms = ms_max / args.steps
     lay = work["layer"]
