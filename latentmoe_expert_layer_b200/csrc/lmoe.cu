@@ -52,7 +52,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 enum Variant { V_SMALL = 0, V_LARGE = 1, V_SMALL4 = 2, V_LARGE4 = 3 };
 constexpr int V_BN[4] = {64, 256, 64, 192};
 constexpr int V_STAGES[4] = {8, 4, 7, 4};
-constexpr int V_BOXN[4] = {16, 64, 16, 64};
+constexpr int V_BOXN[4] = {16, 256, 16, 192};  // one token box per stage at prefill sizes
 constexpr bool V_FP4[4] = {false, false, true, true};
 constexpr int V_ACC_SPLIT[4] = {4, 1, 2, 1};  // decode-sized tiles rotate over independent accumulators
 // K stages of one token tile's activation scales that fit resident in TMEM (0: per-stage copies)
