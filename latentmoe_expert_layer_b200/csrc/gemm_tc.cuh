@@ -120,7 +120,7 @@ template <int BN_MAX, int STAGES, bool FP4, int ACC_SPLIT, int RES_STAGES>
 struct GemmSmem {
   static constexpr int NRA = (BN_MAX + 127) / 128;                    // 128-row scale atoms of B
   static constexpr int B_STAGE_BYTES = BN_MAX * 128;
-  static constexpr int SFA_STAGE_BYTES = FP4 ? 4 * SF_ATOM_BYTES : 0;
+  static constexpr int SFA_STAGE_BYTES = FP4 ? 4 * SF_ATOM_BYTES * SF_WREP : 0;  // replicated weight atoms
   static constexpr int SFB_STAGE_BYTES = FP4 ? 4 * NRA * SF_ATOM_BYTES : 0;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES + SFA_STAGE_BYTES + SFB_STAGE_BYTES;
   static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           if constexpr (FP4) {
             uint8_t* ssfa = sb + S::B_STAGE_BYTES;
             uint8_t* ssfb = ssfa + S::SFA_STAGE_BYTES;
-            bulk_load(ssfa, pr.w_sf + ((long long)(un.a_row >> 7) * pr.w_atoms_k + kb * 4) * SF_ATOM_BYTES,
+            bulk_load(ssfa, pr.w_sf + ((long long)(un.a_row >> 7) * pr.w_atoms_k + kb * 4) * (SF_ATOM_BYTES * SF_WREP),
                       S::SFA_STAGE_BYTES, &full[stage]);
             if (fill)
               bulk_load(ssfb, pr.act_sf + ((long long)un.tile * pr.act_sf_stages + kb) * S::SFB_STAGE_BYTES,
@@ -456,9 +456,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               sfb_pitch = nra;
             }
             if (++sf_slot == S::SF_SLOTS) sf_slot = 0;
+            // weight scales: two copies of two replicated atoms each (K atoms 0-1, then 2-3)
+            tcgen05_cp_128x256b(t_sfa, smem_desc_sf_pair(ssfa));
+            tcgen05_cp_128x256b(t_sfa + 8, smem_desc_sf_pair(ssfa + 2 * SF_ATOM_BYTES * SF_WREP));
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              tcgen05_cp_32x128b_x4(t_sfa + 4 * k, smem_desc_sf_atom(ssfa + k * SF_ATOM_BYTES));
               if (fill)
                 for (int ra = 0; ra < nra; ++ra)
                   tcgen05_cp_32x128b_x4(t_sfb + 4 * (k * sfb_pitch + ra),

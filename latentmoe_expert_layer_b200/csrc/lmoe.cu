@@ -51,7 +51,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 // tiles (tensor-core bound at prefill sizes), each in bf16 and in NVFP4.
 enum Variant { V_SMALL = 0, V_LARGE = 1, V_SMALL4 = 2, V_LARGE4 = 3 };
 constexpr int V_BN[4] = {64, 256, 64, 192};
-constexpr int V_STAGES[4] = {8, 4, 7, 4};
+constexpr int V_STAGES[4] = {8, 4, 6, 4};
 constexpr int V_BOXN[4] = {16, 256, 16, 192};  // one token box per stage at prefill sizes
 constexpr bool V_FP4[4] = {false, false, true, true};
 constexpr int V_ACC_SPLIT[4] = {4, 1, 2, 1};  // decode-sized tiles rotate over independent accumulators
@@ -784,7 +784,9 @@ lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream
     // quantise W1, W2, W_s1, W_s2 on the device; keep only codes, scale atoms and tensor scales
     __nv_bfloat16* ws2_tmp = nullptr;
     ok = ok && dalloc(&ws2_tmp, (size_t)d * ms) && conv(w->ws2, d, ms, ms, ws2_tmp, ms, 0);
-    auto sf_bytes = [](long long rows, int K) { return (size_t)(rows / 128) * sf_atoms_k(K) * SF_ATOM_BYTES; };
+    auto sf_bytes = [](long long rows, int K) {
+      return (size_t)(rows / 128) * sf_atoms_k(K) * SF_ATOM_BYTES * SF_WREP;
+    };
     ok = ok && dalloc(&c->w1q, (size_t)N * m * l / 2) && dalloc(&c->w1_sf, sf_bytes((long long)N * m, l));
     ok = ok && dalloc(&c->w2q, (size_t)N * l * m / 2) && dalloc(&c->w2_sf, sf_bytes((long long)N * l, m));
     ok = ok && dalloc(&c->ws1q, (size_t)ms * d / 2) && dalloc(&c->ws1_sf, sf_bytes(ms, d));
@@ -1097,9 +1099,10 @@ lmoe_status lmoe_export_nvfp4(lmoe_handle c, int32_t which, int32_t index, uint8
   if (cudaMemcpy(gscale_host, c->wg + gi, sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess) return LMOE_ERR_CUDA;
   // the matrix's scale atoms are contiguous (its rows start on a 128-row tile)
   const int atoms_k = sf_atoms_k(K);
-  const size_t atom_bytes = (size_t)(rows / 128) * atoms_k * SF_ATOM_BYTES;
+  const size_t atom_bytes = (size_t)(rows / 128) * atoms_k * SF_ATOM_BYTES * SF_WREP;
   std::vector<uint8_t> tmp(atom_bytes);
-  if (cudaMemcpy(tmp.data(), atoms + (row0 / 128) * atoms_k * SF_ATOM_BYTES, atom_bytes, cudaMemcpyDeviceToHost) !=
+  if (cudaMemcpy(tmp.data(), atoms + (row0 / 128) * atoms_k * SF_ATOM_BYTES * SF_WREP, atom_bytes,
+                 cudaMemcpyDeviceToHost) !=
       cudaSuccess)
     return LMOE_ERR_CUDA;
   for (long long r = 0; r < rows; ++r)

@@ -202,10 +202,16 @@ __host__ __device__ __forceinline__ long long act_sf_offset(long long tile, int 
   return (((tile * stages + st) * 4 + ka) * nra + (j >> 7)) * 512 + (j & 31) * 16 + ((j & 127) >> 5) * 4 + s;
 }
 
-// Byte offset of the scale of (row r, 16-element block kb) inside a weight-scale atom array with
-// `atoms_k` K atoms per 128-row tile.
-__host__ __device__ __forceinline__ long long sf_atom_offset(long long r, int kb, int atoms_k) {
-  return ((r >> 7) * atoms_k + (kb >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (kb & 3);
+// Weight-scale atoms are stored replicated: each 512-byte atom four times in a row (2 KB), the
+// image tcgen05.cp.128x256b turns into the scale columns of all four TMEM lane quadrants (lane L
+// reads bytes 16 L .. 16 L + 15 of the 2 KB block), so one copy instruction moves two K atoms.
+constexpr int SF_WREP = 4;
+
+// Byte offset of the scale of (row r, 16-element block kb), copy `rep` (0..3), inside a
+// weight-scale array with `atoms_k` K atoms per 128-row tile.
+__host__ __device__ __forceinline__ long long sf_atom_offset(long long r, int kb, int atoms_k, int rep = 0) {
+  return ((r >> 7) * atoms_k + (kb >> 2)) * (512 * SF_WREP) + rep * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 +
+         (kb & 3);
 }
 
 __host__ __device__ __forceinline__ int sf_atoms_k(int K) { return ((K + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K) * 4; }
@@ -266,7 +272,8 @@ __global__ void quant_weight_kernel(const __nv_bfloat16* __restrict__ w, long lo
     uint32_t c[2];
     const uint32_t sb = mse ? nvfp4_block_mse(v, g, c) : nvfp4_block(v, g, c);
     *reinterpret_cast<uint2*>(codes + r * (K / 2) + kb * 8) = make_uint2(c[0], c[1]);
-    sf_atoms[sf_atom_offset(r, kb, atoms_k)] = (uint8_t)sb;
+#pragma unroll
+    for (int rp = 0; rp < SF_WREP; ++rp) sf_atoms[sf_atom_offset(r, kb, atoms_k, rp)] = (uint8_t)sb;
     if (kb == 0 && r % rows_per_group == 0) g_out[grp] = g;
   }
 }

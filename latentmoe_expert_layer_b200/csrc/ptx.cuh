@@ -165,6 +165,25 @@ __device__ __forceinline__ void tcgen05_cp_32x128b_x4(uint32_t dst_tmem, uint64_
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(dst_tmem), "l"(src_desc) : "memory");
 }
 
+// Copy a 128-row x 256-bit shared-memory matrix into 8 consecutive TMEM columns of lanes 0..127
+// (lane L gets row L: its first 16 bytes in columns 0-3, its second 16 bytes in columns 4-7).
+__device__ __forceinline__ void tcgen05_cp_128x256b(uint32_t dst_tmem, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(dst_tmem), "l"(src_desc) : "memory");
+}
+
+// Shared-memory descriptor of two replicated weight-scale atoms (2 KB each, back to back) as the
+// 128-row x 256-bit source of tcgen05_cp_128x256b, without swizzle: 8-row core matrices of 128
+// contiguous bytes, 128 bytes apart along the rows (stride byte offset); the second 16 bytes of
+// every row 2048 bytes further (leading byte offset).
+__device__ __forceinline__ uint64_t smem_desc_sf_pair(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(2048u >> 4) << 16;  // leading byte offset: the next K core matrix
+  d |= static_cast<uint64_t>(128u >> 4) << 32;   // stride byte offset: next 8 rows
+  d |= static_cast<uint64_t>(1) << 46;           // descriptor version (sm_100)
+  return d;                                      // swizzle mode 0: none
+}
+
 // Shared-memory descriptor of a 32-row x 16-byte block without swizzle (8-row core matrices of 128
 // contiguous bytes, 128 bytes apart).  Used as the tcgen05.cp source of one scale atom.
 __device__ __forceinline__ uint64_t smem_desc_sf_atom(uint32_t smem_addr) {
