@@ -144,8 +144,13 @@ typedef enum {
   LMOE_BUF_H = 5,          /* bf16 [T, l]   latent h = W_down x (UNSUPPORTED for a standard MoE) */
   LMOE_BUF_Z = 6,          /* bf16 [T, l + m_s] columns 0..l-1: latent sum z; the rest: sqrelu(W_s1 x) */
   LMOE_BUF_U = 7,          /* bf16 [T*K, m] expert hidden activations, grouped rows (bf16 precision) */
-  /* NVFP4 precision only: packed E2M1 codes [rows, K/2] and row-major E4M3 scales
-   * [rows, 16 * ceil(K / 256)] of the quantised activations, and the fp32 shared-expert output */
+  /* NVFP4 precision only: packed E2M1 codes [rows, K/2] (element 2i in the low nibble) and the E4M3
+   * block scales of the quantised activations, and the fp32 shared-expert output.  Scales are in
+   * tile-local 512-byte atoms, the layout the block-scaled GEMM reads: with the forward's token tile
+   * of R rows (64 when T*K <= 48*N, else 192), nra = ceil(R / 128), S = ceil(K / 256), the scale of
+   * row j of tile tile (grouped tensors: tiles restart at each expert's first row) and 16-element
+   * block b is at byte (((tile*S + b/16)*4 + (b/4)%4)*nra + j/128)*512 + (j%32)*16 + ((j%128)/32)*4
+   * + b%4.  The count covers the allocation for max_tokens. */
   LMOE_BUF_XQ = 8,         /* x codes [T, d/2] */
   LMOE_BUF_X_SF = 9,       /* x scales */
   LMOE_BUF_HQ = 10,        /* h codes, grouped rows [T*K, l/2] */
