@@ -48,11 +48,11 @@ DEFAULT_STEPS.update({"decode_small": 400, "decode_nvfp4": 400, "prefill_nvfp4":
 # captured (TRAFFIC_SOURCES_SHA256); otherwise the roofline reports no traffic.
 TRAFFIC_RATIO = {
     ("bf16", "decode", "expert_up"): 0.998, ("bf16", "decode", "expert_down"): 1.002,
-    ("nvfp4", "decode", "expert_up"): 1.040, ("nvfp4", "decode", "expert_down"): 1.119,
-    ("bf16", "prefill", "expert_up"): 0.987, ("bf16", "prefill", "expert_down"): 1.008,
+    ("nvfp4", "decode", "expert_up"): 1.385, ("nvfp4", "decode", "expert_down"): 1.493,
+    ("bf16", "prefill", "expert_up"): 0.983, ("bf16", "prefill", "expert_down"): 0.995,
 }
 TRAFFIC_SOURCES = ("gemm_tc.cuh", "ptx.cuh", "nvfp4.cuh", "lmoe.cu")
-TRAFFIC_SOURCES_SHA256 = "60bc4c0ef1e0f155c59701185d66cc95d66e7ab037e55d7a86961a917628ce5d"
+TRAFFIC_SOURCES_SHA256 = "dc2fdaee937be0a25a464d9b8ec07484161a6cb3c9bad3665aaef758d8e3c9ad"
 
 
 def gemm_sources_sha256() -> str:
