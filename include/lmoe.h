@@ -150,7 +150,8 @@ typedef enum {
    * of R rows (64 when T*K <= 48*N, else 192), nra = ceil(R / 128), S = ceil(K / 256), the scale of
    * row j of tile tile (grouped tensors: tiles restart at each expert's first row) and 16-element
    * block b is at byte (((tile*S + b/16)*4 + (b/4)%4)*nra + j/128)*512 + (j%32)*16 + ((j%128)/32)*4
-   * + b%4.  The count covers the allocation for max_tokens. */
+   * + b%4; with 192-row tiles every atom is stored four times in a row (multiply the atom index, the
+   * part before *512, by 4 and add 512 per copy).  The count covers the allocation for max_tokens. */
   LMOE_BUF_XQ = 8,         /* x codes [T, d/2] */
   LMOE_BUF_X_SF = 9,       /* x scales */
   LMOE_BUF_HQ = 10,        /* h codes, grouped rows [T*K, l/2] */

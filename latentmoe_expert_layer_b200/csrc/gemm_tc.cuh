@@ -121,7 +121,11 @@ struct GemmSmem {
   static constexpr int NRA = (BN_MAX + 127) / 128;                    // 128-row scale atoms of B
   static constexpr int B_STAGE_BYTES = BN_MAX * 128;
   static constexpr int SFA_STAGE_BYTES = FP4 ? 4 * SF_ATOM_BYTES * SF_WREP : 0;  // replicated weight atoms
-  static constexpr int SFB_STAGE_BYTES = FP4 ? 4 * NRA * SF_ATOM_BYTES : 0;
+  // activation scales of the variants without resident scales (prefill sizes) are stored replicated
+  // like the weight scales, so one 128x256b copy moves both 128-row atoms of a K atom
+  static constexpr int SFB_REP = (FP4 && RES_STAGES == 0) ? SF_WREP : 1;
+  static_assert(SFB_REP == 1 || NRA == 2, "replicated activation scales pair the two row atoms of a K atom");
+  static constexpr int SFB_STAGE_BYTES = FP4 ? 4 * NRA * SF_ATOM_BYTES * SFB_REP : 0;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES + SFA_STAGE_BYTES + SFB_STAGE_BYTES;
   static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
   static constexpr int BAR_OFF = EPI_OFF + 4 * EPI_STAGE_BYTES;
@@ -453,18 +457,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               sfb_pitch = S::NRA;
             } else {
               t_sfb = tmem_base + S::SFB_COL0 + (uint32_t)(sf_slot * 16 * S::NRA);
-              sfb_pitch = nra;
+              sfb_pitch = S::SFB_REP > 1 ? S::NRA : nra;
             }
             if (++sf_slot == S::SF_SLOTS) sf_slot = 0;
             // weight scales: two copies of two replicated atoms each (K atoms 0-1, then 2-3)
             tcgen05_cp_128x256b(t_sfa, smem_desc_sf_pair(ssfa));
             tcgen05_cp_128x256b(t_sfa + 8, smem_desc_sf_pair(ssfa + 2 * SF_ATOM_BYTES * SF_WREP));
+            if constexpr (S::SFB_REP > 1) {
+              // both row atoms of K atom k (replicated, 2 KB apart) in one copy: columns 8k .. 8k + 7
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              if (fill)
-                for (int ra = 0; ra < nra; ++ra)
-                  tcgen05_cp_32x128b_x4(t_sfb + 4 * (k * sfb_pitch + ra),
-                                        smem_desc_sf_atom(ssfb + (k * S::NRA + ra) * SF_ATOM_BYTES));
+              for (int k = 0; k < 4; ++k)
+                tcgen05_cp_128x256b(t_sfb + 8 * k, smem_desc_sf_pair(ssfb + k * 2 * SF_ATOM_BYTES * SF_WREP));
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                if (fill)
+                  for (int ra = 0; ra < nra; ++ra)
+                    tcgen05_cp_32x128b_x4(t_sfb + 4 * (k * sfb_pitch + ra),
+                                          smem_desc_sf_atom(ssfb + (k * S::NRA + ra) * SF_ATOM_BYTES));
+              }
             }
 #pragma unroll
             for (int k = 0; k < 4; ++k, ++mma_i)  // K = 64 E2M1 per MMA: +32 bytes = +2 in the address field
@@ -607,9 +618,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(pr.out) + row * pr.ldo + f / 2) =
                 make_uint4(cw[0], cw[1], cw[2], cw[3]);
             // the two blocks are adjacent bytes of one atom row (f is a multiple of 32)
-            *reinterpret_cast<uint16_t*>(
-                pr.out_sf + act_sf_offset(un.tile, c * 32 + lane, f / 16, pr.out_sf_stages, S::NRA)) =
-                (uint16_t)sbs;
+            for (int rp = 0; rp < S::SFB_REP; ++rp)
+              *reinterpret_cast<uint16_t*>(pr.out_sf + act_sf_offset(un.tile, c * 32 + lane, f / 16, pr.out_sf_stages,
+                                                                     S::NRA, rp, S::SFB_REP)) = (uint16_t)sbs;
           }
         } else if (f32_out) {
           float* s32 = reinterpret_cast<float*>(stg);

@@ -51,7 +51,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 // tiles (tensor-core bound at prefill sizes), each in bf16 and in NVFP4.
 enum Variant { V_SMALL = 0, V_LARGE = 1, V_SMALL4 = 2, V_LARGE4 = 3 };
 constexpr int V_BN[4] = {64, 256, 64, 192};
-constexpr int V_STAGES[4] = {8, 4, 6, 4};
+constexpr int V_STAGES[4] = {8, 4, 6, 3};
 constexpr int V_BOXN[4] = {16, 256, 16, 192};  // one token box per stage at prefill sizes
 constexpr bool V_FP4[4] = {false, false, true, true};
 constexpr int V_ACC_SPLIT[4] = {4, 1, 2, 1};  // decode-sized tiles rotate over independent accumulators
@@ -174,7 +174,7 @@ struct lmoe_ctx {
   size_t sf_bytes_tiles(long long tiles_small, long long tiles_large, int K) const {
     const long long st = (K + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K;
     const long long a = tiles_small * st * 4 * ((V_BN[V_SMALL4] + 127) / 128) * 512;
-    const long long b = tiles_large * st * 4 * ((V_BN[V_LARGE4] + 127) / 128) * 512;
+    const long long b = tiles_large * st * 4 * ((V_BN[V_LARGE4] + 127) / 128) * 512 * SF_WREP;  // replicated
     return (size_t)(a > b ? a : b);
   }
   size_t sf_bytes_dense(int K) const {
@@ -485,9 +485,10 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
   amax_act_kernel<<<grid_for((long long)T * d / 8, 256), 256, 0, s>>>(
       reinterpret_cast<const __nv_bfloat16*>(x), (long long)T * d / 8, amax_x);
   const int nra = (V_BN[vg] + 127) / 128;  // scale row atoms per token tile of the FP4 variant
+  const int sf_reps = vg == V_LARGE4 ? SF_WREP : 1;  // the prefill variant reads replicated scale atoms
   quant_act_kernel<<<grid_for((long long)T * d / 16, 256), 256, 0, s>>>(
       reinterpret_cast<const __nv_bfloat16*>(x), d, nullptr, T, T, nullptr, nullptr, N, V_BN[vg], nra, amax_x, c->xq,
-      c->x_sf, g_x, c->status);
+      c->x_sf, g_x, c->status, sf_reps);
   amax_act_kernel<<<grid_for((long long)T * l / 8, 256), 256, 0, s>>>(c->h, (long long)T * l / 8, amax_h);
   chk(cudaGetLastError());
   mark(2);
@@ -514,12 +515,12 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
       idx, gate, c->chunk_base, T, N, K, ct, c->row_of, c->tok_of_row, c->gate_of_row, c->status);
   quant_act_kernel<<<grid_for((long long)T * l / 16, 256), 256, 0, s>>>(c->h, l, nullptr, T, T, nullptr, nullptr, N,
                                                                          V_BN[vg], 0, amax_h, c->hq_tok, c->h_sf_tok,
-                                                                         g_h, c->status);
+                                                                         g_h, c->status, 1);
   {
     long long blocks = (TK + 7) / 8;  // one warp per row
     if (blocks > 16LL * c->num_sms) blocks = 16LL * c->num_sms;
     gather_act_q_kernel<<<(int)blocks, 256, 0, s>>>(c->hq_tok, c->h_sf_tok, l, c->tok_of_row, TK, T, c->offsets,
-                                                     c->tile0, N, V_BN[vg], nra, c->hq, c->h_sf, c->status);
+                                                     c->tile0, N, V_BN[vg], nra, c->hq, c->h_sf, c->status, sf_reps);
   }
   chk(cudaGetLastError());
   mark(5);

@@ -197,9 +197,12 @@ __device__ __forceinline__ uint32_t nvfp4_block_fast(const float (&v)[16], float
 // major: atom (ka, ra) at ((tile * stages + st) * 4 + ka) * nra + ra.  Inside an atom the layout is the
 // weight atoms' one.  Each K atom's scales must start on a 4-column-aligned TMEM address for the
 // block-scaled MMA, hence one atom (one tcgen05.cp) per K atom and 128 tokens even for short tiles.
-__host__ __device__ __forceinline__ long long act_sf_offset(long long tile, int j, int kb16, int stages, int nra) {
+__host__ __device__ __forceinline__ long long act_sf_offset(long long tile, int j, int kb16, int stages, int nra,
+                                                           int rep = 0, int reps = 1) {
   const int st = kb16 >> 4, ka = (kb16 >> 2) & 3, s = kb16 & 3;
-  return (((tile * stages + st) * 4 + ka) * nra + (j >> 7)) * 512 + (j & 31) * 16 + ((j & 127) >> 5) * 4 + s;
+  // reps > 1: every atom stored `reps` times in a row (copy `rep` here), as for the weight scales
+  return (((((tile * stages + st) * 4 + ka) * nra + (j >> 7)) * reps) + rep) * 512 + (j & 31) * 16 +
+         ((j & 127) >> 5) * 4 + s;
 }
 
 // Weight-scale atoms are stored replicated: each 512-byte atom four times in a row (2 KB), the
@@ -310,7 +313,7 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, con
                                  long long n_rows, int n_src_rows, const int* __restrict__ offsets,
                                  const int* __restrict__ tile0, int n_experts, int tile_rows, int nra,
                                  const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes,
-                                 uint8_t* __restrict__ sf, float* __restrict__ g_out, unsigned* status) {
+                                 uint8_t* __restrict__ sf, float* __restrict__ g_out, unsigned* status, int reps) {
   const int nb = K / 16;
   const int stages = (K + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K;
   const float g = tensor_scale_from_amax(__uint_as_float(amax_bits[0]));
@@ -360,7 +363,9 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, con
     uint32_t c[2];
     const uint32_t sb = nvfp4_block_exact(v, g, c);
     *reinterpret_cast<uint2*>(codes + r * (K / 2) + kb * 8) = make_uint2(c[0], c[1]);
-    if (nra > 0) sf[act_sf_offset(tile, j, kb, stages, nra)] = (uint8_t)sb;
+    if (nra > 0) {
+      for (int rp = 0; rp < reps; ++rp) sf[act_sf_offset(tile, j, kb, stages, nra, rp, reps)] = (uint8_t)sb;
+    }
     else sf[r * nb + kb] = (uint8_t)sb;  // plain row-major scales
   }
 }
@@ -376,7 +381,8 @@ __global__ void __launch_bounds__(256)
     gather_act_q_kernel(const uint8_t* __restrict__ codes_tok, const uint8_t* __restrict__ sf_tok, int K,
                         const int* __restrict__ tok_of_row, long long n_rows, int n_tok,
                         const int* __restrict__ offsets, const int* __restrict__ tile0, int n_experts, int tile_rows,
-                        int nra, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, unsigned* status) {
+                        int nra, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, unsigned* status,
+                        int reps) {
   const int lane = threadIdx.x & 31;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
   const int row_bytes = K / 2, nb = K / 16;
@@ -399,9 +405,11 @@ __global__ void __launch_bounds__(256)
     for (int c = lane * 16; c < row_bytes; c += 32 * 16)
       *reinterpret_cast<uint4*>(codes + r * row_bytes + c) =
           *reinterpret_cast<const uint4*>(codes_tok + (long long)t * row_bytes + c);
-    for (int q = lane; q < nb / 4; q += 32)
-      *reinterpret_cast<uint32_t*>(sf + act_sf_offset(tile, j, 4 * q, stages, nra)) =
-          *reinterpret_cast<const uint32_t*>(sf_tok + (long long)t * nb + 4 * q);
+    for (int q = lane; q < nb / 4; q += 32) {
+      const uint32_t v = *reinterpret_cast<const uint32_t*>(sf_tok + (long long)t * nb + 4 * q);
+      for (int rp = 0; rp < reps; ++rp)
+        *reinterpret_cast<uint32_t*>(sf + act_sf_offset(tile, j, 4 * q, stages, nra, rp, reps)) = v;
+    }
   }
 }
 
