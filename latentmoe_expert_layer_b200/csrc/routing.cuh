@@ -40,15 +40,13 @@ __global__ void router_f32_kernel(const __nv_bfloat16* __restrict__ x, const flo
 }
 
 // ------------------------------------------------------------------------------------------------
-// top-K + softmax + per-chunk expert histogram.  One block per chunk of `chunk_tokens` consecutive
-// tokens, one warp per token.  Lane j holds the candidates j, j + 32, ... (P of them); it sorts them
-// once (bitonic network in registers, order: value desc, index asc).  Then K rounds of a warp
-// arg-max over the lanes' current heads pick the experts in output order; only the lane that owned
-// the winner shifts its sorted list by one.  Requires K <= 32 and N <= 32 * P.
+// top-K + softmax + per-chunk expert histogram.  A chunk of `chunk_tokens` consecutive tokens is
+// handled by `parts` blocks, one warp per token.  Lane j holds the candidates j, j + 32, ... (P of
+// them) as order-preserving 32-bit keys.  The K-th largest key X is built two bits at a time from
+// warp-wide counts; the selection is every key above X plus the lowest expert indices among the keys
+// equal to X (ranked with ballots in index order); a warp bitonic sort puts the K selections in
+// output order (value desc, index asc).  Requires K <= 32 and N <= 32 * P.
 // ------------------------------------------------------------------------------------------------
-__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
-  return va > vb || (va == vb && ia < ib);
-}
 
 template <int P>
 __global__ void __launch_bounds__(1024)
@@ -193,7 +191,8 @@ inline cudaError_t launch_topk_hist(int n_chunks, int parts, cudaStream_t s, con
 }
 
 // ------------------------------------------------------------------------------------------------
-// Expert totals, exclusive offsets, per-chunk bases and the grouped-GEMM unit lists.
+// Expert totals, exclusive offsets, per-chunk bases, first token tiles and each expert's first unit
+// in the two grouped-GEMM unit lists (build_units_kernel then writes the lists over the whole grid).
 // Single block of 1024 threads; thread e owns expert e (N <= 1024).
 // ------------------------------------------------------------------------------------------------
 struct UnitListSpec {
@@ -348,9 +347,11 @@ __global__ void __launch_bounds__(256)
 }
 
 // ------------------------------------------------------------------------------------------------
-// Stable row assignment.  One warp per chunk walks the chunk's assignments in (token, slot) order,
-// 32 at a time: lanes holding the same expert are ranked with __match_any_sync, and a per-expert
-// running base (from scan_units_kernel) gives each assignment its grouped row.
+// Stable row assignment.  One block per chunk; its W warps take contiguous parts of the chunk's
+// assignments in (token, slot) order.  Each warp counts its part per expert, the per-warp bases
+// follow from the chunk's per-expert base (scan_units_kernel) and the earlier warps' counts, and then
+// each warp walks its part 32 at a time: lanes holding the same expert are ranked with
+// __match_any_sync on top of the warp's running base.  W = 1 (32 threads) works as well.
 // ------------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
     assign_rows_kernel(const int* __restrict__ topk_idx, const float* __restrict__ topk_gate,
