@@ -52,15 +52,21 @@ TRAFFIC_RATIO = {
     ("bf16", "prefill", "expert_up"): 0.982, ("bf16", "prefill", "expert_down"): 0.993,
 }
 TRAFFIC_SOURCES = ("gemm_tc.cuh", "ptx.cuh", "nvfp4.cuh", "lmoe.cu")
-TRAFFIC_SOURCES_SHA256 = "9c0631a36f70a7748548e60017a96c818de08e26cddaa3aa7b8af8d320e9c901"
+TRAFFIC_SOURCES_SHA256 = "66bdba2299abce8c6abe29f480a83eae0daeb46152f95da3a8dac9fe660bb35a"
 
 
 def gemm_sources_sha256() -> str:
+    """SHA-256 of the GEMM's code: the sources with comments removed and whitespace runs collapsed, so
+    that editing a comment does not invalidate a capture (string literals are kept as they are)."""
     import hashlib
+    import re
+    token = re.compile(r'"(?:\\.|[^"\\])*"|//[^\n]*|/\*.*?\*/', re.S)
     h = hashlib.sha256()
     for f in TRAFFIC_SOURCES:
-        with open(os.path.join(ROOT, "latentmoe_expert_layer_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "latentmoe_expert_layer_b200", "csrc", f)) as fh:
+            src = fh.read()
+        code = token.sub(lambda m: m.group(0) if m.group(0).startswith('"') else " ", src)
+        h.update(" ".join(code.split()).encode())
     return h.hexdigest()
 
 

@@ -11,9 +11,12 @@
 // Two operand formats (template flag FP4):
 //   bf16   kind::f16, 64 elements (128 bytes) of K per pipeline stage
 //   NVFP4  kind::mxf4nvf4 with 16-element E4M3 block scales, 256 E2M1 elements (128 bytes) of K per
-//          stage; weight scales arrive as 512-byte atoms by bulk copy, activation scales are staged
-//          into atoms by the producer warp, and the MMA issuer moves both into TMEM with tcgen05.cp.
-//          The epilogue multiplies by the two fp32 tensor scales.
+//          stage.  Scales arrive by bulk copy in 512-byte atoms and the MMA issuer moves them into
+//          TMEM with tcgen05.cp: weight atoms are stored replicated (two 128x256b copies per stage);
+//          the decode variant keeps a token tile's activation scales resident in TMEM across the
+//          tile's units (copied by its first unit), the prefill variant reads replicated activation
+//          atoms (one 128x256b copy per K atom).  The epilogue multiplies by the two fp32 tensor
+//          scales.
 //
 // Roles (192 threads):
 //   warp 0      producer: streams W and activation tiles (TMA) and scales into a STAGES-deep ring

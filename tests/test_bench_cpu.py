@@ -59,13 +59,16 @@ def test_standard_moe_experts_work_in_d():
 def test_traffic_hash_is_deterministic_and_covers_the_gemm_sources(tmp_path, monkeypatch):
     h = bench.gemm_sources_sha256()
     assert len(h) == 64 and h == bench.gemm_sources_sha256()
-    # a changed source file changes the hash (the bench then reports no traffic)
+    # changed code changes the hash (the bench then reports no traffic); comments do not
     csrc = tmp_path / "latentmoe_expert_layer_b200" / "csrc"
     csrc.mkdir(parents=True)
     for f in bench.TRAFFIC_SOURCES:
         (csrc / f).write_bytes(open(os.path.join(ROOT, "latentmoe_expert_layer_b200", "csrc", f), "rb").read())
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.gemm_sources_sha256() == h
-    with open(csrc / bench.TRAFFIC_SOURCES[0], "ab") as fh:
-        fh.write(b"\n")
+    with open(csrc / bench.TRAFFIC_SOURCES[0], "a") as fh:   # a comment: same code
+        fh.write("\n// a note\n/* another */\n")
+    assert bench.gemm_sources_sha256() == h
+    with open(csrc / bench.TRAFFIC_SOURCES[0], "a") as fh:   # changed code
+        fh.write("\nconstexpr int kProbe = 1;\n")
     assert bench.gemm_sources_sha256() != h
