@@ -1,7 +1,10 @@
 """Throughput of the B200 LatentMoE layer (Super shape) on seeded synthetic inputs.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|skewed|tiny]
-                    [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--no-cpu-baseline]
+
+Workloads (lmoe_inputs): decode (default), prefill, skewed, tiny, decode_nvfp4, prefill_nvfp4, the
+Ultra-width and standard-MoE variants, and the small profiling cases.
 
 One step = one full forward of the layer (router, top-K, dispatch, W_down, routed experts, combine,
 W_up, shared expert) over one batch.  The default workload is the Super-shaped decode/verify batch
@@ -12,8 +15,9 @@ Prints ONE JSON line on rank 0.  `value` is whole-job tokens/s with inputs resid
 is the same through lmoe_forward_host (pinned host x in, y/idx/gate out, copies inside the timed
 region); `roofline` reports the dominant kernel's algorithmic bytes (or FLOPs) per launch over its
 CUDA-event duration against the measured peak, from a second, identical timed loop that records the
-library's per-stage events (`profiled_ms_per_step`; the headline loop runs without them); `cpu_baseline` times the fp64 oracle on a bounded
-sample on the host cores.  `--impl reference` times that oracle alone as the reference arm.
+library's per-stage events (`profiled_ms_per_step`; the headline loop runs without them);
+`cpu_baseline` times the fp64 oracle on a bounded sample on the host cores.  `--impl reference`
+times that oracle alone as the reference arm.
 """
 from __future__ import annotations
 
