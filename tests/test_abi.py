@@ -58,6 +58,10 @@ def test_create_rejects_bad_config_without_touching_a_gpu(libmod):
     assert libmod.lib.lmoe_create(ctypes.byref(bad), 0, ctypes.byref(h)) == 1
     bad = libmod._Config(256, 64, 16, 4, 128, 256, 64, 1, 0, 2)     # unknown weight-scale rule
     assert libmod.lib.lmoe_create(ctypes.byref(bad), 0, ctypes.byref(h)) == 1
+    bad = libmod._Config(256, 0, 16, 4, 128, 256, 64, 1, 0, 0)      # standard MoE (latent 0) in NVFP4
+    assert libmod.lib.lmoe_create(ctypes.byref(bad), 0, ctypes.byref(h)) == 3
+    bad = libmod._Config(256, -64, 16, 4, 128, 256, 64, 0, 0, 0)    # negative latent
+    assert libmod.lib.lmoe_create(ctypes.byref(bad), 0, ctypes.byref(h)) == 1
     assert libmod.lib.lmoe_forward(None, None, 0, None, None, None, None) == 1
     del cfg
 
