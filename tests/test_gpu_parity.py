@@ -205,3 +205,34 @@ def test_standard_rejects_projections_and_nvfp4():
     with pytest.raises(RuntimeError):     # W_down / W_up given to a layer without projections
         layer.load_weights(dev["w_router"], dev["w_down"], dev["w_up"], dev["w1"], dev["w2"], dev["ws1"], dev["ws2"])
     layer.close()
+
+
+def test_cuda_graph_replay_matches_eager(superlayer):
+    """lmoe_forward makes no host synchronisation or allocation, so a forward can be captured in a
+    CUDA graph; replaying it gives the eager call's outputs bit for bit."""
+    _, _, layer = superlayer
+    wl = inp.workload("decode")
+    x = to_dev(inp.make_x(wl), "bf16")
+    y = torch.empty((wl.tokens, wl.shape.d), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((wl.tokens, wl.shape.top_k), dtype=torch.int32, device="cuda")
+    gate = torch.empty((wl.tokens, wl.shape.top_k), dtype=torch.float32, device="cuda")
+    layer.forward(x, y, idx, gate)
+    torch.cuda.synchronize()
+    ref = (y.clone(), idx.clone(), gate.clone())
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):                 # warm-up on the stream the capture will use
+        layer.forward(x, y, idx, gate)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer.forward(x, y, idx, gate)
+    for t in (y, idx, gate):
+        t.zero_()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert torch.equal(y, ref[0]) and torch.equal(idx, ref[1]) and torch.equal(gate, ref[2])
+    del graph
