@@ -236,3 +236,22 @@ def test_cuda_graph_replay_matches_eager(superlayer):
     assert layer.device_status() == 0
     assert torch.equal(y, ref[0]) and torch.equal(idx, ref[1]) and torch.equal(gate, ref[2])
     del graph
+
+
+@pytest.mark.parametrize("k", [1, 16])
+def test_degenerate_top_k(k):
+    """K = 1 (every gate exactly 1) and K = N (every expert selected, softmax over all logits), on
+    the tiny layer's weights."""
+    base = inp.workload("tiny")
+    wl = dataclasses.replace(base, shape=dataclasses.replace(base.shape, top_k=k))
+    w = inp.make_weights(base)
+    layer = make_layer(wl, w, device_weights(w), wl.tokens)
+    try:
+        st = _compare(layer, oracle_weights(w, False), inp.make_x(wl), k)
+        _check_dispatch(layer, st["idx"], wl.shape.n_experts)
+        if k == 1:
+            assert np.all(st["gate"] == 1.0)
+        else:
+            assert np.array_equal(np.sort(st["idx"], axis=1), np.tile(np.arange(16), (wl.tokens, 1)))
+    finally:
+        layer.close()
