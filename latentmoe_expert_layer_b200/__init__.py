@@ -124,9 +124,13 @@ def route_noalloc(logits: torch.Tensor, top_k: int, bias: Optional[torch.Tensor]
 
 
 class LatentMoE:
-    """One LatentMoE layer on one GPU.
+    """One LatentMoE layer on one GPU (lmoe_create / lmoe_load_weights / lmoe_forward).
 
-    shape: object with d, latent, n_experts, top_k, expert_ffn, shared_ffn attributes.
+    shape: object with d, latent, n_experts, top_k, expert_ffn, shared_ffn attributes; latent = 0
+        builds the standard MoE without W_down / W_up (experts work in d; bf16 only).
+    max_tokens: the largest T a forward may pass (sizes the workspace).
+    precision: "bf16", or "nvfp4" for block-scaled FP4 routed and shared experts.
+    router_bias: a per-expert fp32 bias is added to the router logits (load_weights' b_router).
     weight_scale: NVFP4 weight block scales, "amax" or "mse" (lmoe_weight_scale).
     """
 
