@@ -1,0 +1,154 @@
+"""Expert-parallel data movement (latentmoe_expert_layer_b200.ep) on CPU ranks over gloo.
+
+The compute steps are the oracle's (test side only); the module under test moves the latent rows,
+expert ids, gates and outputs between ranks.  Every rank's y must equal the single-process oracle
+layer on its tokens, for several world sizes, ragged token counts and a rank without tokens."""
+import math
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+from latentmoe_expert_layer_b200 import ep  # noqa: E402
+from oracle import lmoe_oracle as lo  # noqa: E402
+
+D, L, N, K, M, MS = 8, 4, 16, 3, 6, 5
+
+
+class _W:
+    """A small float64 layer (router, W_down, W_up, experts, shared expert)."""
+
+    def __init__(self, seed):
+        rng = np.random.default_rng(seed)
+        self.w_router = rng.standard_normal((N, D))
+        self.b_router = None
+        self.w_down = rng.standard_normal((L, D)) / math.sqrt(D)
+        self.w_up = rng.standard_normal((D, L)) / math.sqrt(L)
+        self._w1 = rng.standard_normal((N, M, L)) / math.sqrt(L)
+        self._w2 = rng.standard_normal((N, L, M)) / math.sqrt(M)
+        self.ws1 = rng.standard_normal((MS, D)) / math.sqrt(D)
+        self.ws2 = rng.standard_normal((D, MS)) / math.sqrt(MS)
+        self.n_experts = N
+
+    def w1(self, e):
+        return self._w1[e]
+
+    def w2(self, e):
+        return self._w2[e]
+
+
+def _tokens(world):
+    counts = [5 + 3 * r for r in range(world)]
+    if world >= 4:
+        counts[2] = 0            # a rank without tokens still takes part in every exchange
+    return counts
+
+
+def _callables(W, rank, part):
+    def route(x):
+        xn = x.numpy()
+        logits = lo.router_logits(xn, W.w_router)
+        idx = lo.topk(logits, K)
+        gate = lo.softmax_gates(logits, idx)
+        return torch.from_numpy(idx), torch.from_numpy(gate), torch.from_numpy(xn @ W.w_down.T)
+
+    def experts(rows, counts, gates):
+        out = torch.empty_like(rows)
+        off = 0
+        for e_local, c in enumerate(counts.tolist()):
+            e = part.first(rank) + e_local
+            r = rows[off:off + c].numpy()
+            o = lo.sqrelu(r @ W.w1(e).T) @ W.w2(e).T
+            out[off:off + c] = torch.from_numpy(o) * gates[off:off + c, None]
+            off += c
+        return out
+
+    def output(z, x):
+        s = lo.sqrelu(x.numpy() @ W.ws1.T) @ W.ws2.T
+        return torch.from_numpy(z.numpy() @ W.w_up.T + s)
+
+    return route, experts, output
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        W = _W(5)
+        counts = _tokens(world)
+        x_all = np.random.default_rng(6).standard_normal((sum(counts), D))
+        start = sum(counts[:rank])
+        x = torch.from_numpy(x_all[start:start + counts[rank]].copy())
+        part = ep.ExpertPartition(N, world)
+        y, idx, gate = ep.ep_forward(x, part, *_callables(W, rank, part))
+        ref = lo.forward(W, x_all, K)
+        sl = slice(start, start + counts[rank])
+        q.put((rank, np.abs(y.numpy() - ref["y"][sl]).max() if counts[rank] else 0.0,
+               bool(np.array_equal(idx.numpy(), ref["idx"][sl])), y.shape[0]))
+    finally:
+        dist.destroy_process_group()
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ep_forward_matches_single_process_layer(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    counts = _tokens(world)
+    for rank, err, same_idx, n in res:
+        assert n == counts[rank]
+        assert same_idx
+        assert err < 1e-12, (rank, err)
+
+
+def test_dispatch_plan_groups_by_owner_in_token_slot_order():
+    rng = np.random.default_rng(7)
+    idx = torch.from_numpy(np.stack([rng.choice(N, K, replace=False) for _ in range(11)]))
+    part = ep.ExpertPartition(N, 4)
+    plan = ep.plan_dispatch(idx, part)
+    order = plan.order.numpy()
+    assert sorted(order.tolist()) == list(range(idx.numel()))          # every assignment once
+    owners = (idx.reshape(-1).numpy() // part.per_rank)[order]
+    assert np.all(np.diff(owners) >= 0)                                  # grouped by destination
+    for r in range(4):
+        a = order[owners == r]
+        assert np.all(np.diff(a) > 0)                                    # (token, slot) order inside
+        assert len(a) == plan.send_counts[r]
+
+
+def test_grouping_by_local_expert_is_stable_and_checks_ownership():
+    eids = torch.tensor([9, 8, 9, 11, 8, 8])
+    order, counts = ep.group_by_local_expert(eids, first=8, per_rank=4)
+    assert order.tolist() == [1, 4, 5, 0, 2, 3] and counts.tolist() == [3, 2, 0, 1]
+    with pytest.raises(ValueError):
+        ep.group_by_local_expert(torch.tensor([3]), first=8, per_rank=4)
+    with pytest.raises(ValueError):
+        ep.ExpertPartition(10, 4)
+
+
+def test_latent_dispatch_moves_d_over_l_fewer_bytes():
+    # Super shape: d = 4096, l = 1024, K = 22; the latent rows are 4x smaller than rows in d
+    assert ep.dispatch_bytes(256, 22, 1024) * 4 == ep.dispatch_bytes(256, 22, 4096)
+    assert ep.dispatch_bytes(1, 22, 1024) == 22 * 1024 * 2
