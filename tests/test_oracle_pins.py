@@ -564,6 +564,21 @@ def test_super_shape_matches_architecture_table():
         vals["experts_per_layer"], vals["top_k"], vals["moe_latent_dim"])
 
 
+def test_ultra_shape_matches_the_ultra_summary():
+    vals = {}
+    with open(os.path.join(GOLDEN, "ultra_layer_shape.txt")) as fh:
+        for line in fh:
+            if line.startswith("#") or not line.strip():
+                continue
+            k, v = line.split()
+            vals[k] = int(v)
+    u = inp.ULTRA
+    assert (u.n_experts, u.top_k, u.expert_ffn, u.shared_ffn) == (
+        vals["experts_per_layer"], vals["top_k"], vals["expert_hidden"], vals["shared_expert_hidden"])
+    # not on that page: Super's model and latent dimensions are kept
+    assert (u.d, u.latent) == (inp.SUPER.d, inp.SUPER.latent)
+
+
 def test_bf16_rounding_is_nearest_even():
     x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9, -2.5], np.float32)
     b = inp.bf16_bits_to_f32(inp.f32_to_bf16_bits(x))
