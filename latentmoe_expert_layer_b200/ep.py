@@ -7,12 +7,19 @@ LatentMoE dispatches the l-dimensional latent h = W_down x instead of x, d / l t
 Each of G ranks owns a contiguous range of N / G experts.  A forward on rank r, for its own tokens:
 
   1. route     idx, gate (router in d) and h = W_down x, locally;
-  2. dispatch  every assignment (t, k) goes to the owner of idx[t, k]: its latent row h[t], its expert
-               id and its gate travel in one all-to-all each, in (token, slot) order per destination;
-  3. experts   the owner groups the received rows by local expert (stably, in arrival order) and runs
-               its experts on them, the gate folded into the output;
-  4. return    the outputs travel back to their source rank (the reverse all-to-all);
-  5. combine   z[t] = sum_k o[t, k] in slot order, then y = W_up z + shared expert (x), locally.
+  2. dispatch  a token's latent row h[t] travels ONCE to every rank that owns at least one of its K
+               experts (one row per (token, destination) pair, not per assignment); beside it go the
+               assignments themselves: (pair index, expert id) and the gate, in (token, slot) order;
+  3. experts   the owner expands the pairs to assignment rows, groups them by local expert (stably,
+               in arrival order) and runs its experts, the gate folded into the output;
+  4. reduce    the owner sums the outputs of each (token, source rank) pair in slot order, so one
+               partial latent sum per pair goes back: at most min(K, G) rows of l per token;
+  5. return    the partial sums travel back to their source rank (the reverse all-to-all);
+  6. combine   z[t] = sum of the partial sums in ascending owner-rank order, then
+               y = W_up z + shared expert (x), locally.
+
+The sum in z is the same set of K gated expert outputs as the single-GPU layer's slot-order sum,
+grouped by owner rank first; the two differ only in floating-point rounding.
 
 This module is the data movement only.  The compute steps are callables (route, experts, output), so
 the same plan runs with the library's kernels on GPUs over NCCL or, in the tests, with any reference
@@ -28,7 +35,7 @@ import torch
 import torch.distributed as dist
 
 __all__ = ["ExpertPartition", "DispatchPlan", "plan_dispatch", "group_by_local_expert", "dispatch_bytes",
-           "ep_forward"]
+           "exchange_bytes", "reduce_pairs", "ep_forward"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -54,17 +61,41 @@ class ExpertPartition:
 
 @dataclasses.dataclass
 class DispatchPlan:
-    order: torch.Tensor        # [T*K] assignments (t*K + k) in send order: by destination, then (t, k)
-    send_counts: torch.Tensor  # [G] assignments sent to each rank
+    """Send order of one rank's routing, grouped by destination rank.
+
+    pairs: the (token, destination) pairs, sorted by (destination, token); one latent row each.
+    assignments: the (token, slot) assignments t*K + k, sorted by (destination, token, slot); the
+    pairs of one destination are numbered from 0 in that destination's segment."""
+    pair_tok: torch.Tensor       # [P] token of each pair, in send order
+    pair_counts: torch.Tensor    # [G] pairs (= latent rows) sent to each rank
+    order: torch.Tensor          # [T*K] assignments in send order
+    assign_pair: torch.Tensor    # [T*K] pair index of each sent assignment, within its destination
+    send_counts: torch.Tensor    # [G] assignments sent to each rank
+
+
+def _exclusive_cumsum(c: torch.Tensor) -> torch.Tensor:
+    return torch.cumsum(c, 0) - c
 
 
 def plan_dispatch(idx: torch.Tensor, part: ExpertPartition) -> DispatchPlan:
-    """Send order of the (token, slot) assignments: grouped by owning rank, (token, slot) order
-    within a rank (a stable sort of the owners)."""
+    """Pairs and assignments of idx [T, K] in send order (a stable sort of the owners keeps the
+    (token, slot) order inside each destination)."""
+    t, k = idx.shape
     flat = idx.reshape(-1).to(torch.int64)
     dest = part.owner(flat)
     _, order = torch.sort(dest, stable=True)
-    return DispatchPlan(order, torch.bincount(dest, minlength=part.world))
+    dest_s = dest[order]
+    tok_s = torch.div(order, max(k, 1), rounding_mode="floor")
+    key = dest_s * max(t, 1) + tok_s                       # nondecreasing along the send order
+    new = torch.ones_like(key, dtype=torch.bool)
+    if key.numel() > 1:
+        new[1:] = key[1:] != key[:-1]
+    pair_global = torch.cumsum(new.to(torch.int64), 0) - 1
+    pair_dest = dest_s[new]
+    pair_counts = torch.bincount(pair_dest, minlength=part.world)
+    assign_pair = pair_global - _exclusive_cumsum(pair_counts)[dest_s]
+    return DispatchPlan(tok_s[new], pair_counts, order, assign_pair,
+                        torch.bincount(dest, minlength=part.world))
 
 
 def group_by_local_expert(expert: torch.Tensor, first: int, per_rank: int) -> Tuple[torch.Tensor, torch.Tensor]:
@@ -76,10 +107,41 @@ def group_by_local_expert(expert: torch.Tensor, first: int, per_rank: int) -> Tu
     return order, torch.bincount(local, minlength=per_rank)
 
 
+def reduce_pairs(o: torch.Tensor, pair: torch.Tensor, n_pairs: int) -> torch.Tensor:
+    """Sum the rows of o [A, w] that share a pair id, in row order.
+
+    pair [A] must be nondecreasing (the assignments of one pair arrive together, in slot order) and
+    every id in [0, n_pairs) must occur; the result is [n_pairs, w], row p the slot-order sum of p's
+    rows.  The loop runs over the slot position, at most min(K, experts per rank) times."""
+    if pair.numel() and (bool((pair[1:] < pair[:-1]).any()) or int(pair[0]) < 0
+                         or int(pair[-1]) >= n_pairs):
+        raise ValueError("pair ids must be nondecreasing and inside [0, n_pairs)")
+    n = torch.bincount(pair, minlength=n_pairs) if pair.numel() else torch.zeros(n_pairs, dtype=torch.int64, device=pair.device)
+    if n_pairs and int(n.min()) == 0:
+        raise ValueError("a dispatched pair carries no assignment")
+    start = _exclusive_cumsum(n)
+    out = torch.zeros((n_pairs,) + tuple(o.shape[1:]), dtype=o.dtype, device=o.device)
+    for j in range(int(n.max()) if n_pairs else 0):
+        sel = torch.nonzero(n > j).reshape(-1)
+        out[sel] += o[start[sel] + j]
+    return out
+
+
 def dispatch_bytes(tokens: int, top_k: int, width: int, elem_bytes: int = 2) -> int:
-    """Bytes of dispatched rows for `tokens` tokens: one row of `width` elements per assignment
-    (the same again on the way back)."""
+    """Upper bound on the dispatched row bytes of `tokens` tokens: one row of `width` elements per
+    assignment, reached when every expert of a token sits on a different rank (G >= K)."""
     return tokens * top_k * width * elem_bytes
+
+
+def exchange_bytes(plan: DispatchPlan, width: int, elem_bytes: int = 2, gate_bytes: int = 4) -> dict:
+    """Bytes one rank sends in each direction for a plan: latent rows (one per pair) plus the
+    assignment metadata (pair index and expert id as int64, the gate) on the way out, one partial
+    latent sum per pair (elem_bytes each) on the way back."""
+    pairs = int(plan.pair_counts.sum())
+    assigns = int(plan.send_counts.sum())
+    return {"rows": pairs * width * elem_bytes,
+            "metadata": assigns * (2 * 8 + gate_bytes),
+            "return": pairs * width * elem_bytes}
 
 
 def _exchange(send: torch.Tensor, send_counts: list, recv_counts: list, group) -> torch.Tensor:
@@ -92,37 +154,52 @@ def ep_forward(x: torch.Tensor, part: ExpertPartition,
                route: Callable[[torch.Tensor], Tuple[torch.Tensor, torch.Tensor, torch.Tensor]],
                experts: Callable[[torch.Tensor, torch.Tensor, torch.Tensor], torch.Tensor],
                output: Callable[[torch.Tensor, torch.Tensor], torch.Tensor],
-               group: Optional["dist.ProcessGroup"] = None):
+               group: Optional["dist.ProcessGroup"] = None, stats: Optional[dict] = None):
     """One expert-parallel forward of this rank's tokens x [T, d].
 
     route(x)                         -> idx [T, K] (global expert ids), gate [T, K], h [T, l]
     experts(rows, counts, gates)     -> o [R, l]: rows grouped by local expert (counts per local
                                         expert, in order), outputs already multiplied by the gates
     output(z, x)                     -> y [T, d] from the latent sum z [T, l]
-    Every rank calls this at the same point (it runs five all-to-alls).  Returns (y, idx, gate)."""
+    Every rank calls this at the same point (it runs five all-to-alls).  If `stats` is a dict it
+    receives this rank's sent pair and assignment counts.  Returns (y, idx, gate)."""
     rank = dist.get_rank(group)
     idx, gate, h = route(x)
     t, k = idx.shape
+    width = h.shape[1]
     plan = plan_dispatch(idx, part)
-    send_counts = plan.send_counts.tolist()
-    recv_counts_t = torch.empty(part.world, dtype=torch.int64, device=plan.send_counts.device)
-    dist.all_to_all_single(recv_counts_t, plan.send_counts.to(torch.int64), group=group)
-    recv_counts = recv_counts_t.tolist()
+    send_cnt = torch.stack([plan.pair_counts, plan.send_counts], 1).to(torch.int64)   # [G, 2]
+    recv_cnt = torch.empty_like(send_cnt)
+    dist.all_to_all_single(recv_cnt, send_cnt, group=group)
+    pairs_out, assigns_out = plan.pair_counts.tolist(), plan.send_counts.tolist()
+    pairs_in, assigns_in = recv_cnt[:, 0].tolist(), recv_cnt[:, 1].tolist()
+    if stats is not None:
+        stats.update(pairs=int(sum(pairs_out)), assignments=int(sum(assigns_out)))
 
-    tok = torch.div(plan.order, k, rounding_mode="floor")
-    rows = _exchange(h[tok], send_counts, recv_counts, group)
-    eids = _exchange(idx.reshape(-1)[plan.order].to(torch.int64), send_counts, recv_counts, group)
-    gates = _exchange(gate.reshape(-1)[plan.order], send_counts, recv_counts, group)
+    # dispatch: one latent row per (token, destination); (pair, expert id) and gate per assignment
+    rows = _exchange(h[plan.pair_tok], pairs_out, pairs_in, group)
+    meta = torch.stack([plan.assign_pair, idx.reshape(-1)[plan.order].to(torch.int64)], 1)
+    meta = _exchange(meta, assigns_out, assigns_in, group)
+    gates = _exchange(gate.reshape(-1)[plan.order], assigns_out, assigns_in, group)
 
-    gorder, counts = group_by_local_expert(eids, part.first(rank), part.per_rank)
-    o_grouped = experts(rows[gorder], counts, gates[gorder])
+    # owner side: pair ids local to each source become ids into `rows`
+    src = torch.repeat_interleave(torch.arange(part.world, device=meta.device),
+                                  torch.tensor(assigns_in, device=meta.device))
+    pin = torch.tensor(pairs_in, dtype=torch.int64, device=meta.device)
+    if meta.shape[0] and (bool((meta[:, 0] < 0).any()) or bool((meta[:, 0] >= pin[src]).any())):
+        raise ValueError("an assignment names a pair its source did not send")
+    pair = _exclusive_cumsum(pin)[src] + meta[:, 0]
+    gorder, counts = group_by_local_expert(meta[:, 1], part.first(rank), part.per_rank)
+    o_grouped = experts(rows[pair[gorder]], counts, gates[gorder])
     o_arrival = torch.empty_like(o_grouped)
     o_arrival[gorder] = o_grouped
-    back = _exchange(o_arrival, recv_counts, send_counts, group)   # the reverse exchange
-    o = torch.empty((t * k, h.shape[1]), dtype=back.dtype, device=back.device)
-    o[plan.order] = back
-    o = o.reshape(t, k, h.shape[1])
-    z = o[:, 0].clone()
-    for s in range(1, k):           # slot order
-        z += o[:, s]
+    partial = reduce_pairs(o_arrival, pair, rows.shape[0])
+
+    # the reverse exchange, then the owner-rank-ordered sum on the source side
+    back = _exchange(partial, pairs_in, pairs_out, group)
+    z = torch.zeros((t, width), dtype=back.dtype, device=back.device)
+    off = 0
+    for c in pairs_out:                 # destinations in ascending rank order; tokens distinct in each
+        z[plan.pair_tok[off:off + c]] += back[off:off + c]
+        off += c
     return output(z, x), idx, gate

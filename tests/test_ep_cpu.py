@@ -1,8 +1,9 @@
 """Expert-parallel data movement (latentmoe_expert_layer_b200.ep) on CPU ranks over gloo.
 
-The compute steps are the oracle's (test side only); the module under test moves the latent rows,
-expert ids, gates and outputs between ranks.  Every rank's y must equal the single-process oracle
-layer on its tokens, for several world sizes, ragged token counts and a rank without tokens."""
+The compute steps are the oracle's (test side only); the module under test moves the latent rows
+(one per (token, destination rank) pair), the assignments' expert ids and gates, and the pre-reduced
+partial sums between ranks.  Every rank's y must equal the single-process oracle layer on its tokens,
+for several world sizes, ragged token counts and a rank without tokens."""
 import math
 import os
 import socket
@@ -89,11 +90,14 @@ def _worker(rank, world, port, q):
         start = sum(counts[:rank])
         x = torch.from_numpy(x_all[start:start + counts[rank]].copy())
         part = ep.ExpertPartition(N, world)
-        y, idx, gate = ep.ep_forward(x, part, *_callables(W, rank, part))
+        stats = {}
+        y, idx, gate = ep.ep_forward(x, part, *_callables(W, rank, part), stats=stats)
         ref = lo.forward(W, x_all, K)
         sl = slice(start, start + counts[rank])
+        owners = {(t, int(e) // part.per_rank) for t, row in enumerate(ref["idx"][sl]) for e in row}
         q.put((rank, np.abs(y.numpy() - ref["y"][sl]).max() if counts[rank] else 0.0,
-               bool(np.array_equal(idx.numpy(), ref["idx"][sl])), y.shape[0]))
+               bool(np.array_equal(idx.numpy(), ref["idx"][sl])), y.shape[0],
+               stats["pairs"] == len(owners), stats["assignments"] == counts[rank] * K))
     finally:
         dist.destroy_process_group()
 
@@ -117,9 +121,10 @@ def test_ep_forward_matches_single_process_layer(world):
         p.join(timeout=60)
         assert p.exitcode == 0
     counts = _tokens(world)
-    for rank, err, same_idx, n in res:
+    for rank, err, same_idx, n, pairs_ok, assigns_ok in res:
         assert n == counts[rank]
         assert same_idx
+        assert pairs_ok and assigns_ok      # one latent row per distinct (token, owner) pair
         assert err < 1e-12, (rank, err)
 
 
@@ -152,3 +157,66 @@ def test_latent_dispatch_moves_d_over_l_fewer_bytes():
     # Super shape: d = 4096, l = 1024, K = 22; the latent rows are 4x smaller than rows in d
     assert ep.dispatch_bytes(256, 22, 1024) * 4 == ep.dispatch_bytes(256, 22, 4096)
     assert ep.dispatch_bytes(1, 22, 1024) == 22 * 1024 * 2
+
+
+def _pairs_bruteforce(idx, part):
+    """(token, owner) pairs sorted by (owner, token), and each assignment's pair index within its
+    owner's segment, by plain loops."""
+    pairs = sorted({(int(e) // part.per_rank, t) for t, row in enumerate(idx.tolist()) for e in row})
+    seg = {}
+    for o, t in pairs:
+        seg.setdefault(o, []).append(t)
+    sent = sorted(((int(e) // part.per_rank, t, s) for t, row in enumerate(idx.tolist())
+                   for s, e in enumerate(row)))
+    return pairs, [seg[o].index(t) for o, t, _ in sent]
+
+
+@pytest.mark.parametrize("world", [1, 2, 4, 8, 16])
+def test_pairs_match_bruteforce(world):
+    rng = np.random.default_rng(11 + world)
+    idx = torch.from_numpy(np.stack([rng.choice(N, K, replace=False) for _ in range(13)]))
+    part = ep.ExpertPartition(N, world)
+    plan = ep.plan_dispatch(idx, part)
+    pairs, assign_pair = _pairs_bruteforce(idx, part)
+    assert plan.pair_tok.tolist() == [t for _, t in pairs]
+    assert plan.pair_counts.tolist() == [sum(1 for o, _ in pairs if o == r) for r in range(world)]
+    assert plan.assign_pair.tolist() == assign_pair
+    assert int(plan.pair_counts.sum()) <= min(K, world) * idx.shape[0]
+    if world == 1:                                           # one rank: every token is one pair
+        assert plan.pair_tok.tolist() == list(range(idx.shape[0]))
+    if world == N:                                           # one expert per rank: a pair per assignment
+        assert int(plan.pair_counts.sum()) == idx.numel()
+
+
+def test_plan_of_no_tokens_is_empty():
+    plan = ep.plan_dispatch(torch.zeros((0, K), dtype=torch.int64), ep.ExpertPartition(N, 4))
+    assert plan.pair_tok.numel() == 0 and plan.order.numel() == 0
+    assert plan.pair_counts.tolist() == [0] * 4 and plan.send_counts.tolist() == [0] * 4
+
+
+def test_reduce_pairs_sums_in_row_order_and_checks_ids():
+    o = torch.tensor([[1.0], [2.0], [4.0], [8.0], [16.0]], dtype=torch.float64)
+    out = ep.reduce_pairs(o, torch.tensor([0, 0, 1, 2, 2]), 3)
+    assert out.reshape(-1).tolist() == [3.0, 4.0, 24.0]
+    # the order is the row order: (1e16 + 1) - 1e16 loses the 1, 1e16 - 1e16 + 1 keeps it
+    big = torch.tensor([[1e16], [1.0], [-1e16]], dtype=torch.float64)
+    assert float(ep.reduce_pairs(big, torch.tensor([0, 0, 0]), 1)) == 0.0
+    assert float(ep.reduce_pairs(big[[0, 2, 1]], torch.tensor([0, 0, 0]), 1)) == 1.0
+    assert ep.reduce_pairs(o[:0], torch.zeros(0, dtype=torch.int64), 0).shape == (0, 1)
+    for bad, n in (([1, 0, 0, 1, 2], 3), ([0, 0, 1, 2, 3], 3), ([0, 0, 2, 2, 2], 3)):
+        with pytest.raises(ValueError):
+            ep.reduce_pairs(o, torch.tensor(bad), n)
+
+
+def test_exchange_bytes_at_the_super_shape():
+    # Super shape (l = 1024, N = 512, K = 22) over 8 ranks: at most 8 latent rows per token leave a
+    # rank instead of 22, and the same count of partial sums comes back
+    rng = np.random.default_rng(3)
+    t = 64
+    idx = torch.from_numpy(np.stack([rng.choice(512, 22, replace=False) for _ in range(t)]))
+    plan = ep.plan_dispatch(idx, ep.ExpertPartition(512, 8))
+    b = ep.exchange_bytes(plan, 1024)
+    pairs = int(plan.pair_counts.sum())
+    assert b["rows"] == b["return"] == pairs * 1024 * 2
+    assert b["metadata"] == t * 22 * 20
+    assert b["rows"] <= 8 * t * 1024 * 2 < ep.dispatch_bytes(t, 22, 1024)
