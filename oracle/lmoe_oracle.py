@@ -30,7 +30,7 @@ expert at a time, so the Super shape (2.9 G parameters) never needs more than a 
 """
 from __future__ import annotations
 
-from typing import Optional, Sequence
+from typing import Optional
 
 import numpy as np
 
@@ -38,7 +38,7 @@ import lmoe_inputs as inp
 
 __all__ = [
     "lift", "OracleWeights", "router_logits", "topk", "softmax_gates", "sqrelu", "dispatch",
-    "near_tie_tokens", "forward",
+    "near_tie_tokens", "expert_rows", "forward",
 ]
 
 
@@ -141,17 +141,29 @@ def near_tie_tokens(logits: np.ndarray, k: int, eps: float) -> np.ndarray:
     return m
 
 
-def forward(w: OracleWeights, x: np.ndarray, k: int, idx: Optional[np.ndarray] = None,
-            experts: Optional[Sequence[int]] = None):
+def expert_rows(w: OracleWeights, h: np.ndarray, idx: np.ndarray, gate: np.ndarray, e: int):
+    """Gate-weighted outputs g * W2_e sqrelu(W1_e h[t]) of expert e for the tokens t that selected it.
+    Returns (tokens, rows [n, width of h]); rows is None when no token selected e."""
+    tt, kk = np.nonzero(idx == e)
+    if tt.size == 0:
+        return tt, None
+    u = sqrelu(h[tt] @ w.w1(e).T)
+    o = u @ w.w2(e).T
+    return tt, gate[tt, kk][:, None] * o
+
+
+def forward(w: OracleWeights, x: np.ndarray, k: int, idx: Optional[np.ndarray] = None, map_fn=map):
     """Full layer forward in float64.
 
     x      [T, d] float64 (the exact bf16 values the device sees)
     k      top-K
     idx    optional forced routing [T, K] (used to re-evaluate tokens whose GPU routing differs at a
            near-tie); gates are then the softmax of the oracle's own logits at those experts.
+    map_fn how the per-expert work is mapped over the experts (the built-in map, or a thread pool's
+           map, which keeps the order); z adds the experts' rows in expert order either way.
     Returns dict with y [T, d], idx [T, K], gate [T, K], logits [T, N], h [T, l], z [T, l].
 
-    A layer without W_down / W_up (w.w_down with zero rows) is the standard MoE these replace
+    A layer given without W_down / W_up (w.w_down with zero rows) is the standard MoE these replace
     ("Nemotron 3 Super" notes, section 3.2): the experts run on x itself (d -> m -> d) and
     y = z + W_s2 sqrelu(W_s1 x).
     """
@@ -162,14 +174,10 @@ def forward(w: OracleWeights, x: np.ndarray, k: int, idx: Optional[np.ndarray] =
     standard = w.w_down.shape[0] == 0
     h = x if standard else x @ w.w_down.T
     z = np.zeros_like(h)
-    for e in range(w.n_experts):
-        tt, kk = np.nonzero(idx == e)
-        if tt.size == 0:
-            continue
-        u = sqrelu(h[tt] @ w.w1(e).T)
-        o = u @ w.w2(e).T
-        # each token selects an expert at most once, so tt has no repeats
-        z[tt] += gate[tt, kk][:, None] * o
+    # each token selects an expert at most once, so a token appears once in an expert's rows
+    for tt, rows in map_fn(lambda e: expert_rows(w, h, idx, gate, e), range(w.n_experts)):
+        if rows is not None:
+            z[tt] += rows
     s = sqrelu(x @ w.ws1.T) @ w.ws2.T
     y = (z if standard else z @ w.w_up.T) + s
     return {"y": y, "idx": idx, "gate": gate, "logits": logits, "h": h, "z": z}

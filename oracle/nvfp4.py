@@ -24,7 +24,7 @@ inside a GEMM epilogue, before any tensor-wide amax exists) use the static g = 1
 """
 from __future__ import annotations
 
-from typing import Optional, Sequence
+from typing import Optional
 
 import numpy as np
 
@@ -33,7 +33,7 @@ from . import lmoe_oracle as lo
 __all__ = [
     "E2M1_VALUES", "e2m1_encode", "e2m1_decode", "e4m3_encode", "e4m3_decode", "tensor_scale",
     "quantize", "quantize_mse", "mse_candidates", "block_sq_error", "dequantize", "qdq", "bf16_round",
-    "forward_nvfp4",
+    "expert_rows_nvfp4", "forward_nvfp4",
 ]
 
 E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
@@ -232,8 +232,25 @@ def qdq(a: np.ndarray, g: Optional[np.float32] = None, quantizer=None) -> np.nda
     return dequantize(c, s, gg)
 
 
+def expert_rows_nvfp4(w: "lo.OracleWeights", hq: np.ndarray, idx: np.ndarray, gate: np.ndarray, e: int,
+                      weight_quantize=None):
+    """Gate-weighted outputs of expert e in the NVFP4 layer for the tokens that selected it:
+    g * qdq(W2_e) qdq(sqrelu(qdq(W1_e) hq), g = 1), hq being the tokens' already quantised latents.
+    Returns (tokens, rows); rows is None when no token selected e."""
+    tt, kk = np.nonzero(idx == e)
+    if tt.size == 0:
+        return tt, None
+    wq = weight_quantize or quantize
+    w1 = qdq(w.w1(e).astype(np.float32), quantizer=wq)
+    w2 = qdq(w.w2(e).astype(np.float32), quantizer=wq)
+    u = lo.sqrelu(hq[tt] @ w1.T)
+    o = qdq(u.astype(np.float32), F32(1.0)) @ w2.T
+    return tt, gate[tt, kk][:, None] * o
+
+
 def forward_nvfp4(w: "lo.OracleWeights", x: np.ndarray, k: int, idx: Optional[np.ndarray] = None,
-                  g_x: Optional[np.float32] = None, g_h: Optional[np.float32] = None, weight_quantize=None):
+                  g_x: Optional[np.float32] = None, g_h: Optional[np.float32] = None, weight_quantize=None,
+                  map_fn=map):
     """Layer forward with NVFP4 routed and shared experts (weights and activations); router,
     W_down and W_up stay at the device's bf16 values.
 
@@ -242,7 +259,9 @@ def forward_nvfp4(w: "lo.OracleWeights", x: np.ndarray, k: int, idx: Optional[np
 
     g_x / g_h: per-call activation scales.  They depend on the whole call's x / h, so a caller that
     evaluates a sample of tokens passes the full batch's values.
-    weight_quantize: the weights' quantiser (quantize, the default, or quantize_mse)."""
+    weight_quantize: the weights' quantiser (quantize, the default, or quantize_mse).
+    map_fn: how the per-expert work is mapped over the experts (see lmoe_oracle.forward); z adds the
+    experts' rows in expert order either way."""
     wq = weight_quantize or quantize
     logits = lo.router_logits(x, w.w_router, w.b_router)
     if idx is None:
@@ -257,15 +276,9 @@ def forward_nvfp4(w: "lo.OracleWeights", x: np.ndarray, k: int, idx: Optional[np
     xq = qdq(x.astype(np.float32), g_x)
     one = F32(1.0)
     z = np.zeros_like(h)
-    for e in range(w.n_experts):
-        tt, kk = np.nonzero(idx == e)
-        if tt.size == 0:
-            continue
-        w1 = qdq(w.w1(e).astype(np.float32), quantizer=wq)
-        w2 = qdq(w.w2(e).astype(np.float32), quantizer=wq)
-        u = lo.sqrelu(hq[tt] @ w1.T)
-        o = qdq(u.astype(np.float32), one) @ w2.T
-        z[tt] += gate[tt, kk][:, None] * o
+    for tt, rows in map_fn(lambda e: expert_rows_nvfp4(w, hq, idx, gate, e, wq), range(w.n_experts)):
+        if rows is not None:
+            z[tt] += rows
     ws1 = qdq(w.ws1.astype(np.float32), quantizer=wq)
     ws2 = qdq(w.ws2.astype(np.float32), quantizer=wq)
     us = lo.sqrelu(xq @ ws1.T)
