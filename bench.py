@@ -1,15 +1,17 @@
 """Throughput of the B200 LatentMoE layer (Super shape) on seeded synthetic inputs.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
-                    [--no-cpu-baseline]
+                    [--no-cpu-baseline] [--no-prefill]
 
 Workloads (lmoe_inputs): decode (default), prefill, skewed, tiny, decode_nvfp4, prefill_nvfp4, the
 Ultra-width and standard-MoE variants, and the small profiling cases.
 
 One step = one full forward of the layer (router, top-K, dispatch, W_down, routed experts, combine,
 W_up, shared expert) over one batch.  The default workload is the Super-shaped decode/verify batch
-(T = 256).  With N > 1 (torchrun, one process per GPU) every rank runs an independent replica:
-the layer has no cross-GPU step, so nothing is exchanged and scaling is weak.
+(T = 256); the same run then also times the T = 16384 prefill batch on the same layer and reports it
+as the line's "prefill" object (its own steps, roofline, e2e and cpu_baseline), so one line carries
+both halves of the metric.  With N > 1 (torchrun, one process per GPU) every rank runs an
+independent replica: the layer has no cross-GPU step, so nothing is exchanged and scaling is weak.
 
 Prints ONE JSON line on rank 0.  `value` is whole-job tokens/s with inputs resident in HBM; `e2e`
 is the same through lmoe_forward_host (pinned host x in, y/idx/gate out, copies inside the timed
@@ -166,7 +168,7 @@ def algorithmic_work(wl, counts: np.ndarray):
             "touched_experts": touched, "expert_weight_bytes": int(2 * w_exp)}
 
 
-def make_device_layer(wl, device):
+def make_device_layer(wl, device, max_tokens=None):
     import torch
 
     import latentmoe_expert_layer_b200 as lm
@@ -177,7 +179,7 @@ def make_device_layer(wl, device):
     if wl.shape.latent == 0:          # a standard MoE has no projections
         dev["w_down"] = dev["w_up"] = None
     b = torch.from_numpy(w.b_router).to(device) if w.b_router is not None else None
-    layer = lm.LatentMoE(wl.shape, wl.tokens, precision=wl.precision, router_bias=wl.router_bias,
+    layer = lm.LatentMoE(wl.shape, max_tokens or wl.tokens, precision=wl.precision, router_bias=wl.router_bias,
                          device=device.index)
     layer.load_weights(b_router=b, **dev)
     torch.cuda.synchronize(device)
@@ -272,14 +274,21 @@ def run_reference(args, wl, rank):
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args, wl, rank, world):
+def load_stats(counts: np.ndarray, tokens: int) -> dict:
+    """Per-expert load of one forward, from the assignment count of every expert."""
+    c = np.asarray(counts, np.float64)
+    return {"max_over_mean": float(c.max() / max(c.mean(), 1e-30)), "zero_load_experts": int((c == 0).sum()),
+            "hottest_share_of_tokens": float(c.max() / tokens), "touched_experts": int((c > 0).sum())}
+
+
+def measure(layer, w, wl, steps, warmup, world, device, with_cpu_baseline):
+    """Time `steps` forwards of workload wl on the loaded layer (after `warmup` untimed ones) and
+    return its line's fields: the headline loop without stage events, a second identical loop with
+    the library's per-stage events (stage breakdown, dominant kernel), and the end-to-end loop
+    through lmoe_forward_host.  Durations are device-timed and taken as the max over ranks."""
     import torch
     import torch.distributed as dist
 
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    layer, w = make_device_layer(wl, device)
     x_bits = inp.make_x(wl)
     x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).to(device)
     t = wl.tokens
@@ -292,7 +301,7 @@ def run_ours(args, wl, rank, world):
         if world > 1:
             dist.barrier()
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         layer.forward(x, y, idx, gate)
     torch.cuda.synchronize(device)
     st = layer.device_status()
@@ -304,24 +313,23 @@ def run_ours(args, wl, rank, world):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(device)
-    with ClockSampler(local) as clk:
+    with ClockSampler(device.index) as clk:
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             layer.forward(x, y, idx, gate)
         e1.record(stream)
         torch.cuda.synchronize(device)
     barrier()
     ms_max = max_over_ranks(e0.elapsed_time(e1), world, device)
 
-    # ---- the same timed loop again with the library's per-stage CUDA events (recorded on the
-    #      launching stream between kernels): the stage breakdown and the dominant kernel's launch
-    #      duration for the roofline.  The events lengthen a step by a few percent, which is why the
-    #      headline loop above runs without them ----
+    # ---- the same loop with the library's per-stage CUDA events (recorded on the launching stream
+    #      between kernels): stage breakdown and the dominant kernel's launch duration.  The events
+    #      lengthen a step by a few percent, which is why the headline loop runs without them ----
     layer.profile(True)
     barrier()
     torch.cuda.synchronize(device)
     e0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         layer.forward(x, y, idx, gate)
     e1.record(stream)
     torch.cuda.synchronize(device)
@@ -337,7 +345,7 @@ def run_ours(args, wl, rank, world):
     yh = torch.empty((t, wl.shape.d), dtype=torch.bfloat16).pin_memory()
     ih = torch.empty((t, wl.shape.top_k), dtype=torch.int32).pin_memory()
     gh = torch.empty((t, wl.shape.top_k), dtype=torch.float32).pin_memory()
-    e2e_steps = max(1, min(args.steps, 200))
+    e2e_steps = max(1, min(steps, 200))
     for _ in range(2):
         layer.forward_host(xh, yh, ih, gh)
     torch.cuda.synchronize(device)
@@ -349,61 +357,49 @@ def run_ours(args, wl, rank, world):
     torch.cuda.synchronize(device)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
 
-    if rank != 0:
-        layer.close()
-        return
     work = algorithmic_work(wl, counts)
     pk, pk_kind = peaks()
+    p_tc = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    tc_src = pk_kind + " bf16 (sustained)"
+    if wl.precision == "nvfp4":  # no measured FP4 peak: bf16 measured x the nominal 4x FP4/BF16 ratio
+        p_tc *= 4.0
+        tc_src = pk_kind + " bf16 (sustained) x nominal FP4/BF16 ratio 4"
     # dominant kernel: the stage with the largest device time
     dom = max(stage_ms, key=stage_ms.get)
     per_launch_ms = stage_ms[dom] / max(1, recorded)
     decode_like = wl.tokens * wl.shape.top_k <= 48 * wl.shape.n_experts
+    roof = None
     if dom in ("expert_up", "expert_down"):
         unit_work = work[dom]
-    else:
-        unit_work = None
-    roof = None
-    if unit_work is not None:
         ratio = TRAFFIC_RATIO.get((wl.precision, "decode" if decode_like else "prefill", dom))
         traffic = None
         if ratio is not None and gemm_sources_sha256() == TRAFFIC_SOURCES_SHA256:
             traffic = ratio * unit_work["bytes"]
+        gbs = unit_work["bytes"] / (per_launch_ms * 1e-3) / 1e9
+        tfs = unit_work["flops"] / (per_launch_ms * 1e-3) / 1e12
+        both = {"hbm_frac": gbs / pk["hbm_gbs"], "tc_frac": tfs / p_tc}
         if decode_like:
-            ach = unit_work["bytes"] / (per_launch_ms * 1e-3) / 1e9
-            roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": ach / pk["hbm_gbs"], "traffic": traffic, "algorithmic_bytes": unit_work["bytes"],
-                    "launch_ms": per_launch_ms, "peak_source": pk_kind}
+            roof = {"kernel": dom, "bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": gbs / pk["hbm_gbs"], "traffic": traffic, "algorithmic_bytes": unit_work["bytes"],
+                    "launch_ms": per_launch_ms, "peak_source": pk_kind, **both}
         else:
-            ach = unit_work["flops"] / (per_launch_ms * 1e-3) / 1e12
-            p = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-            src = pk_kind + " bf16 (sustained)"
-            if wl.precision == "nvfp4":  # no measured FP4 peak: bf16 measured x the nominal 4x FP4/BF16 ratio
-                p *= 4.0
-                src = pk_kind + " bf16 (sustained) x nominal FP4/BF16 ratio 4"
-            roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": p, "unit": "TFLOP/s",
-                    "frac": ach / p, "traffic": traffic, "algorithmic_flops": unit_work["flops"],
-                    "algorithmic_bytes": unit_work["bytes"],
-                    "launch_ms": per_launch_ms, "peak_source": src}
-    step_ms = ms_max / args.steps
+            roof = {"kernel": dom, "bound": "tensor", "achieved": tfs, "peak": p_tc, "unit": "TFLOP/s",
+                    "frac": tfs / p_tc, "traffic": traffic, "algorithmic_flops": unit_work["flops"],
+                    "algorithmic_bytes": unit_work["bytes"], "launch_ms": per_launch_ms, "peak_source": tc_src,
+                    **both}
+    step_ms = ms_max / steps
     lay = work["layer"]
     layer_roof = {"bytes_per_step": lay["bytes"], "flops_per_step": lay["flops"],
                   "hbm_frac": lay["bytes"] / (step_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                   "tc_frac_of_bf16_peak": lay["flops"] / (step_ms * 1e-3) / 1e12 /
                   pk.get("bf16_tflops_sustained", pk["bf16_tflops"])}
-    line = {
-        "metric": METRIC,
-        "value": whole_job_tokens_per_s(world, t, args.steps, ms_max),
+    out = {
+        "value": whole_job_tokens_per_s(world, t, steps, ms_max),
         "unit": "tokens/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
+        "steps": steps,
+        "warmup": warmup,
         "ms_per_step": step_ms,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
         "dtype": "nvfp4+bf16" if wl.precision == "nvfp4" else "bf16",
-        "data": "synthetic: seeded N(0,1/fan_in) weights, N(0,1) x, bf16" +
-                (" (experts and shared expert quantised to NVFP4 on the device)" if wl.precision == "nvfp4" else ""),
         "config": {"workload": wl.name, "tokens": t, "d": wl.shape.d, "latent": wl.shape.latent,
                    "experts": wl.shape.n_experts, "top_k": wl.shape.top_k, "expert_ffn": wl.shape.expert_ffn,
                    "shared_ffn": wl.shape.shared_ffn, "precision": wl.precision,
@@ -412,18 +408,47 @@ def run_ours(args, wl, rank, world):
                          f"({work['touched_experts']} experts, {work['expert_weight_bytes'] / 1e9:.2f} GB)"},
         "roofline": roof,
         "layer_roofline": layer_roof,
+        "load": load_stats(counts, t),
         "stages_ms_per_step": {k: v / max(1, recorded) for k, v in stage_ms.items()},
-        "profiled_ms_per_step": prof_ms_max / args.steps,
+        "profiled_ms_per_step": prof_ms_max / steps,
         "e2e": {"value": whole_job_tokens_per_s(world, t, e2e_steps, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": t * wl.shape.d * 2,
                 "d2h_bytes_per_step": t * wl.shape.d * 2 + t * wl.shape.top_k * 8, "steps": e2e_steps},
-        "gpu_launches": launches * args.steps,
+        "gpu_launches": launches * steps,
         "clocks": clk.summary(),
     }
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, w)
+    if with_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, w)
+    return out
+
+
+# The default run covers both halves of the metric: the decode batch (T = 256) is the headline
+# line, the prefill batch (T = 16384, the same layer's weights) its "prefill" object.
+PREFILL_OF = {"decode": "prefill", "decode_nvfp4": "prefill_nvfp4"}
+
+
+def run_ours(args, wl, rank, world):
+    import torch
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    pwl = inp.workload(PREFILL_OF[wl.name]) if (wl.name in PREFILL_OF and not args.no_prefill) else None
+    layer, w = make_device_layer(wl, device, max_tokens=max(wl.tokens, pwl.tokens if pwl else 0))
+    cpu = world == 1 and rank == 0 and not args.no_cpu_baseline
+    line = {"metric": METRIC, "n_gpus": world, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "data": "synthetic: seeded N(0,1/fan_in) weights, N(0,1) x, bf16" +
+                    (" (experts and shared expert quantised to NVFP4 on the device)" if wl.precision == "nvfp4"
+                     else "")}
+    line.update(measure(layer, w, wl, args.steps, args.warmup, world, device, cpu))
+    if pwl is not None:
+        psteps = min(args.steps, DEFAULT_STEPS[pwl.name])
+        p = measure(layer, w, pwl, psteps, args.warmup, world, device, cpu)
+        line["prefill"] = p
+        line["gpu_launches"] += p["gpu_launches"]
     layer.close()
-    print(json.dumps(line), flush=True)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def main():
@@ -434,6 +459,8 @@ def main():
     ap.add_argument("--workload", default="decode", choices=sorted(inp.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="decode workloads only: skip the prefill half of the line")
     args = ap.parse_args()
     wl = inp.workload(args.workload)
     if args.steps is None:

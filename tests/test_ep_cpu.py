@@ -6,7 +6,6 @@ partial sums between ranks.  Every rank's y must equal the single-process oracle
 for several world sizes, ragged token counts and a rank without tokens."""
 import math
 import os
-import socket
 import sys
 
 import numpy as np
@@ -79,10 +78,11 @@ def _callables(W, rank, part):
     return route, experts, output
 
 
-def _worker(rank, world, port, q):
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+def _worker(rank, world, init_file, q):
     import datetime
-    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    # rendezvous through a file in the test's own temporary directory (no port to race for)
+    dist.init_process_group("gloo", init_method="file://" + init_file, rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
     try:
         W = _W(5)
         counts = _tokens(world)
@@ -102,18 +102,13 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def _free_port():
-    with socket.socket() as s:
-        s.bind(("127.0.0.1", 0))
-        return s.getsockname()[1]
-
 
 @pytest.mark.parametrize("world", [2, 4])
-def test_ep_forward_matches_single_process_layer(world):
+def test_ep_forward_matches_single_process_layer(world, tmp_path):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    init_file = str(tmp_path / "rendezvous")
+    procs = [ctx.Process(target=_worker, args=(r, world, init_file, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = sorted(q.get(timeout=180) for _ in range(world))

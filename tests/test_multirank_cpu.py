@@ -5,7 +5,6 @@ collectives are the timing reductions.  These tests run those reductions, the wh
 throughput arithmetic and the reference arm's rank handling as two CPU processes."""
 import json
 import os
-import socket
 import subprocess
 import sys
 
@@ -20,16 +19,12 @@ sys.path.insert(0, ROOT)
 import bench  # noqa: E402
 
 
-def _free_port() -> int:
-    with socket.socket() as s:
-        s.bind(("127.0.0.1", 0))
-        return s.getsockname()[1]
 
-
-def _worker(rank, world, port, q):
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+def _worker(rank, world, init_file, q):
     import datetime
-    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    # rendezvous through a file in the test's own temporary directory (no port to race for)
+    dist.init_process_group("gloo", init_method="file://" + init_file, rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
     try:
         # rank r "measured" (r + 1) * 10 ms: the job time is the slowest rank's
         ms = bench.max_over_ranks(10.0 * (rank + 1), world, torch.device("cpu"))
@@ -40,11 +35,11 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_max_over_ranks_gloo_world2():
-    world, port = 2, _free_port()
+def test_max_over_ranks_gloo_world2(tmp_path):
+    world, init_file = 2, str(tmp_path / "rendezvous")
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, init_file, q)) for r in range(world)]
     for p in procs:
         p.start()
     out = sorted(q.get(timeout=120) for _ in range(world))
