@@ -236,6 +236,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // the next launch may begin (its CTAs take SMs as this grid's CTAs exit)
+  griddep_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -267,6 +269,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // everything above is this CTA's own set-up; from here on the kernel reads what earlier launches
+  // wrote (unit lists, activations, scales, addends)
+  griddep_wait();
 
   const int num_units = args.n_pre_units + ((args.units != nullptr) ? *args.num_units : args.main_dense_units);
   // Every role walks the same sequence of units, published by the producer through the unit ring

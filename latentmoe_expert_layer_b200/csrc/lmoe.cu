@@ -14,6 +14,7 @@
 
 #include "../../include/lmoe.h"
 #include "gemm_tc.cuh"
+#include "route_fused.cuh"
 #include "routing.cuh"
 
 using namespace lmoe;
@@ -128,6 +129,7 @@ struct lmoe_ctx {
   GemmUnit* units2 = nullptr;
   int* num_units = nullptr;  // [2]
   unsigned* status = nullptr;
+  unsigned* route_bar = nullptr;  // [2] grid barrier of the fused decode routing kernel (zero at rest)
   int* work_counters = nullptr;  // [kCounters] per-launch unit counters and (last two) activation amax
                                  // bits, all zeroed at the start of a forward
   static constexpr int kCounters = 10;
@@ -226,7 +228,7 @@ void free_all(lmoe_ctx* c) {
                   c->ws2_sf, c->wg,     c->w_amax, c->xq,        c->x_sf,       c->hq,         c->h_sf,
                   c->hq_tok, c->h_sf_tok,
                   c->uq,     c->u_sf,   c->usq,    c->us_sf,     c->act_g,      c->tile0,      c->unit_u0,
-                  c->router_part};
+                  c->router_part, c->route_bar};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -259,9 +261,8 @@ lmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LMOE_OK : LMO
 template <int V>
 cudaError_t launch_gemm_v(const CUtensorMap& w0, const CUtensorMap& a0, const CUtensorMap& w1, const CUtensorMap& a1,
                           const GemmArgs& a, int grid, cudaStream_t s) {
-  gemm_tc_kernel<VT<V>::BN, VT<V>::ST, VT<V>::BOX, VT<V>::F4, VT<V>::AS, VT<V>::RS>
-      <<<grid, GEMM_THREADS, VT<V>::smem(), s>>>(w0, a0, w1, a1, a);
-  return cudaGetLastError();
+  return launch_pdl(gemm_tc_kernel<VT<V>::BN, VT<V>::ST, VT<V>::BOX, VT<V>::F4, VT<V>::AS, VT<V>::RS>, grid,
+                    GEMM_THREADS, VT<V>::smem(), s, w0, a0, w1, a1, a);
 }
 
 // A bf16 problem with its epilogue; K in elements (multiple of 64).
@@ -420,7 +421,10 @@ cudaError_t launch_split_reduce(lmoe_ctx* c, int ks, long long stride, int T, in
 //                        the slice sum writes the logits and h
 //   bf16, larger T       one launch: W_down (EPI_BF16 into h) as its dense pre problem, the router
 //                        rows K-sliced into fp32 partials as its main problem; then the slice sum
-cudaError_t router_stage(lmoe_ctx* c, const void* x, int T, cudaStream_t s, int& launches) {
+//   defer_sum: at decode sizes with the stacked rows, leave the slice sum to the fused routing kernel
+//   (only the GEMM is enqueued; *ks_out receives its slice count)
+cudaError_t router_stage(lmoe_ctx* c, const void* x, int T, cudaStream_t s, int& launches, bool defer_sum = false,
+                         int* ks_out = nullptr) {
   const lmoe_config& g = c->cfg;
   const int N = g.n_experts, l = g.latent, d = g.d;
   const int vd = T <= 512 ? V_SMALL : V_LARGE;
@@ -448,6 +452,11 @@ cudaError_t router_stage(lmoe_ctx* c, const void* x, int T, cudaStream_t s, int&
     p.split_stride = (long long)T * rows;
     gl.main_dense(c->fused_router ? c->map_rd : c->map_r, c->map_x[vd], p, rows, T);
     if ((e = gl.run(s)) != cudaSuccess) return e;
+    if (ks_out) *ks_out = ks;
+    if (defer_sum && c->fused_router) {
+      launches += 1;
+      return cudaSuccess;
+    }
     launches += 2;
     return launch_split_reduce(c, ks, p.split_stride, T, N, rows - N, s);
   }
@@ -472,6 +481,71 @@ cudaError_t launch_build_units(const lmoe_ctx* c, cudaStream_t s, const UnitList
   if (blocks > 4LL * c->num_sms) blocks = 4LL * c->num_sms;
   build_units_kernel<<<(int)blocks, 256, 0, s>>>(c->counts, c->offsets, c->tile0, c->cfg.n_experts, l1, l2);
   return cudaGetLastError();
+}
+
+// The decode routing chain as one cooperative launch (route_fused.cuh): slice sum of the router
+// GEMM (ks slices), top-K, expert scan, unit lists, stable rows and the gather into h_perm; it also
+// zeroes the unit counters of the expert launches that follow.
+constexpr int kRouteFusedThreads = 256;
+
+template <int P>
+cudaError_t launch_route_fused_p(const RouteFusedArgs& a, int grid, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kRouteFusedThreads);
+  cfg.dynamicSmemBytes = route_fused_smem(a.N, kRouteFusedThreads / 32);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, route_fused_kernel<P>, a);
+}
+
+cudaError_t launch_route_fused(lmoe_ctx* c, int T, int ks, int nch, int ct, int* idx, float* gate,
+                               const UnitListSpec& l1, const UnitListSpec& l2, cudaStream_t s) {
+  const lmoe_config& g = c->cfg;
+  RouteFusedArgs a;
+  memset(&a, 0, sizeof(a));
+  a.part = c->router_part;
+  a.ks = ks;
+  a.slice_stride = (long long)T * (g.n_experts + g.latent);
+  a.bias = c->b_router;
+  a.T = T;
+  a.N = g.n_experts;
+  a.K = g.top_k;
+  a.l = g.latent;
+  a.chunk_tokens = ct;
+  a.n_chunks = nch;
+  a.logits = c->logits;
+  a.h = c->h;
+  a.idx = idx;
+  a.gate = gate;
+  a.chunk_counts = c->chunk_counts;
+  a.counts = c->counts;
+  a.offsets = c->offsets;
+  a.tile0 = c->tile0;
+  a.l1 = l1;
+  a.l2 = l2;
+  a.row_of = c->row_of;
+  a.tok_of_row = c->tok_of_row;
+  a.gate_of_row = c->gate_of_row;
+  a.h_perm = c->h_perm;
+  a.zero_words = c->work_counters;
+  a.n_zero = lmoe_ctx::kCounters;
+  a.bar = c->route_bar;
+  a.status = c->status;
+  a.timeout_ns = c->timeout_ns;
+  const int grid = nch > c->num_sms ? nch : c->num_sms;  // one block per SM; the first nch own a chunk
+  switch (topk_lane_candidates(g.n_experts)) {
+    case 1: return launch_route_fused_p<1>(a, grid, s);
+    case 2: return launch_route_fused_p<2>(a, grid, s);
+    case 4: return launch_route_fused_p<4>(a, grid, s);
+    case 8: return launch_route_fused_p<8>(a, grid, s);
+    case 16: return launch_route_fused_p<16>(a, grid, s);
+    default: return launch_route_fused_p<32>(a, grid, s);
+  }
 }
 
 // NVFP4 forward: router, W_down and W_up in bf16; routed and shared experts as block-scaled FP4 GEMMs.
@@ -503,7 +577,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
 
   // 1. router logits and h = W_down x (bf16)
   chk(router_stage(c, x, T, s, launches));
-  mark(1);
+  if (!mark(1)) return e;
   // 2. quantise x (dynamic tensor scale); amax of h
   amax_act_kernel<<<grid_for((long long)T * d / 8, 256), 256, 0, s>>>(
       reinterpret_cast<const __nv_bfloat16*>(x), (long long)T * d / 8, amax_x);
@@ -514,7 +588,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
       c->x_sf, g_x, c->status, sf_reps);
   amax_act_kernel<<<grid_for((long long)T * l / 8, 256), 256, 0, s>>>(c->h, (long long)T * l / 8, amax_h);
   chk(cudaGetLastError());
-  mark(2);
+  if (!mark(2)) return e;
   // 3. top-K + softmax + per-chunk histogram
   int ct;
   const int nch = n_chunks_for(T, N, &ct);
@@ -523,7 +597,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
     if (parts > 1) chk(cudaMemsetAsync(c->chunk_counts, 0, (size_t)N * nch * sizeof(int), s));
     chk(launch_topk_hist(nch, parts, s, c->logits, c->b_router, T, N, K, ct, idx, gate, c->chunk_counts));
   }
-  mark(3);
+  if (!mark(3)) return e;
   // 4. expert offsets and grouped-GEMM unit lists
   UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1, c->unit_u0};
   UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2, c->unit_u0 + N + 1};
@@ -531,7 +605,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
                                                               c->chunk_base, l1, l2, c->tile0, c->status);
   chk(cudaGetLastError());
   chk(launch_build_units(c, s, l1, l2));
-  mark(4);
+  if (!mark(4)) return e;
   // 5. stable grouping; h quantised once per token, then its rows copied into grouped order with
   //    their scales in the expert GEMM's tile-local atoms
   assign_rows_kernel<<<nch, 32 * kAssignWarps, kAssignWarps * N * sizeof(int), s>>>(
@@ -546,7 +620,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
                                                      c->tile0, N, V_BN[vg], nra, c->hq, c->h_sf, c->status, sf_reps);
   }
   chk(cudaGetLastError());
-  mark(5);
+  if (!mark(5)) return e;
   // 6. expert up (FP4): u = NVFP4(sqrelu(W1_e h)); shared up u_s = NVFP4(sqrelu(W_s1 x))
   GemmProblem shared_up = problem4(d, EPI_SQRELU_NVFP4, c->usq, ms / 2, c->ws1_sf, c->wg + 2 * N, ms, c->x_sf, g_x);
   shared_up.out_sf = c->us_sf;
@@ -565,7 +639,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
     gl.main_dense(c->map_ws1q, c->map_xq[vg], shared_up, ms, T);
     chk(gl.run(s));
   }
-  mark(6);
+  if (!mark(6)) return e;
   // 7. expert down (FP4) with the gate folded in: o = g * (W2_e u); y_s = W_s2 u_s (fp32)
   const GemmProblem shared_down = problem4(ms, EPI_F32, c->y_s, d, c->ws2_sf, c->wg + 2 * N + 1, d, c->us_sf, one);
   {
@@ -581,10 +655,10 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
     gl.main_dense(c->map_ws2q, c->map_usq[vg], shared_down, d, T);
     chk(gl.run(s));
   }
-  mark(7);
+  if (!mark(7)) return e;
   // 8. latent combine: zu[:, :l] = sum_k o[row_of[t, k]]
   chk(launch_combine(c->num_sms, s, c->o, c->row_of, T, K, l, c->zu, l + ms, TKmax, c->status));
-  mark(8);
+  if (!mark(8)) return e;
   // 9. y = W_up z + y_s (bf16 GEMM)
   {
     GemmLaunch gl(c, vd, 6);
@@ -594,7 +668,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
     gl.main_dense(c->map_wup, c->map_z[vd], p, d, T);
     chk(gl.run(s));
   }
-  mark(9);
+  if (!mark(9)) return e;
   launches += 13 + (split ? 0 : 2);
   return e;
 }
@@ -664,7 +738,7 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   ok = ok && dalloc(&c->h_perm, tk * le) && dalloc(&c->u, tk * m) && dalloc(&c->o, tk * le);
   ok = ok && dalloc(&c->zu, T * (l + ms));
   ok = ok && dalloc(&c->units1, c->max_units1) && dalloc(&c->units2, c->max_units2) && dalloc(&c->num_units, 2);
-  ok = ok && dalloc(&c->status, 1) && dalloc(&c->work_counters, lmoe_ctx::kCounters);
+  ok = ok && dalloc(&c->status, 1) && dalloc(&c->work_counters, lmoe_ctx::kCounters) && dalloc(&c->route_bar, 2);
   ok = ok && dalloc(&c->tile0, N + 1) && dalloc(&c->unit_u0, 2 * (N + 1));
   {
     // router K-slice partials: stacked router + W_down rows at decode sizes, router rows otherwise
@@ -689,6 +763,7 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
     return LMOE_ERR_OOM;
   }
   cudaMemset(c->status, 0, sizeof(unsigned));
+  cudaMemset(c->route_bar, 0, 2 * sizeof(unsigned));
   // rows that no expert writes must still be finite for the MMA (they are masked in the epilogue)
   cudaMemset(c->h_perm, 0, tk * le * 2);
   cudaMemset(c->u, 0, tk * m * 2);
@@ -729,6 +804,19 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   }
   ok = ok && cudaFuncSetAttribute(reinterpret_cast<const void*>(scan_units_kernel),
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kScanSmemMax) == cudaSuccess;
+  {
+    // the attribute belongs to the kernel, not to this handle: size it for the largest N any handle
+    // may have, so that creating a layer never lowers another layer's limit
+    const int rsm = (int)route_fused_smem(1024, kRouteFusedThreads / 32);
+    const void* rk[] = {reinterpret_cast<const void*>(route_fused_kernel<1>),
+                        reinterpret_cast<const void*>(route_fused_kernel<2>),
+                        reinterpret_cast<const void*>(route_fused_kernel<4>),
+                        reinterpret_cast<const void*>(route_fused_kernel<8>),
+                        reinterpret_cast<const void*>(route_fused_kernel<16>),
+                        reinterpret_cast<const void*>(route_fused_kernel<32>)};
+    for (const void* f : rk)
+      ok = ok && cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, rsm) == cudaSuccess;
+  }
   if (!ok || cudaDeviceSynchronize() != cudaSuccess) {
     free_all(c);
     delete c;
@@ -912,12 +1000,18 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   };
   const bool prof = c->prof_on && c->prof_n < lmoe_ctx::kProfMax;
   cudaEvent_t* ev = prof ? &c->prof_ev[(size_t)c->prof_n * (LMOE_NUM_STAGES + 1)] : nullptr;
+  // stage boundary: record the profiling event; false once any launch has failed, so that no later
+  // kernel runs on routing state a failed launch did not write
   auto mark = [&](int i) {
     if (prof) chk(cudaEventRecord(ev[i], s));
+    return e == cudaSuccess;
   };
   int launches = 0;
-  chk(cudaMemsetAsync(c->work_counters, 0, lmoe_ctx::kCounters * sizeof(int), s));
-  mark(0);
+  // Decode sizes with the stacked router rows (bf16): the routing chain is one cooperative kernel,
+  // which also zeroes the unit counters of the launches after it
+  const bool fused_route = !c->nvfp4 && c->fused_router && vd == V_SMALL && vg == V_SMALL && c->route_bar;
+  if (!fused_route) chk(cudaMemsetAsync(c->work_counters, 0, lmoe_ctx::kCounters * sizeof(int), s));
+  if (!mark(0)) return cuda_status(e);
   if (c->nvfp4) {
     const cudaError_t r = forward_nvfp4(c, x, T, y, idx, gate, s, mark, launches);
     chk(r);
@@ -931,9 +1025,11 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   // inside the expert launches as dense pre problems, and the output GEMM only does W_up z + y_s.
   const bool split = vd == V_SMALL && vg == V_SMALL && c->y_s != nullptr;
 
-  // 1. router logits and the latent h = W_down x
-  chk(router_stage(c, x, T, s, launches));
-  mark(1);
+  // 1. router logits and the latent h = W_down x (with the fused routing kernel: the router GEMM's
+  //    K-slice partials, summed by that kernel)
+  int rks = 1;
+  chk(router_stage(c, x, T, s, launches, fused_route, &rks));
+  if (!mark(1)) return cuda_status(e);
   // 2. shared expert, first matrix: zu[:, l:] = sqrelu(W_s1 x)   (inside the expert-up launch when split)
   const GemmProblem shared_up = problem(d, EPI_SQRELU_BF16, c->zu, l + ms, l);
   if (!split) {
@@ -942,38 +1038,46 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
     chk(g.run(s));
     launches += 1;
   }
-  mark(2);
-  // 3. top-K + softmax + per-chunk histogram
+  if (!mark(2)) return cuda_status(e);
   int ct;
   const int nch = n_chunks_for(T, N, &ct);
-  {
-    const int parts = topk_parts(ct);
-    if (parts > 1) chk(cudaMemsetAsync(c->chunk_counts, 0, (size_t)N * nch * sizeof(int), s));
-    chk(launch_topk_hist(nch, parts, s, c->logits, c->b_router, T, N, K, ct, idx, gate, c->chunk_counts));
-  }
-  mark(3);
-  // 4. expert offsets and grouped-GEMM unit lists
   UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1, c->unit_u0};
   UnitListSpec l2{c->units2, c->num_units + 1, le, V_BN[vg], c->max_units2, c->unit_u0 + N + 1};
-  scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(c->chunk_counts, nch, N, c->counts, c->offsets,
-                                                              c->chunk_base, l1, l2, c->tile0, c->status);
-  chk(cudaGetLastError());
-  chk(launch_build_units(c, s, l1, l2));
-  mark(4);
-  // 5. stable grouping, then the gather of latent rows into grouped order
-  assign_rows_kernel<<<nch, 32 * kAssignWarps, kAssignWarps * N * sizeof(int), s>>>(
-      idx, gate, c->chunk_base, T, N, K, ct, c->row_of, c->tok_of_row, c->gate_of_row, c->status);
-  chk(cudaGetLastError());
-  {
-    long long warps = (TK + GATHER_ROWS - 1) / GATHER_ROWS;
-    long long blocks = (warps + 7) / 8;
-    if (blocks > (long long)c->num_sms * 8) blocks = (long long)c->num_sms * 8;
-    // a standard MoE's experts read x itself
-    const __nv_bfloat16* src = c->standard ? reinterpret_cast<const __nv_bfloat16*>(x) : c->h;
-    gather_rows_kernel<<<(int)blocks, 256, 0, s>>>(src, c->tok_of_row, TK, T, le, c->h_perm, c->status);
+  if (fused_route) {
+    // 3-5. slice sum, top-K, expert scan, unit lists, stable rows and gather in one launch
+    chk(launch_route_fused(c, T, rks, nch, ct, idx, gate, l1, l2, s));
+    if (!mark(3)) return cuda_status(e);
+    if (!mark(4)) return cuda_status(e);
+    if (!mark(5)) return cuda_status(e);
+  } else {
+    // 3. top-K + softmax + per-chunk histogram
+    {
+      const int parts = topk_parts(ct);
+      if (parts > 1) chk(cudaMemsetAsync(c->chunk_counts, 0, (size_t)N * nch * sizeof(int), s));
+      chk(launch_topk_hist(nch, parts, s, c->logits, c->b_router, T, N, K, ct, idx, gate, c->chunk_counts));
+    }
+    if (!mark(3)) return cuda_status(e);
+    // 4. expert offsets and grouped-GEMM unit lists
+    scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(c->chunk_counts, nch, N, c->counts, c->offsets,
+                                                                c->chunk_base, l1, l2, c->tile0, c->status);
     chk(cudaGetLastError());
+    chk(launch_build_units(c, s, l1, l2));
+    if (!mark(4)) return cuda_status(e);
+    // 5. stable grouping, then the gather of latent rows into grouped order
+    assign_rows_kernel<<<nch, 32 * kAssignWarps, kAssignWarps * N * sizeof(int), s>>>(
+        idx, gate, c->chunk_base, T, N, K, ct, c->row_of, c->tok_of_row, c->gate_of_row, c->status);
+    chk(cudaGetLastError());
+    {
+      long long warps = (TK + GATHER_ROWS - 1) / GATHER_ROWS;
+      long long blocks = (warps + 7) / 8;
+      if (blocks > (long long)c->num_sms * 8) blocks = (long long)c->num_sms * 8;
+      // a standard MoE's experts read x itself
+      const __nv_bfloat16* src = c->standard ? reinterpret_cast<const __nv_bfloat16*>(x) : c->h;
+      gather_rows_kernel<<<(int)blocks, 256, 0, s>>>(src, c->tok_of_row, TK, T, le, c->h_perm, c->status);
+      chk(cudaGetLastError());
+    }
+    if (!mark(5)) return cuda_status(e);
   }
-  mark(5);
   // 6. expert up: u = sqrelu(W1_e h)
   {
     GemmLaunch g(c, vg, 4);
@@ -982,7 +1086,7 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
                    0);
     chk(g.run(s));
   }
-  mark(6);
+  if (!mark(6)) return cuda_status(e);
   // 7. expert down with the gate folded in: o = g * (W2_e u); when split, also y_s = W_s2 u_s (fp32)
   {
     GemmLaunch g(c, vg, 5);
@@ -999,7 +1103,7 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
     chk(g.run(s));
     launches += 1;
   }
-  mark(7);
+  if (!mark(7)) return cuda_status(e);
   // 8. latent combine: zu[:, :l] = sum_k o[row_of[t, k]]; a standard MoE's combine writes
   //    y = sum_k o[row_of[t, k]] + y_s and the layer ends here
   if (c->standard)
@@ -1007,9 +1111,9 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
                        c->status, c->y_s, d));
   else
     chk(launch_combine(c->num_sms, s, c->o, c->row_of, T, K, l, c->zu, l + ms, TKmax, c->status));
-  mark(8);
+  if (!mark(8)) return cuda_status(e);
   if (c->standard) {
-    mark(9);
+    if (!mark(9)) return cuda_status(e);
     launches += 8;
     c->launches = launches;
     if (prof) ++c->prof_n;
@@ -1029,8 +1133,8 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
     }
     chk(g.run(s));
   }
-  mark(9);
-  launches += 9;
+  if (!mark(9)) return cuda_status(e);
+  launches += fused_route ? 5 : 9;
   c->launches = launches;
   if (prof) ++c->prof_n;
   c->last_T = T;
@@ -1137,6 +1241,8 @@ lmoe_status lmoe_get_device_status(lmoe_handle c) {
   unsigned st = 0;
   if (cudaMemcpy(&st, c->status, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return LMOE_ERR_CUDA;
   cudaMemset(c->status, 0, sizeof(unsigned));
+  // a bounded wait that gave up may have left the routing kernel's grid barrier mid-phase
+  if (st & DEV_STATUS_TIMEOUT) cudaMemset(c->route_bar, 0, 2 * sizeof(unsigned));
   if (st & DEV_STATUS_TIMEOUT) return LMOE_ERR_DEVICE_TIMEOUT;
   if (st & DEV_STATUS_BAD_INDEX) return LMOE_ERR_DEVICE_INDEX;
   return LMOE_OK;

@@ -77,6 +77,16 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 }
 
 // ------------------------------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with the programmatic-serialisation attribute
+// may start while its predecessor in the stream is still running; it must not read the
+// predecessor's results (or write what the predecessor reads) before griddep_wait(), which returns
+// once the predecessor grid has completed and its memory is visible.  griddep_launch_dependents()
+// lets this kernel's own dependent launch begin early.  Both are no-ops for an ordinary launch.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
+// ------------------------------------------------------------------------------------------------
 // TMA (tiled tensor loads into shared memory, completion signalled on an mbarrier)
 // ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

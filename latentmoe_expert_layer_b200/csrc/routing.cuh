@@ -13,6 +13,9 @@
 // folded into o by the second expert GEMM's epilogue).
 #pragma once
 #include <cuda_bf16.h>
+
+#include <utility>
+
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
 
@@ -48,6 +51,99 @@ __global__ void router_f32_kernel(const __nv_bfloat16* __restrict__ x, const flo
 // output order (value desc, index asc).  Requires K <= 32 and N <= 32 * P.
 // ------------------------------------------------------------------------------------------------
 
+// One token's top-K on one warp: val[i] is logit e = 32 i + lane (bias not included; the caller
+// loads every candidate first, so that all its loads are in flight together).  Writes the K expert
+// ids and softmax gates of the token (slot r at out_idx[r], out_gate[r]) and counts the selections
+// into the shared-memory histogram s_counts.  s_key / s_idx: 32 words each of warp-private scratch.
+template <int P>
+__device__ __forceinline__ void topk_one_token(const float (&val)[P], const float* __restrict__ bias, int n_experts,
+                                               int k, uint32_t* s_key, int* s_idx, int* __restrict__ out_idx,
+                                               float* __restrict__ out_gate, int* s_counts) {
+  const int lane = threadIdx.x & 31;
+  // order-preserving keys: a larger logit has a larger key, -0 and +0 share one; padding is 0
+  uint32_t key[P];
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+    const int e = i * 32 + lane;
+    if (e < n_experts) {
+      const uint32_t u = __float_as_uint(__fadd_rn(val[i] + (bias ? bias[e] : 0.f), 0.f));
+      key[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    } else {
+      key[i] = 0u;
+    }
+  }
+  // the K-th largest key X: the largest value with at least K keys >= X, built two bits at a
+  // time (three independent warp-wide counts per step)
+  uint32_t X = 0u;
+#pragma unroll 1
+  for (int b = 30; b >= 0; b -= 2) {
+    const uint32_t Y1 = X | (1u << b), Y2 = X | (2u << b), Y3 = X | (3u << b);
+    int c1 = 0, c2 = 0, c3 = 0;
+#pragma unroll
+    for (int i = 0; i < P; ++i) {
+      c1 += key[i] >= Y1;
+      c2 += key[i] >= Y2;
+      c3 += key[i] >= Y3;
+    }
+    c1 = __reduce_add_sync(0xffffffffu, c1);
+    c2 = __reduce_add_sync(0xffffffffu, c2);
+    c3 = __reduce_add_sync(0xffffffffu, c3);
+    X = c3 >= k ? Y3 : c2 >= k ? Y2 : c1 >= k ? Y1 : X;
+  }
+  // selected: every key above X, then the lowest expert indices among the keys equal to X
+  int above = 0;
+#pragma unroll
+  for (int i = 0; i < P; ++i) above += key[i] > X;
+  const int need = k - __reduce_add_sync(0xffffffffu, above);
+  const unsigned lt = (1u << lane) - 1u;
+  int tie_base = 0, pos_base = 0;
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+    const unsigned tie = __ballot_sync(0xffffffffu, key[i] == X);
+    const bool sel = key[i] > X || (key[i] == X && tie_base + __popc(tie & lt) < need);
+    tie_base += __popc(tie);
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    if (sel) {
+      const int pos = pos_base + __popc(sb & lt);
+      s_key[pos] = key[i];
+      s_idx[pos] = i * 32 + lane;
+    }
+    pos_base += __popc(sb);
+  }
+  __syncwarp();
+  uint32_t mk = lane < k ? s_key[lane] : 0u;
+  int mi = lane < k ? s_idx[lane] : 0x7fffffff;
+  __syncwarp();
+  // bitonic sort of the K selections over the warp: key descending, then index ascending
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint32_t ok = __shfl_xor_sync(0xffffffffu, mk, stride);
+      const int oi = __shfl_xor_sync(0xffffffffu, mi, stride);
+      const bool other_better = ok > mk || (ok == mk && oi < mi);
+      const bool keep_better = ((lane & stride) == 0) == ((lane & size) == 0);
+      if (keep_better == other_better) {
+        mk = ok;
+        mi = oi;
+      }
+    }
+  }
+  const uint32_t ub = (mk & 0x80000000u) ? (mk & 0x7fffffffu) : ~mk;
+  const float sel_v = __uint_as_float(ub);
+  // softmax over the selected logits (lane r holds slot r); the max is slot 0
+  const float vmax = __shfl_sync(0xffffffffu, sel_v, 0);
+  const float ex = (lane < k) ? expf(sel_v - vmax) : 0.f;
+  float sum = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane < k) {
+    out_idx[lane] = mi;
+    out_gate[lane] = ex / sum;
+    atomicAdd(&s_counts[mi], 1);
+  }
+}
+
 template <int P>
 __global__ void __launch_bounds__(1024)
     topk_hist_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int n_experts,
@@ -63,93 +159,15 @@ __global__ void __launch_bounds__(1024)
   const int sub = (chunk_tokens + parts - 1) / parts;
   const int t_begin = chunk * chunk_tokens + part * sub;
   const int t_end = min(min(T, (chunk + 1) * chunk_tokens), t_begin + sub);
+  uint32_t* s_key = reinterpret_cast<uint32_t*>(s_counts + n_experts) + warp * 64;
+  int* s_idx = reinterpret_cast<int*>(s_key + 32);
   for (int t = t_begin + warp; t < t_end; t += nwarps) {
     const float* lrow = logits + (long long)t * n_experts;
-    // order-preserving keys: a larger logit has a larger key, -0 and +0 share one; padding is 0
-    uint32_t key[P];
+    float val[P];
 #pragma unroll
-    for (int i = 0; i < P; ++i) {
-      const int e = i * 32 + lane;
-      if (e < n_experts) {
-        const uint32_t u = __float_as_uint(__fadd_rn(lrow[e] + (bias ? bias[e] : 0.f), 0.f));
-        key[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-      } else {
-        key[i] = 0u;
-      }
-    }
-    // the K-th largest key X: the largest value with at least K keys >= X, built two bits at a
-    // time (three independent warp-wide counts per step)
-    uint32_t X = 0u;
-#pragma unroll 1
-    for (int b = 30; b >= 0; b -= 2) {
-      const uint32_t Y1 = X | (1u << b), Y2 = X | (2u << b), Y3 = X | (3u << b);
-      int c1 = 0, c2 = 0, c3 = 0;
-#pragma unroll
-      for (int i = 0; i < P; ++i) {
-        c1 += key[i] >= Y1;
-        c2 += key[i] >= Y2;
-        c3 += key[i] >= Y3;
-      }
-      c1 = __reduce_add_sync(0xffffffffu, c1);
-      c2 = __reduce_add_sync(0xffffffffu, c2);
-      c3 = __reduce_add_sync(0xffffffffu, c3);
-      X = c3 >= k ? Y3 : c2 >= k ? Y2 : c1 >= k ? Y1 : X;
-    }
-    // selected: every key above X, then the lowest expert indices among the keys equal to X
-    int above = 0;
-#pragma unroll
-    for (int i = 0; i < P; ++i) above += key[i] > X;
-    const int need = k - __reduce_add_sync(0xffffffffu, above);
-    const unsigned lt = (1u << lane) - 1u;
-    int tie_base = 0, pos_base = 0;
-    uint32_t* s_key = reinterpret_cast<uint32_t*>(s_counts + n_experts) + warp * 64;
-    int* s_idx = reinterpret_cast<int*>(s_key + 32);
-#pragma unroll
-    for (int i = 0; i < P; ++i) {
-      const unsigned tie = __ballot_sync(0xffffffffu, key[i] == X);
-      const bool sel = key[i] > X || (key[i] == X && tie_base + __popc(tie & lt) < need);
-      tie_base += __popc(tie);
-      const unsigned sb = __ballot_sync(0xffffffffu, sel);
-      if (sel) {
-        const int pos = pos_base + __popc(sb & lt);
-        s_key[pos] = key[i];
-        s_idx[pos] = i * 32 + lane;
-      }
-      pos_base += __popc(sb);
-    }
-    __syncwarp();
-    uint32_t mk = lane < k ? s_key[lane] : 0u;
-    int mi = lane < k ? s_idx[lane] : 0x7fffffff;
-    __syncwarp();
-    // bitonic sort of the K selections over the warp: key descending, then index ascending
-#pragma unroll
-    for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        const uint32_t ok = __shfl_xor_sync(0xffffffffu, mk, stride);
-        const int oi = __shfl_xor_sync(0xffffffffu, mi, stride);
-        const bool other_better = ok > mk || (ok == mk && oi < mi);
-        const bool keep_better = ((lane & stride) == 0) == ((lane & size) == 0);
-        if (keep_better == other_better) {
-          mk = ok;
-          mi = oi;
-        }
-      }
-    }
-    const uint32_t ub = (mk & 0x80000000u) ? (mk & 0x7fffffffu) : ~mk;
-    const float sel_v = __uint_as_float(ub);
-    const int sel_i = mi;
-    // softmax over the selected logits (lane r holds slot r); the max is slot 0
-    const float vmax = __shfl_sync(0xffffffffu, sel_v, 0);
-    const float ex = (lane < k) ? expf(sel_v - vmax) : 0.f;
-    float sum = ex;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane < k) {
-      topk_idx[(long long)t * k + lane] = sel_i;
-      topk_gate[(long long)t * k + lane] = ex / sum;
-      atomicAdd(&s_counts[sel_i], 1);
-    }
+    for (int i = 0; i < P; ++i) val[i] = (i * 32 + lane < n_experts) ? lrow[i * 32 + lane] : 0.f;
+    topk_one_token<P>(val, bias, n_experts, k, s_key, s_idx, topk_idx + (long long)t * k, topk_gate + (long long)t * k,
+                      s_counts);
   }
   __syncthreads();
   // expert-major layout [N][n_chunks]: the scan reads one expert's chunks contiguously; blocks that
@@ -475,6 +493,8 @@ template <bool BATCH>
 __global__ void combine_kernel(const __nv_bfloat16* __restrict__ o, const int* __restrict__ row_of, int T, int k,
                                int latent, __nv_bfloat16* __restrict__ zu, long long ld_zu, long long n_rows,
                                unsigned* status, const float* __restrict__ add, long long ld_add) {
+  griddep_launch_dependents();
+  griddep_wait();  // o comes from the launch before
   const int vpr = latent / 8;  // 8 bf16 per thread
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long t = gid / vpr;
@@ -578,16 +598,33 @@ __global__ void __launch_bounds__(256)
 
 // combine over T tokens of `latent` columns: the batched variant while the grid is below ~8 warps
 // per SM
+// Launch with programmatic stream serialisation (the kernel calls griddep_wait before it reads what
+// the previous launch wrote): its launch and set-up overlap the previous kernel's tail.
+template <typename... P, typename... A>
+cudaError_t launch_pdl(void (*kernel)(P...), int grid, int threads, size_t smem, cudaStream_t s, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
+
 inline cudaError_t launch_combine(int num_sms, cudaStream_t s, const __nv_bfloat16* o, const int* row_of, int T,
                                   int k, int latent, __nv_bfloat16* out, long long ld_out, long long n_rows,
                                   unsigned* status, const float* add = nullptr, long long ld_add = 0) {
   const long long threads = (long long)T * (latent / 8);
   const int blocks = (int)((threads + 255) / 256);
   if (threads <= (long long)num_sms * 256)
-    combine_kernel<true><<<blocks, 256, 0, s>>>(o, row_of, T, k, latent, out, ld_out, n_rows, status, add, ld_add);
-  else
-    combine_kernel<false><<<blocks, 256, 0, s>>>(o, row_of, T, k, latent, out, ld_out, n_rows, status, add, ld_add);
-  return cudaGetLastError();
+    return launch_pdl(combine_kernel<true>, blocks, 256, 0, s, o, row_of, T, k, latent, out, ld_out, n_rows, status,
+                      add, ld_add);
+  return launch_pdl(combine_kernel<false>, blocks, 256, 0, s, o, row_of, T, k, latent, out, ld_out, n_rows, status,
+                    add, ld_add);
 }
 
 // ------------------------------------------------------------------------------------------------

@@ -254,3 +254,16 @@ def test_degenerate_top_k(k):
             assert np.array_equal(np.sort(st["idx"], axis=1), np.tile(np.arange(16), (wl.tokens, 1)))
     finally:
         layer.close()
+
+
+def test_a_second_layer_does_not_disturb_the_first(superlayer):
+    """Kernel attributes are process-wide: creating a layer of another shape (here N = 16 experts)
+    must not change what an existing layer's forward can launch."""
+    import latentmoe_expert_layer_b200 as lm
+    w, _, layer = superlayer
+    wl = inp.workload("decode")
+    small = lm.LatentMoE(dataclasses.replace(inp.TINY, latent=0), 16)
+    try:
+        compare_bf16(layer, oracle_weights(w, False), inp.make_x(wl, tokens=64), wl.shape.top_k)
+    finally:
+        small.close()
