@@ -66,6 +66,12 @@ typedef struct {
                           NVFP4 needs d, latent, expert_ffn and shared_ffn to be multiples of 128 */
   int32_t has_router_bias; /* 1: a per-expert fp32 bias is added to the router logits */
   int32_t weight_scale;    /* NVFP4 weight block scales (lmoe_weight_scale); ignored for bf16 */
+  int32_t ep_world;        /* expert parallelism: 0 or 1 = this layer holds every expert; G in 2..8 = this
+                              layer is rank ep_rank of G ranks and holds only experts [ep_rank * N / G,
+                              (ep_rank + 1) * N / G) (bf16 LatentMoE only; N a multiple of 16 * G).  Such a
+                              layer runs through lmoe_ep_dispatch / lmoe_ep_experts / lmoe_ep_combine, and
+                              lmoe_forward returns LMOE_ERR_UNSUPPORTED */
+  int32_t ep_rank;         /* 0 .. ep_world - 1 */
 } lmoe_config;
 
 /* How the NVFP4 quantiser picks a weight block's E4M3 scale.  AMAX: s = E4M3(amax_block / (6 g)).
@@ -85,8 +91,9 @@ typedef struct {
   const float* b_router; /* [N] fp32, or NULL (required iff has_router_bias) */
   const void* w_down;    /* [l, d]   (W_down); NULL for a standard MoE (latent == 0), else required */
   const void* w_up;      /* [d, l]   (W_up); NULL for a standard MoE, else required */
-  const void* w1;        /* [N, m, l] expert up matrices ([N, m, d] for a standard MoE) */
-  const void* w2;        /* [N, l, m] expert down matrices ([N, d, m] for a standard MoE) */
+  const void* w1;        /* [N, m, l] expert up matrices ([N, m, d] for a standard MoE; [N / G, m, l], the
+                            owned experts in order, for an expert-parallel layer) */
+  const void* w2;        /* [N, l, m] expert down matrices (likewise) */
   const void* ws1;       /* [m_s, d] shared expert */
   const void* ws2;       /* [d, m_s] shared expert */
   int32_t dtype;         /* lmoe_dtype */
@@ -217,6 +224,59 @@ lmoe_status lmoe_profile_read(lmoe_handle h, double* stage_ms /* [LMOE_NUM_STAGE
 lmoe_status lmoe_route_noalloc(const float* logits, const float* bias, int32_t T, int32_t n_experts, int32_t top_k,
                                int32_t* topk_idx, float* topk_gate, int32_t* counts, int32_t* offsets,
                                int32_t* row_of, uint32_t* status, void* stream);
+
+/* ------------------------------------------------------------------------------------------------
+ * Expert parallelism ("Nemotron 3 Super" notes, section 3.2: the routing traffic of distributed MoE
+ * grows with the dispatched vectors' width times K; LatentMoE dispatches the l-wide latent h = W_down x
+ * instead of x).  G ranks (one layer handle each, created with ep_world = G) each own N / G
+ * consecutive experts and replicate the router, W_down, W_up and the shared expert.  A forward of a
+ * rank's T tokens is three calls with two exchanges between them, done by the caller (for example an
+ * all-to-all over NCCL):
+ *
+ *   1. lmoe_ep_dispatch  (every rank, its own tokens)  routing and the send plan: one latent row per
+ *      (token, owner rank) pair, pairs in (destination, token) order, and per assignment in
+ *      (destination, token, slot) order its pair index within the destination and its expert id local
+ *      to the destination, with the gate.
+ *      exchange: rows, assignments and gates to their destinations (sizes from `counts`);
+ *   2. lmoe_ep_experts   (every rank, the rows it received)  the owned experts, gate folded in, and
+ *      the sum of each pair's gated outputs in slot order: one fp32 partial latent sum per pair.
+ *      exchange: partial sums back to their sources, in the order the rows came;
+ *   3. lmoe_ep_combine   (every rank, its own tokens)  z[t] = the token's partial sums in ascending
+ *      owner-rank order, then y = W_up z + W_s2 sqrelu(W_s1 x).
+ *
+ * z is the single-GPU layer's K gated expert outputs grouped by owner rank; the two differ only in
+ * rounding.  At most min(K, G) latent rows of l per token cross in each direction instead of K rows of
+ * d.  All pointers are device pointers, 16-byte aligned; calls are enqueued on `stream`; the handle's
+ * workspace is shared by the three calls, so one rank's calls must not overlap each other.
+ * ------------------------------------------------------------------------------------------------ */
+
+/* Step 1.  x [T, d] bf16 in.  Out, with P = pairs and A = T * K assignments:
+ *   topk_idx [T, K] int32 (global expert ids), topk_gate [T, K] fp32
+ *   send_rows [T * min(K, G), l] bf16: rows 0 .. P-1 are the latent rows of the pairs in send order
+ *   send_meta [T * K, 2] int32: per assignment in send order, (pair index within its destination,
+ *             expert id local to the destination)
+ *   send_gate [T * K] fp32: per assignment in send order
+ *   counts    [G, 2] int32: pairs and assignments sent to each destination (destinations in order)
+ *   tok_pairs [T, min(K, G)] int32: the send-order indices of token t's pairs, ascending destination,
+ *             then -1
+ * Errors: UNSUPPORTED unless the handle is expert-parallel; SHAPE for T outside 0 .. max_tokens. */
+lmoe_status lmoe_ep_dispatch(lmoe_handle h, const void* x, int32_t T, int32_t* topk_idx, float* topk_gate,
+                             void* send_rows, int32_t* send_meta, float* send_gate, int32_t* counts,
+                             int32_t* tok_pairs, void* stream);
+
+/* Step 2.  recv_rows [R, l] bf16: the latent rows received (any order of sources); recv_meta [A, 2]
+ * int32: per received assignment, (row of recv_rows, expert id local to this rank), with the rows
+ * nondecreasing (each source's assignments arrive in its send order, sources one after another);
+ * recv_gate [A] fp32.  Out: partial [R, l] fp32, row r = sum over the assignments of row r, in arrival
+ * order, of gate * W2_e sqrelu(W1_e recv_rows[r]).  R <= ep_world * max_tokens * min(K, G) and
+ * A <= ep_world * max_tokens * K, else SHAPE.  A row with no assignment gets zeros. */
+lmoe_status lmoe_ep_experts(lmoe_handle h, const void* recv_rows, int32_t R, const int32_t* recv_meta,
+                            const float* recv_gate, int32_t A, float* partial, void* stream);
+
+/* Step 3.  x [T, d] bf16 (the tokens of step 1); back [P, l] fp32: the partial sums returned for this
+ * rank's pairs, in send order; tok_pairs from step 1.  Out: y [T, d] bf16. */
+lmoe_status lmoe_ep_combine(lmoe_handle h, const void* x, int32_t T, const float* back, const int32_t* tok_pairs,
+                            void* y, void* stream);
 
 /* Failure-detection self-test.  Enqueues on `stream` one kernel that waits, with the bounded
  * mbarrier wait that every pipelined kernel of the library uses, on a barrier that nothing ever

@@ -36,13 +36,15 @@ DTYPE = {torch.bfloat16: 0, torch.float32: 1}
 # every extern "C" symbol declared in include/lmoe.h
 SYMBOLS = ("lmoe_create", "lmoe_load_weights", "lmoe_forward", "lmoe_forward_host", "lmoe_get_device_status",
            "lmoe_inspect", "lmoe_profile", "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_export_nvfp4",
-           "lmoe_selftest_wait_timeout", "lmoe_status_string", "lmoe_destroy")
+           "lmoe_selftest_wait_timeout", "lmoe_status_string", "lmoe_destroy", "lmoe_ep_dispatch", "lmoe_ep_experts",
+           "lmoe_ep_combine")
 STAGES = ("router", "shared_up", "topk", "grouping", "scatter", "expert_up", "expert_down", "combine", "output")
 
 
 class _Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("d", "latent", "n_experts", "top_k", "expert_ffn", "shared_ffn",
-                                             "max_tokens", "precision", "has_router_bias", "weight_scale")]
+                                             "max_tokens", "precision", "has_router_bias", "weight_scale",
+                                             "ep_world", "ep_rank")]
 
 
 class _Weights(ctypes.Structure):
@@ -63,13 +65,16 @@ lib.lmoe_profile_read.argtypes = [_vp, ctypes.POINTER(ctypes.c_double), ctypes.P
 lib.lmoe_route_noalloc.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.lmoe_export_nvfp4.argtypes = [_vp, _i32, _i32, _vp, _vp, _vp]
 lib.lmoe_selftest_wait_timeout.argtypes = [_vp, ctypes.c_uint64, _vp]
+lib.lmoe_ep_dispatch.argtypes = [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.lmoe_ep_experts.argtypes = [_vp, _vp, _i32, _vp, _vp, _i32, _vp, _vp]
+lib.lmoe_ep_combine.argtypes = [_vp, _vp, _i32, _vp, _vp, _vp, _vp]
 lib.lmoe_status_string.argtypes = [ctypes.c_int]
 lib.lmoe_status_string.restype = ctypes.c_char_p
 lib.lmoe_destroy.argtypes = [_vp]
 lib.lmoe_destroy.restype = None
 for _f in ("lmoe_create", "lmoe_load_weights", "lmoe_forward", "lmoe_forward_host", "lmoe_get_device_status",
            "lmoe_inspect", "lmoe_profile", "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_export_nvfp4",
-           "lmoe_selftest_wait_timeout"):
+           "lmoe_selftest_wait_timeout", "lmoe_ep_dispatch", "lmoe_ep_experts", "lmoe_ep_combine"):
     getattr(lib, _f).restype = ctypes.c_int
 
 
@@ -143,18 +148,23 @@ class LatentMoE:
     precision: "bf16", or "nvfp4" for block-scaled FP4 routed and shared experts.
     router_bias: a per-expert fp32 bias is added to the router logits (load_weights' b_router).
     weight_scale: NVFP4 weight block scales, "amax" or "mse" (lmoe_weight_scale).
+    ep_world, ep_rank: expert parallelism; with ep_world = G >= 2 this layer is rank ep_rank of G and
+        holds only experts [ep_rank * N / G, (ep_rank + 1) * N / G) (load_weights' w1 / w2 hold those);
+        it runs through ep_dispatch / ep_experts / ep_combine instead of forward.
     """
 
     def __init__(self, shape, max_tokens: int, precision: str = "bf16", router_bias: bool = False,
-                 device: int = 0, weight_scale: str = "amax"):
+                 device: int = 0, weight_scale: str = "amax", ep_world: int = 0, ep_rank: int = 0):
         cfg = _Config(shape.d, shape.latent, shape.n_experts, shape.top_k, shape.expert_ffn, shape.shared_ffn,
-                      max_tokens, PREC[precision], int(router_bias), WSCALE[weight_scale])
+                      max_tokens, PREC[precision], int(router_bias), WSCALE[weight_scale], ep_world, ep_rank)
         h = _vp()
         _check(lib.lmoe_create(ctypes.byref(cfg), device, ctypes.byref(h)), "lmoe_create")
         self._h = h
         self.shape = shape
         self.max_tokens = max_tokens
         self.device = torch.device("cuda", device)
+        self.ep_world = ep_world if ep_world > 1 else 0
+        self.ep_rank = ep_rank if ep_world > 1 else 0
 
     def load_weights(self, w_router, w_down, w_up, w1, w2, ws1, ws2, b_router=None, stream=None) -> None:
         # a standard MoE (latent == 0) passes w_down = w_up = None
@@ -189,6 +199,46 @@ class LatentMoE:
         """x, y, idx, gate are CPU tensors (pinned for asynchronous copies)."""
         _check(lib.lmoe_forward_host(self._h, _ptr(x), x.shape[0], _ptr(y), _ptr(idx), _ptr(gate),
                                      self._stream(stream)), "lmoe_forward_host")
+
+    # ------------------------------------------------------------------ expert parallelism
+    def ep_dispatch(self, x: torch.Tensor, stream=None) -> dict:
+        """Step 1 (lmoe_ep_dispatch): routing and the send plan of this rank's tokens x [T, d].
+        Returns device tensors idx, gate, send_rows (first P rows valid), send_meta, send_gate (first
+        A entries valid), counts [G, 2] (pairs, assignments per destination) and tok_pairs."""
+        t, s, g = x.shape[0], self.shape, self.ep_world
+        gp = min(s.top_k, g)
+        dev = self.device
+        out = {"idx": torch.empty((t, s.top_k), dtype=torch.int32, device=dev),
+               "gate": torch.empty((t, s.top_k), dtype=torch.float32, device=dev),
+               "send_rows": torch.empty((t * gp, s.latent), dtype=torch.bfloat16, device=dev),
+               "send_meta": torch.empty((t * s.top_k, 2), dtype=torch.int32, device=dev),
+               "send_gate": torch.empty((t * s.top_k,), dtype=torch.float32, device=dev),
+               "counts": torch.empty((g, 2), dtype=torch.int32, device=dev),
+               "tok_pairs": torch.empty((t, gp), dtype=torch.int32, device=dev)}
+        _check(lib.lmoe_ep_dispatch(self._h, _ptr(x), t, _ptr(out["idx"]), _ptr(out["gate"]), _ptr(out["send_rows"]),
+                                    _ptr(out["send_meta"]), _ptr(out["send_gate"]), _ptr(out["counts"]),
+                                    _ptr(out["tok_pairs"]), self._stream(stream)), "lmoe_ep_dispatch")
+        return out
+
+    def ep_experts(self, recv_rows: torch.Tensor, recv_meta: torch.Tensor, recv_gate: torch.Tensor,
+                   stream=None) -> torch.Tensor:
+        """Step 2 (lmoe_ep_experts): this rank's experts on the received latent rows [R, l]; recv_meta
+        [A, 2] (row of recv_rows, local expert id), rows nondecreasing; recv_gate [A].  Returns the fp32
+        partial sums [R, l]."""
+        r, a = recv_rows.shape[0], recv_meta.shape[0]
+        partial = torch.empty((r, self.shape.latent), dtype=torch.float32, device=self.device)
+        _check(lib.lmoe_ep_experts(self._h, _ptr(recv_rows), r, _ptr(recv_meta) if a else None,
+                                   _ptr(recv_gate) if a else None, a, _ptr(partial), self._stream(stream)),
+               "lmoe_ep_experts")
+        return partial
+
+    def ep_combine(self, x: torch.Tensor, back: torch.Tensor, tok_pairs: torch.Tensor, stream=None) -> torch.Tensor:
+        """Step 3 (lmoe_ep_combine): y [T, d] from this rank's tokens x, the fp32 partial sums returned
+        for its pairs (send order) and tok_pairs from ep_dispatch."""
+        y = torch.empty((x.shape[0], self.shape.d), dtype=torch.bfloat16, device=self.device)
+        _check(lib.lmoe_ep_combine(self._h, _ptr(x), x.shape[0], _ptr(back), _ptr(tok_pairs), _ptr(y),
+                                   self._stream(stream)), "lmoe_ep_combine")
+        return y
 
     def device_status(self) -> int:
         return lib.lmoe_get_device_status(self._h)

@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "../../include/lmoe.h"
+#include "ep.cuh"
 #include "gemm_tc.cuh"
 #include "route_fused.cuh"
 #include "routing.cuh"
@@ -95,6 +96,10 @@ struct lmoe_ctx {
   bool fused_router = false;
   bool standard = false;  // latent == 0: a standard MoE, experts d -> m -> d, no W_down / W_up
   int le = 0;             // width the routed experts work in: latent, or d for a standard MoE
+  int ep_world = 0;       // expert parallelism: G ranks (>= 2), this one ep_rank, owning n_local experts
+  int ep_rank = 0;
+  int n_local = 0;        // experts whose weights this handle holds (N, or N / G)
+  long long tk_exp = 0;   // capacity in assignments of the expert-side buffers
   unsigned long long timeout_ns = kDefaultTimeoutNs;
 
   // weights (library-owned)
@@ -130,6 +135,9 @@ struct lmoe_ctx {
   int* num_units = nullptr;  // [2]
   unsigned* status = nullptr;
   unsigned* route_bar = nullptr;  // [2] grid barrier of the fused decode routing kernel (zero at rest)
+  int* ep_ids = nullptr;          // [tk_exp] expert parallelism: received assignments' local experts
+  int* ep_src = nullptr;          // [tk_exp] and their rows in the received latent rows
+  int* ep_send_tok = nullptr;     // [max_tokens * min(K, G)] token of each sent pair
   int* work_counters = nullptr;  // [kCounters] per-launch unit counters and (last two) activation amax
                                  // bits, all zeroed at the start of a forward
   static constexpr int kCounters = 10;
@@ -228,7 +236,7 @@ void free_all(lmoe_ctx* c) {
                   c->ws2_sf, c->wg,     c->w_amax, c->xq,        c->x_sf,       c->hq,         c->h_sf,
                   c->hq_tok, c->h_sf_tok,
                   c->uq,     c->u_sf,   c->usq,    c->us_sf,     c->act_g,      c->tile0,      c->unit_u0,
-                  c->router_part, c->route_bar};
+                  c->router_part, c->route_bar, c->ep_ids, c->ep_src, c->ep_send_tok};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -474,12 +482,23 @@ cudaError_t router_stage(lmoe_ctx* c, const void* x, int T, cudaStream_t s, int&
   return launch_split_reduce(c, ks, p.split_stride, T, N, 0, s);
 }
 
+// Tensor maps of the activations x [T, d] for both bf16 variants, cached by (pointer, T).
+bool set_x_maps(lmoe_ctx* c, const void* x, int T) {
+  if (x == c->x_cached && T == c->x_cached_T) return true;
+  for (int v = 0; v < 2; ++v)
+    if (!make_map(&c->map_x[v], x, T, c->cfg.d, c->cfg.d, V_BOXN[v])) return false;
+  c->x_cached = x;
+  c->x_cached_T = T;
+  return true;
+}
+
 // The two grouped-GEMM unit lists from the scan's first units: one unit per thread.
-cudaError_t launch_build_units(const lmoe_ctx* c, cudaStream_t s, const UnitListSpec& l1, const UnitListSpec& l2) {
+cudaError_t launch_build_units(const lmoe_ctx* c, cudaStream_t s, const UnitListSpec& l1, const UnitListSpec& l2,
+                               int n_experts) {
   const long long cap = (long long)c->max_units1 + c->max_units2;
   long long blocks = (cap + 255) / 256;
   if (blocks > 4LL * c->num_sms) blocks = 4LL * c->num_sms;
-  build_units_kernel<<<(int)blocks, 256, 0, s>>>(c->counts, c->offsets, c->tile0, c->cfg.n_experts, l1, l2);
+  build_units_kernel<<<(int)blocks, 256, 0, s>>>(c->counts, c->offsets, c->tile0, n_experts, l1, l2);
   return cudaGetLastError();
 }
 
@@ -604,7 +623,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
   scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(c->chunk_counts, nch, N, c->counts, c->offsets,
                                                               c->chunk_base, l1, l2, c->tile0, c->status);
   chk(cudaGetLastError());
-  chk(launch_build_units(c, s, l1, l2));
+  chk(launch_build_units(c, s, l1, l2, N));
   if (!mark(4)) return e;
   // 5. stable grouping; h quantised once per token, then its rows copied into grouped order with
   //    their scales in the expert GEMM's tile-local atoms
@@ -708,8 +727,15 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   if (g.precision == LMOE_PREC_NVFP4 &&
       (g.d % 128 || g.latent % 128 || g.expert_ffn % 128 || g.shared_ffn % 128))
     return LMOE_ERR_UNSUPPORTED;
+  if (g.ep_world < 0 || (g.ep_world > 1 && (g.ep_rank < 0 || g.ep_rank >= g.ep_world))) return LMOE_ERR_INVALID_ARG;
+  const bool ep = g.ep_world > 1;
+  if (ep && (g.ep_world > EP_MAX_WORLD || g.n_experts % g.ep_world || g.precision != LMOE_PREC_BF16 ||
+             g.latent == 0))
+    return LMOE_ERR_UNSUPPORTED;
   const long long tk = (long long)g.max_tokens * g.top_k;
-  if (tk > 0x7fffffffLL / 2) return LMOE_ERR_UNSUPPORTED;
+  // expert-side capacity: an expert-parallel rank may receive every rank's assignments
+  const long long tk_exp = ep ? tk * g.ep_world : tk;
+  if (tk_exp > 0x7fffffffLL / 2) return LMOE_ERR_UNSUPPORTED;
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) return LMOE_ERR_NO_DEVICE;
   cudaDeviceProp prop;
@@ -726,16 +752,25 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   c->standard = l == 0;
   const int le = c->standard ? d : l;
   c->le = le;
+  c->ep_world = ep ? g.ep_world : 0;
+  c->ep_rank = ep ? g.ep_rank : 0;
+  c->n_local = ep ? N / g.ep_world : N;
+  c->tk_exp = tk_exp;
+  const int NL = c->n_local;
   const int nft1 = (m + BLOCK_M - 1) / BLOCK_M, nft2 = (le + BLOCK_M - 1) / BLOCK_M;
-  c->max_units1 = (int)(nft1 * (N + (tk + V_BN[V_SMALL] - 1) / V_BN[V_SMALL]));
-  c->max_units2 = (int)(nft2 * (N + (tk + V_BN[V_SMALL] - 1) / V_BN[V_SMALL]));
+  c->max_units1 = (int)(nft1 * (NL + (tk_exp + V_BN[V_SMALL] - 1) / V_BN[V_SMALL]));
+  c->max_units2 = (int)(nft2 * (NL + (tk_exp + V_BN[V_SMALL] - 1) / V_BN[V_SMALL]));
   bool ok = true;
   ok = ok && dalloc(&c->logits, T * N) && dalloc(&c->idx, tk) && dalloc(&c->gate, tk);
   ok = ok && dalloc(&c->chunk_counts, 128LL * N) && dalloc(&c->chunk_base, 128LL * N);
   ok = ok && dalloc(&c->counts, N) && dalloc(&c->offsets, N + 1);
-  ok = ok && dalloc(&c->row_of, tk) && dalloc(&c->tok_of_row, tk) && dalloc(&c->gate_of_row, tk);
+  ok = ok && dalloc(&c->row_of, tk_exp) && dalloc(&c->tok_of_row, tk_exp) && dalloc(&c->gate_of_row, tk_exp);
   if (!c->standard) ok = ok && dalloc(&c->h, T * l);
-  ok = ok && dalloc(&c->h_perm, tk * le) && dalloc(&c->u, tk * m) && dalloc(&c->o, tk * le);
+  ok = ok && dalloc(&c->h_perm, tk_exp * le) && dalloc(&c->u, tk_exp * m) && dalloc(&c->o, tk_exp * le);
+  if (ep) {
+    const int gp = g.top_k < g.ep_world ? g.top_k : g.ep_world;
+    ok = ok && dalloc(&c->ep_ids, tk_exp) && dalloc(&c->ep_src, tk_exp) && dalloc(&c->ep_send_tok, T * gp);
+  }
   ok = ok && dalloc(&c->zu, T * (l + ms));
   ok = ok && dalloc(&c->units1, c->max_units1) && dalloc(&c->units2, c->max_units2) && dalloc(&c->num_units, 2);
   ok = ok && dalloc(&c->status, 1) && dalloc(&c->work_counters, lmoe_ctx::kCounters) && dalloc(&c->route_bar, 2);
@@ -765,12 +800,12 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   cudaMemset(c->status, 0, sizeof(unsigned));
   cudaMemset(c->route_bar, 0, 2 * sizeof(unsigned));
   // rows that no expert writes must still be finite for the MMA (they are masked in the epilogue)
-  cudaMemset(c->h_perm, 0, tk * le * 2);
-  cudaMemset(c->u, 0, tk * m * 2);
+  cudaMemset(c->h_perm, 0, tk_exp * le * 2);
+  cudaMemset(c->u, 0, tk_exp * m * 2);
   cudaMemset(c->zu, 0, T * (l + ms) * 2);
   for (int v = 0; v < 2; ++v) {
-    ok = ok && make_map(&c->map_hperm[v], c->h_perm, tk, le, le, V_BOXN[v]);
-    ok = ok && make_map(&c->map_u[v], c->u, tk, m, m, V_BOXN[v]);
+    ok = ok && make_map(&c->map_hperm[v], c->h_perm, tk_exp, le, le, V_BOXN[v]);
+    ok = ok && make_map(&c->map_u[v], c->u, tk_exp, m, m, V_BOXN[v]);
     ok = ok && make_map(&c->map_zu[v], c->zu, T, l + ms, l + ms, V_BOXN[v]);
     if (!c->standard) ok = ok && make_map(&c->map_z[v], c->zu, T, l, l + ms, V_BOXN[v]);
     ok = ok && make_map(&c->map_us[v], c->zu + l, T, ms, l + ms, V_BOXN[v]);
@@ -892,8 +927,9 @@ lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream
   if (!c->standard) ok = ok && conv(w->w_up, d, l, l, c->w_cat, l + ms, 0);
   ok = ok && conv(w->ws2, d, ms, ms, c->w_cat, l + ms, l);
   ok = ok && dalloc(&c->ws1, (size_t)ms * d) && conv(w->ws1, ms, d, d, c->ws1, d, 0);
-  ok = ok && dalloc(&c->w1, (size_t)N * m * le) && conv(w->w1, (long long)N * m, le, le, c->w1, le, 0);
-  ok = ok && dalloc(&c->w2, (size_t)N * le * m) && conv(w->w2, (long long)N * le, m, m, c->w2, m, 0);
+  const int NL = c->n_local;  // the experts this handle holds
+  ok = ok && dalloc(&c->w1, (size_t)NL * m * le) && conv(w->w1, (long long)NL * m, le, le, c->w1, le, 0);
+  ok = ok && dalloc(&c->w2, (size_t)NL * le * m) && conv(w->w2, (long long)NL * le, m, m, c->w2, m, 0);
   if (!ok) return LMOE_ERR_OOM;
   if (c->nvfp4) {
     // quantise W1, W2, W_s1, W_s2 on the device; keep only codes, scale atoms and tensor scales
@@ -958,8 +994,8 @@ lmoe_status lmoe_load_weights(lmoe_handle c, const lmoe_weights* w, void* stream
   ok = ok && make_map(&c->map_ws2, c->w_cat + l, d, ms, l + ms, BLOCK_M);
   if (!c->nvfp4) {
     ok = ok && make_map(&c->map_ws1, c->ws1, ms, d, d, BLOCK_M);
-    ok = ok && make_map(&c->map_w1, c->w1, (uint64_t)N * m, le, le, BLOCK_M);
-    ok = ok && make_map(&c->map_w2, c->w2, (uint64_t)N * le, m, m, BLOCK_M);
+    ok = ok && make_map(&c->map_w1, c->w1, (uint64_t)NL * m, le, le, BLOCK_M);
+    ok = ok && make_map(&c->map_w2, c->w2, (uint64_t)NL * le, m, m, BLOCK_M);
   }
   if (!ok) return LMOE_ERR_CUDA;
   c->loaded = true;
@@ -971,6 +1007,7 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   if (!c) return LMOE_ERR_INVALID_ARG;
   if (T < 0 || T > c->cfg.max_tokens) return LMOE_ERR_SHAPE;
   if (!c->loaded) return LMOE_ERR_NOT_LOADED;
+  if (c->ep_world > 1) return LMOE_ERR_UNSUPPORTED;  // an expert-parallel rank runs the lmoe_ep_* steps
   if (T == 0) return LMOE_OK;
   if (!x || !y) return LMOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y) || (topk_idx && !aligned16(topk_idx)) || (topk_gate && !aligned16(topk_gate)))
@@ -985,13 +1022,7 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   const int vd = T <= 512 ? V_SMALL : V_LARGE;
   const int vg = TK <= 48LL * N ? V_SMALL : V_LARGE;
 
-  if (x != c->x_cached || T != c->x_cached_T) {
-    bool ok = true;
-    for (int v = 0; v < 2; ++v) ok = ok && make_map(&c->map_x[v], x, T, d, d, V_BOXN[v]);
-    if (!ok) return LMOE_ERR_CUDA;
-    c->x_cached = x;
-    c->x_cached_T = T;
-  }
+  if (!set_x_maps(c, x, T)) return LMOE_ERR_CUDA;
   int* idx = topk_idx ? topk_idx : c->idx;
   float* gate = topk_gate ? topk_gate : c->gate;
   cudaError_t e = cudaSuccess;
@@ -1061,7 +1092,7 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
     scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(c->chunk_counts, nch, N, c->counts, c->offsets,
                                                                 c->chunk_base, l1, l2, c->tile0, c->status);
     chk(cudaGetLastError());
-    chk(launch_build_units(c, s, l1, l2));
+    chk(launch_build_units(c, s, l1, l2, N));
     if (!mark(4)) return cuda_status(e);
     // 5. stable grouping, then the gather of latent rows into grouped order
     assign_rows_kernel<<<nch, 32 * kAssignWarps, kAssignWarps * N * sizeof(int), s>>>(
@@ -1169,6 +1200,158 @@ lmoe_status lmoe_forward_host(lmoe_handle c, const void* x_host, int32_t T, void
   if (gate_host && cudaMemcpyAsync(gate_host, c->gate_dev, ib, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return LMOE_ERR_CUDA;
   return LMOE_OK;
+}
+
+// ---------------------------------------------------------------------------------------- expert parallelism
+lmoe_status lmoe_ep_dispatch(lmoe_handle c, const void* x, int32_t T, int32_t* topk_idx, float* topk_gate,
+                             void* send_rows, int32_t* send_meta, float* send_gate, int32_t* counts,
+                             int32_t* tok_pairs, void* stream) {
+  if (!c) return LMOE_ERR_INVALID_ARG;
+  if (c->ep_world < 2) return LMOE_ERR_UNSUPPORTED;
+  if (T < 0 || T > c->cfg.max_tokens) return LMOE_ERR_SHAPE;
+  if (!c->loaded) return LMOE_ERR_NOT_LOADED;
+  if (T == 0) return LMOE_OK;
+  const void* ptrs[] = {x, topk_idx, topk_gate, send_rows, send_meta, send_gate, counts, tok_pairs};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const lmoe_config& g = c->cfg;
+  const int N = g.n_experts, K = g.top_k, G = c->ep_world;
+  const int GP = K < G ? K : G;
+  if (!set_x_maps(c, x, T)) return LMOE_ERR_CUDA;
+  cudaError_t e = cudaMemsetAsync(c->work_counters, 0, lmoe_ctx::kCounters * sizeof(int), s);
+  int launches = 0;
+  if (e == cudaSuccess) e = router_stage(c, x, T, s, launches);
+  int ct;
+  const int nch = n_chunks_for(T, N, &ct);
+  const int parts = topk_parts(ct);
+  if (e == cudaSuccess && parts > 1) e = cudaMemsetAsync(c->chunk_counts, 0, (size_t)N * nch * sizeof(int), s);
+  if (e == cudaSuccess)
+    e = launch_topk_hist(nch, parts, s, c->logits, c->b_router, T, N, K, ct, topk_idx, topk_gate, c->chunk_counts);
+  if (e == cudaSuccess) {
+    ep_plan_kernel<<<1, EP_PLAN_THREADS, 0, s>>>(topk_idx, topk_gate, T, K, N, N / G, G, GP, counts, c->ep_send_tok,
+                                                 send_meta, send_gate, tok_pairs, c->status);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) {
+    long long blocks = ((long long)T * GP + 7) / 8;  // one warp per row
+    if (blocks > 8LL * c->num_sms) blocks = 8LL * c->num_sms;
+    ep_gather_send_kernel<<<(int)blocks, 256, 0, s>>>(c->h, c->ep_send_tok, counts, G, T, g.latent,
+                                                      reinterpret_cast<__nv_bfloat16*>(send_rows), c->status);
+    e = cudaGetLastError();
+  }
+  c->last_T = T;
+  return cuda_status(e);
+}
+
+lmoe_status lmoe_ep_experts(lmoe_handle c, const void* recv_rows, int32_t R, const int32_t* recv_meta,
+                            const float* recv_gate, int32_t A, float* partial, void* stream) {
+  if (!c) return LMOE_ERR_INVALID_ARG;
+  if (c->ep_world < 2) return LMOE_ERR_UNSUPPORTED;
+  if (!c->loaded) return LMOE_ERR_NOT_LOADED;
+  const lmoe_config& g = c->cfg;
+  const int K = g.top_k, G = c->ep_world, l = g.latent, m = g.expert_ffn, NL = c->n_local;
+  const long long GP = K < G ? K : G;
+  if (R < 0 || A < 0 || (long long)R > (long long)G * g.max_tokens * GP || A > c->tk_exp) return LMOE_ERR_SHAPE;
+  if (R == 0) return LMOE_OK;
+  if (!recv_rows || !partial || !aligned16(recv_rows) || !aligned16(partial)) return LMOE_ERR_INVALID_ARG;
+  if (A > 0 && (!recv_meta || !recv_gate || !aligned16(recv_meta) || !aligned16(recv_gate)))
+    return LMOE_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (A == 0) return cuda_status(cudaMemsetAsync(partial, 0, (size_t)R * l * sizeof(float), s));
+  cudaError_t e = cudaMemsetAsync(c->work_counters, 0, lmoe_ctx::kCounters * sizeof(int), s);
+  auto chk = [&](cudaError_t r) {
+    if (e == cudaSuccess) e = r;
+    return e == cudaSuccess;
+  };
+  // the received assignments, grouped stably (arrival order) by local expert: the single-GPU
+  // dispatch kernels with the assignments as "tokens" of one slot each
+  ep_split_meta_kernel<<<(int)((A + 255) / 256 < 4 * c->num_sms ? (A + 255) / 256 : 4 * c->num_sms), 256, 0, s>>>(
+      recv_meta, A, c->ep_ids, c->ep_src);
+  if (!chk(cudaGetLastError())) return cuda_status(e);
+  int ct;
+  const int nch = n_chunks_for(A, NL, &ct);
+  ids_hist_kernel<<<nch, 256, NL * sizeof(int), s>>>(c->ep_ids, A, NL, ct, c->chunk_counts);
+  if (!chk(cudaGetLastError())) return cuda_status(e);
+  const int vg = A <= 48LL * NL ? V_SMALL : V_LARGE;
+  UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1, c->unit_u0};
+  UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2, c->unit_u0 + g.n_experts + 1};
+  scan_units_kernel<<<1, 1024, scan_smem_bytes(NL, nch), s>>>(c->chunk_counts, nch, NL, c->counts, c->offsets,
+                                                               c->chunk_base, l1, l2, c->tile0, c->status);
+  if (!chk(cudaGetLastError()) || !chk(launch_build_units(c, s, l1, l2, NL))) return cuda_status(e);
+  assign_rows_kernel<<<nch, 32 * kAssignWarps, kAssignWarps * NL * sizeof(int), s>>>(
+      c->ep_ids, recv_gate, c->chunk_base, A, NL, 1, ct, c->row_of, c->tok_of_row, c->gate_of_row, c->status);
+  if (!chk(cudaGetLastError())) return cuda_status(e);
+  {
+    long long blocks = ((long long)A + 7) / 8;  // one warp per grouped row
+    if (blocks > 8LL * c->num_sms) blocks = 8LL * c->num_sms;
+    gather_src_kernel<<<(int)blocks, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(recv_rows), R, c->ep_src,
+                                                  c->tok_of_row, A, A, l, c->h_perm, c->status);
+    if (!chk(cudaGetLastError())) return cuda_status(e);
+  }
+  // the owned experts, gate folded into the second GEMM
+  {
+    GemmLaunch gl(c, vg, 4);
+    gl.main_grouped(c->map_w1, c->map_hperm[vg], problem(l, EPI_SQRELU_BF16, c->u, m), c->units1, c->num_units, m, 0);
+    if (!chk(gl.run(s))) return cuda_status(e);
+  }
+  {
+    GemmLaunch gl(c, vg, 5);
+    GemmProblem p = problem(m, EPI_ROWSCALE_BF16, c->o, l);
+    p.row_scale = c->gate_of_row;
+    gl.main_grouped(c->map_w2, c->map_u[vg], p, c->units2, c->num_units + 1, l, 0);
+    if (!chk(gl.run(s))) return cuda_status(e);
+  }
+  // one fp32 partial latent sum per received row
+  {
+    long long blocks = ((long long)R * (l / 8) + 255) / 256;
+    if (blocks > 8LL * c->num_sms) blocks = 8LL * c->num_sms;
+    ep_pair_reduce_kernel<<<(int)blocks, 256, 0, s>>>(c->o, c->row_of, c->ep_src, A, A, R, l, partial, c->status);
+    chk(cudaGetLastError());
+  }
+  return cuda_status(e);
+}
+
+lmoe_status lmoe_ep_combine(lmoe_handle c, const void* x, int32_t T, const float* back, const int32_t* tok_pairs,
+                            void* y, void* stream) {
+  if (!c) return LMOE_ERR_INVALID_ARG;
+  if (c->ep_world < 2) return LMOE_ERR_UNSUPPORTED;
+  if (T < 0 || T > c->cfg.max_tokens) return LMOE_ERR_SHAPE;
+  if (!c->loaded) return LMOE_ERR_NOT_LOADED;
+  if (T == 0) return LMOE_OK;
+  const void* ptrs[] = {x, back, tok_pairs, y};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LMOE_ERR_INVALID_ARG;
+  DeviceGuard dg(c->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const lmoe_config& g = c->cfg;
+  const int K = g.top_k, G = c->ep_world, d = g.d, l = g.latent, ms = g.shared_ffn;
+  const int GP = K < G ? K : G;
+  const int vd = T <= 512 ? V_SMALL : V_LARGE;
+  if (!set_x_maps(c, x, T)) return LMOE_ERR_CUDA;
+  cudaError_t e = cudaMemsetAsync(c->work_counters, 0, lmoe_ctx::kCounters * sizeof(int), s);
+  if (e == cudaSuccess) {
+    // z = the token's partial sums in ascending owner order, into zu[:, :l]
+    long long blocks = ((long long)T * (l / 8) + 255) / 256;
+    if (blocks > 8LL * c->num_sms) blocks = 8LL * c->num_sms;
+    ep_combine_kernel<<<(int)blocks, 256, 0, s>>>(back, T * GP, tok_pairs, T, GP, l, c->zu, l + ms, c->status);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) {
+    // shared expert, first matrix: zu[:, l:] = sqrelu(W_s1 x)
+    GemmLaunch gl(c, vd, 3);
+    gl.main_dense(c->map_ws1, c->map_x[vd], problem(d, EPI_SQRELU_BF16, c->zu, l + ms, l), ms, T);
+    e = gl.run(s);
+  }
+  if (e == cudaSuccess) {
+    // y = [z | sqrelu(W_s1 x)] [W_up | W_s2]^T
+    GemmLaunch gl(c, vd, 6);
+    gl.main_dense(c->map_cat, c->map_zu[vd], problem(l + ms, EPI_BF16, y, d), d, T);
+    e = gl.run(s);
+  }
+  return cuda_status(e);
 }
 
 lmoe_status lmoe_export_nvfp4(lmoe_handle c, int32_t which, int32_t index, uint8_t* codes_host, uint8_t* scales_host,

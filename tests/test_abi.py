@@ -28,7 +28,7 @@ def test_header_declares_the_boundary():
                                   "lmoe_get_device_status", "lmoe_inspect", "lmoe_profile",
                                   "lmoe_profile_read", "lmoe_route_noalloc", "lmoe_export_nvfp4",
                                   "lmoe_selftest_wait_timeout", "lmoe_status_string",
-                                  "lmoe_destroy"])
+                                  "lmoe_destroy", "lmoe_ep_dispatch", "lmoe_ep_experts", "lmoe_ep_combine"])
 
 
 def test_library_exports_every_declared_symbol(libmod):
@@ -63,6 +63,18 @@ def test_create_rejects_bad_config_without_touching_a_gpu(libmod):
     bad = libmod._Config(256, -64, 16, 4, 128, 256, 64, 0, 0, 0)    # negative latent
     assert libmod.lib.lmoe_create(ctypes.byref(bad), 0, ctypes.byref(h)) == 1
     assert libmod.lib.lmoe_forward(None, None, 0, None, None, None, None) == 1
+    # expert parallelism: world above 8, rank outside the world, N not divisible, NVFP4, standard MoE
+    bad = libmod._Config(256, 64, 16, 4, 128, 256, 64, 0, 0, 0, 9, 0)
+    assert libmod.lib.lmoe_create(ctypes.byref(bad), 0, ctypes.byref(h)) == 3
+    bad = libmod._Config(256, 64, 16, 4, 128, 256, 64, 0, 0, 0, 2, 2)
+    assert libmod.lib.lmoe_create(ctypes.byref(bad), 0, ctypes.byref(h)) == 1
+    bad = libmod._Config(256, 64, 16, 4, 128, 256, 64, 0, 0, 0, 3, 0)
+    assert libmod.lib.lmoe_create(ctypes.byref(bad), 0, ctypes.byref(h)) == 3
+    bad = libmod._Config(256, 128, 16, 4, 128, 256, 64, 1, 0, 0, 2, 0)
+    assert libmod.lib.lmoe_create(ctypes.byref(bad), 0, ctypes.byref(h)) == 3
+    bad = libmod._Config(256, 0, 16, 4, 128, 256, 64, 0, 0, 0, 2, 0)
+    assert libmod.lib.lmoe_create(ctypes.byref(bad), 0, ctypes.byref(h)) == 3
+    assert libmod.lib.lmoe_ep_dispatch(None, None, 0, None, None, None, None, None, None, None, None) == 1
     del cfg
 
 
