@@ -208,14 +208,19 @@ struct lmoe_ctx {
 
 namespace {
 
+// Makes `dev` current for the call, restoring the caller's device afterwards.  cudaSetDevice runs even
+// when the device is already current: it also binds the device's primary context to the calling
+// host thread, which the driver-API tensor-map encoder needs (a thread that has made no runtime call
+// yet has no current context).
 struct DeviceGuard {
   int prev = -1;
-  explicit DeviceGuard(int dev) {
+  int dev;
+  explicit DeviceGuard(int d) : dev(d) {
     cudaGetDevice(&prev);
-    if (prev != dev) cudaSetDevice(dev);
+    cudaSetDevice(dev);
   }
   ~DeviceGuard() {
-    if (prev >= 0) cudaSetDevice(prev);
+    if (prev >= 0 && prev != dev) cudaSetDevice(prev);
   }
 };
 

@@ -21,10 +21,15 @@ Each of G ranks owns a contiguous range of N / G experts.  A forward on rank r, 
 The sum in z is the same set of K gated expert outputs as the single-GPU layer's slot-order sum,
 grouped by owner rank first; the two differ only in floating-point rounding.
 
-This module is the data movement only.  The compute steps are callables (route, experts, output), so
-the same plan runs with the library's kernels on GPUs over NCCL or, in the tests, with any reference
-implementation on CPU ranks over gloo.  Collectives are the torch.distributed ones; the exchanged
-sizes are agreed with one all-to-all of per-destination counts (its result is read on the host).
+Two drivers of the same plan:
+  ep_forward          the compute steps are callables (route, experts, output), so the plan runs with
+                      any implementation; the tests run it on CPU ranks over gloo with the oracle;
+  ep_forward_library  the compute steps are the library's lmoe_ep_dispatch / lmoe_ep_experts /
+                      lmoe_ep_combine on a layer created with ep_world = G (its plan is built on the
+                      device), and the exchanges are all-to-alls of the process group (NCCL on GPUs).
+Collectives are the torch.distributed ones.  The exchanged sizes are agreed with one all-to-all of
+per-destination counts, whose result is the only value read back on the host (the split sizes of
+the other all-to-alls).  Partial sums travel at no less than fp32.
 """
 from __future__ import annotations
 
@@ -35,7 +40,7 @@ import torch
 import torch.distributed as dist
 
 __all__ = ["ExpertPartition", "DispatchPlan", "plan_dispatch", "group_by_local_expert", "dispatch_bytes",
-           "exchange_bytes", "reduce_pairs", "ep_forward"]
+           "exchange_bytes", "reduce_pairs", "ep_forward", "ep_forward_library"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -191,8 +196,11 @@ def ep_forward(x: torch.Tensor, part: ExpertPartition,
     pair = _exclusive_cumsum(pin)[src] + meta[:, 0]
     gorder, counts = group_by_local_expert(meta[:, 1], part.first(rank), part.per_rank)
     o_grouped = experts(rows[pair[gorder]], counts, gates[gorder])
-    o_arrival = torch.empty_like(o_grouped)
-    o_arrival[gorder] = o_grouped
+    # each pair's slot-order sum, and its trip back, at no less than fp32 (a bf16 sum would add one
+    # rounding per pair to z)
+    o_arrival = torch.empty(o_grouped.shape, dtype=torch.promote_types(o_grouped.dtype, torch.float32),
+                            device=o_grouped.device)
+    o_arrival[gorder] = o_grouped.to(o_arrival.dtype)
     partial = reduce_pairs(o_arrival, pair, rows.shape[0])
 
     # the reverse exchange, then the owner-rank-ordered sum on the source side
@@ -203,3 +211,50 @@ def ep_forward(x: torch.Tensor, part: ExpertPartition,
         z[plan.pair_tok[off:off + c]] += back[off:off + c]
         off += c
     return output(z, x), idx, gate
+
+
+def ep_forward_library(layer, x: torch.Tensor, group: Optional["dist.ProcessGroup"] = None,
+                       stats: Optional[dict] = None):
+    """One expert-parallel forward of this rank's tokens x [T, d] (bf16, on this rank's GPU) with the
+    library's three steps on `layer` (a LatentMoE created with ep_world = the group's size and
+    ep_rank = this rank).  Every rank calls this at the same point (five all-to-alls).  The plan and
+    every row move on the device; the per-destination counts are the one value read on the host.
+    Returns (y [T, d] bf16, idx [T, K], gate [T, K])."""
+    world = dist.get_world_size(group)
+    if layer.ep_world != world:
+        raise ValueError("the layer's ep_world must equal the process group's size")
+    t, width = x.shape[0], layer.shape.latent
+    dev = x.device
+    if t:
+        plan = layer.ep_dispatch(x)
+        send_cnt = plan["counts"].to(torch.int64)
+    else:
+        plan = None
+        send_cnt = torch.zeros((world, 2), dtype=torch.int64, device=dev)
+    recv_cnt = torch.empty_like(send_cnt)
+    dist.all_to_all_single(recv_cnt, send_cnt, group=group)
+    cnt = torch.stack([send_cnt, recv_cnt]).cpu()          # the only host round trip
+    pairs_out, assigns_out = cnt[0, :, 0].tolist(), cnt[0, :, 1].tolist()
+    pairs_in, assigns_in = cnt[1, :, 0].tolist(), cnt[1, :, 1].tolist()
+    if stats is not None:
+        stats.update(pairs=int(sum(pairs_out)), assignments=int(sum(assigns_out)))
+    p_out, a_out = sum(pairs_out), sum(assigns_out)
+    empty = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)
+    send_rows = plan["send_rows"][:p_out] if plan is not None else empty((0, width), torch.bfloat16)
+    send_meta = plan["send_meta"][:a_out] if plan is not None else empty((0, 2), torch.int32)
+    send_gate = plan["send_gate"][:a_out] if plan is not None else empty((0,), torch.float32)
+    rows = _exchange(send_rows, pairs_out, pairs_in, group)
+    meta = _exchange(send_meta, assigns_out, assigns_in, group)
+    gates = _exchange(send_gate, assigns_out, assigns_in, group)
+    # pair indices local to each source become rows of `rows` (sources arrive in rank order)
+    row_base = _exclusive_cumsum(torch.tensor(pairs_in, dtype=torch.int64, device=dev))
+    src = torch.repeat_interleave(torch.arange(world, device=dev), torch.tensor(assigns_in, device=dev))
+    meta = torch.stack([(meta[:, 0].to(torch.int64) + row_base[src]).to(torch.int32), meta[:, 1]], 1).contiguous()
+    partial = layer.ep_experts(rows.contiguous(), meta, gates.contiguous()) if rows.shape[0] else \
+        empty((0, width), torch.float32)
+    back = _exchange(partial, pairs_in, pairs_out, group)
+    if plan is None:
+        return empty((0, layer.shape.d), torch.bfloat16), empty((0, layer.shape.top_k), torch.int32), \
+            empty((0, layer.shape.top_k), torch.float32)
+    y = layer.ep_combine(x, back.contiguous(), plan["tok_pairs"])
+    return y, plan["idx"], plan["gate"]

@@ -78,6 +78,64 @@ def _callables(W, rank, part):
     return route, experts, output
 
 
+def _bf16_callables(W, rank, part):
+    """The oracle's steps with bf16 latent rows and bf16 expert outputs, as a bf16 device layer would
+    send and produce them."""
+    route, experts, output = _callables(W, rank, part)
+
+    def route16(x):
+        idx, gate, h = route(x)
+        return idx, gate, h.to(torch.bfloat16)
+
+    def experts16(rows, counts, gates):
+        return experts(rows.to(torch.float64), counts, gates.to(torch.float64)).to(torch.bfloat16)
+
+    def output16(z, x):
+        return output(z.to(torch.float64), x)
+
+    return route16, experts16, output16
+
+
+def _worker_bf16(rank, world, init_file, q):
+    import datetime
+    dist.init_process_group("gloo", init_method="file://" + init_file, rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        W = _W(5)
+        counts = _tokens(world)
+        x_all = np.random.default_rng(6).standard_normal((sum(counts), D))
+        start = sum(counts[:rank])
+        x = torch.from_numpy(x_all[start:start + counts[rank]].copy())
+        part = ep.ExpertPartition(N, world)
+        y, idx, _ = ep.ep_forward(x, part, *_bf16_callables(W, rank, part))
+        ref = lo.forward(W, x_all, K)
+        sl = slice(start, start + counts[rank])
+        rms = float(np.sqrt(np.mean(ref["y"] ** 2)))
+        err = float(np.abs(y.numpy() - ref["y"][sl]).max()) if counts[rank] else 0.0
+        q.put((rank, err / rms, bool(np.array_equal(idx.numpy(), ref["idx"][sl]))))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ep_forward_with_bf16_rows_stays_within_the_bf16_tolerance(world, tmp_path):
+    """bf16 rows and bf16 expert outputs: the pair partial sums travel at fp32, so y stays within
+    the layer's bf16 tolerance (2e-2 x RMS) of the fp64 oracle."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    init_file = str(tmp_path / "rendezvous")
+    procs = [ctx.Process(target=_worker_bf16, args=(r, world, init_file, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, rel, same_idx in res:
+        assert same_idx
+        assert rel < 2e-2, (rank, rel)
+
+
 def _worker(rank, world, init_file, q):
     import datetime
     # rendezvous through a file in the test's own temporary directory (no port to race for)

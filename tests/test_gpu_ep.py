@@ -129,3 +129,88 @@ def test_ep_layer_rejects_the_single_gpu_forward():
         layer.forward(x)
     assert e.value.code == 6 or e.value.code == 3   # not loaded, or unsupported once loaded
     layer.close()
+
+
+class _ThreadRanks:
+    """Stand-in for the two torch.distributed calls ep_forward_library makes (get_world_size and
+    all_to_all_single), for ranks that are host threads of one process: each rank deposits its input
+    chunks, and after a barrier takes the chunks addressed to it, in source-rank order.  Only the
+    host threads meet here; no kernel waits on another rank's kernel."""
+
+    def __init__(self, world):
+        import threading
+        self.world = world
+        self.barrier = threading.Barrier(world, timeout=120)
+        self.slots = [None] * world
+        self.rank_of = {}
+
+    def get_world_size(self, group=None):
+        return self.world
+
+    def all_to_all_single(self, out, inp, output_split_sizes=None, input_split_sizes=None, group=None):
+        import threading
+        r = self.rank_of[threading.get_ident()]
+        sizes = input_split_sizes or [inp.shape[0] // self.world] * self.world
+        offs = np.concatenate([[0], np.cumsum(sizes)]).astype(int)
+        self.slots[r] = [inp[offs[g]:offs[g + 1]] for g in range(self.world)]
+        self.barrier.wait()
+        parts = [self.slots[src][r] for src in range(self.world)]
+        if out.numel():
+            out.copy_(torch.cat(parts))
+        self.barrier.wait()
+
+
+@pytest.mark.parametrize("world,tokens", [(2, [21, 30]), (4, [9, 14, 0, 25])])
+def test_ep_forward_library_over_thread_ranks(world, tokens, monkeypatch):
+    """ep.ep_forward_library end to end (plan, the five all-to-alls, the three library steps),
+    with the collectives replaced by _ThreadRanks; y of every rank matches the oracle's layer."""
+    import threading
+
+    from latentmoe_expert_layer_b200 import ep
+    wl = inp.Workload("ep", SMALL, sum(tokens), 9, 10, "bf16", "bf16")
+    w = inp.make_weights(wl)
+    x_all = inp.make_x(wl)
+    starts = np.concatenate([[0], np.cumsum(tokens)])
+    xs = [to_dev(x_all[starts[r]:starts[r + 1]], "bf16") for r in range(world)]
+    layers = _layers(SMALL, w, world, max(tokens))
+    fake = _ThreadRanks(world)
+    monkeypatch.setattr(ep, "dist", fake)
+    out, errors = [None] * world, []
+
+    def run(r):
+        try:
+            fake.rank_of[threading.get_ident()] = r
+            stats = {}
+            y, idx, gate = ep.ep_forward_library(layers[r], xs[r], stats=stats)
+            torch.cuda.synchronize()
+            out[r] = (bf16_to_np(y), idx.cpu().numpy(), gate.cpu().numpy(), stats)
+        except Exception as e:  # pragma: no cover - reported below
+            errors.append(e)
+            fake.barrier.abort()
+
+    threads = [threading.Thread(target=run, args=(r,)) for r in range(world)]
+    try:
+        for th in threads:
+            th.start()
+        for th in threads:
+            th.join(timeout=300)
+        assert not errors, errors
+        for layer in layers:
+            assert layer.device_status() == 0
+        ow = lo.OracleWeights(w)
+        x64 = lo.lift(x_all, "bf16")
+        full = oracle_routing(ow, x64, SMALL.top_k)
+        idx_all = np.concatenate([o[1] for o in out])
+        gate_all = np.concatenate([o[2] for o in out])
+        diff, _ = check_routing(idx_all, gate_all, full, SMALL.top_k)
+        ref = oracle_forward(ow, x64, SMALL.top_k)
+        yref = ref["y"].copy()
+        if diff.any():
+            yref[diff] = oracle_forward(ow, x64[diff], SMALL.top_k, idx=idx_all[diff])["y"]
+        rel = check_y(np.concatenate([o[0] for o in out]), yref)
+        for r in range(world):
+            assert out[r][3]["assignments"] == tokens[r] * SMALL.top_k
+        print(f"ep_forward_library over {world} thread ranks: max|err|/RMS {rel:.3g}")
+    finally:
+        for layer in layers:
+            layer.close()
