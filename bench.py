@@ -50,15 +50,17 @@ DEFAULT_STEPS.update({"decode_small": 400, "decode_nvfp4": 400, "prefill_nvfp4":
 # dram__bytes_write.sum from ncu section captures, summarised under profiles/): the decode NVFP4
 # capture is the full workload; the bf16 ones are smaller cases of the same regime (Super dims with
 # 128 experts: T = 64 for decode, T = 4096 for prefill), scaled to a launch by its algorithmic
-# bytes, which grow with the units processed.  Valid only while the GEMM's sources are the ones
+# bytes, which grow with the units processed.  The prefill ratios hold where the library runs the
+# same GEMM variants as the capture (expert up on one CTA: at least one full 256-token tile per
+# expert on average; expert down as CTA pairs).  Valid only while the GEMM's sources are the ones
 # captured (TRAFFIC_SOURCES_SHA256); otherwise the roofline reports no traffic.
 TRAFFIC_RATIO = {
-    ("bf16", "decode", "expert_up"): 0.999, ("bf16", "decode", "expert_down"): 1.002,
-    ("nvfp4", "decode", "expert_up"): 1.385, ("nvfp4", "decode", "expert_down"): 1.493,
-    ("bf16", "prefill", "expert_up"): 0.982, ("bf16", "prefill", "expert_down"): 0.993,
+    ("bf16", "decode", "expert_up"): 0.997, ("bf16", "decode", "expert_down"): 1.000,
+    ("nvfp4", "decode", "expert_up"): 1.383, ("nvfp4", "decode", "expert_down"): 1.495,
+    ("bf16", "prefill", "expert_up"): 0.983, ("bf16", "prefill", "expert_down"): 1.078,
 }
 TRAFFIC_SOURCES = ("gemm_tc.cuh", "ptx.cuh", "nvfp4.cuh", "lmoe.cu")
-TRAFFIC_SOURCES_SHA256 = "66bdba2299abce8c6abe29f480a83eae0daeb46152f95da3a8dac9fe660bb35a"
+TRAFFIC_SOURCES_SHA256 = "4f02f2b87ddc50eed6580fd1c8a0cad66e5e560d65211f48d36f132c82826b1f"
 
 
 def gemm_sources_sha256() -> str:
@@ -371,7 +373,9 @@ def measure(layer, w, wl, steps, warmup, world, device, with_cpu_baseline):
     roof = None
     if dom in ("expert_up", "expert_down"):
         unit_work = work[dom]
-        ratio = TRAFFIC_RATIO.get((wl.precision, "decode" if decode_like else "prefill", dom))
+        regime = "decode" if decode_like else ("prefill" if wl.tokens * wl.shape.top_k >= 256 * wl.shape.n_experts
+                                                 else "skewed")
+        ratio = TRAFFIC_RATIO.get((wl.precision, regime, dom))
         traffic = None
         if ratio is not None and gemm_sources_sha256() == TRAFFIC_SOURCES_SHA256:
             traffic = ratio * unit_work["bytes"]

@@ -115,10 +115,12 @@ constexpr int SF_ATOM_BYTES = 512;
 // RES_STAGES > 0 (FP4): room for the activation scales of one token tile over up to RES_STAGES
 // K stages, kept in TMEM across consecutive units of that tile (problems with sfb_resident): the
 // tile's first unit loads and copies them stage by stage, its later units reuse them.
-template <int BN_MAX, int STAGES, bool FP4, int ACC_SPLIT, int RES_STAGES>
+// PAIR: the CTA is one of a pair sharing cta_group::2 MMAs (M = 256); it holds half of the token
+// tile's rows per stage.
+template <int BN_MAX, int STAGES, bool FP4, int ACC_SPLIT, int RES_STAGES, bool PAIR = false>
 struct GemmSmem {
   static constexpr int NRA = (BN_MAX + 127) / 128;                    // 128-row scale atoms of B
-  static constexpr int B_STAGE_BYTES = BN_MAX * 128;
+  static constexpr int B_STAGE_BYTES = (PAIR ? BN_MAX / 2 : BN_MAX) * 128;
   static constexpr int SFA_STAGE_BYTES = FP4 ? 4 * SF_ATOM_BYTES * SF_WREP : 0;  // replicated weight atoms
   // activation scales of the variants without resident scales (prefill sizes) are stored replicated
   // like the weight scales, so one 128x256b copy moves both 128-row atoms of a K atom
@@ -158,7 +160,7 @@ struct GemmSmem {
   static_assert(ALLOC <= 232448, "shared memory per CTA");
 };
 
-template <int BN_MAX>
+template <int BN_MAX, int TILE_M>
 __device__ __forceinline__ GemmUnit dense_unit(const GemmProblem& p, int u) {
   GemmUnit r;
   // K slices outermost; token tiles of one weight tile run on adjacent CTAs, so the weight tile is
@@ -169,10 +171,10 @@ __device__ __forceinline__ GemmUnit dense_unit(const GemmProblem& p, int u) {
   r.kslice = ks;
   const int tt = u % p.dense_ttiles;
   const int ft = u / p.dense_ttiles;
-  r.a_row = ft * BLOCK_M;
+  r.a_row = ft * TILE_M;
   r.f0 = r.a_row;
   r.b_row = tt * BN_MAX;
-  const int mv = min(BLOCK_M, p.dense_feat - r.f0);
+  const int mv = min(TILE_M, p.dense_feat - r.f0);
   const int nv = min(BN_MAX, p.dense_tokens - r.b_row);
   r.nm = nv | (mv << 16);
   r.tile = tt;
@@ -193,16 +195,27 @@ __device__ __forceinline__ void unit_k_range(const GemmProblem& p, const GemmUni
 
 // Global unit u of the launch: which problem it belongs to, and its tile.  The pre problem's units
 // come first (measured: spreading them through the expert units was slower at decode sizes).
-template <int BN_MAX>
-__device__ __forceinline__ GemmUnit unit_at(const GemmArgs& a, int u, int& pid) {
+// In a CTA pair a unit covers 256 weight rows; each CTA of the pair sees its own 128 (unit_at
+// returns the CTA's half: rows and first feature shifted by 128 * rank, valid features clamped).
+template <int BN_MAX, int TILE_M>
+__device__ __forceinline__ GemmUnit unit_at(const GemmArgs& a, int u, int& pid, uint32_t pair_rank = 0) {
+  GemmUnit r;
   if (u < a.n_pre_units) {
     pid = 1;
-    return dense_unit<BN_MAX>(a.prob[1], u);
+    r = dense_unit<BN_MAX, TILE_M>(a.prob[1], u);
+  } else {
+    pid = 0;
+    u -= a.n_pre_units;
+    r = (a.units != nullptr) ? a.units[u] : dense_unit<BN_MAX, TILE_M>(a.prob[0], u);
   }
-  pid = 0;
-  u -= a.n_pre_units;
-  if (a.units != nullptr) return a.units[u];
-  return dense_unit<BN_MAX>(a.prob[0], u);
+  if (TILE_M > BLOCK_M) {
+    const int sh = BLOCK_M * (int)pair_rank;
+    r.a_row += sh;
+    r.f0 += sh;
+    const int mv = max(0, min(BLOCK_M, (r.nm >> 16) - sh));
+    r.nm = (r.nm & 0xFFFF) | (mv << 16);
+  }
+  return r;
 }
 
 __device__ __forceinline__ uint16_t f32_to_bf16_rn(float v) {
@@ -213,14 +226,25 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rn(float v) {
 // ACC_SPLIT > 1: consecutive MMAs of a tile rotate over ACC_SPLIT independent partial accumulators,
 // summed by the epilogue.  With few tokens (N = 16..64) one MMA is far shorter than the tensor pipe's
 // latency, and MMAs chained on one accumulator would each wait for the previous one.
-template <int BN_MAX, int STAGES, int BOXN, bool FP4, int ACC_SPLIT, int RES_STAGES>
+//
+// PAIR (bf16 only): the grid is made of clusters of two CTAs that share cta_group::2 MMAs of
+// M = 256 weight rows.  Each CTA loads its own 128 weight rows and half of the token tile (the even
+// CTA tokens 0..N/2-1, the odd one N/2..N-1) into its shared memory; the even CTA's producer expects
+// both halves' bytes on its stage barrier, its MMA issuer runs the pair's MMAs and commits them to
+// both CTAs' barriers, and each CTA's epilogue drains its own half of the accumulator from its own
+// TMEM.  Per stage an SM then reads 32 KB for 128 x 256 x 64 MACs instead of 48 KB.  Both CTAs
+// walk the same unit sequence: static claims by pair, or dynamic claims taken by the even CTA and
+// passed to the odd one through a mailbox in its shared memory.
+template <int BN_MAX, int STAGES, int BOXN, bool FP4, int ACC_SPLIT, int RES_STAGES, bool PAIR>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_w0, const __grid_constant__ CUtensorMap map_act0,
                    const __grid_constant__ CUtensorMap map_w1, const __grid_constant__ CUtensorMap map_act1,
                    const GemmArgs args) {
-  using S = GemmSmem<BN_MAX, STAGES, FP4, ACC_SPLIT, RES_STAGES>;
+  using S = GemmSmem<BN_MAX, STAGES, FP4, ACC_SPLIT, RES_STAGES, PAIR>;
+  constexpr int TILE_M = PAIR ? 2 * BLOCK_M : BLOCK_M;
   static_assert(BN_MAX % BOXN == 0 && BOXN % 8 == 0, "token box must tile the token block");
   static_assert(BN_MAX % 16 == 0 && BN_MAX <= 256, "MMA N limit");
+  static_assert(!PAIR || (!FP4 && ACC_SPLIT == 1 && BOXN == BN_MAX / 2), "pair variant: bf16, one box per half");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
@@ -230,12 +254,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint64_t* drain = tempty + 2;
   uint64_t* ufull = drain + 1;              // unit ring: producer -> MMA issuer and epilogue warps
   uint64_t* uempty = ufull + UNIT_RING;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(uempty + UNIT_RING);
+  uint64_t* mfull = uempty + UNIT_RING;     // claim mailbox (pair, dynamic): even -> odd CTA
+  uint64_t* mempty = mfull + UNIT_RING;     //   odd -> even CTA (the slot may be rewritten)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mempty + UNIT_RING);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* unit_ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  volatile int* mailbox = reinterpret_cast<volatile int*>(tmem_slot + 2 + UNIT_RING);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t prank = PAIR ? cluster_ctarank() : 0u;  // rank in the pair; 0 issues the MMAs
+  const bool issuer = prank == 0;
   // the next launch may begin (its CTAs take SMs as this grid's CTAs exit)
   griddep_launch_dependents();
 
@@ -246,12 +275,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], PAIR ? 8 : 4);  // a pair's issuer waits for both CTAs' epilogue warps
     }
     mbar_init(drain, 1);
     for (int i = 0; i < UNIT_RING; ++i) {
       mbar_init(&ufull[i], 1);
       mbar_init(&uempty[i], 5);  // the MMA issuer and the four epilogue warps
+      mbar_init(&mfull[i], 1);
+      mbar_init(&mempty[i], 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -264,9 +295,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       tma_prefetch_desc(&map_act1);
     }
   }
-  if (warp == 1) tmem_alloc(tmem_slot, S::TMEM_COLS);
+  if (warp == 1) {
+    if constexpr (PAIR) tmem_alloc_pair(tmem_slot, S::TMEM_COLS);
+    else tmem_alloc(tmem_slot, S::TMEM_COLS);
+  }
   tc_fence_before();
   __syncthreads();
+  // a pair's barriers and TMEM are set up on both sides before either CTA signals the other
+  if constexpr (PAIR) cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // everything above is this CTA's own set-up; from here on the kernel reads what earlier launches
@@ -297,7 +333,40 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int n_pre = args.n_pre_units;
       const int chunk = args.chunk > 0 ? args.chunk : 1;
       const int n_claims = n_pre + (num_units - n_pre + chunk - 1) / chunk;
-      int claim = args.dynamic ? atomicAdd(args.work_counter, 1) : (int)blockIdx.x;
+      // a pair is one worker: claims by pair index, or the even CTA's dynamic claims forwarded
+      const int worker = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+      const int n_workers = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+      int mslot = 0;
+      uint32_t mphase = 0;
+      auto take_claim = [&]() -> int {
+        if constexpr (PAIR) {
+          int cl = n_claims;
+          if (issuer) {
+            if (!mbar_wait_bounded_cluster(&mempty[mslot], mphase ^ 1u, abort_flag, tmo)) {
+              ok = false;
+              return n_claims;
+            }
+            cl = atomicAdd(args.work_counter, 1);
+            st_cluster_u32(cluster_addr((const void*)&mailbox[mslot], 1), (uint32_t)cl);
+            mbar_arrive_cluster(cluster_addr(&mfull[mslot], 1));
+          } else {
+            if (!mbar_wait_bounded_cluster(&mfull[mslot], mphase, abort_flag, tmo)) {
+              ok = false;
+              return n_claims;
+            }
+            cl = mailbox[mslot];
+            mbar_arrive_cluster(cluster_addr(&mempty[mslot], 0));
+          }
+          if (++mslot == UNIT_RING) {
+            mslot = 0;
+            mphase ^= 1u;
+          }
+          return cl;
+        } else {
+          return atomicAdd(args.work_counter, 1);
+        }
+      };
+      int claim = args.dynamic ? take_claim() : worker;
       int u_next = num_units, u_end = num_units;
       auto open_claim = [&]() {
         if (claim < n_claims) {
@@ -324,11 +393,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         if (u < 0) break;
         if (++u_next >= u_end) {
-          claim = args.dynamic ? atomicAdd(args.work_counter, 1) : claim + (int)gridDim.x;
+          claim = args.dynamic ? take_claim() : claim + n_workers;
           open_claim();
         }
         int pid;
-        const GemmUnit un = unit_at<BN_MAX>(args, u, pid);
+        const GemmUnit un = unit_at<BN_MAX, TILE_M>(args, u, pid, prank);
         const GemmProblem& pr = args.prob[pid];
         const CUtensorMap* mw = pid ? &map_w1 : &map_w0;
         const CUtensorMap* ma = pid ? &map_act1 : &map_act0;
@@ -344,7 +413,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           fill = !res || key != res_key;
           res_key = res ? key : -1;
         }
-        const uint32_t bytes = A_STAGE_BYTES + nbox * BOXN * 128 + S::SFA_STAGE_BYTES + (fill ? S::SFB_STAGE_BYTES : 0);
+        uint32_t bytes = A_STAGE_BYTES + nbox * BOXN * 128 + S::SFA_STAGE_BYTES + (fill ? S::SFB_STAGE_BYTES : 0);
+        // pair: one box per CTA, the odd CTA's tokens start half the MMA's N further; the even CTA's
+        // stage barrier expects both CTAs' bytes
+        int b_row = un.b_row;
+        if constexpr (PAIR) {
+          b_row += (int)prank * (((nv + 15) & ~15) >> 1);
+          bytes = 2u * (A_STAGE_BYTES + BOXN * 128);
+        }
         // x coordinate of a stage in the tensor maps: 128 bytes = 64 bf16 elements or 128 FP4 bytes
         const int kx = FP4 ? 128 : BLOCK_K;
         int kb0, kb1;
@@ -356,10 +432,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
           uint8_t* sa = smem + stage * S::STAGE_BYTES;
           uint8_t* sb = sa + A_STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d(sa, mw, &full[stage], kb * kx, un.a_row, pol_w);
-          for (int i = 0; i < nbox; ++i)
-            tma_load_2d(sb + i * BOXN * 128, ma, &full[stage], kb * kx, un.b_row + i * BOXN, pol_a);
+          if constexpr (PAIR) {
+            if (issuer) mbar_arrive_expect_tx(&full[stage], bytes);
+            const uint32_t bar = cluster_addr(&full[stage], 0);
+            tma_load_2d_pair(sa, mw, bar, kb * kx, un.a_row, pol_w);
+            tma_load_2d_pair(sb, ma, bar, kb * kx, b_row, pol_a);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            tma_load_2d(sa, mw, &full[stage], kb * kx, un.a_row, pol_w);
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d(sb + i * BOXN * 128, ma, &full[stage], kb * kx, b_row + i * BOXN, pol_a);
+          }
           if constexpr (FP4) {
             uint8_t* ssfa = sb + S::B_STAGE_BYTES;
             uint8_t* ssfb = ssfa + S::SFA_STAGE_BYTES;
@@ -376,9 +459,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
         }
       }
-      if (!ok) {
-        // Give every load still in flight a bounded chance to land before the CTA exits.
-        atomicOr(args.status, DEV_STATUS_TIMEOUT);
+      if (!ok) atomicOr(args.status, DEV_STATUS_TIMEOUT);
+      if (!ok && issuer) {
+        // Give every load still in flight a bounded chance to land before the CTA exits (a pair's
+        // loads all complete on the even CTA's barriers).
         volatile int never = 0;
         int s = stage, p = phase;
         for (int i = 0; i < STAGES && i < issued; ++i) {
@@ -393,7 +477,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (PAIR && !issuer && lane == 0) {
+      // the odd CTA of a pair issues nothing; it only keeps its unit ring moving
+      int uslot = 0;
+      uint32_t uphase = 0;
+      while (true) {
+        if (!mbar_wait_bounded(&ufull[uslot], uphase, abort_flag, tmo)) {
+          atomicOr(args.status, DEV_STATUS_TIMEOUT);
+          break;
+        }
+        const int u = unit_ring[uslot];
+        mbar_arrive(&uempty[uslot]);
+        if (++uslot == UNIT_RING) {
+          uslot = 0;
+          uphase ^= 1u;
+        }
+        if (u < 0) break;
+      }
+    } else if (lane == 0) {
       int sf_slot = 0;
       int stage = 0;
       uint32_t phase = 0;
@@ -416,11 +517,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         if (u < 0) break;
         int pid;
-        const GemmUnit un = unit_at<BN_MAX>(args, u, pid);
+        const GemmUnit un = unit_at<BN_MAX, TILE_M>(args, u, pid, prank);
         const int nkb = args.prob[pid].num_k_blocks;
         const int nv = un.nm & 0xFFFF;
         const uint32_t n_mma = (uint32_t)((nv + 15) & ~15);
-        const uint32_t idesc = FP4 ? idesc_nvf4(BLOCK_M, n_mma) : idesc_bf16_f32(BLOCK_M, n_mma);
+        const uint32_t idesc = FP4 ? idesc_nvf4(BLOCK_M, n_mma) : idesc_bf16_f32(TILE_M, n_mma);
         const int nra = (int)((n_mma + 127) >> 7);
         // res: this unit's activation scales live in the resident columns (filled by the tile's first
         // unit, whose copies the tensor pipe runs after the previous tile's MMAs)
@@ -485,26 +586,34 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int k = 0; k < 4; ++k, ++mma_i)  // K = 64 E2M1 per MMA: +32 bytes = +2 in the address field
               umma_nvf4(d_tmem + (uint32_t)((mma_i % ACC_SPLIT) * BN_MAX), da + 2 * k, db + 2 * k, idesc, t_sfa + 4 * k,
                         t_sfb + 4 * k * sfb_pitch, mma_i >= ACC_SPLIT);
+          } else if constexpr (PAIR) {
+#pragma unroll
+            for (int k = 0; k < BLOCK_K / 16; ++k, ++mma_i)
+              umma_bf16_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, mma_i >= 1);
           } else {
 #pragma unroll
             for (int k = 0; k < BLOCK_K / 16; ++k, ++mma_i)  // K = 16 bf16 per MMA: +32 bytes = +2 in the address field
               umma_bf16(d_tmem + (uint32_t)((mma_i % ACC_SPLIT) * BN_MAX), da + 2 * k, db + 2 * k, idesc,
                         mma_i >= ACC_SPLIT);
           }
-          umma_commit(&empty[stage]);
+          // the stage is free again in both CTAs of a pair once these MMAs have read it
+          if constexpr (PAIR) umma_commit_pair(&empty[stage], 3);
+          else umma_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        if constexpr (PAIR) umma_commit_pair(&tfull[acc], 3);
+        else umma_commit(&tfull[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       if (!ok) atomicOr(args.status, DEV_STATUS_TIMEOUT);
       // every MMA this thread issued completes before TMEM is released
-      umma_commit(drain);
+      if constexpr (PAIR) umma_commit_pair(drain, 1);
+      else umma_commit(drain);
       volatile int never = 0;
       mbar_wait_bounded(drain, 0, &never, 100000000ull);
     }
@@ -532,7 +641,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
       if (u < 0) break;
       int pid;
-      const GemmUnit un = unit_at<BN_MAX>(args, u, pid);
+      const GemmUnit un = unit_at<BN_MAX, TILE_M>(args, u, pid, prank);
       const GemmProblem& pr = args.prob[pid];
       const int nv = un.nm & 0xFFFF;
       const int mv = un.nm >> 16;
@@ -566,7 +675,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           // accumulator fully read by this warp: hand it back to the MMA issuer
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[acc]);
+          if (lane == 0) {
+            if constexpr (PAIR) mbar_arrive_remote(cluster_addr(&tempty[acc], 0));
+            else mbar_arrive(&tempty[acc]);
+          }
         }
         if constexpr (FP4) {
 #pragma unroll
@@ -671,9 +783,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  // a pair's MMAs read both CTAs' shared memory and write both CTAs' TMEM: neither CTA releases
+  // either before the even CTA's MMAs have drained
+  if constexpr (PAIR) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, S::TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
+    else tmem_dealloc(tmem_base, S::TMEM_COLS);
   }
 }
 

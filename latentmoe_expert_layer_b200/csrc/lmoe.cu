@@ -50,22 +50,29 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 }
 
 // GEMM shapes: small token tiles with a deep ring (weight streaming at decode sizes) and large token
-// tiles (tensor-core bound at prefill sizes), each in bf16 and in NVFP4.
-enum Variant { V_SMALL = 0, V_LARGE = 1, V_SMALL4 = 2, V_LARGE4 = 3 };
-constexpr int V_BN[4] = {64, 256, 64, 192};
-constexpr int V_STAGES[4] = {8, 4, 6, 3};
-constexpr int V_BOXN[4] = {16, 256, 16, 192};  // one token box per stage at prefill sizes
-constexpr bool V_FP4[4] = {false, false, true, true};
-constexpr int V_ACC_SPLIT[4] = {4, 1, 2, 1};  // decode-sized tiles rotate over independent accumulators
+// tiles (tensor-core bound at prefill sizes), each in bf16 and in NVFP4.  The bf16 large-tile variant
+// runs as CTA pairs (cta_group::2 MMAs over 256 weight rows x 256 tokens; each CTA loads 128 weight
+// rows and 128 tokens per stage).  V_LARGE1 is the same token tile on one CTA with 128 weight rows:
+// the prefill expert-up GEMM uses it, because its 2688 features would leave half of every 11th pair
+// tile empty (measured: the pair variant was 7 % slower there, the down GEMM and the dense GEMMs
+// faster).
+enum Variant { V_SMALL = 0, V_LARGE = 1, V_SMALL4 = 2, V_LARGE4 = 3, V_LARGE1 = 4 };
+constexpr int V_BN[5] = {64, 256, 64, 192, 256};
+constexpr int V_STAGES[5] = {8, 6, 6, 3, 4};
+constexpr int V_BOXN[5] = {16, 128, 16, 192, 256};  // one token box per stage (per CTA) at prefill sizes
+constexpr bool V_FP4[5] = {false, false, true, true, false};
+constexpr int V_ACC_SPLIT[5] = {4, 1, 2, 1, 1};  // decode-sized tiles rotate over independent accumulators
 // K stages of one token tile's activation scales that fit resident in TMEM (0: per-stage copies)
-constexpr int V_RES[4] = {0, 0, 12, 0};
+constexpr int V_RES[5] = {0, 0, 12, 0, 0};
+constexpr bool V_PAIR[5] = {false, true, false, false, false};
+constexpr int V_TILE_M[5] = {128, 256, 128, 128, 128};  // weight rows per unit
 
 template <int V>
 struct VT {
   static constexpr int BN = V_BN[V], ST = V_STAGES[V], BOX = V_BOXN[V], AS = V_ACC_SPLIT[V], RS = V_RES[V];
-  static constexpr bool F4 = V_FP4[V];
-  static void* fn() { return reinterpret_cast<void*>(gemm_tc_kernel<BN, ST, BOX, F4, AS, RS>); }
-  static int smem() { return GemmSmem<BN, ST, F4, AS, RS>::ALLOC; }
+  static constexpr bool F4 = V_FP4[V], PR = V_PAIR[V];
+  static void* fn() { return reinterpret_cast<void*>(gemm_tc_kernel<BN, ST, BOX, F4, AS, RS, PR>); }
+  static int smem() { return GemmSmem<BN, ST, F4, AS, RS, PR>::ALLOC; }
 };
 
 // 2-D byte tensor map (packed NVFP4 codes): rows x cols_bytes, 128-byte x box_rows tiles, 128-byte swizzle.
@@ -91,6 +98,7 @@ struct lmoe_ctx {
   lmoe_config cfg{};
   int device = 0;
   int num_sms = 148;
+  int pair_workers = 74;  // CTA pairs of the pair variant that can be resident at once
   bool loaded = false;
   bool router_f32 = false;
   bool fused_router = false;
@@ -144,6 +152,7 @@ struct lmoe_ctx {
   static constexpr int kAmaxX = 8, kAmaxH = 9;
   int max_units1 = 0, max_units2 = 0;
   CUtensorMap map_hperm[2]{}, map_u[2]{}, map_zu[2]{};
+  CUtensorMap map_hperm1{};  // h_perm with the single-CTA large token tile (expert up, V_LARGE1)
   CUtensorMap map_z[2]{}, map_us[2]{};  // the z and u_s column blocks of zu
   float* y_s = nullptr;                 // [min(T_max, 512), d] fp32: W_s2 u_s at decode sizes
 
@@ -274,8 +283,8 @@ lmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LMOE_OK : LMO
 template <int V>
 cudaError_t launch_gemm_v(const CUtensorMap& w0, const CUtensorMap& a0, const CUtensorMap& w1, const CUtensorMap& a1,
                           const GemmArgs& a, int grid, cudaStream_t s) {
-  return launch_pdl(gemm_tc_kernel<VT<V>::BN, VT<V>::ST, VT<V>::BOX, VT<V>::F4, VT<V>::AS, VT<V>::RS>, grid,
-                    GEMM_THREADS, VT<V>::smem(), s, w0, a0, w1, a1, a);
+  return launch_pdl(gemm_tc_kernel<VT<V>::BN, VT<V>::ST, VT<V>::BOX, VT<V>::F4, VT<V>::AS, VT<V>::RS, VT<V>::PR>,
+                    grid, GEMM_THREADS, VT<V>::smem(), s, VT<V>::PR ? 2 : 1, w0, a0, w1, a1, a);
 }
 
 // A bf16 problem with its epilogue; K in elements (multiple of 64).
@@ -311,7 +320,7 @@ GemmProblem problem4(int K, int epi, void* out, long long ldo, const uint8_t* w_
 
 // Make `p` a dense problem over feat x tokens with the token tile of variant v.
 int set_dense(GemmProblem& p, int v, int feat, int tokens) {
-  p.dense_ftiles = (feat + BLOCK_M - 1) / BLOCK_M;
+  p.dense_ftiles = (feat + V_TILE_M[v] - 1) / V_TILE_M[v];
   p.dense_ttiles = (tokens + V_BN[v] - 1) / V_BN[v];
   p.dense_feat = feat;
   p.dense_tokens = tokens;
@@ -380,16 +389,20 @@ struct GemmLaunch {
       w1 = w0;
       a1 = a0;
     }
-    int grid = c->num_sms;
+    // one worker per SM, or per pair of SMs for the pair variant (grid = 2 x workers)
+    const int per = V_PAIR[v] ? 2 : 1;
+    int grid = V_PAIR[v] ? c->pair_workers : c->num_sms;
     if (a.units == nullptr) {
       const int total = a.n_pre_units + a.main_dense_units;
       if (total < grid) grid = total;
     }
     if (grid < 1) grid = 1;
+    grid *= per;
     switch (v) {
       case V_SMALL: return launch_gemm_v<V_SMALL>(*w0, *a0, *w1, *a1, a, grid, s);
       case V_LARGE: return launch_gemm_v<V_LARGE>(*w0, *a0, *w1, *a1, a, grid, s);
       case V_SMALL4: return launch_gemm_v<V_SMALL4>(*w0, *a0, *w1, *a1, a, grid, s);
+      case V_LARGE1: return launch_gemm_v<V_LARGE1>(*w0, *a0, *w1, *a1, a, grid, s);
       default: return launch_gemm_v<V_LARGE4>(*w0, *a0, *w1, *a1, a, grid, s);
     }
   }
@@ -527,8 +540,13 @@ cudaError_t launch_route_fused_p(const RouteFusedArgs& a, int grid, cudaStream_t
   return cudaLaunchKernelEx(&cfg, route_fused_kernel<P>, a);
 }
 
+// Experts whose first matrix the fused routing kernel prefetches into L2 for the expert-up launch.
+constexpr int kPrefetchExperts = 6;
+
+// fp4_x: NVFP4 experts (the layer input x, quantised here with h); nullptr for bf16 experts.
 cudaError_t launch_route_fused(lmoe_ctx* c, int T, int ks, int nch, int ct, int* idx, float* gate,
-                               const UnitListSpec& l1, const UnitListSpec& l2, cudaStream_t s) {
+                               const UnitListSpec& l1, const UnitListSpec& l2, cudaStream_t s,
+                               const void* fp4_x = nullptr) {
   const lmoe_config& g = c->cfg;
   RouteFusedArgs a;
   memset(&a, 0, sizeof(a));
@@ -557,7 +575,30 @@ cudaError_t launch_route_fused(lmoe_ctx* c, int T, int ks, int nch, int ct, int*
   a.gate_of_row = c->gate_of_row;
   a.h_perm = c->h_perm;
   a.zero_words = c->work_counters;
-  a.n_zero = lmoe_ctx::kCounters;
+  a.n_zero = lmoe_ctx::kAmaxX;  // the unit counters (the activation maxima are zeroed before the launch)
+  if (!fp4_x && c->ws1 && c->w1) {
+    // bf16 experts: the expert-up launch reads W_s1 first (its dense pre problem), then the experts
+    // in index order; about 80 MB of it goes to L2 while this kernel runs
+    a.pf_ptr[0] = reinterpret_cast<const uint8_t*>(c->ws1);
+    a.pf_bytes[0] = (long long)g.shared_ffn * g.d * 2;
+    a.pf_ptr[1] = reinterpret_cast<const uint8_t*>(c->w1);
+    a.pf_bytes[1] = (long long)(c->n_local < kPrefetchExperts ? c->n_local : kPrefetchExperts) * g.expert_ffn * c->le * 2;
+  }
+  if (fp4_x) {
+    a.fp4 = 1;
+    a.x = reinterpret_cast<const __nv_bfloat16*>(fp4_x);
+    a.d = g.d;
+    a.amax = reinterpret_cast<unsigned*>(c->work_counters + lmoe_ctx::kAmaxX);
+    a.act_g = c->act_g;
+    a.xq = c->xq;
+    a.x_sf = c->x_sf;
+    a.hq_tok = c->hq_tok;
+    a.h_sf_tok = c->h_sf_tok;
+    a.hq = c->hq;
+    a.h_sf = c->h_sf;
+    a.tile_tokens4 = l1.tile_tokens;
+    a.nra4 = (l1.tile_tokens + 127) / 128;
+  }
   a.bar = c->route_bar;
   a.status = c->status;
   a.timeout_ns = c->timeout_ns;
@@ -599,52 +640,66 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
     return (int)(b < 1 ? 1 : b);
   };
 
-  // 1. router logits and h = W_down x (bf16)
-  chk(router_stage(c, x, T, s, launches));
-  if (!mark(1)) return e;
-  // 2. quantise x (dynamic tensor scale); amax of h
-  amax_act_kernel<<<grid_for((long long)T * d / 8, 256), 256, 0, s>>>(
-      reinterpret_cast<const __nv_bfloat16*>(x), (long long)T * d / 8, amax_x);
+  // Decode sizes with the stacked router rows: the routing chain, the activation maxima, the x and h
+  // quantisers and the grouped copy of h are one cooperative kernel
+  const bool fused = vd == V_SMALL && vg == V_SMALL4 && c->fused_router && c->route_bar;
   const int nra = (V_BN[vg] + 127) / 128;  // scale row atoms per token tile of the FP4 variant
   const int sf_reps = vg == V_LARGE4 ? SF_WREP : 1;  // the prefill variant reads replicated scale atoms
-  quant_act_kernel<<<grid_for((long long)T * d / 16, 256), 256, 0, s>>>(
-      reinterpret_cast<const __nv_bfloat16*>(x), d, nullptr, T, T, nullptr, nullptr, N, V_BN[vg], nra, amax_x, c->xq,
-      c->x_sf, g_x, c->status, sf_reps);
-  amax_act_kernel<<<grid_for((long long)T * l / 8, 256), 256, 0, s>>>(c->h, (long long)T * l / 8, amax_h);
-  chk(cudaGetLastError());
-  if (!mark(2)) return e;
-  // 3. top-K + softmax + per-chunk histogram
-  int ct;
-  const int nch = n_chunks_for(T, N, &ct);
-  {
-    const int parts = topk_parts(ct);
-    if (parts > 1) chk(cudaMemsetAsync(c->chunk_counts, 0, (size_t)N * nch * sizeof(int), s));
-    chk(launch_topk_hist(nch, parts, s, c->logits, c->b_router, T, N, K, ct, idx, gate, c->chunk_counts));
+  // 1. router logits and h = W_down x (bf16)
+  int rks = 1;
+  chk(router_stage(c, x, T, s, launches, fused, &rks));
+  if (!mark(1)) return e;
+  if (fused) {
+    int ct;
+    const int nch = n_chunks_for(T, N, &ct);
+    UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1, c->unit_u0, V_TILE_M[vg]};
+    UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2, c->unit_u0 + N + 1, V_TILE_M[vg]};
+    chk(launch_route_fused(c, T, rks, nch, ct, idx, gate, l1, l2, s, x));
+    for (int i = 2; i <= 5; ++i)
+      if (!mark(i)) return e;
+  } else {
+    // 2. quantise x (dynamic tensor scale); amax of h
+    amax_act_kernel<<<grid_for((long long)T * d / 8, 256), 256, 0, s>>>(
+        reinterpret_cast<const __nv_bfloat16*>(x), (long long)T * d / 8, amax_x);
+    quant_act_kernel<<<grid_for((long long)T * d / 16, 256), 256, 0, s>>>(
+        reinterpret_cast<const __nv_bfloat16*>(x), d, nullptr, T, T, nullptr, nullptr, N, V_BN[vg], nra, amax_x, c->xq,
+        c->x_sf, g_x, c->status, sf_reps);
+    amax_act_kernel<<<grid_for((long long)T * l / 8, 256), 256, 0, s>>>(c->h, (long long)T * l / 8, amax_h);
+    chk(cudaGetLastError());
+    if (!mark(2)) return e;
+    // 3. top-K + softmax + per-chunk histogram
+    int ct;
+    const int nch = n_chunks_for(T, N, &ct);
+    {
+      const int parts = topk_parts(ct);
+      if (parts > 1) chk(cudaMemsetAsync(c->chunk_counts, 0, (size_t)N * nch * sizeof(int), s));
+      chk(launch_topk_hist(nch, parts, s, c->logits, c->b_router, T, N, K, ct, idx, gate, c->chunk_counts));
+    }
+    if (!mark(3)) return e;
+    // 4. expert offsets and grouped-GEMM unit lists
+    UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1, c->unit_u0, V_TILE_M[vg]};
+    UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2, c->unit_u0 + N + 1, V_TILE_M[vg]};
+    scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(c->chunk_counts, nch, N, c->counts, c->offsets,
+                                                                c->chunk_base, l1, l2, c->tile0, c->status);
+    chk(cudaGetLastError());
+    chk(launch_build_units(c, s, l1, l2, N));
+    if (!mark(4)) return e;
+    // 5. stable grouping; h quantised once per token, then its rows copied into grouped order with
+    //    their scales in the expert GEMM's tile-local atoms
+    assign_rows_kernel<<<nch, 32 * kAssignWarps, kAssignWarps * N * sizeof(int), s>>>(
+        idx, gate, c->chunk_base, T, N, K, ct, c->row_of, c->tok_of_row, c->gate_of_row, c->status);
+    quant_act_kernel<<<grid_for((long long)T * l / 16, 256), 256, 0, s>>>(c->h, l, nullptr, T, T, nullptr, nullptr, N,
+                                                                           V_BN[vg], 0, amax_h, c->hq_tok, c->h_sf_tok,
+                                                                           g_h, c->status, 1);
+    {
+      long long blocks = (TK + 7) / 8;  // one warp per row
+      if (blocks > 16LL * c->num_sms) blocks = 16LL * c->num_sms;
+      gather_act_q_kernel<<<(int)blocks, 256, 0, s>>>(c->hq_tok, c->h_sf_tok, l, c->tok_of_row, TK, T, c->offsets,
+                                                       c->tile0, N, V_BN[vg], nra, c->hq, c->h_sf, c->status, sf_reps);
+    }
+    chk(cudaGetLastError());
+    if (!mark(5)) return e;
   }
-  if (!mark(3)) return e;
-  // 4. expert offsets and grouped-GEMM unit lists
-  UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1, c->unit_u0};
-  UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2, c->unit_u0 + N + 1};
-  scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(c->chunk_counts, nch, N, c->counts, c->offsets,
-                                                              c->chunk_base, l1, l2, c->tile0, c->status);
-  chk(cudaGetLastError());
-  chk(launch_build_units(c, s, l1, l2, N));
-  if (!mark(4)) return e;
-  // 5. stable grouping; h quantised once per token, then its rows copied into grouped order with
-  //    their scales in the expert GEMM's tile-local atoms
-  assign_rows_kernel<<<nch, 32 * kAssignWarps, kAssignWarps * N * sizeof(int), s>>>(
-      idx, gate, c->chunk_base, T, N, K, ct, c->row_of, c->tok_of_row, c->gate_of_row, c->status);
-  quant_act_kernel<<<grid_for((long long)T * l / 16, 256), 256, 0, s>>>(c->h, l, nullptr, T, T, nullptr, nullptr, N,
-                                                                         V_BN[vg], 0, amax_h, c->hq_tok, c->h_sf_tok,
-                                                                         g_h, c->status, 1);
-  {
-    long long blocks = (TK + 7) / 8;  // one warp per row
-    if (blocks > 16LL * c->num_sms) blocks = 16LL * c->num_sms;
-    gather_act_q_kernel<<<(int)blocks, 256, 0, s>>>(c->hq_tok, c->h_sf_tok, l, c->tok_of_row, TK, T, c->offsets,
-                                                     c->tile0, N, V_BN[vg], nra, c->hq, c->h_sf, c->status, sf_reps);
-  }
-  chk(cudaGetLastError());
-  if (!mark(5)) return e;
   // 6. expert up (FP4): u = NVFP4(sqrelu(W1_e h)); shared up u_s = NVFP4(sqrelu(W_s1 x))
   GemmProblem shared_up = problem4(d, EPI_SQRELU_NVFP4, c->usq, ms / 2, c->ws1_sf, c->wg + 2 * N, ms, c->x_sf, g_x);
   shared_up.out_sf = c->us_sf;
@@ -693,7 +748,7 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
     chk(gl.run(s));
   }
   if (!mark(9)) return e;
-  launches += 13 + (split ? 0 : 2);
+  launches += fused ? 5 : 13 + (split ? 0 : 2);
   return e;
 }
 
@@ -810,6 +865,7 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
   cudaMemset(c->zu, 0, T * (l + ms) * 2);
   for (int v = 0; v < 2; ++v) {
     ok = ok && make_map(&c->map_hperm[v], c->h_perm, tk_exp, le, le, V_BOXN[v]);
+    if (v == V_LARGE) ok = ok && make_map(&c->map_hperm1, c->h_perm, tk_exp, le, le, V_BOXN[V_LARGE1]);
     ok = ok && make_map(&c->map_u[v], c->u, tk_exp, m, m, V_BOXN[v]);
     ok = ok && make_map(&c->map_zu[v], c->zu, T, l + ms, l + ms, V_BOXN[v]);
     if (!c->standard) ok = ok && make_map(&c->map_z[v], c->zu, T, l, l + ms, V_BOXN[v]);
@@ -823,6 +879,28 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
                                   VT<V_SMALL4>::smem()) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(VT<V_LARGE4>::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   VT<V_LARGE4>::smem()) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(VT<V_LARGE1>::fn(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  VT<V_LARGE1>::smem()) == cudaSuccess;
+  if (ok) {
+    // a pair's two CTAs sit in one GPC: size the pair variant's grid to the pairs that fit at once
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(c->num_sms);
+    cfg.blockDim = dim3(GEMM_THREADS);
+    cfg.dynamicSmemBytes = VT<V_LARGE>::smem();
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int nc = 0;
+    if (cudaOccupancyMaxActiveClusters(&nc, VT<V_LARGE>::fn(), &cfg) != cudaSuccess || nc < 1) {
+      cudaGetLastError();
+      nc = c->num_sms / 2;
+    }
+    c->pair_workers = nc < c->num_sms / 2 ? nc : c->num_sms / 2;
+  }
   if (ok && c->nvfp4) {
     // scale padding (beyond K / 16) must read as zero; stale rows must hold finite scales
     cudaMemset(c->x_sf, 0, c->sf_bytes_dense(d));
@@ -1077,8 +1155,13 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   if (!mark(2)) return cuda_status(e);
   int ct;
   const int nch = n_chunks_for(T, N, &ct);
-  UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1, c->unit_u0};
-  UnitListSpec l2{c->units2, c->num_units + 1, le, V_BN[vg], c->max_units2, c->unit_u0 + N + 1};
+  // the expert-up GEMM's variant.  With at least a full token tile per expert on average (prefill),
+  // the single-CTA one (same token tile as the pair), which has no half-empty pair tiles at 2688
+  // features; with fewer (skewed loads: most experts hold one partial tile and stream their weights),
+  // the pair, whose deeper ring keeps more weight bytes in flight (measured: 0.79 vs 0.85 ms there)
+  const int vu = (vg == V_LARGE && TK >= (long long)V_BN[V_LARGE1] * N) ? V_LARGE1 : vg;
+  UnitListSpec l1{c->units1, c->num_units, m, V_BN[vu], c->max_units1, c->unit_u0, V_TILE_M[vu]};
+  UnitListSpec l2{c->units2, c->num_units + 1, le, V_BN[vg], c->max_units2, c->unit_u0 + N + 1, V_TILE_M[vg]};
   if (fused_route) {
     // 3-5. slice sum, top-K, expert scan, unit lists, stable rows and gather in one launch
     chk(launch_route_fused(c, T, rks, nch, ct, idx, gate, l1, l2, s));
@@ -1116,10 +1199,10 @@ lmoe_status lmoe_forward(lmoe_handle c, const void* x, int32_t T, void* y, int32
   }
   // 6. expert up: u = sqrelu(W1_e h)
   {
-    GemmLaunch g(c, vg, 4);
+    GemmLaunch g(c, vu, 4);
     if (split) g.pre_dense(c->map_ws1, c->map_x[vd], shared_up, ms, T);
-    g.main_grouped(c->map_w1, c->map_hperm[vg], problem(le, EPI_SQRELU_BF16, c->u, m), c->units1, c->num_units, m,
-                   0);
+    g.main_grouped(c->map_w1, vu == V_LARGE1 ? c->map_hperm1 : c->map_hperm[vg], problem(le, EPI_SQRELU_BF16, c->u, m),
+                   c->units1, c->num_units, m, 0);
     chk(g.run(s));
   }
   if (!mark(6)) return cuda_status(e);
@@ -1281,8 +1364,9 @@ lmoe_status lmoe_ep_experts(lmoe_handle c, const void* recv_rows, int32_t R, con
   ids_hist_kernel<<<nch, 256, NL * sizeof(int), s>>>(c->ep_ids, A, NL, ct, c->chunk_counts);
   if (!chk(cudaGetLastError())) return cuda_status(e);
   const int vg = A <= 48LL * NL ? V_SMALL : V_LARGE;
-  UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1, c->unit_u0};
-  UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2, c->unit_u0 + g.n_experts + 1};
+  UnitListSpec l1{c->units1, c->num_units, m, V_BN[vg], c->max_units1, c->unit_u0, V_TILE_M[vg]};
+  UnitListSpec l2{c->units2, c->num_units + 1, l, V_BN[vg], c->max_units2, c->unit_u0 + g.n_experts + 1,
+                  V_TILE_M[vg]};
   scan_units_kernel<<<1, 1024, scan_smem_bytes(NL, nch), s>>>(c->chunk_counts, nch, NL, c->counts, c->offsets,
                                                                c->chunk_base, l1, l2, c->tile0, c->status);
   if (!chk(cudaGetLastError()) || !chk(launch_build_units(c, s, l1, l2, NL))) return cuda_status(e);
@@ -1582,7 +1666,7 @@ extern "C" lmoe_status lmoe_route_noalloc(const float* logits, const float* bias
   if (launch_topk_hist(nch, 1, s, logits, bias, T, N, K, ct, topk_idx, topk_gate, chunk_counts) !=
       cudaSuccess)
     return LMOE_ERR_CUDA;
-  UnitListSpec none{nullptr, nullptr, 0, 64, 0, nullptr};
+  UnitListSpec none{nullptr, nullptr, 0, 64, 0, nullptr, BLOCK_M};
   scan_units_kernel<<<1, 1024, scan_smem_bytes(N, nch), s>>>(chunk_counts, nch, N, counts, offsets, chunk_base,
                                                               none, none, nullptr, status);
   if (cudaGetLastError() != cudaSuccess) return LMOE_ERR_CUDA;

@@ -309,18 +309,17 @@ __global__ void amax_act_kernel(const __nv_bfloat16* __restrict__ a, long long n
 // / tile_rows.  nra == 0: scales in plain row-major bytes [n_rows, K/16] instead of atoms.  One
 // thread per 16-element block; tensor scale from amax_bits[0], also written to *g_out.
 // ------------------------------------------------------------------------------------------------
-__global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, const int* __restrict__ src_rows,
-                                 long long n_rows, int n_src_rows, const int* __restrict__ offsets,
-                                 const int* __restrict__ tile0, int n_experts, int tile_rows, int nra,
-                                 const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes,
-                                 uint8_t* __restrict__ sf, float* __restrict__ g_out, unsigned* status, int reps) {
+// The blocks i = i0, i0 + stride, ... of quant_act_kernel (shared with the fused decode routing).
+__device__ __forceinline__ void quant_act_blocks(const __nv_bfloat16* __restrict__ a, int K,
+                                                 const int* __restrict__ src_rows, long long n_rows, int n_src_rows,
+                                                 const int* __restrict__ offsets, const int* __restrict__ tile0,
+                                                 int n_experts, int tile_rows, int nra, float g,
+                                                 uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                                                 unsigned* status, int reps, long long i0, long long stride) {
   const int nb = K / 16;
   const int stages = (K + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K;
-  const float g = tensor_scale_from_amax(__uint_as_float(amax_bits[0]));
-  if (blockIdx.x == 0 && threadIdx.x == 0 && g_out) *g_out = g;
   const long long total = n_rows * nb;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
+  for (long long i = i0; i < total; i += stride) {
     const long long r = i / nb;
     const int kb = (int)(i - r * nb);
     long long sr = r;
@@ -351,7 +350,7 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, con
     float v[16];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const uint4 q = src[h];
+      const uint4 q = __ldcg(src + h);  // L2: the fused routing reads h written by other blocks
       const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -370,6 +369,17 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, con
   }
 }
 
+__global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, const int* __restrict__ src_rows,
+                                 long long n_rows, int n_src_rows, const int* __restrict__ offsets,
+                                 const int* __restrict__ tile0, int n_experts, int tile_rows, int nra,
+                                 const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes,
+                                 uint8_t* __restrict__ sf, float* __restrict__ g_out, unsigned* status, int reps) {
+  const float g = tensor_scale_from_amax(__uint_as_float(amax_bits[0]));
+  if (blockIdx.x == 0 && threadIdx.x == 0 && g_out) *g_out = g;
+  quant_act_blocks(a, K, src_rows, n_rows, n_src_rows, offsets, tile0, n_experts, tile_rows, nra, g, codes, sf, status,
+                   reps, (long long)blockIdx.x * blockDim.x + threadIdx.x, (long long)gridDim.x * blockDim.x);
+}
+
 // ------------------------------------------------------------------------------------------------
 // Grouped copy of per-token NVFP4 rows: grouped row r gets the codes of token tok_of_row[r]
 // (quantised once per token: a row's codes and block scales depend only on its values and the
@@ -377,18 +387,21 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, con
 // row; K is a multiple of 128, so a row is a whole number of 512-byte code chunks and 4-byte scale
 // groups, and the four scales of one K atom of a row are four adjacent bytes of the atom.
 // ------------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256)
-    gather_act_q_kernel(const uint8_t* __restrict__ codes_tok, const uint8_t* __restrict__ sf_tok, int K,
-                        const int* __restrict__ tok_of_row, long long n_rows, int n_tok,
-                        const int* __restrict__ offsets, const int* __restrict__ tile0, int n_experts, int tile_rows,
-                        int nra, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, unsigned* status,
-                        int reps) {
+// Rows r = r0, r0 + stride, ... of gather_act_q_kernel, one per warp (shared with the fused decode
+// routing, which wrote the routing maps and the per-token codes earlier in the same launch: every
+// read of them goes through L2).
+__device__ __forceinline__ void gather_act_q_rows(const uint8_t* __restrict__ codes_tok,
+                                                  const uint8_t* __restrict__ sf_tok, int K,
+                                                  const int* __restrict__ tok_of_row, long long n_rows, int n_tok,
+                                                  const int* __restrict__ offsets, const int* __restrict__ tile0,
+                                                  int n_experts, int tile_rows, int nra, uint8_t* __restrict__ codes,
+                                                  uint8_t* __restrict__ sf, unsigned* status, int reps, long long r0,
+                                                  long long stride) {
   const int lane = threadIdx.x & 31;
-  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
   const int row_bytes = K / 2, nb = K / 16;
   const int stages = (K + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K;
-  for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < n_rows; r += nwarps) {
-    const int t = tok_of_row[r];
+  for (long long r = r0; r < n_rows; r += stride) {
+    const int t = __ldcg(tok_of_row + r);
     if (t < 0 || t >= n_tok) {
       if (lane == 0) atomicOr(status, DEV_STATUS_BAD_INDEX);
       continue;
@@ -396,21 +409,32 @@ __global__ void __launch_bounds__(256)
     int lo = 0, hi = n_experts - 1;  // largest expert whose first row is <= r
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (__ldg(offsets + mid) <= r) lo = mid;
+      if (__ldcg(offsets + mid) <= r) lo = mid;
       else hi = mid - 1;
     }
-    const int local = (int)(r - __ldg(offsets + lo));
-    const long long tile = __ldg(tile0 + lo) + local / tile_rows;
+    const int local = (int)(r - __ldcg(offsets + lo));
+    const long long tile = __ldcg(tile0 + lo) + local / tile_rows;
     const int j = local % tile_rows;
     for (int c = lane * 16; c < row_bytes; c += 32 * 16)
       *reinterpret_cast<uint4*>(codes + r * row_bytes + c) =
-          *reinterpret_cast<const uint4*>(codes_tok + (long long)t * row_bytes + c);
+          __ldcg(reinterpret_cast<const uint4*>(codes_tok + (long long)t * row_bytes + c));
     for (int q = lane; q < nb / 4; q += 32) {
-      const uint32_t v = *reinterpret_cast<const uint32_t*>(sf_tok + (long long)t * nb + 4 * q);
+      const uint32_t v = __ldcg(reinterpret_cast<const unsigned int*>(sf_tok + (long long)t * nb + 4 * q));
       for (int rp = 0; rp < reps; ++rp)
         *reinterpret_cast<uint32_t*>(sf + act_sf_offset(tile, j, 4 * q, stages, nra, rp, reps)) = v;
     }
   }
+}
+
+__global__ void __launch_bounds__(256)
+    gather_act_q_kernel(const uint8_t* __restrict__ codes_tok, const uint8_t* __restrict__ sf_tok, int K,
+                        const int* __restrict__ tok_of_row, long long n_rows, int n_tok,
+                        const int* __restrict__ offsets, const int* __restrict__ tile0, int n_experts, int tile_rows,
+                        int nra, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, unsigned* status,
+                        int reps) {
+  gather_act_q_rows(codes_tok, sf_tok, K, tok_of_row, n_rows, n_tok, offsets, tile0, n_experts, tile_rows, nra, codes,
+                    sf, status, reps, ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5,
+                    ((long long)gridDim.x * blockDim.x) >> 5);
 }
 
 }  // namespace lmoe

@@ -17,6 +17,15 @@
 //   -------  grid barrier
 //   phase 3  all blocks: the gather h_perm[r] = h[tok_of_row[r]]
 //
+// NVFP4 experts (fp4 != 0): phase 1 also takes max |x| and max |h| (of the bf16 h) over the grid;
+// in phase 2 the blocks without a chunk quantise x (the shared expert's input, in the expert
+// launch's dense tile atoms) and h once per token with the dynamic tensor scales; phase 3 copies
+// each grouped row's h codes and scales (tile-local atoms) instead of gathering bf16 rows.
+//
+// While the routing chain runs, HBM is almost idle: at the start every block asks L2 to fetch its
+// share of up to two weight ranges that the next launch (the expert-up GEMM) reads first (bf16
+// experts: the shared expert's first matrix and the lowest experts' first matrices).
+//
 // The grid barrier is self-resetting (an arrival count and a generation word, both zero when the
 // layer is created) and its wait is bounded by wall-clock time: on expiry the block raises
 // DEV_STATUS_TIMEOUT and returns (the host then resets the barrier words when it reads the status).
@@ -24,6 +33,7 @@
 #pragma once
 #include <cuda_bf16.h>
 
+#include "nvfp4.cuh"
 #include "ptx.cuh"
 #include "routing.cuh"
 
@@ -55,6 +65,24 @@ struct RouteFusedArgs {
   unsigned* bar;               // [2]: grid-barrier arrival count, generation
   unsigned* status;
   unsigned long long timeout_ns;
+  // NVFP4 experts
+  int fp4;
+  const __nv_bfloat16* x;      // [T, d] layer input
+  int d;
+  unsigned* amax;              // [2]: max |x|, max |h| as float bits (zero at launch)
+  float* act_g;                // [2] out: tensor scales g_x, g_h
+  uint8_t* xq;                 // [T, d / 2] x codes
+  uint8_t* x_sf;               //   x block scales, dense tile-local atoms
+  uint8_t* hq_tok;             // [T, l / 2] h codes per token
+  uint8_t* h_sf_tok;           // [T, l / 16] h block scales per token (plain)
+  uint8_t* hq;                 // [T * K, l / 2] grouped h codes
+  uint8_t* h_sf;               //   grouped h block scales, tile-local atoms
+  int tile_tokens4;            // token tile of the FP4 expert variant
+  int nra4;                    // its 128-row scale atoms per tile
+  // L2 prefetch of the next launch's first weights: ranges of pf_bytes[i] (multiples of 16, 16-byte
+  // aligned; 0: none)
+  const uint8_t* pf_ptr[2];
+  long long pf_bytes[2];
 };
 
 // Grid-wide barrier of a cooperative launch (every block resident).  Returns false, with
@@ -158,6 +186,13 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteFusedArgs a
   const int t_begin = b * a.chunk_tokens, t_end = min(a.T, t_begin + a.chunk_tokens);
 
   // ------------------------------------------------------------------ phase 1
+  if (tid < 2 && a.pf_bytes[tid] > 0) {
+    // this block's share of range tid, in pieces of at most 64 KB
+    const long long per = ((a.pf_bytes[tid] + G - 1) / G + 15) & ~15LL;
+    const long long lo = min(a.pf_bytes[tid], (long long)b * per), hi = min(a.pf_bytes[tid], lo + per);
+    for (long long o = lo; o < hi; o += 65536)
+      prefetch_l2_bulk(a.pf_ptr[tid] + o, (uint32_t)min(65536LL, hi - o));
+  }
   int* s_counts = smem_i;  // [N]
   for (int e = tid; e < N; e += blockDim.x) s_counts[e] = 0;
   if (b == 0)
@@ -190,6 +225,7 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteFusedArgs a
   }
   // latent rows of all tokens, over the whole grid: h = bf16(sum of the W_down slices), 4 columns
   // per thread
+  float amax_h = 0.f;  // NVFP4: max |h| of this thread's bf16 values
   {
     const int vpr = l / 4;
     const long long n = (long long)a.T * vpr;
@@ -210,6 +246,33 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteFusedArgs a
       pk.x = *reinterpret_cast<uint32_t*>(&lo);
       pk.y = *reinterpret_cast<uint32_t*>(&hi);
       *reinterpret_cast<uint2*>(a.h + t * l + col) = pk;
+      if (a.fp4) {
+        const float2 fl = __bfloat1622float2(lo), fh = __bfloat1622float2(hi);
+        amax_h = fmaxf(amax_h, fmaxf(fmaxf(fabsf(fl.x), fabsf(fl.y)), fmaxf(fabsf(fh.x), fabsf(fh.y))));
+      }
+    }
+  }
+  if (a.fp4) {
+    // max |x| over the grid (8 bf16 per load), then one atomic per warp for each maximum
+    float amax_x = 0.f;
+    const long long n8 = (long long)a.T * a.d / 8;
+    for (long long i = (long long)b * blockDim.x + tid; i < n8; i += (long long)G * blockDim.x) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(a.x) + i);
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(p2[j]);
+        amax_x = fmaxf(amax_x, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      amax_x = fmaxf(amax_x, __shfl_xor_sync(0xffffffffu, amax_x, o));
+      amax_h = fmaxf(amax_h, __shfl_xor_sync(0xffffffffu, amax_h, o));
+    }
+    if (lane == 0) {
+      if (amax_x > 0.f) atomicMax(a.amax, __float_as_uint(amax_x));
+      if (amax_h > 0.f) atomicMax(a.amax + 1, __float_as_uint(amax_h));
     }
   }
   __syncthreads();
@@ -228,7 +291,8 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteFusedArgs a
     int* s_hist = s_u2 + (N + 1);        // [W][N] per-warp counts, then per-warp running bases
     __shared__ int s_warp[4 * 33];
     const int tile = a.l1.tile_tokens;
-    const int nft1 = (a.l1.feat + BLOCK_M - 1) / BLOCK_M, nft2 = (a.l2.feat + BLOCK_M - 1) / BLOCK_M;
+    const int nft1 = (a.l1.feat + a.l1.tile_rows - 1) / a.l1.tile_rows;
+    const int nft2 = (a.l2.feat + a.l2.tile_rows - 1) / a.l2.tile_rows;
     // per-expert totals and this chunk's prefix: chunk rows are expert-contiguous, so a warp's
     // loads for one chunk are coalesced; sixteen chunks in flight per thread
     for (int e = tid; e < N; e += blockDim.x) {
@@ -305,8 +369,8 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteFusedArgs a
         const int cnt = s_off[ex + 1] - s_off[ex];
         const int nv = min(L.tile_tokens, cnt - tt * L.tile_tokens);
         int4* dst = reinterpret_cast<int4*>(&L.units[u]);
-        dst[0] = make_int4(ex * L.feat + ft * BLOCK_M, s_off[ex] + tt * L.tile_tokens, ft * BLOCK_M,
-                           nv | (min(BLOCK_M, L.feat - ft * BLOCK_M) << 16));
+        dst[0] = make_int4(ex * L.feat + ft * L.tile_rows, s_off[ex] + tt * L.tile_tokens, ft * L.tile_rows,
+                           nv | (min(L.tile_rows, L.feat - ft * L.tile_rows) << 16));
         dst[1] = make_int4(s_t0[ex] + tt, 0, 0, 0);
       }
     }
@@ -365,8 +429,33 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteFusedArgs a
       }
     }
   }
+  if (a.fp4) {
+    // x and h quantised with the tensor scales from the grid's maxima: the blocks without a chunk,
+    // or every block (after its chunk's work) when all blocks own a chunk
+    const int qn = G > nch ? G - nch : G, qb = G > nch ? b - nch : b;
+    if (qb >= 0) {
+      const float g_x = tensor_scale_from_amax(__uint_as_float(__ldcg(a.amax)));
+      const float g_h = tensor_scale_from_amax(__uint_as_float(__ldcg(a.amax + 1)));
+      if (qb == 0 && tid == 0) {
+        a.act_g[0] = g_x;
+        a.act_g[1] = g_h;
+      }
+      const long long i0 = (long long)qb * blockDim.x + tid, st = (long long)qn * blockDim.x;
+      quant_act_blocks(a.x, a.d, nullptr, a.T, a.T, nullptr, nullptr, N, a.tile_tokens4, a.nra4, g_x, a.xq, a.x_sf,
+                       a.status, 1, i0, st);
+      quant_act_blocks(a.h, l, nullptr, a.T, a.T, nullptr, nullptr, N, a.tile_tokens4, 0, g_h, a.hq_tok, a.h_sf_tok,
+                       a.status, 1, i0, st);
+    }
+  }
 
   if (!grid_barrier_bounded(a.bar, a.timeout_ns, a.status)) return;
+
+  if (a.fp4) {
+    // ------------------------------------------------------------------ phase 3 (NVFP4)
+    gather_act_q_rows(a.hq_tok, a.h_sf_tok, l, a.tok_of_row, (long long)a.T * K, a.T, a.offsets, a.tile0, N,
+                      a.tile_tokens4, a.nra4, a.hq, a.h_sf, a.status, 1, (long long)b * W + warp, (long long)G * W);
+    return;
+  }
 
   // ------------------------------------------------------------------ phase 3
   // h_perm[r] = h[tok_of_row[r]] over the whole grid: a warp copies four rows at a time, all of a

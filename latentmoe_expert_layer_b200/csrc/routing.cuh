@@ -220,6 +220,7 @@ struct UnitListSpec {
   int tile_tokens;     // tokens per unit (the GEMM variant's BN_MAX)
   int max_units;       // capacity
   int* u0;             // [N + 1] first unit of each expert, then the total (written by the scan)
+  int tile_rows;       // weight rows per unit: 128, or 256 for the CTA-pair variant
 };
 
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp, int& total) {
@@ -316,7 +317,7 @@ __global__ void __launch_bounds__(1024)
   for (int li = 0; li < 2; ++li) {
     const UnitListSpec& L = li ? l2 : l1;
     if (L.units == nullptr) continue;
-    const int nft = (L.feat + BLOCK_M - 1) / BLOCK_M;
+    const int nft = (L.feat + L.tile_rows - 1) / L.tile_rows;
     const int ntt = (c_e + L.tile_tokens - 1) / L.tile_tokens;
     const int nu = (e < n_experts) ? ntt * nft : 0;
     int nu_total;
@@ -352,12 +353,12 @@ __global__ void __launch_bounds__(256)
       else hi = mid - 1;
     }
     const int ex = lo;
-    const int nft = (L.feat + BLOCK_M - 1) / BLOCK_M;
+    const int nft = (L.feat + L.tile_rows - 1) / L.tile_rows;
     const int local = u - __ldg(L.u0 + ex);
     const int tt = local / nft, ft = local - tt * nft;
     const int nv = min(L.tile_tokens, __ldg(counts + ex) - tt * L.tile_tokens);
-    const int4 g = make_int4(ex * L.feat + ft * BLOCK_M, __ldg(offsets + ex) + tt * L.tile_tokens, ft * BLOCK_M,
-                             nv | (min(BLOCK_M, L.feat - ft * BLOCK_M) << 16));
+    const int4 g = make_int4(ex * L.feat + ft * L.tile_rows, __ldg(offsets + ex) + tt * L.tile_tokens,
+                             ft * L.tile_rows, nv | (min(L.tile_rows, L.feat - ft * L.tile_rows) << 16));
     int4* dst = reinterpret_cast<int4*>(&L.units[u]);
     dst[0] = g;
     dst[1] = make_int4(__ldg(tile0 + ex) + tt, 0, 0, 0);
@@ -601,17 +602,25 @@ __global__ void __launch_bounds__(256)
 // Launch with programmatic stream serialisation (the kernel calls griddep_wait before it reads what
 // the previous launch wrote): its launch and set-up overlap the previous kernel's tail.
 template <typename... P, typename... A>
-cudaError_t launch_pdl(void (*kernel)(P...), int grid, int threads, size_t smem, cudaStream_t s, A&&... args) {
+cudaError_t launch_pdl(void (*kernel)(P...), int grid, int threads, size_t smem, cudaStream_t s, int cluster,
+                       A&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (cluster > 1) {  // clusters of `cluster` consecutive CTAs (grid is a multiple of it)
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
 }
 
@@ -621,9 +630,9 @@ inline cudaError_t launch_combine(int num_sms, cudaStream_t s, const __nv_bfloat
   const long long threads = (long long)T * (latent / 8);
   const int blocks = (int)((threads + 255) / 256);
   if (threads <= (long long)num_sms * 256)
-    return launch_pdl(combine_kernel<true>, blocks, 256, 0, s, o, row_of, T, k, latent, out, ld_out, n_rows, status,
+    return launch_pdl(combine_kernel<true>, blocks, 256, 0, s, 1, o, row_of, T, k, latent, out, ld_out, n_rows, status,
                       add, ld_add);
-  return launch_pdl(combine_kernel<false>, blocks, 256, 0, s, o, row_of, T, k, latent, out, ld_out, n_rows, status,
+  return launch_pdl(combine_kernel<false>, blocks, 256, 0, s, 1, o, row_of, T, k, latent, out, ld_out, n_rows, status,
                     add, ld_add);
 }
 

@@ -53,6 +53,21 @@ def test_tiny_ragged_tokens(tiny, t):
     compare_bf16(layer, oracle_weights(w, False), x, wl.shape.top_k)
 
 
+@pytest.mark.parametrize("t", [600, 1000])
+def test_tiny_shape_at_prefill_sizes(t):
+    """Past 512 tokens the dense and grouped GEMMs run as CTA pairs over 256 weight rows.  The tiny
+    layer's weight blocks are narrower than a pair (router 16 rows, W_down 64, experts 128 and 64), so
+    the odd CTA of every pair holds no valid rows, and the token tiles end ragged."""
+    wl = dataclasses.replace(inp.workload("tiny"), tokens=t)
+    w = inp.make_weights(wl)
+    layer = make_layer(wl, w, device_weights(w), t)
+    try:
+        st = compare_bf16(layer, oracle_weights(w, False), inp.make_x(wl), wl.shape.top_k)
+        check_dispatch(layer, st["idx"], wl.shape.n_experts)
+    finally:
+        layer.close()
+
+
 def test_tiny_deterministic(tiny):
     wl, w, layer = tiny
     x = inp.make_x(wl)
