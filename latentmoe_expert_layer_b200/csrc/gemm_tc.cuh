@@ -54,7 +54,8 @@ enum EpiKind : int {
 // EPI_SQRELU_NVFP4); tile: token-tile id (NVFP4 activation scales are stored per token tile).
 struct GemmUnit {
   int a_row, b_row, f0, nm;
-  int tile, kslice, pad1, pad2;  // kslice: K slice of a split dense unit (0 otherwise)
+  int tile, kslice, pad1, pad2;  // kslice: K slice of a split dense unit (0 otherwise); in the
+                                 // kernel's unit ring pad1 = problem, pad2 = unit (-1: no more units)
 };
 
 // One GEMM problem of a launch: K extent, epilogue, NVFP4 scales, and (for dense problems) the grid.
@@ -131,6 +132,8 @@ struct GemmSmem {
   static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
   static constexpr int BAR_OFF = EPI_OFF + 4 * EPI_STAGE_BYTES;
   static constexpr int BYTES = BAR_OFF + 512;
+  // barrier block: 2 * STAGES + 21 mbarriers, TMEM slot and abort flag, unit ring, claim mailbox
+  static_assert(16 * STAGES + 176 + 32 * UNIT_RING + 4 * UNIT_RING <= 512, "barrier block overflows");
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment of the base
   // TMEM: two accumulator buffers (double buffering), each ACC_SPLIT partial fp32 accumulators of
   // BN_MAX columns; then (FP4) SF_SLOTS rotating slots of weight scales (SFA: 4 MMAs x 4 columns per
@@ -258,8 +261,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint64_t* mempty = mfull + UNIT_RING;     //   odd -> even CTA (the slot may be rewritten)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mempty + UNIT_RING);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* unit_ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
-  volatile int* mailbox = reinterpret_cast<volatile int*>(tmem_slot + 2 + UNIT_RING);
+  // unit ring entries: the producer publishes each unit's whole descriptor (16-byte aligned: the
+  // barrier block is 16 * STAGES + 176 bytes long), so the MMA issuer and the epilogue start a unit
+  // without a global-memory round trip
+  int4* unit_ring = reinterpret_cast<int4*>(tmem_slot + 2);
+  volatile int* mailbox = reinterpret_cast<volatile int*>(unit_ring + 2 * UNIT_RING);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -379,13 +385,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       open_claim();
       int res_key = -1;  // (token tile, problem) whose activation scales are resident in TMEM
       auto wait0 = [&](uint64_t* bar, uint32_t par) -> bool { return mbar_wait_bounded(bar, par, abort_flag, tmo); };
+      // the next unit's descriptor is read one unit ahead: its global load lands while this unit's
+      // loads are issued
+      GemmUnit nxt = {};
+      int nxt_pid = 0;
+      if (u_next < num_units) nxt = unit_at<BN_MAX, TILE_M>(args, u_next, nxt_pid, prank);
       while (ok) {
         if (!wait0(&uempty[uslot], uphase ^ 1u)) {
           ok = false;
           break;
         }
         const int u = u_next < num_units ? u_next : -1;
-        unit_ring[uslot] = u;
+        GemmUnit un = nxt;
+        const int pid = nxt_pid;
+        un.pad1 = pid;
+        un.pad2 = u;
+        unit_ring[2 * uslot] = make_int4(un.a_row, un.b_row, un.f0, un.nm);
+        unit_ring[2 * uslot + 1] = make_int4(un.tile, un.kslice, un.pad1, un.pad2);
         mbar_arrive(&ufull[uslot]);
         if (++uslot == UNIT_RING) {
           uslot = 0;
@@ -396,8 +412,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           claim = args.dynamic ? take_claim() : claim + n_workers;
           open_claim();
         }
-        int pid;
-        const GemmUnit un = unit_at<BN_MAX, TILE_M>(args, u, pid, prank);
+        if (u_next < num_units) nxt = unit_at<BN_MAX, TILE_M>(args, u_next, nxt_pid, prank);
         const GemmProblem& pr = args.prob[pid];
         const CUtensorMap* mw = pid ? &map_w1 : &map_w0;
         const CUtensorMap* ma = pid ? &map_act1 : &map_act0;
@@ -486,7 +501,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           atomicOr(args.status, DEV_STATUS_TIMEOUT);
           break;
         }
-        const int u = unit_ring[uslot];
+        const int u = unit_ring[2 * uslot + 1].w;
         mbar_arrive(&uempty[uslot]);
         if (++uslot == UNIT_RING) {
           uslot = 0;
@@ -509,15 +524,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           ok = false;
           break;
         }
-        const int u = unit_ring[uslot];
+        const int4 e0 = unit_ring[2 * uslot], e1 = unit_ring[2 * uslot + 1];
         mbar_arrive(&uempty[uslot]);
         if (++uslot == UNIT_RING) {
           uslot = 0;
           uphase ^= 1u;
         }
-        if (u < 0) break;
-        int pid;
-        const GemmUnit un = unit_at<BN_MAX, TILE_M>(args, u, pid, prank);
+        if (e1.w < 0) break;
+        const GemmUnit un = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+        const int pid = e1.z;
         const int nkb = args.prob[pid].num_k_blocks;
         const int nv = un.nm & 0xFFFF;
         const uint32_t n_mma = (uint32_t)((nv + 15) & ~15);
@@ -632,16 +647,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (lane == 0) atomicOr(args.status, DEV_STATUS_TIMEOUT);
         break;
       }
-      const int u = unit_ring[uslot];
+      const int4 e0 = unit_ring[2 * uslot], e1 = unit_ring[2 * uslot + 1];
       __syncwarp();
       if (lane == 0) mbar_arrive(&uempty[uslot]);
       if (++uslot == UNIT_RING) {
         uslot = 0;
         uphase ^= 1u;
       }
-      if (u < 0) break;
-      int pid;
-      const GemmUnit un = unit_at<BN_MAX, TILE_M>(args, u, pid, prank);
+      if (e1.w < 0) break;
+      const GemmUnit un = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+      const int pid = e1.z;
       const GemmProblem& pr = args.prob[pid];
       const int nv = un.nm & 0xFFFF;
       const int mv = un.nm >> 16;

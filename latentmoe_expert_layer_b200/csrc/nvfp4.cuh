@@ -309,7 +309,17 @@ __global__ void amax_act_kernel(const __nv_bfloat16* __restrict__ a, long long n
 // / tile_rows.  nra == 0: scales in plain row-major bytes [n_rows, K/16] instead of atoms.  One
 // thread per 16-element block; tensor scale from amax_bits[0], also written to *g_out.
 // ------------------------------------------------------------------------------------------------
+// Loads of routing maps and activations in the shared device functions below.  SAME_LAUNCH: the
+// data was written earlier in the same launch by other blocks (the fused decode routing), so it is
+// read through L2 only; otherwise it is read-only for the kernel and may be cached on the SM.
+template <bool SAME_LAUNCH, typename V>
+__device__ __forceinline__ V ld_act(const V* p) {
+  if constexpr (SAME_LAUNCH) return __ldcg(p);
+  else return __ldg(p);
+}
+
 // The blocks i = i0, i0 + stride, ... of quant_act_kernel (shared with the fused decode routing).
+template <bool SAME_LAUNCH>
 __device__ __forceinline__ void quant_act_blocks(const __nv_bfloat16* __restrict__ a, int K,
                                                  const int* __restrict__ src_rows, long long n_rows, int n_src_rows,
                                                  const int* __restrict__ offsets, const int* __restrict__ tile0,
@@ -350,7 +360,7 @@ __device__ __forceinline__ void quant_act_blocks(const __nv_bfloat16* __restrict
     float v[16];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const uint4 q = __ldcg(src + h);  // L2: the fused routing reads h written by other blocks
+      const uint4 q = ld_act<SAME_LAUNCH>(src + h);
       const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -376,8 +386,9 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, con
                                  uint8_t* __restrict__ sf, float* __restrict__ g_out, unsigned* status, int reps) {
   const float g = tensor_scale_from_amax(__uint_as_float(amax_bits[0]));
   if (blockIdx.x == 0 && threadIdx.x == 0 && g_out) *g_out = g;
-  quant_act_blocks(a, K, src_rows, n_rows, n_src_rows, offsets, tile0, n_experts, tile_rows, nra, g, codes, sf, status,
-                   reps, (long long)blockIdx.x * blockDim.x + threadIdx.x, (long long)gridDim.x * blockDim.x);
+  quant_act_blocks<false>(a, K, src_rows, n_rows, n_src_rows, offsets, tile0, n_experts, tile_rows, nra, g, codes, sf,
+                          status, reps, (long long)blockIdx.x * blockDim.x + threadIdx.x,
+                          (long long)gridDim.x * blockDim.x);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -388,8 +399,8 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, con
 // groups, and the four scales of one K atom of a row are four adjacent bytes of the atom.
 // ------------------------------------------------------------------------------------------------
 // Rows r = r0, r0 + stride, ... of gather_act_q_kernel, one per warp (shared with the fused decode
-// routing, which wrote the routing maps and the per-token codes earlier in the same launch: every
-// read of them goes through L2).
+// routing, which wrote the routing maps and the per-token codes earlier in the same launch).
+template <bool SAME_LAUNCH>
 __device__ __forceinline__ void gather_act_q_rows(const uint8_t* __restrict__ codes_tok,
                                                   const uint8_t* __restrict__ sf_tok, int K,
                                                   const int* __restrict__ tok_of_row, long long n_rows, int n_tok,
@@ -401,7 +412,7 @@ __device__ __forceinline__ void gather_act_q_rows(const uint8_t* __restrict__ co
   const int row_bytes = K / 2, nb = K / 16;
   const int stages = (K + NVFP4_STAGE_K - 1) / NVFP4_STAGE_K;
   for (long long r = r0; r < n_rows; r += stride) {
-    const int t = __ldcg(tok_of_row + r);
+    const int t = ld_act<SAME_LAUNCH>(tok_of_row + r);
     if (t < 0 || t >= n_tok) {
       if (lane == 0) atomicOr(status, DEV_STATUS_BAD_INDEX);
       continue;
@@ -409,17 +420,17 @@ __device__ __forceinline__ void gather_act_q_rows(const uint8_t* __restrict__ co
     int lo = 0, hi = n_experts - 1;  // largest expert whose first row is <= r
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (__ldcg(offsets + mid) <= r) lo = mid;
+      if (ld_act<SAME_LAUNCH>(offsets + mid) <= r) lo = mid;
       else hi = mid - 1;
     }
-    const int local = (int)(r - __ldcg(offsets + lo));
-    const long long tile = __ldcg(tile0 + lo) + local / tile_rows;
+    const int local = (int)(r - ld_act<SAME_LAUNCH>(offsets + lo));
+    const long long tile = ld_act<SAME_LAUNCH>(tile0 + lo) + local / tile_rows;
     const int j = local % tile_rows;
     for (int c = lane * 16; c < row_bytes; c += 32 * 16)
       *reinterpret_cast<uint4*>(codes + r * row_bytes + c) =
-          __ldcg(reinterpret_cast<const uint4*>(codes_tok + (long long)t * row_bytes + c));
+          ld_act<SAME_LAUNCH>(reinterpret_cast<const uint4*>(codes_tok + (long long)t * row_bytes + c));
     for (int q = lane; q < nb / 4; q += 32) {
-      const uint32_t v = __ldcg(reinterpret_cast<const unsigned int*>(sf_tok + (long long)t * nb + 4 * q));
+      const uint32_t v = ld_act<SAME_LAUNCH>(reinterpret_cast<const unsigned int*>(sf_tok + (long long)t * nb + 4 * q));
       for (int rp = 0; rp < reps; ++rp)
         *reinterpret_cast<uint32_t*>(sf + act_sf_offset(tile, j, 4 * q, stages, nra, rp, reps)) = v;
     }
@@ -432,8 +443,8 @@ __global__ void __launch_bounds__(256)
                         const int* __restrict__ offsets, const int* __restrict__ tile0, int n_experts, int tile_rows,
                         int nra, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, unsigned* status,
                         int reps) {
-  gather_act_q_rows(codes_tok, sf_tok, K, tok_of_row, n_rows, n_tok, offsets, tile0, n_experts, tile_rows, nra, codes,
-                    sf, status, reps, ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5,
+  gather_act_q_rows<false>(codes_tok, sf_tok, K, tok_of_row, n_rows, n_tok, offsets, tile0, n_experts, tile_rows, nra,
+                           codes, sf, status, reps, ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5,
                     ((long long)gridDim.x * blockDim.x) >> 5);
 }
 

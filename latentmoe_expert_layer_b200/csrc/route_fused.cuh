@@ -441,9 +441,9 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteFusedArgs a
         a.act_g[1] = g_h;
       }
       const long long i0 = (long long)qb * blockDim.x + tid, st = (long long)qn * blockDim.x;
-      quant_act_blocks(a.x, a.d, nullptr, a.T, a.T, nullptr, nullptr, N, a.tile_tokens4, a.nra4, g_x, a.xq, a.x_sf,
+      quant_act_blocks<true>(a.x, a.d, nullptr, a.T, a.T, nullptr, nullptr, N, a.tile_tokens4, a.nra4, g_x, a.xq, a.x_sf,
                        a.status, 1, i0, st);
-      quant_act_blocks(a.h, l, nullptr, a.T, a.T, nullptr, nullptr, N, a.tile_tokens4, 0, g_h, a.hq_tok, a.h_sf_tok,
+      quant_act_blocks<true>(a.h, l, nullptr, a.T, a.T, nullptr, nullptr, N, a.tile_tokens4, 0, g_h, a.hq_tok, a.h_sf_tok,
                        a.status, 1, i0, st);
     }
   }
@@ -452,7 +452,7 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteFusedArgs a
 
   if (a.fp4) {
     // ------------------------------------------------------------------ phase 3 (NVFP4)
-    gather_act_q_rows(a.hq_tok, a.h_sf_tok, l, a.tok_of_row, (long long)a.T * K, a.T, a.offsets, a.tile0, N,
+    gather_act_q_rows<true>(a.hq_tok, a.h_sf_tok, l, a.tok_of_row, (long long)a.T * K, a.T, a.offsets, a.tile0, N,
                       a.tile_tokens4, a.nra4, a.hq, a.h_sf, a.status, 1, (long long)b * W + warp, (long long)G * W);
     return;
   }

@@ -98,6 +98,11 @@ WORKLOADS: Dict[str, Workload] = {
     # experts, ~2.3 GB on the device
     "prefill_small": Workload("prefill_small", dataclasses.replace(SUPER, n_experts=128), 4096, 1, 3, "bf16", "bf16",
                               description="Super dims with 128 experts, T=4096 (~704 tokens per expert)"),
+    # profiling case: the NVFP4 prefill GEMM's regime (~704 tokens per expert, 192-token tiles) with
+    # 128 experts, under 1 GB on the device
+    "prefill_small_nvfp4": Workload("prefill_small_nvfp4", dataclasses.replace(SUPER, n_experts=128), 4096, 1, 3,
+                                    "bf16", "nvfp4",
+                                    description="NVFP4 Super dims with 128 experts, T=4096 (~704 tokens per expert)"),
     # small NVFP4 layers: several 128-row tiles, a ragged 256-element K stage (m = 384), both the
     # decode-sized (~10 tokens per expert) and the prefill-sized (~256 per expert) GEMM shapes
     "nvfp4_tiny": Workload("nvfp4_tiny", LayerShape(512, 256, 16, 4, 384, 512), 40, 7, 8, "bf16", "nvfp4",
