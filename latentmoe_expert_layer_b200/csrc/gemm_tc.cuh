@@ -105,7 +105,7 @@ struct GemmArgs {
   unsigned long long timeout_ns;
 };
 
-constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_THREADS = 192;  // producer warp, MMA warp and four epilogue warps (the default)
 constexpr int UNIT_RING = 4;
 constexpr int BLOCK_M = 128;
 constexpr int BLOCK_K = 64;                 // bf16 elements per stage (one 128-byte swizzle row)
@@ -118,7 +118,7 @@ constexpr int SF_ATOM_BYTES = 512;
 // tile's first unit loads and copies them stage by stage, its later units reuse them.
 // PAIR: the CTA is one of a pair sharing cta_group::2 MMAs (M = 256); it holds half of the token
 // tile's rows per stage.
-template <int BN_MAX, int STAGES, bool FP4, int ACC_SPLIT, int RES_STAGES, bool PAIR = false>
+template <int BN_MAX, int STAGES, bool FP4, int ACC_SPLIT, int RES_STAGES, bool PAIR = false, int EPIW = 4>
 struct GemmSmem {
   static constexpr int NRA = (BN_MAX + 127) / 128;                    // 128-row scale atoms of B
   static constexpr int B_STAGE_BYTES = (PAIR ? BN_MAX / 2 : BN_MAX) * 128;
@@ -130,7 +130,7 @@ struct GemmSmem {
   static constexpr int SFB_STAGE_BYTES = FP4 ? 4 * NRA * SF_ATOM_BYTES * SFB_REP : 0;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES + SFA_STAGE_BYTES + SFB_STAGE_BYTES;
   static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
-  static constexpr int BAR_OFF = EPI_OFF + 4 * EPI_STAGE_BYTES;
+  static constexpr int BAR_OFF = EPI_OFF + EPIW * EPI_STAGE_BYTES;
   static constexpr int BYTES = BAR_OFF + 512;
   // barrier block: 2 * STAGES + 21 mbarriers, TMEM slot and abort flag, unit ring, claim mailbox
   static_assert(16 * STAGES + 176 + 32 * UNIT_RING + 4 * UNIT_RING <= 512, "barrier block overflows");
@@ -238,12 +238,17 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rn(float v) {
 // TMEM.  Per stage an SM then reads 32 KB for 128 x 256 x 64 MACs instead of 48 KB.  Both CTAs
 // walk the same unit sequence: static claims by pair, or dynamic claims taken by the even CTA and
 // passed to the odd one through a mailbox in its shared memory.
-template <int BN_MAX, int STAGES, int BOXN, bool FP4, int ACC_SPLIT, int RES_STAGES, bool PAIR>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+//
+// EPIW epilogue warps (4 or 8): with 8, two warps share each TMEM lane quadrant and take alternate
+// 32-token chunks of a tile (for epilogues that cost more than the tile's MMAs, such as the NVFP4
+// quantisation of u after short-K units).
+template <int BN_MAX, int STAGES, int BOXN, bool FP4, int ACC_SPLIT, int RES_STAGES, bool PAIR, int EPIW>
+__global__ void __launch_bounds__(64 + 32 * EPIW, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_w0, const __grid_constant__ CUtensorMap map_act0,
                    const __grid_constant__ CUtensorMap map_w1, const __grid_constant__ CUtensorMap map_act1,
                    const GemmArgs args) {
-  using S = GemmSmem<BN_MAX, STAGES, FP4, ACC_SPLIT, RES_STAGES, PAIR>;
+  using S = GemmSmem<BN_MAX, STAGES, FP4, ACC_SPLIT, RES_STAGES, PAIR, EPIW>;
+  static_assert(EPIW == 4 || EPIW == 8, "one or two epilogue warps per TMEM lane quadrant");
   constexpr int TILE_M = PAIR ? 2 * BLOCK_M : BLOCK_M;
   static_assert(BN_MAX % BOXN == 0 && BOXN % 8 == 0, "token box must tile the token block");
   static_assert(BN_MAX % 16 == 0 && BN_MAX <= 256, "MMA N limit");
@@ -281,12 +286,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], PAIR ? 8 : 4);  // a pair's issuer waits for both CTAs' epilogue warps
+      mbar_init(&tempty[b], PAIR ? 2 * EPIW : EPIW);  // a pair's issuer waits for both CTAs' epilogue warps
     }
     mbar_init(drain, 1);
     for (int i = 0; i < UNIT_RING; ++i) {
       mbar_init(&ufull[i], 1);
-      mbar_init(&uempty[i], 5);  // the MMA issuer and the four epilogue warps
+      mbar_init(&uempty[i], 1 + EPIW);  // the MMA issuer and the epilogue warps
       mbar_init(&mfull[i], 1);
       mbar_init(&mempty[i], 1);
     }
@@ -634,9 +639,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ epilogue (warps 2..5)
+    // ------------------------------------------------------------------ epilogue (warps 2..)
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    uint8_t* stg = smem + S::EPI_OFF + q * EPI_STAGE_BYTES;
+    const int ew = warp - 2;
+    const int c_first = ew >> 2, c_step = EPIW >> 2;  // this warp's 32-token chunks of a tile
+    uint8_t* stg = smem + S::EPI_OFF + ew * EPI_STAGE_BYTES;
     int acc = 0;
     uint32_t acc_phase = 0;
     int uslot = 0;
@@ -675,7 +682,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int nchunks = (nv + 31) >> 5;
       const bool feat_ok = (q * 32) < mv;
       const int f = un.f0 + q * 32;  // first feature of this warp's 32
-      for (int c = 0; c < nchunks; ++c) {
+      if (c_first >= nchunks) {
+        // no chunk of this tile for this warp: the accumulator is free as far as it is concerned
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_remote(cluster_addr(&tempty[acc], 0));
+          else mbar_arrive(&tempty[acc]);
+        }
+      }
+      for (int c = c_first; c < nchunks; c += c_step) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), r);
         tmem_ld_wait();
@@ -686,7 +702,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(r2[j]));
         }
-        if (c == nchunks - 1) {
+        if (c + c_step >= nchunks) {
           // accumulator fully read by this warp: hand it back to the MMA issuer
           tc_fence_before();
           __syncwarp();

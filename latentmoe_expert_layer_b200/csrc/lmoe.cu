@@ -65,14 +65,18 @@ constexpr int V_ACC_SPLIT[5] = {4, 1, 2, 1, 1};  // decode-sized tiles rotate ov
 // K stages of one token tile's activation scales that fit resident in TMEM (0: per-stage copies)
 constexpr int V_RES[5] = {0, 0, 12, 0, 0};
 constexpr bool V_PAIR[5] = {false, true, false, false, false};
+// epilogue warps: eight for the NVFP4 prefill variant, whose fc1 epilogue (squared ReLU and the NVFP4
+// quantisation of u) costs more than the MMAs of a K = 1024 unit
+constexpr int V_EPIW[5] = {4, 4, 4, 8, 4};
 constexpr int V_TILE_M[5] = {128, 256, 128, 128, 128};  // weight rows per unit
 
 template <int V>
 struct VT {
   static constexpr int BN = V_BN[V], ST = V_STAGES[V], BOX = V_BOXN[V], AS = V_ACC_SPLIT[V], RS = V_RES[V];
   static constexpr bool F4 = V_FP4[V], PR = V_PAIR[V];
-  static void* fn() { return reinterpret_cast<void*>(gemm_tc_kernel<BN, ST, BOX, F4, AS, RS, PR>); }
-  static int smem() { return GemmSmem<BN, ST, F4, AS, RS, PR>::ALLOC; }
+  static constexpr int EW = V_EPIW[V], THREADS = 64 + 32 * V_EPIW[V];
+  static void* fn() { return reinterpret_cast<void*>(gemm_tc_kernel<BN, ST, BOX, F4, AS, RS, PR, EW>); }
+  static int smem() { return GemmSmem<BN, ST, F4, AS, RS, PR, EW>::ALLOC; }
 };
 
 // 2-D byte tensor map (packed NVFP4 codes): rows x cols_bytes, 128-byte x box_rows tiles, 128-byte swizzle.
@@ -283,8 +287,9 @@ lmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LMOE_OK : LMO
 template <int V>
 cudaError_t launch_gemm_v(const CUtensorMap& w0, const CUtensorMap& a0, const CUtensorMap& w1, const CUtensorMap& a1,
                           const GemmArgs& a, int grid, cudaStream_t s) {
-  return launch_pdl(gemm_tc_kernel<VT<V>::BN, VT<V>::ST, VT<V>::BOX, VT<V>::F4, VT<V>::AS, VT<V>::RS, VT<V>::PR>,
-                    grid, GEMM_THREADS, VT<V>::smem(), s, VT<V>::PR ? 2 : 1, w0, a0, w1, a1, a);
+  return launch_pdl(
+      gemm_tc_kernel<VT<V>::BN, VT<V>::ST, VT<V>::BOX, VT<V>::F4, VT<V>::AS, VT<V>::RS, VT<V>::PR, VT<V>::EW>, grid,
+      VT<V>::THREADS, VT<V>::smem(), s, VT<V>::PR ? 2 : 1, w0, a0, w1, a1, a);
 }
 
 // A bf16 problem with its epilogue; K in elements (multiple of 64).
@@ -885,7 +890,7 @@ lmoe_status lmoe_create(const lmoe_config* cfg, int device, lmoe_handle* out) {
     // a pair's two CTAs sit in one GPC: size the pair variant's grid to the pairs that fit at once
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(c->num_sms);
-    cfg.blockDim = dim3(GEMM_THREADS);
+    cfg.blockDim = dim3(VT<V_LARGE>::THREADS);
     cfg.dynamicSmemBytes = VT<V_LARGE>::smem();
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
