@@ -48,19 +48,20 @@ DEFAULT_STEPS.update({"decode_small": 400, "decode_nvfp4": 400, "prefill_nvfp4":
 
 # DRAM traffic per launch of the expert GEMMs over their algorithmic bytes (dram__bytes_read.sum +
 # dram__bytes_write.sum from ncu section captures, summarised under profiles/): the decode NVFP4
-# capture is the full workload; the bf16 ones are smaller cases of the same regime (Super dims with
-# 128 experts: T = 64 for decode, T = 4096 for prefill), scaled to a launch by its algorithmic
+# capture is the full workload; the others are smaller cases of the same regime (Super dims with
+# 128 experts: T = 64 for decode, T = 4096 for bf16 and NVFP4 prefill), scaled to a launch by its algorithmic
 # bytes, which grow with the units processed.  The prefill ratios hold where the library runs the
 # same GEMM variants as the capture (expert up on one CTA: at least one full 256-token tile per
 # expert on average; expert down as CTA pairs).  Valid only while the GEMM's sources are the ones
 # captured (TRAFFIC_SOURCES_SHA256); otherwise the roofline reports no traffic.
 TRAFFIC_RATIO = {
-    ("bf16", "decode", "expert_up"): 0.997, ("bf16", "decode", "expert_down"): 1.000,
-    ("nvfp4", "decode", "expert_up"): 1.383, ("nvfp4", "decode", "expert_down"): 1.495,
-    ("bf16", "prefill", "expert_up"): 0.983, ("bf16", "prefill", "expert_down"): 1.078,
+    ("bf16", "decode", "expert_up"): 0.998, ("bf16", "decode", "expert_down"): 1.001,
+    ("nvfp4", "decode", "expert_up"): 1.381, ("nvfp4", "decode", "expert_down"): 1.494,
+    ("bf16", "prefill", "expert_up"): 0.982, ("bf16", "prefill", "expert_down"): 1.014,
+    ("nvfp4", "prefill", "expert_up"): 1.459, ("nvfp4", "prefill", "expert_down"): 1.245,
 }
 TRAFFIC_SOURCES = ("gemm_tc.cuh", "ptx.cuh", "nvfp4.cuh", "lmoe.cu")
-TRAFFIC_SOURCES_SHA256 = "4f02f2b87ddc50eed6580fd1c8a0cad66e5e560d65211f48d36f132c82826b1f"
+TRAFFIC_SOURCES_SHA256 = "2dff12f96abd7ae190ff6b0dc62d52d33004f3c50642f6457b85138f7da9073a"
 
 
 def gemm_sources_sha256() -> str:
