@@ -120,7 +120,13 @@ lmoe_status lmoe_forward(lmoe_handle h, const void* x, int32_t T, void* y, int32
 
 /* Same as lmoe_forward, with x/y/topk_idx/topk_gate in HOST memory (pinned memory gives
  * asynchronous copies).  The host-to-device copy of x, the layer and the device-to-host copies of
- * the outputs are all enqueued on `stream`; the caller synchronises before reading the outputs. */
+ * the outputs are all ordered after earlier work on `stream`, and later work on `stream` is ordered
+ * after them; the caller synchronises before reading the outputs.  BF16 layers with T >= 8192 run
+ * the batch in chunks of 4096 tokens: each chunk's input copy and output copies run on two streams
+ * the handle creates on first use, overlapping the layer's work on the neighbouring chunks.  Every
+ * token's routing is the one-call forward's; y can differ from it in rounding only (the chunks'
+ * expert-up GEMM may take another tile shape).  Staging buffers for max_tokens are allocated on the
+ * first call. */
 lmoe_status lmoe_forward_host(lmoe_handle h, const void* x_host, int32_t T, void* y_host, int32_t* topk_idx_host,
                               float* topk_gate_host, void* stream);
 

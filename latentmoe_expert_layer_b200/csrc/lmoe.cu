@@ -170,6 +170,9 @@ struct lmoe_ctx {
   __nv_bfloat16* y_dev = nullptr;
   int* idx_dev = nullptr;
   float* gate_dev = nullptr;
+  // chunked host forward: copy streams and their events (created on first use)
+  cudaStream_t host_in = nullptr, host_out = nullptr;
+  std::vector<cudaEvent_t> host_ev;
 
   int last_T = 0;
 
@@ -757,6 +760,73 @@ cudaError_t forward_nvfp4(lmoe_ctx* c, const void* x, int T, void* y, int* idx, 
   return e;
 }
 
+// Host-buffer forwards of large bf16 batches run in chunks of kHostChunk tokens, so that the copy of
+// one chunk's input and of another chunk's outputs overlap the layer's work on a third.  Each
+// chunk still streams every expert's weights once, so chunks stay large (at 4096 tokens the layer
+// is tensor-bound, not weight-bound).  NVFP4 layers are not chunked: their activation tensor
+// scales are taken over the whole call's tokens.
+constexpr int kHostChunk = 4096;
+
+int host_chunk_tokens(const lmoe_ctx* c, int T) {
+  if (c->nvfp4 || T < 2 * kHostChunk) return T;
+  return kHostChunk;
+}
+
+// Chunk i: its input copy on host_in, its forward on s once that copy is done, its output copies on
+// host_out once the forward is done.  The call forks from s (so the previous call's forward has
+// finished reading x_dev before this call overwrites it) and joins back into s.
+lmoe_status forward_host_chunked(lmoe_ctx* c, const void* x_host, int T, void* y_host, int* idx_host,
+                                 float* gate_host, cudaStream_t s, int chunk) {
+  const lmoe_config& g = c->cfg;
+  const int n = (T + chunk - 1) / chunk;
+  if (!c->host_in) {
+    if (cudaStreamCreateWithFlags(&c->host_in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&c->host_out, cudaStreamNonBlocking) != cudaSuccess)
+      return LMOE_ERR_CUDA;
+  }
+  const size_t need = 2 * (size_t)n + 2;
+  while (c->host_ev.size() < need) {
+    cudaEvent_t e;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return LMOE_ERR_CUDA;
+    c->host_ev.push_back(e);
+  }
+  cudaEvent_t* ev = c->host_ev.data();  // [0] fork, [1] join, [2 + 2i] input i copied, [3 + 2i] chunk i done
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  if (!ok(cudaEventRecord(ev[0], s)) || !ok(cudaStreamWaitEvent(c->host_in, ev[0], 0)) ||
+      !ok(cudaStreamWaitEvent(c->host_out, ev[0], 0)))
+    return LMOE_ERR_CUDA;
+  const size_t row = (size_t)g.d * 2;
+  for (int i = 0; i < n; ++i) {
+    const size_t t0 = (size_t)i * chunk, tn = (size_t)(T - (int)t0 < chunk ? T - (int)t0 : chunk);
+    if (!ok(cudaMemcpyAsync(reinterpret_cast<uint8_t*>(c->x_dev) + t0 * row,
+                            reinterpret_cast<const uint8_t*>(x_host) + t0 * row, tn * row, cudaMemcpyHostToDevice,
+                            c->host_in)) ||
+        !ok(cudaEventRecord(ev[2 + 2 * i], c->host_in)))
+      return LMOE_ERR_CUDA;
+  }
+  for (int i = 0; i < n; ++i) {
+    const size_t t0 = (size_t)i * chunk, tn = (size_t)(T - (int)t0 < chunk ? T - (int)t0 : chunk);
+    const size_t k0 = t0 * g.top_k, kn = tn * g.top_k;
+    if (!ok(cudaStreamWaitEvent(s, ev[2 + 2 * i], 0))) return LMOE_ERR_CUDA;
+    const lmoe_status st = lmoe_forward(c, reinterpret_cast<uint8_t*>(c->x_dev) + t0 * row, (int)tn,
+                                        reinterpret_cast<uint8_t*>(c->y_dev) + t0 * row, c->idx_dev + k0,
+                                        c->gate_dev + k0, s);
+    if (st != LMOE_OK) return st;
+    if (!ok(cudaEventRecord(ev[3 + 2 * i], s)) || !ok(cudaStreamWaitEvent(c->host_out, ev[3 + 2 * i], 0)) ||
+        !ok(cudaMemcpyAsync(reinterpret_cast<uint8_t*>(y_host) + t0 * row,
+                            reinterpret_cast<const uint8_t*>(c->y_dev) + t0 * row, tn * row, cudaMemcpyDeviceToHost,
+                            c->host_out)))
+      return LMOE_ERR_CUDA;
+    if (idx_host && !ok(cudaMemcpyAsync(idx_host + k0, c->idx_dev + k0, kn * 4, cudaMemcpyDeviceToHost, c->host_out)))
+      return LMOE_ERR_CUDA;
+    if (gate_host &&
+        !ok(cudaMemcpyAsync(gate_host + k0, c->gate_dev + k0, kn * 4, cudaMemcpyDeviceToHost, c->host_out)))
+      return LMOE_ERR_CUDA;
+  }
+  if (!ok(cudaEventRecord(ev[1], c->host_out)) || !ok(cudaStreamWaitEvent(s, ev[1], 0))) return LMOE_ERR_CUDA;
+  return LMOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1282,6 +1352,8 @@ lmoe_status lmoe_forward_host(lmoe_handle c, const void* x_host, int32_t T, void
       return LMOE_ERR_OOM;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int chunk = host_chunk_tokens(c, T);
+  if (chunk < T) return forward_host_chunked(c, x_host, T, y_host, idx_host, gate_host, s, chunk);
   const size_t bytes = (size_t)T * g.d * 2;
   if (cudaMemcpyAsync(c->x_dev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return LMOE_ERR_CUDA;
   lmoe_status st = lmoe_forward(c, c->x_dev, T, c->y_dev, c->idx_dev, c->gate_dev, stream);
@@ -1595,6 +1667,9 @@ void lmoe_destroy(lmoe_handle c) {
     DeviceGuard dg(c->device);
     cudaDeviceSynchronize();
     for (auto& e : c->prof_ev) cudaEventDestroy(e);
+    for (auto& e : c->host_ev) cudaEventDestroy(e);
+    if (c->host_in) cudaStreamDestroy(c->host_in);
+    if (c->host_out) cudaStreamDestroy(c->host_out);
     free_all(c);
   }
   delete c;

@@ -12,8 +12,8 @@ import torch
 
 import lmoe_inputs as inp
 from oracle import lmoe_oracle as lo
-from lmoe_testlib import (bf16_to_np, check_dispatch, compare_bf16, device_weights, host_weights, make_layer,
-                          oracle_weights, run_layer, to_dev)
+from lmoe_testlib import (Y_TOL_BF16, bf16_to_np, check_dispatch, compare_bf16, device_weights, host_weights,
+                          make_layer, oracle_weights, run_layer, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -130,6 +130,34 @@ def test_prefill_sampled_parity_and_full_dispatch(superlayer):
     print(f"prefill: rel err {st['rel_err']:.3g} on {st['tokens_y_checked']} tokens, logit err "
           f"{st['logit_err']:.3g}, routing checked on {st['tokens_routed_checked']} tokens, near ties "
           f"{st['near_ties']}, routing diffs {st['routing_diffs']}")
+
+
+def test_prefill_host_forward_in_chunks_matches_device_forward(superlayer):
+    """lmoe_forward_host splits the 16384-token batch into 4096-token chunks whose copies overlap the
+    neighbouring chunks' compute.  Every token's routing equals the one-call device forward's bit for
+    bit; y equals it within the parity tolerance (the chunks' expert-up GEMM runs as CTA pairs, the
+    one-call forward's on one CTA)."""
+    w, _, layer = superlayer
+    wl = inp.workload("prefill")
+    x_np = inp.make_x(wl)
+    y_dev, idx_dev, gate_dev = run_layer(layer, x_np)
+    xh = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty((wl.tokens, wl.shape.d), dtype=torch.bfloat16).pin_memory()
+    ih = torch.empty((wl.tokens, wl.shape.top_k), dtype=torch.int32).pin_memory()
+    gh = torch.empty((wl.tokens, wl.shape.top_k), dtype=torch.float32).pin_memory()
+    for _ in range(2):  # twice: the second call's input copies must wait for the first call's layer
+        yh.zero_()
+        layer.forward_host(xh, yh, ih, gh)
+        torch.cuda.synchronize()
+        assert layer.device_status() == 0
+        assert np.array_equal(ih.numpy(), idx_dev)
+        assert np.array_equal(gh.numpy(), gate_dev)
+        y_host = bf16_to_np(yh)
+        rms = np.sqrt(np.mean(y_dev ** 2))
+        err = np.abs(y_host - y_dev).max()
+        assert err <= Y_TOL_BF16 * rms, f"chunked host forward differs: {err:.3g} vs RMS {rms:.3g}"
+    print(f"prefill host forward in chunks: max|dy|/RMS {err / rms:.3g}, "
+          f"bit-identical y: {bool(np.array_equal(y_host, y_dev))}")
 
 
 @pytest.fixture(scope="module")
