@@ -55,13 +55,13 @@ DEFAULT_STEPS.update({"decode_small": 400, "decode_nvfp4": 400, "prefill_nvfp4":
 # expert on average; expert down as CTA pairs).  Valid only while the GEMM's sources are the ones
 # captured (TRAFFIC_SOURCES_SHA256); otherwise the roofline reports no traffic.
 TRAFFIC_RATIO = {
-    ("bf16", "decode", "expert_up"): 0.999, ("bf16", "decode", "expert_down"): 1.002,
-    ("nvfp4", "decode", "expert_up"): 1.383, ("nvfp4", "decode", "expert_down"): 1.496,
-    ("bf16", "prefill", "expert_up"): 0.982, ("bf16", "prefill", "expert_down"): 1.018,
-    ("nvfp4", "prefill", "expert_up"): 1.461, ("nvfp4", "prefill", "expert_down"): 1.247,
+    ("bf16", "decode", "expert_up"): 0.997, ("bf16", "decode", "expert_down"): 1.001,
+    ("nvfp4", "decode", "expert_up"): 1.382, ("nvfp4", "decode", "expert_down"): 1.494,
+    ("bf16", "prefill", "expert_up"): 0.982, ("bf16", "prefill", "expert_down"): 1.029,
+    ("nvfp4", "prefill", "expert_up"): 1.460, ("nvfp4", "prefill", "expert_down"): 1.246,
 }
 TRAFFIC_SOURCES = ("gemm_tc.cuh", "ptx.cuh", "nvfp4.cuh", "lmoe.cu")
-TRAFFIC_SOURCES_SHA256 = "48c96b284fafc2ee762ee4f565732f0d5bd5efda40b10f8aecba3e1d6c863842"
+TRAFFIC_SOURCES_SHA256 = "e96e97b9d221e6a37ee1cd5030aa01b7fea8ef5535f5c81f9f5815fc4182206c"
 
 
 def gemm_sources_sha256() -> str:

@@ -796,35 +796,40 @@ lmoe_status forward_host_chunked(lmoe_ctx* c, const void* x_host, int T, void* y
       !ok(cudaStreamWaitEvent(c->host_out, ev[0], 0)))
     return LMOE_ERR_CUDA;
   const size_t row = (size_t)g.d * 2;
-  for (int i = 0; i < n; ++i) {
+  lmoe_status st = LMOE_OK;
+  for (int i = 0; i < n && st == LMOE_OK; ++i) {
     const size_t t0 = (size_t)i * chunk, tn = (size_t)(T - (int)t0 < chunk ? T - (int)t0 : chunk);
     if (!ok(cudaMemcpyAsync(reinterpret_cast<uint8_t*>(c->x_dev) + t0 * row,
                             reinterpret_cast<const uint8_t*>(x_host) + t0 * row, tn * row, cudaMemcpyHostToDevice,
                             c->host_in)) ||
         !ok(cudaEventRecord(ev[2 + 2 * i], c->host_in)))
-      return LMOE_ERR_CUDA;
+      st = LMOE_ERR_CUDA;
   }
-  for (int i = 0; i < n; ++i) {
+  for (int i = 0; i < n && st == LMOE_OK; ++i) {
     const size_t t0 = (size_t)i * chunk, tn = (size_t)(T - (int)t0 < chunk ? T - (int)t0 : chunk);
     const size_t k0 = t0 * g.top_k, kn = tn * g.top_k;
-    if (!ok(cudaStreamWaitEvent(s, ev[2 + 2 * i], 0))) return LMOE_ERR_CUDA;
-    const lmoe_status st = lmoe_forward(c, reinterpret_cast<uint8_t*>(c->x_dev) + t0 * row, (int)tn,
-                                        reinterpret_cast<uint8_t*>(c->y_dev) + t0 * row, c->idx_dev + k0,
-                                        c->gate_dev + k0, s);
-    if (st != LMOE_OK) return st;
+    if (!ok(cudaStreamWaitEvent(s, ev[2 + 2 * i], 0))) {
+      st = LMOE_ERR_CUDA;
+      break;
+    }
+    st = lmoe_forward(c, reinterpret_cast<uint8_t*>(c->x_dev) + t0 * row, (int)tn,
+                      reinterpret_cast<uint8_t*>(c->y_dev) + t0 * row, c->idx_dev + k0, c->gate_dev + k0, s);
+    if (st != LMOE_OK) break;
     if (!ok(cudaEventRecord(ev[3 + 2 * i], s)) || !ok(cudaStreamWaitEvent(c->host_out, ev[3 + 2 * i], 0)) ||
         !ok(cudaMemcpyAsync(reinterpret_cast<uint8_t*>(y_host) + t0 * row,
                             reinterpret_cast<const uint8_t*>(c->y_dev) + t0 * row, tn * row, cudaMemcpyDeviceToHost,
-                            c->host_out)))
-      return LMOE_ERR_CUDA;
-    if (idx_host && !ok(cudaMemcpyAsync(idx_host + k0, c->idx_dev + k0, kn * 4, cudaMemcpyDeviceToHost, c->host_out)))
-      return LMOE_ERR_CUDA;
-    if (gate_host &&
-        !ok(cudaMemcpyAsync(gate_host + k0, c->gate_dev + k0, kn * 4, cudaMemcpyDeviceToHost, c->host_out)))
-      return LMOE_ERR_CUDA;
+                            c->host_out)) ||
+        (idx_host && !ok(cudaMemcpyAsync(idx_host + k0, c->idx_dev + k0, kn * 4, cudaMemcpyDeviceToHost, c->host_out))) ||
+        (gate_host &&
+         !ok(cudaMemcpyAsync(gate_host + k0, c->gate_dev + k0, kn * 4, cudaMemcpyDeviceToHost, c->host_out))))
+      st = LMOE_ERR_CUDA;
   }
-  if (!ok(cudaEventRecord(ev[1], c->host_out)) || !ok(cudaStreamWaitEvent(s, ev[1], 0))) return LMOE_ERR_CUDA;
-  return LMOE_OK;
+  // join both copy streams back into the caller's stream, on the error paths too, so that a
+  // synchronisation of that stream covers every copy this call enqueued
+  const bool joined = ok(cudaEventRecord(ev[1], c->host_in)) && ok(cudaStreamWaitEvent(s, ev[1], 0)) &&
+                      ok(cudaEventRecord(ev[1], c->host_out)) && ok(cudaStreamWaitEvent(s, ev[1], 0));
+  if (st == LMOE_OK && !joined) st = LMOE_ERR_CUDA;
+  return st;
 }
 
 }  // namespace
