@@ -57,11 +57,11 @@ DEFAULT_STEPS.update({"decode_small": 400, "decode_nvfp4": 400, "prefill_nvfp4":
 TRAFFIC_RATIO = {
     ("bf16", "decode", "expert_up"): 0.997, ("bf16", "decode", "expert_down"): 1.001,
     ("nvfp4", "decode", "expert_up"): 1.382, ("nvfp4", "decode", "expert_down"): 1.494,
-    ("bf16", "prefill", "expert_up"): 0.982, ("bf16", "prefill", "expert_down"): 1.029,
-    ("nvfp4", "prefill", "expert_up"): 1.460, ("nvfp4", "prefill", "expert_down"): 1.246,
+    ("bf16", "prefill", "expert_up"): 0.982, ("bf16", "prefill", "expert_down"): 1.066,
+    ("nvfp4", "prefill", "expert_up"): 1.462, ("nvfp4", "prefill", "expert_down"): 1.246,
 }
 TRAFFIC_SOURCES = ("gemm_tc.cuh", "ptx.cuh", "nvfp4.cuh", "lmoe.cu")
-TRAFFIC_SOURCES_SHA256 = "e96e97b9d221e6a37ee1cd5030aa01b7fea8ef5535f5c81f9f5815fc4182206c"
+TRAFFIC_SOURCES_SHA256 = "1f79b6d41f17bb69eec54cc37e63ce8600503863bcafe7e6a16440a17a1cd993"
 
 
 def gemm_sources_sha256() -> str:

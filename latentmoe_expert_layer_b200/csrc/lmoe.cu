@@ -548,9 +548,6 @@ cudaError_t launch_route_fused_p(const RouteFusedArgs& a, int grid, cudaStream_t
   return cudaLaunchKernelEx(&cfg, route_fused_kernel<P>, a);
 }
 
-// Experts whose first matrix the fused routing kernel prefetches into L2 for the expert-up launch.
-constexpr int kPrefetchExperts = 6;
-
 // fp4_x: NVFP4 experts (the layer input x, quantised here with h); nullptr for bf16 experts.
 cudaError_t launch_route_fused(lmoe_ctx* c, int T, int ks, int nch, int ct, int* idx, float* gate,
                                const UnitListSpec& l1, const UnitListSpec& l2, cudaStream_t s,
@@ -584,14 +581,6 @@ cudaError_t launch_route_fused(lmoe_ctx* c, int T, int ks, int nch, int ct, int*
   a.h_perm = c->h_perm;
   a.zero_words = c->work_counters;
   a.n_zero = lmoe_ctx::kAmaxX;  // the unit counters (the activation maxima are zeroed before the launch)
-  if (!fp4_x && c->ws1 && c->w1) {
-    // bf16 experts: the expert-up launch reads W_s1 first (its dense pre problem), then the experts
-    // in index order; about 80 MB of it goes to L2 while this kernel runs
-    a.pf_ptr[0] = reinterpret_cast<const uint8_t*>(c->ws1);
-    a.pf_bytes[0] = (long long)g.shared_ffn * g.d * 2;
-    a.pf_ptr[1] = reinterpret_cast<const uint8_t*>(c->w1);
-    a.pf_bytes[1] = (long long)(c->n_local < kPrefetchExperts ? c->n_local : kPrefetchExperts) * g.expert_ffn * c->le * 2;
-  }
   if (fp4_x) {
     a.fp4 = 1;
     a.x = reinterpret_cast<const __nv_bfloat16*>(fp4_x);

@@ -213,13 +213,6 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(uint32_t m, uint32_t n) {
          | ((m >> 4) << 24);  // M / 16   (bit 23 = 0: E4M3 scales; bit 31 = 0: K = 64)
 }
 
-// Start fetching `bytes` (multiple of 16) of global memory at `p` (16-byte aligned) into L2; the
-// instruction does not wait for the data.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
-               : "memory");
-}
-
 // Bulk copy (no tensor map) of `bytes` (multiple of 16, 16-byte aligned) into shared memory.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
   asm volatile(

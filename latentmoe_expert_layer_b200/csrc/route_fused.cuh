@@ -22,10 +22,6 @@
 // launch's dense tile atoms) and h once per token with the dynamic tensor scales; phase 3 copies
 // each grouped row's h codes and scales (tile-local atoms) instead of gathering bf16 rows.
 //
-// While the routing chain runs, HBM is almost idle: at the start every block asks L2 to fetch its
-// share of up to two weight ranges that the next launch (the expert-up GEMM) reads first (bf16
-// experts: the shared expert's first matrix and the lowest experts' first matrices).
-//
 // The grid barrier is self-resetting (an arrival count and a generation word, both zero when the
 // layer is created) and its wait is bounded by wall-clock time: on expiry the block raises
 // DEV_STATUS_TIMEOUT and returns (the host then resets the barrier words when it reads the status).
@@ -79,10 +75,6 @@ struct RouteFusedArgs {
   uint8_t* h_sf;               //   grouped h block scales, tile-local atoms
   int tile_tokens4;            // token tile of the FP4 expert variant
   int nra4;                    // its 128-row scale atoms per tile
-  // L2 prefetch of the next launch's first weights: ranges of pf_bytes[i] (multiples of 16, 16-byte
-  // aligned; 0: none)
-  const uint8_t* pf_ptr[2];
-  long long pf_bytes[2];
 };
 
 // Grid-wide barrier of a cooperative launch (every block resident).  Returns false, with
@@ -186,13 +178,6 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteFusedArgs a
   const int t_begin = b * a.chunk_tokens, t_end = min(a.T, t_begin + a.chunk_tokens);
 
   // ------------------------------------------------------------------ phase 1
-  if (tid < 2 && a.pf_bytes[tid] > 0) {
-    // this block's share of range tid, in pieces of at most 64 KB
-    const long long per = ((a.pf_bytes[tid] + G - 1) / G + 15) & ~15LL;
-    const long long lo = min(a.pf_bytes[tid], (long long)b * per), hi = min(a.pf_bytes[tid], lo + per);
-    for (long long o = lo; o < hi; o += 65536)
-      prefetch_l2_bulk(a.pf_ptr[tid] + o, (uint32_t)min(65536LL, hi - o));
-  }
   int* s_counts = smem_i;  // [N]
   for (int e = tid; e < N; e += blockDim.x) s_counts[e] = 0;
   if (b == 0)
