@@ -18,11 +18,12 @@
 //          atoms (one 128x256b copy per K atom).  The epilogue multiplies by the two fp32 tensor
 //          scales.
 //
-// Roles (192 threads):
-//   warp 0      producer: streams W and activation tiles (TMA) and scales into a STAGES-deep ring
+// Roles (64 + 32 * EPIW threads; EPIW = 4 epilogue warps, or 8 for the NVFP4 prefill variant):
+//   warp 0      producer: streams W and activation tiles (TMA) and scales into a STAGES-deep ring,
+//               and publishes each unit's descriptor to the other roles through a shared-memory ring
 //   warp 1      MMA issuer: allocates TMEM, one lane issues tcgen05 MMAs into one of two TMEM
 //               accumulators (double buffered, so the epilogue of tile i overlaps the MMAs of i+1)
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes 32*(w%4)..),
+//   warps 2..   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes 32*(w%4)..),
 //               elementwise op, transpose through shared memory, vector stores
 //
 // Work units are (weight row block, token block) pairs.  Dense GEMMs enumerate them from the
