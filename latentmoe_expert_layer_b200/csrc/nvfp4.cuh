@@ -400,7 +400,9 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ a, int K, con
 // ------------------------------------------------------------------------------------------------
 // Rows r = r0, r0 + stride, ... of gather_act_q_kernel, one per warp (shared with the fused decode
 // routing, which wrote the routing maps and the per-token codes earlier in the same launch).
-template <bool SAME_LAUNCH>
+// MAPS_SMEM: offsets and tile0 point to copies in shared memory (the per-row expert search then
+// costs no memory round trips).
+template <bool SAME_LAUNCH, bool MAPS_SMEM = false>
 __device__ __forceinline__ void gather_act_q_rows(const uint8_t* __restrict__ codes_tok,
                                                   const uint8_t* __restrict__ sf_tok, int K,
                                                   const int* __restrict__ tok_of_row, long long n_rows, int n_tok,
@@ -420,11 +422,11 @@ __device__ __forceinline__ void gather_act_q_rows(const uint8_t* __restrict__ co
     int lo = 0, hi = n_experts - 1;  // largest expert whose first row is <= r
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (ld_act<SAME_LAUNCH>(offsets + mid) <= r) lo = mid;
+      if ((MAPS_SMEM ? offsets[mid] : ld_act<SAME_LAUNCH>(offsets + mid)) <= r) lo = mid;
       else hi = mid - 1;
     }
-    const int local = (int)(r - ld_act<SAME_LAUNCH>(offsets + lo));
-    const long long tile = ld_act<SAME_LAUNCH>(tile0 + lo) + local / tile_rows;
+    const int local = (int)(r - (MAPS_SMEM ? offsets[lo] : ld_act<SAME_LAUNCH>(offsets + lo)));
+    const long long tile = (MAPS_SMEM ? tile0[lo] : ld_act<SAME_LAUNCH>(tile0 + lo)) + local / tile_rows;
     const int j = local % tile_rows;
     for (int c = lane * 16; c < row_bytes; c += 32 * 16)
       *reinterpret_cast<uint4*>(codes + r * row_bytes + c) =

@@ -437,7 +437,16 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteFusedArgs a
 
   if (a.fp4) {
     // ------------------------------------------------------------------ phase 3 (NVFP4)
-    gather_act_q_rows<true>(a.hq_tok, a.h_sf_tok, l, a.tok_of_row, (long long)a.T * K, a.T, a.offsets, a.tile0, N,
+    // the expert offsets and first token tiles, once per block into shared memory: every row's
+    // expert search then runs there
+    int* s_offm = smem_i;            // [N + 1]
+    int* s_t0m = smem_i + (N + 1);   // [N + 1]
+    for (int e = tid; e <= N; e += blockDim.x) {
+      s_offm[e] = __ldcg(a.offsets + e);
+      s_t0m[e] = __ldcg(a.tile0 + e);
+    }
+    __syncthreads();
+    gather_act_q_rows<true, true>(a.hq_tok, a.h_sf_tok, l, a.tok_of_row, (long long)a.T * K, a.T, s_offm, s_t0m, N,
                       a.tile_tokens4, a.nra4, a.hq, a.h_sf, a.status, 1, (long long)b * W + warp, (long long)G * W);
     return;
   }
