@@ -55,13 +55,13 @@ DEFAULT_STEPS.update({"decode_small": 400, "decode_nvfp4": 400, "prefill_nvfp4":
 # expert on average; expert down as CTA pairs).  Valid only while the GEMM's sources are the ones
 # captured (TRAFFIC_SOURCES_SHA256); otherwise the roofline reports no traffic.
 TRAFFIC_RATIO = {
-    ("bf16", "decode", "expert_up"): 0.997, ("bf16", "decode", "expert_down"): 1.001,
-    ("nvfp4", "decode", "expert_up"): 1.382, ("nvfp4", "decode", "expert_down"): 1.494,
-    ("bf16", "prefill", "expert_up"): 0.982, ("bf16", "prefill", "expert_down"): 1.066,
-    ("nvfp4", "prefill", "expert_up"): 1.462, ("nvfp4", "prefill", "expert_down"): 1.246,
+    ("bf16", "decode", "expert_up"): 0.998, ("bf16", "decode", "expert_down"): 1.001,
+    ("nvfp4", "decode", "expert_up"): 1.384, ("nvfp4", "decode", "expert_down"): 1.494,
+    ("bf16", "prefill", "expert_up"): 0.982, ("bf16", "prefill", "expert_down"): 1.051,
+    ("nvfp4", "prefill", "expert_up"): 1.457, ("nvfp4", "prefill", "expert_down"): 1.246,
 }
 TRAFFIC_SOURCES = ("gemm_tc.cuh", "ptx.cuh", "nvfp4.cuh", "lmoe.cu")
-TRAFFIC_SOURCES_SHA256 = "1f79b6d41f17bb69eec54cc37e63ce8600503863bcafe7e6a16440a17a1cd993"
+TRAFFIC_SOURCES_SHA256 = "5aeb9bc3143e270f9362e872b6c4cf2a8d1ca6985c385975e30c8f2bc0ccc353"
 
 
 def gemm_sources_sha256() -> str:
