@@ -132,6 +132,29 @@ def test_prefill_sampled_parity_and_full_dispatch(superlayer):
           f"{st['near_ties']}, routing diffs {st['routing_diffs']}")
 
 
+def test_decode_host_forward_matches_device_forward(superlayer):
+    """lmoe_forward_host at decode size (one call, no chunks): copies in, the layer, copies out, all on
+    the caller's stream; the results equal the device-buffer forward's bit for bit, and a call with
+    NULL idx / gate outputs still writes y."""
+    _, _, layer = superlayer
+    wl = inp.workload("decode")
+    x_np = inp.make_x(wl)
+    y_dev, idx_dev, gate_dev = run_layer(layer, x_np)
+    xh = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.zeros((wl.tokens, wl.shape.d), dtype=torch.bfloat16).pin_memory()
+    ih = torch.empty((wl.tokens, wl.shape.top_k), dtype=torch.int32).pin_memory()
+    gh = torch.empty((wl.tokens, wl.shape.top_k), dtype=torch.float32).pin_memory()
+    layer.forward_host(xh, yh, ih, gh)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert np.array_equal(bf16_to_np(yh), y_dev)
+    assert np.array_equal(ih.numpy(), idx_dev) and np.array_equal(gh.numpy(), gate_dev)
+    yh.zero_()
+    layer.forward_host(xh, yh)
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_to_np(yh), y_dev)
+
+
 def test_prefill_host_forward_in_chunks_matches_device_forward(superlayer):
     """lmoe_forward_host splits the 16384-token batch into 4096-token chunks whose copies overlap the
     neighbouring chunks' compute.  Every token's routing equals the one-call device forward's bit for
